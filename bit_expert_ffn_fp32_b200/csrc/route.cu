@@ -1,0 +1,172 @@
+// Router logits (fixed-order fp32) and top-k gates.
+//
+// Per token a router scores the layer's experts and the top 10 of 512 are used
+// ("个人开发者用 AI 十天写出 Strata 引擎，让 12GB 显存跑起 1250 亿参数的 Qwen 3.8 Flash
+// Next", section "1250 亿参数，每个词只用得上 2%"). The logit's fp32 value is defined
+// by a fixed order of operations (see moe_route in moe.h) that a warp follows
+// natively: lane l owns elements 128i+4l+j, accumulates them with fused
+// multiply-adds chunk by chunk, and the butterfly of shuffles acc += shfl_xor(acc, o)
+// for o = 16..1 is exactly the pairwise combination of the definition.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTokTile = 8;      // tokens per warp
+constexpr int kWarpsPerCta = 4;  // experts per CTA
+
+// One warp = one expert x up to 8 tokens.
+__global__ void __launch_bounds__(kWarpsPerCta * 32)
+    router_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ Wr, const float *__restrict__ bias,
+                         int T, int d, int E, float *__restrict__ logits, int32_t *status) {
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    if (e >= E) return;
+    const int t0 = blockIdx.y * kTokTile;
+    const int nt = min(kTokTile, T - t0);
+    const float *w = Wr + size_t(e) * d + 4 * lane;
+    const uint16_t *xb = x + size_t(t0) * d + 4 * lane;
+    float acc[kTokTile];
+#pragma unroll
+    for (int tt = 0; tt < kTokTile; ++tt) acc[tt] = 0.0f;
+    const int nchunk = d / 128;
+#pragma unroll 4
+    for (int i = 0; i < nchunk; ++i) {
+        const float4 wv = __ldg(reinterpret_cast<const float4 *>(w + 128 * i));
+#pragma unroll
+        for (int tt = 0; tt < kTokTile; ++tt) {
+            if (tt < nt) {
+                const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(xb + size_t(tt) * d + 128 * i));
+                float a = acc[tt];
+                a = __fmaf_rn(bf16_lo(xv.x), wv.x, a);
+                a = __fmaf_rn(bf16_hi(xv.x), wv.y, a);
+                a = __fmaf_rn(bf16_lo(xv.y), wv.z, a);
+                a = __fmaf_rn(bf16_hi(xv.y), wv.w, a);
+                acc[tt] = a;
+            }
+        }
+    }
+#pragma unroll
+    for (int tt = 0; tt < kTokTile; ++tt) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) acc[tt] = __fadd_rn(acc[tt], __shfl_xor_sync(0xffffffffu, acc[tt], o));
+    }
+    if (lane == 0) {
+        const float b = bias ? bias[e] : 0.0f;
+        for (int tt = 0; tt < nt; ++tt) {
+            float v = bias ? __fadd_rn(acc[tt], b) : acc[tt];
+            if (!isfinite(v)) flag(status, MOE_DEV_NONFINITE);
+            logits[size_t(t0 + tt) * E + e] = v;
+        }
+    }
+}
+
+// (v1, i1) comes before (v2, i2): larger logit first, then lower id. NaN never wins.
+__device__ __forceinline__ bool before(float v1, int i1, float v2, int i2) {
+    return v1 > v2 || (v1 == v2 && i1 < i2);
+}
+
+// One warp per token: k rounds of warp-wide arg-max, then softmax over the k.
+__global__ void topk_kernel(const float *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ idx,
+                            float *__restrict__ gate, int32_t *status) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float *row = logits + size_t(t) * E;
+    uint32_t taken[kMaxE / 32 / 32];  // bit m of word m/32: candidate lane + 32*m taken
+#pragma unroll
+    for (int i = 0; i < kMaxE / 1024; ++i) taken[i] = 0;
+    const int per_lane = (E + 31) / 32;
+    bool saw_nan = false;
+    int sel_id[kMaxK];
+    float sel_v[kMaxK];
+    for (int r = 0; r < k; ++r) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int m = 0; m < per_lane; ++m) {
+            const int e = lane + 32 * m;
+            if (e >= E) break;
+            if ((taken[m >> 5] >> (m & 31)) & 1u) continue;
+            const float v = row[e];
+            if (v != v) {
+                saw_nan = true;
+                continue;
+            }
+            if (before(v, e, bv, bi)) {
+                bv = v;
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (before(ov, oi, bv, bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if (bi == 0x7fffffff) {  // only NaN left: no valid choice
+            bi = 0;
+            saw_nan = true;
+        }
+        if ((bi & 31) == lane) {
+            const int m = bi >> 5;
+            taken[m >> 5] |= 1u << (m & 31);
+        }
+        sel_id[r] = bi;
+        sel_v[r] = bv;
+    }
+    if (saw_nan) flag(status, MOE_DEV_NONFINITE);
+    if (lane == 0) {
+        // selection order is by value; sort by id for the output
+        for (int a = 1; a < k; ++a) {
+            const int id = sel_id[a];
+            const float v = sel_v[a];
+            int b = a - 1;
+            while (b >= 0 && sel_id[b] > id) {
+                sel_id[b + 1] = sel_id[b];
+                sel_v[b + 1] = sel_v[b];
+                --b;
+            }
+            sel_id[b + 1] = id;
+            sel_v[b + 1] = v;
+        }
+        float mx = -INFINITY;
+        for (int a = 0; a < k; ++a) mx = fmaxf(mx, sel_v[a]);
+        float z = 0.0f;
+        float ex[kMaxK];
+        for (int a = 0; a < k; ++a) {
+            ex[a] = expf(sel_v[a] - mx);
+            z += ex[a];
+        }
+        const float inv = 1.0f / z;
+        for (int a = 0; a < k; ++a) {
+            idx[size_t(t) * k + a] = sel_id[a];
+            gate[size_t(t) * k + a] = ex[a] * inv;
+        }
+    }
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+MOE_API moe_status moe_route(const uint16_t *x, const float *Wr, const float *bias, int T, int d, int E, int k,
+                             float *logits, int32_t *topk_idx, float *topk_w, int32_t *dev_status,
+                             moe_stream_t stream) {
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+    if (d % 128 || d > kMaxDim || E > kMaxE || k > kMaxK || k > E) return MOE_ERR_UNSUPPORTED;
+    if (int64_t(T) * E >= (int64_t(1) << 31) || int64_t(T) * k >= (int64_t(1) << 31)) return MOE_ERR_OVERFLOW;
+    if (T == 0) return MOE_OK;
+    if (!x || !Wr || !logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = as_cuda(stream);
+    dim3 g1((E + kWarpsPerCta - 1) / kWarpsPerCta, (T + kTokTile - 1) / kTokTile);
+    router_logits_kernel<<<g1, kWarpsPerCta * 32, 0, s>>>(x, Wr, bias, T, d, E, logits, dev_status);
+    const int wpb = 8;
+    topk_kernel<<<(T + wpb - 1) / wpb, wpb * 32, 0, s>>>(logits, T, E, k, topk_idx, topk_w, dev_status);
+    return launch_status();
+}

@@ -1,0 +1,173 @@
+"""Device-resident MoE layers driven through the C ABI.
+
+A ``MoEStack`` owns, for one or more layers of a workload, the fp32 router
+weights (+ optional Zipf bias), the per-layer expert->slot table, and one pool
+of packed experts in HBM (resident routed experts plus one shared expert per
+layer). ``forward`` enqueues the layer's steps on the current stream:
+
+    moe_route -> moe_permute -> moe_cache_lookup -> moe_expert_ffn (routed)
+    -> moe_expert_ffn (shared, as E=1, k=1) -> moe_combine
+
+Inputs are the seeded synthetic tensors of ``synth``; weights are generated on
+the host and packed on the device by ``moe_pack_expert``.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import native, synth
+from .configs import ZIPF_ALPHA, Workload
+
+
+def _t(a, device):
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def upload_expert(ex: dict, fmt: int, d: int, f: int, dst_ptr: int, device, stream=None) -> None:
+    """Pack one canonical expert (numpy) into the device record at dst_ptr."""
+    keep = []
+    mats = []
+    for m in ("gate", "up", "down"):
+        c = ex[m]
+        parts = [_t(c["codes"], device), _t(c["scale"].view(np.int16), device),
+                 _t(None if c["min"] is None else c["min"].view(np.int16), device), _t(c["hi"], device)]
+        keep.append(parts)
+        mats.append(native.qmatrix(parts[0], parts[1], parts[2], parts[3]))
+    native.pack_expert(fmt, d, f, mats[0], mats[1], mats[2], dst_ptr, stream)
+    torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+    del keep
+
+
+@dataclass
+class Buffers:
+    T: int
+    logits: torch.Tensor
+    idx: torch.Tensor
+    w: torch.Tensor
+    counts: torch.Tensor
+    offsets: torch.Tensor
+    sorted_tok: torch.Tensor
+    sorted_j: torch.Tensor
+    inv: torch.Tensor
+    active: torch.Tensor
+    perm_ws: torch.Tensor | None
+    sop: torch.Tensor
+    miss: torch.Tensor
+    miss_count: torch.Tensor
+    h_ws: torch.Tensor
+    h_sh: torch.Tensor
+    y_perm: torch.Tensor
+    y_sh: torch.Tensor
+    y: torch.Tensor
+    status: torch.Tensor
+    sh_offsets: torch.Tensor
+    sh_sorted_tok: torch.Tensor
+    sh_sorted_j: torch.Tensor
+    sh_active: torch.Tensor
+
+
+class MoEStack:
+    def __init__(self, wl: Workload, device="cuda", seed: int | None = None, layers: int | None = None,
+                 alpha: float = ZIPF_ALPHA):
+        self.wl = wl
+        self.device = torch.device(device)
+        self.seed = wl.seed if seed is None else seed
+        self.L = wl.layers if layers is None else layers
+        self.R = wl.resident_count
+        self.slot_bytes = native.expert_bytes(wl.fmt, wl.d, wl.f)
+        if self.slot_bytes == 0:
+            raise ValueError("unsupported shape")
+        self.num_slots = self.L * self.R + self.L
+        self.pool = torch.empty(self.num_slots * self.slot_bytes, dtype=torch.uint8, device=self.device)
+        self.qpool = native.qpool(self.pool, self.slot_bytes, self.num_slots, wl.fmt, wl.d, wl.f)
+        self.Wr, self.bias, self.rank, self.slot_of_host, self.slot_of, self.shared_slot = [], [], [], [], [], []
+        for l in range(self.L):
+            Wr = synth.gen_router(self.seed, l, wl.E, wl.d)
+            rank = synth.gen_rank_perm(self.seed, l, wl.E)
+            bias = synth.zipf_bias(rank, alpha) if wl.zipf else None
+            if self.R >= wl.E:
+                slot = np.arange(wl.E, dtype=np.int32) + l * self.R
+            else:
+                slot = synth.slot_table_by_rank(rank, self.R, l * self.R)
+            self.Wr.append(_t(Wr, self.device))
+            self.bias.append(_t(bias, self.device))
+            self.rank.append(rank)
+            self.slot_of_host.append(slot)
+            self.slot_of.append(_t(slot, self.device))
+            sh = self.L * self.R + l
+            self.shared_slot.append(torch.tensor([sh], dtype=torch.int32, device=self.device))
+            for e in range(wl.E):
+                if slot[e] >= 0:
+                    self._pack(l, e, int(slot[e]))
+            self._pack(l, wl.E, sh)
+        self._bufs: dict[int, Buffers] = {}
+
+    # expert e == E is the layer's shared expert
+    def canonical_expert(self, layer: int, e: int) -> dict:
+        return synth.gen_expert(self.seed, layer, e, self.wl.fmt, self.wl.d, self.wl.f)
+
+    def _pack(self, layer: int, e: int, slot: int) -> None:
+        upload_expert(self.canonical_expert(layer, e), self.wl.fmt, self.wl.d, self.wl.f,
+                      self.pool.data_ptr() + slot * self.slot_bytes, self.device)
+
+    def buffers(self, T: int) -> Buffers:
+        if T in self._bufs:
+            return self._bufs[T]
+        wl, dev = self.wl, self.device
+        n = T * wl.k
+        i32 = dict(dtype=torch.int32, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        pws = native.permute_workspace_bytes(T, wl.k, wl.E)
+        b = Buffers(
+            T=T,
+            logits=torch.empty(max(T, 1), wl.E, **f32), idx=torch.empty(max(n, 1), **i32),
+            w=torch.empty(max(n, 1), **f32), counts=torch.empty(wl.E, **i32), offsets=torch.empty(wl.E + 1, **i32),
+            sorted_tok=torch.empty(max(n, 1), **i32), sorted_j=torch.empty(max(n, 1), **i32),
+            inv=torch.empty(max(n, 1), **i32), active=torch.empty(wl.E + 1, **i32),
+            perm_ws=torch.empty(pws, dtype=torch.uint8, device=dev) if pws else None,
+            sop=torch.empty(max(n, 1), **i32), miss=torch.empty(max(n, 1) * native.MISS_BYTES, dtype=torch.uint8,
+                                                                device=dev),
+            miss_count=torch.zeros(1, **i32),
+            h_ws=torch.empty(max(native.expert_ffn_workspace_bytes(T, wl.k, wl.f), 4), dtype=torch.uint8, device=dev),
+            h_sh=torch.empty(max(native.expert_ffn_workspace_bytes(T, 1, wl.f), 4), dtype=torch.uint8, device=dev),
+            y_perm=torch.zeros(max(n, 1), wl.d, **f32), y_sh=torch.empty(max(T, 1), wl.d, **f32),
+            y=torch.empty(max(T, 1), wl.d, **f32), status=torch.zeros(1, **i32),
+            sh_offsets=torch.tensor([0, T], **i32), sh_sorted_tok=torch.arange(max(T, 1), **i32),
+            sh_sorted_j=torch.zeros(max(T, 1), **i32), sh_active=torch.tensor([1, 0], **i32),
+        )
+        self._bufs[T] = b
+        return b
+
+    def forward(self, layer: int, x: torch.Tensor, b: Buffers | None = None, stream=None) -> Buffers:
+        """Enqueue one layer on x (bf16 bits as int16/uint16-sized tensor [T][d])."""
+        wl = self.wl
+        T = x.shape[0]
+        b = b or self.buffers(T)
+        k, E, d, f = wl.k, wl.E, wl.d, wl.f
+        native.route(x, self.Wr[layer], self.bias[layer], T, d, E, k, b.logits, b.idx, b.w, b.status, stream)
+        native.permute(b.idx, T, k, E, b.counts, b.offsets, b.sorted_tok, b.sorted_j, b.inv, b.active, b.perm_ws,
+                       0 if b.perm_ws is None else b.perm_ws.numel(), b.status, stream)
+        native.cache_lookup(self.slot_of[layer], self.num_slots, layer, b.idx, b.w, b.offsets, b.sorted_tok,
+                            b.sorted_j, T, k, E, b.sop, b.miss, b.miss_count, b.idx.numel(), b.status, stream)
+        native.expert_ffn(self.qpool, self.slot_of[layer], x, T, d, f, E, k, b.offsets, b.sorted_tok, b.sorted_j,
+                          b.active, None, b.y_perm, b.h_ws, b.h_ws.numel(), b.status, stream)
+        native.expert_ffn(self.qpool, self.shared_slot[layer], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
+                          b.sh_sorted_j, b.sh_active, None, b.y_sh, b.h_sh, b.h_sh.numel(), b.status, stream)
+        native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y, stream)
+        return b
+
+    def misses(self, b: Buffers) -> list:
+        """Miss records of the last forward (host copy; synchronises)."""
+        n = int(b.miss_count.item())
+        raw = b.miss[: min(n, b.idx.numel()) * native.MISS_BYTES].cpu().numpy().tobytes()
+        rec = np.frombuffer(raw, dtype=np.dtype([("layer", "<i4"), ("expert", "<i4"), ("token", "<i4"),
+                                                 ("j", "<i4"), ("gate", "<f4")]))
+        return [(int(r["layer"]), int(r["expert"]), int(r["token"]), int(r["j"]), float(r["gate"])) for r in rec]
+
+
+def x_tensor(x_bits: np.ndarray, device="cuda") -> torch.Tensor:
+    """bf16 bit patterns (uint16 numpy) as a device int16 tensor of the same bytes."""
+    return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).to(device)

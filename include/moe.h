@@ -1,0 +1,245 @@
+/*
+ * moe.h -- C ABI of libmoe, a CUDA (sm_100a) library for one sparse
+ * mixture-of-experts FFN layer with 2-bit / 3-bit block-quantised experts.
+ *
+ * The layer follows the MoE block described in
+ *   [SAITO] "个人开发者用 AI 十天写出 Strata 引擎，让 12GB 显存跑起 1250 亿参数的
+ *           Qwen 3.8 Flash Next" (attain.fans repost of an X article),
+ *   [JDSSL] "5070ti16g单卡跑qwen 3.8 flash next 新方案最高90t/s Hermes调用60t/s",
+ *   [EN]    "Running Qwen3.8-Flash-Next on a 12GB GPU: Custom Engine Hits 65 tok/s":
+ * per token a router picks 10 of the layer's 512 experts and one shared expert
+ * always runs ([SAITO] section "1250 亿参数，每个词只用得上 2%"); hot experts sit in a
+ * GPU-memory cache and the others are computed elsewhere ([JDSSL] section
+ * "为什么从 18t/s 变成 60-90t/s"; [SAITO] section "命中率七成，代价是答案会变");
+ * weights come in 2-bit and 3-bit tiers ([EN] section "Detailed Performance
+ * Numbers"). The pages fix none of the arithmetic; each call below states the
+ * definition this library implements.
+ *
+ * Conventions for every call:
+ *  - All array pointers are DEVICE pointers unless a parameter says "host".
+ *    The caller allocates and owns every buffer; the library never allocates,
+ *    frees or synchronises.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and runs asynchronously; results are valid once the stream has
+ *    reached that point.
+ *  - Host-side checks run first: a null required pointer, a negative or
+ *    inconsistent size or an unsupported shape returns an error code at once
+ *    and enqueues nothing. T == 0 is valid and enqueues nothing.
+ *  - Faults only the device can see (an expert id outside [0,E), a slot
+ *    outside the pool, a non-finite logit, too many misses) are OR-ed into
+ *    `*dev_status` (MOE_DEV_* bits) and the kernels finish normally; the
+ *    caller reads the word after synchronising. `dev_status` may be NULL to
+ *    ignore them. Kernels never trap.
+ *  - Calls keep no state between invocations and may run concurrently on
+ *    different streams with disjoint outputs.
+ *  - Shapes: d and f multiples of 256 (d <= 8192, f <= 8192), 1 <= k <= 16,
+ *    k <= E <= 4096, T*k < 2^31.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same handle as cudaStream_t */
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, negative or inconsistent size   */
+    MOE_ERR_UNSUPPORTED = 2, /* shape outside the supported range (see top)   */
+    MOE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required    */
+    MOE_ERR_CUDA = 4,        /* a kernel launch was rejected by the runtime   */
+    MOE_ERR_OVERFLOW = 5     /* a size product overflows                     */
+} moe_status;
+
+/* Device-side status bits, OR-ed into *dev_status. */
+#define MOE_DEV_BAD_INDEX 0x1     /* expert id outside [0,E) or repeated in a token */
+#define MOE_DEV_BAD_SLOT 0x2      /* slot_of entry outside [-1, num_slots)          */
+#define MOE_DEV_NONFINITE 0x4     /* NaN/Inf router logit, or an activation beyond  */
+                                  /* the fp16 range used for tensor-core staging    */
+#define MOE_DEV_MISS_OVERFLOW 0x8 /* more misses than miss_cap                      */
+#define MOE_DEV_TIMEOUT 0x10      /* a bounded in-kernel wait gave up               */
+
+/*
+ * Canonical storage of one quantised matrix [R][K] (host or device memory as
+ * the call states). K runs along 64-weight blocks.
+ *   codes: uint8 [R][K/4]; weight k's 2-bit code (Q2) or low two bits (Q3) at
+ *          byte k/4, bits 2*(k%4) and 2*(k%4)+1 (least significant first).
+ *   hi:    Q3 only, uint8 [R][K/8]; third code bit of weight k at byte k/8, bit k%8.
+ *   scale: fp16 bits [R][K/64], one scale s per block.
+ *   min:   Q2 only, fp16 bits [R][K/64], one offset m per block.
+ * Q2 weight: w = s*q + m, q in {0..3}.  Q3 weight: w = s*(q-4), q in {0..7}.
+ */
+typedef struct moe_qmatrix {
+    const uint8_t *codes;
+    const uint8_t *hi;     /* NULL for Q2 */
+    const uint16_t *scale;
+    const uint16_t *min;   /* NULL for Q3 */
+} moe_qmatrix;
+
+/*
+ * A pool of packed experts in device memory: slot s starts at
+ * base + s*slot_bytes (256-byte aligned, slot_bytes >= moe_expert_bytes()).
+ * Every slot holds one expert (gate [f][d], up [f][d], down [d][f]) in the
+ * library's packed record, written by moe_pack_expert. fmt is 2 (Q2) or 3 (Q3).
+ */
+typedef struct moe_qpool {
+    const void *base;
+    int64_t slot_bytes;
+    int32_t num_slots;
+    int32_t fmt;
+    int32_t d;
+    int32_t f;
+} moe_qpool;
+
+/* One routed (token, expert) pair whose expert has no slot in the pool. */
+typedef struct moe_miss {
+    int32_t layer;
+    int32_t expert;
+    int32_t token;
+    int32_t j;      /* position of the expert in the token's top-k list */
+    float gate;     /* its gate weight */
+} moe_miss;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *moe_status_str(moe_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int moe_version(void);
+
+/* ------------------------------------------------------------------ */
+/* Packing                                                             */
+/* ------------------------------------------------------------------ */
+
+/* Bytes of one packed expert record (a multiple of 256); 0 if the shape is
+ * unsupported. Q2 stores 2.5 bits and Q3 3.25 bits per weight, so a
+ * d=2048, f=768 expert takes 1,474,560 B (Q2) or 1,916,928 B (Q3). */
+size_t moe_expert_bytes(int fmt, int d, int f);
+
+/* Pack one expert from canonical storage (device pointers inside the three
+ * host structs) into a record at dst (device, 256-byte aligned,
+ * moe_expert_bytes() bytes). The record is a bijective re-ordering of the same
+ * bits, arranged for the kernels' loads; its layout is private to the library. */
+moe_status moe_pack_expert(int fmt, int d, int f, const moe_qmatrix *gate, const moe_qmatrix *up,
+                           const moe_qmatrix *down, void *dst, moe_stream_t stream);
+
+/* Same as moe_pack_expert, on the host: canonical host arrays -> host record. */
+moe_status moe_pack_expert_host(int fmt, int d, int f, const moe_qmatrix *gate, const moe_qmatrix *up,
+                                const moe_qmatrix *down, void *dst_host);
+
+/* Inverse of moe_pack_expert_host: host record -> canonical host arrays
+ * (the struct members point at caller-owned writable host buffers). */
+moe_status moe_unpack_expert_host(int fmt, int d, int f, const void *record_host, moe_qmatrix *gate,
+                                  moe_qmatrix *up, moe_qmatrix *down);
+
+/* ------------------------------------------------------------------ */
+/* The layer's steps                                                   */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Router and top-k gates ([SAITO] "1250 亿参数，每个词只用得上 2%": 10 of 512
+ * experts per token; the router is kept on the GPU per "命中率七成，代价是答案会变").
+ *   x       bf16 bits [T][d], row-major
+ *   Wr      fp32 [E][d], row-major
+ *   bias    fp32 [E] or NULL
+ *   logits  fp32 [T][E] (output): the router logit as an fp32 value with a
+ *           fixed order of operations -- d is cut into d/128 chunks; inside
+ *           chunk i accumulator l (0..31) takes elements 128i+4l+j, j=0..3, by
+ *           fused multiply-add, chunks in order; the 32 accumulators are
+ *           combined by acc[l] += acc[l^o] for o = 16,8,4,2,1; the bias is
+ *           added last. d must be a multiple of 128 (256 for the whole library).
+ *   topk_idx int32 [T][k] (output): the k experts that come first in the
+ *           order (logit desc, id asc), listed in ascending id.
+ *   topk_w  fp32 [T][k] (output): softmax of the k selected logits (equal to
+ *           a full softmax renormalised over the selected experts).
+ * A NaN logit sets MOE_DEV_NONFINITE and is never selected.
+ */
+moe_status moe_route(const uint16_t *x, const float *Wr, const float *bias, int T, int d, int E, int k,
+                     float *logits, int32_t *topk_idx, float *topk_w, int32_t *dev_status,
+                     moe_stream_t stream);
+
+/* Workspace bytes moe_permute needs for (T, k, E); may be 0. */
+size_t moe_permute_workspace_bytes(int T, int k, int E);
+
+/*
+ * Token -> expert permutation: the T*k pairs p = t*k + j are sorted by expert
+ * id and, within an expert, by p (a stable counting sort).
+ *   counts   int32 [E]      pairs per expert
+ *   offsets  int32 [E+1]    exclusive prefix sum of counts
+ *   sorted_tok, sorted_j int32 [T*k]: pair at sorted position s
+ *   inv      int32 [T*k]    inv[p] = sorted position of pair p
+ *   active   int32 [E+1]    active[0] = number of experts with >= 1 pair,
+ *                           active[1..] = those expert ids, ascending
+ *   ws       workspace of moe_permute_workspace_bytes() bytes (may be NULL if 0)
+ * Ids outside [0,E) or repeated within a token set MOE_DEV_BAD_INDEX.
+ */
+moe_status moe_permute(const int32_t *topk_idx, int T, int k, int E, int32_t *counts, int32_t *offsets,
+                       int32_t *sorted_tok, int32_t *sorted_j, int32_t *inv, int32_t *active, void *ws,
+                       size_t ws_bytes, int32_t *dev_status, moe_stream_t stream);
+
+/*
+ * Expert-cache lookup ([JDSSL] "为什么从 18t/s 变成 60-90t/s": a GPU-memory cache of
+ * hot experts; [SAITO] "命中率七成，代价是答案会变": experts outside it are computed
+ * on the CPU). Runs after moe_permute on the same routing.
+ *   slot_of      int32 [E]: HBM slot of each expert of this layer, -1 = not resident
+ *   num_slots    slots in the pool (entries >= num_slots set MOE_DEV_BAD_SLOT
+ *                and are treated as misses)
+ *   slot_of_pair int32 [T*k] (output): slot_of[topk_idx[p]] for pair p (-1 = miss)
+ *   miss         moe_miss [miss_cap] (output): every pair whose expert is not
+ *                resident, ordered by (expert, token); entries past miss_cap are
+ *                dropped and set MOE_DEV_MISS_OVERFLOW
+ *   miss_count   int32 [1] (output): the true number of misses
+ */
+moe_status moe_cache_lookup(const int32_t *slot_of, int32_t num_slots, int32_t layer, const int32_t *topk_idx,
+                            const float *topk_w, const int32_t *offsets, const int32_t *sorted_tok,
+                            const int32_t *sorted_j, int T, int k, int E, int32_t *slot_of_pair, moe_miss *miss,
+                            int32_t *miss_count, int32_t miss_cap, int32_t *dev_status, moe_stream_t stream);
+
+/* Workspace bytes moe_expert_ffn_q2/q3 need for (T, k, f). */
+size_t moe_expert_ffn_workspace_bytes(int T, int k, int f);
+
+/*
+ * SwiGLU experts on the packed pool: for every active expert e that has a slot
+ * and every sorted pair s of e (token t = sorted_tok[s]):
+ *     a = Wg_e x_t,  u = Wu_e x_t,  h = silu(a) * u = a / (1 + exp(-a)) * u,
+ *     y_e = Wd_e h.
+ *   W        host pointer to the pool description (W->fmt must match the call)
+ *   slot_of  int32 [E]: slot of each expert, -1 = skip (a miss)
+ *   x        bf16 bits [T][d]
+ *   offsets, sorted_tok, sorted_j, active: from moe_permute
+ *   topk_w   NULL: out is y_perm fp32 [T*k][d], row s = y_e for pair s (rows of
+ *            skipped experts are left untouched);
+ *            non-NULL: out is y fp32 [T][d] and receives y[t] += topk_w[t*k+j] * y_e
+ *            (atomic adds; the caller initialises y).
+ * The shared expert is the case E = 1, k = 1, offsets = {0, T},
+ * sorted_tok[t] = t, sorted_j[t] = 0, active = {1, 0}, slot_of = {its slot}.
+ * Activations are staged as fp16 for the tensor cores; |x| or |h| beyond
+ * 65504 sets MOE_DEV_NONFINITE.
+ */
+moe_status moe_expert_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f,
+                             int E, int k, const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j,
+                             const int32_t *active, const float *topk_w, float *out, void *ws, size_t ws_bytes,
+                             int32_t *dev_status, moe_stream_t stream);
+moe_status moe_expert_ffn_q3(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f,
+                             int E, int k, const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j,
+                             const int32_t *active, const float *topk_w, float *out, void *ws, size_t ws_bytes,
+                             int32_t *dev_status, moe_stream_t stream);
+
+/*
+ * Gate-weighted combine plus the shared expert:
+ *   y[t] = y_shared[t] + sum_{j=0..k-1, slot_of_pair[t*k+j] >= 0} topk_w[t*k+j] * y_perm[inv[t*k+j]]
+ *   y_perm fp32 [T*k][d]; inv, topk_w, slot_of_pair [T*k] (slot_of_pair may be
+ *   NULL = every pair resident); y_shared fp32 [T][d] or NULL (= 0); y fp32 [T][d].
+ */
+moe_status moe_combine(const float *y_perm, const int32_t *inv, const float *topk_w, const int32_t *slot_of_pair,
+                       const float *y_shared, int T, int k, int d, float *y, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,54 @@
+"""Shared helpers for the GPU parity tests (CUDA path vs the CPU oracle)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as orc
+from bit_expert_ffn_fp32_b200 import synth
+from bit_expert_ffn_fp32_b200.layer import MoEStack, x_tensor
+
+OUT_TOL = 2e-3      # max|y - y_ref| / max|y_ref| per layer
+GATE_RTOL = 1e-5
+
+
+def run_layer(stack: MoEStack, layer: int, x_bits: np.ndarray):
+    x = x_tensor(x_bits, stack.device)
+    b = stack.buffers(x.shape[0])
+    b.status.zero_()
+    stack.forward(layer, x, b)
+    torch.cuda.synchronize()
+    return b
+
+
+def oracle_layer(stack: MoEStack, layer: int, x_bits: np.ndarray, tokens=None):
+    wl = stack.wl
+    Wr = stack.Wr[layer].cpu().numpy()
+    bias = None if stack.bias[layer] is None else stack.bias[layer].cpu().numpy()
+    # inputs regenerated from the seeded generator, never read back from the device
+    Wr_gen = synth.gen_router(stack.seed, layer, wl.E, wl.d)
+    assert np.array_equal(Wr, Wr_gen)
+    return orc.layer(x_bits, Wr_gen, bias, lambda e: stack.canonical_expert(layer, e),
+                     stack.canonical_expert(layer, wl.E), wl.k, wl.fmt, slot_of=stack.slot_of_host[layer],
+                     layer_id=layer, tokens=tokens)
+
+
+def rel_err(y: np.ndarray, ref: np.ndarray) -> float:
+    return float(np.max(np.abs(y - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+def check_routing(b, ref, T: int, k: int, E: int):
+    logits = b.logits[:T].cpu().numpy()
+    np.testing.assert_array_equal(logits.view(np.uint32), ref["logit32"].view(np.uint32))
+    idx = b.idx[: T * k].cpu().numpy().reshape(T, k)
+    np.testing.assert_array_equal(idx, ref["idx"])
+    w = b.w[: T * k].cpu().numpy().reshape(T, k)
+    np.testing.assert_allclose(w, ref["gate"], rtol=GATE_RTOL, atol=1e-7)
+    p = ref["perm"]
+    for key, buf in (("counts", b.counts), ("offsets", b.offsets), ("sorted_tok", b.sorted_tok),
+                     ("sorted_j", b.sorted_j), ("inv", b.inv)):
+        n = p[key].shape[0]
+        np.testing.assert_array_equal(buf[:n].cpu().numpy(), p[key], err_msg=key)
+    na = int(p["active"][0])
+    np.testing.assert_array_equal(b.active[: na + 1].cpu().numpy(), p["active"][: na + 1])
+    np.testing.assert_array_equal(b.sop[: T * k].cpu().numpy(), ref["slot_of_pair"])

@@ -1,0 +1,202 @@
+"""CUDA path (through the C ABI) against the CPU oracle on the same seeded inputs.
+
+Indices (router top-k, permutation, cache slots, miss list) must match bit for
+bit, router logits too (the fp32 operation order is part of the definition);
+gates within 1e-5 relative; layer outputs within max|y-y_ref|/max|y_ref| <= 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_expert_ffn_fp32_b200 import configs, native, synth
+from bit_expert_ffn_fp32_b200.layer import MoEStack, x_tensor
+from gpu_util import OUT_TOL, check_routing, oracle_layer, rel_err, run_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(stack, layer, x_bits, tokens=None):
+    wl = stack.wl
+    T = x_bits.shape[0]
+    b = run_layer(stack, layer, x_bits)
+    ref = oracle_layer(stack, layer, x_bits, tokens=tokens)
+    assert int(b.status.item()) == 0
+    check_routing(b, ref, T, wl.k, wl.E)
+    misses = stack.misses(b)
+    assert [m[:4] for m in misses] == [m[:4] for m in ref["misses"]]
+    assert int(b.miss_count.item()) == ref["miss_count"]
+    toks = ref["tokens"]
+    y = b.y[:T].cpu().numpy().astype(np.float64)
+    err = rel_err(y[toks], ref["y_partial"][toks])
+    assert err <= OUT_TOL, err
+    return b, ref, err
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    return MoEStack(configs.TINY)
+
+
+def test_tiny_layer(tiny):
+    x = synth.gen_x(0, 0, configs.TINY.T, configs.TINY.d)
+    _full_check(tiny, 0, x)
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 7, 8, 9, 13, 31, 64])
+def test_tiny_ragged_token_counts(tiny, T):
+    x = synth.gen_x(0, 0, T, configs.TINY.d, stream=100 + T)
+    _full_check(tiny, 0, x)
+
+
+def test_tiny_zero_tokens(tiny):
+    b = tiny.buffers(0)
+    x = torch.empty(0, configs.TINY.d, dtype=torch.int16, device="cuda")
+    tiny.forward(0, x, b)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0 and int(b.active[0].item()) == 0 and int(b.miss_count.item()) == 0
+
+
+def test_tiny_ties_zero_input(tiny):
+    T = 3
+    x = np.zeros((T, configs.TINY.d), np.uint16)
+    b, ref, _ = _full_check(tiny, 0, x)
+    np.testing.assert_array_equal(ref["idx"], np.tile(np.arange(configs.TINY.k), (T, 1)))
+    assert np.all(b.y[:T].cpu().numpy() == 0)
+
+
+@pytest.fixture(scope="module")
+def decode():
+    return MoEStack(configs.DECODE)
+
+
+def test_decode_layer_full_size(decode):
+    for s in range(3):
+        x = synth.gen_x(0, 0, 1, configs.DECODE.d, stream=s)
+        _full_check(decode, 0, x)
+
+
+def test_decode_fused_gate_matches_combine(decode):
+    """moe_expert_ffn with topk_w set (gate-weighted atomic accumulation) equals
+    y_perm + moe_combine."""
+    wl = configs.DECODE
+    x = x_tensor(synth.gen_x(0, 0, 2, wl.d, stream=7))
+    b = decode.buffers(2)
+    decode.forward(0, x, b)
+    y_ref = b.y[:2].clone()
+    y2 = b.y_sh[:2].clone()
+    native.expert_ffn(decode.qpool, decode.slot_of[0], x, 2, wl.d, wl.f, wl.E, wl.k, b.offsets, b.sorted_tok,
+                      b.sorted_j, b.active, b.w, y2, b.h_ws, b.h_ws.numel(), b.status)
+    torch.cuda.synchronize()
+    assert rel_err(y2.cpu().numpy(), y_ref.cpu().numpy()) < 1e-5
+
+
+@pytest.fixture(scope="module")
+def verify():
+    return MoEStack(configs.VERIFY)
+
+
+def test_verify_layer_q3(verify):
+    for s in range(2):
+        x = synth.gen_x(0, 0, configs.VERIFY.T, configs.VERIFY.d, stream=s)
+        _full_check(verify, 0, x)
+
+
+def test_prefill_chunk_routing_and_sampled_outputs():
+    wl = configs.PREFILL
+    stack = MoEStack(wl)
+    x = synth.gen_x(0, 0, wl.T, wl.d)
+    rng = np.random.default_rng(0)
+    toks = sorted(set([0, wl.T - 1] + list(rng.choice(wl.T, 4, replace=False))))
+    b, ref, err = _full_check(stack, 0, x, tokens=toks)
+    counts = b.counts.cpu().numpy()
+    assert counts.sum() == wl.T * wl.k and counts.max() > 500     # Zipf skew present
+
+
+def test_stack48_cache_and_misses():
+    wl = configs.STACK48
+    stack = MoEStack(wl)
+    hits = total = 0
+    for l in range(wl.layers):
+        x = synth.gen_x(0, l, 1, wl.d)
+        b = run_layer(stack, l, x)
+        assert int(b.status.item()) == 0
+        sample_y = l % 6 == 0
+        ref = oracle_layer(stack, l, x, tokens=[0] if sample_y else [])
+        check_routing(b, ref, 1, wl.k, wl.E)
+        assert [m[:4] for m in stack.misses(b)] == [m[:4] for m in ref["misses"]]
+        hits += int((b.sop[: wl.k].cpu().numpy() >= 0).sum())
+        total += wl.k
+        if sample_y:
+            assert rel_err(b.y[:1].cpu().numpy().astype(np.float64), ref["y_partial"][:1]) <= OUT_TOL
+    assert 0 < hits < total
+
+
+# ---------------------------------------------------------------- device-side status
+def test_bad_expert_id_is_flagged(tiny):
+    wl = configs.TINY
+    T, k, E = 4, wl.k, wl.E
+    b = tiny.buffers(T)
+    idx = torch.tensor([[0, 1, 2, 3], [4, 5, 6, 99], [7, 7, 8, 9], [1, 2, 3, 4]], dtype=torch.int32, device="cuda")
+    b.status.zero_()
+    native.permute(idx, T, k, E, b.counts, b.offsets, b.sorted_tok, b.sorted_j, b.inv, b.active, None, 0, b.status)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) & native.DEV_BAD_INDEX
+
+
+def test_bad_slot_and_miss_overflow(tiny):
+    wl = configs.TINY
+    T = 4
+    x = x_tensor(synth.gen_x(0, 0, T, wl.d, stream=3))
+    b = tiny.buffers(T)
+    b.status.zero_()
+    tiny.forward(0, x, b)
+    slot_bad = tiny.slot_of[0].clone()
+    slot_bad[:] = -1
+    e0 = int(b.idx[0].item())
+    slot_bad[e0] = tiny.num_slots + 5        # out of range: flagged, treated as a miss
+    native.cache_lookup(slot_bad, tiny.num_slots, 0, b.idx, b.w, b.offsets, b.sorted_tok, b.sorted_j, T, wl.k, wl.E,
+                        b.sop, b.miss, b.miss_count, 3, b.status)
+    torch.cuda.synchronize()
+    st = int(b.status.item())
+    assert st & native.DEV_BAD_SLOT and st & native.DEV_MISS_OVERFLOW
+    assert int(b.miss_count.item()) == T * wl.k
+    assert np.all(b.sop[: T * wl.k].cpu().numpy() == -1)
+
+
+def test_all_misses_gives_shared_only(tiny):
+    wl = configs.TINY
+    T = 5
+    x_bits = synth.gen_x(0, 0, T, wl.d, stream=4)
+    x = x_tensor(x_bits)
+    b = tiny.buffers(T)
+    saved = tiny.slot_of[0].clone()
+    try:
+        tiny.slot_of[0].fill_(-1)
+        b.status.zero_()
+        tiny.forward(0, x, b)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(b.y[:T].cpu().numpy(), b.y_sh[:T].cpu().numpy())
+        assert int(b.miss_count.item()) == T * wl.k
+    finally:
+        tiny.slot_of[0].copy_(saved)
+
+
+def test_multi_tile_permutation():
+    # T above one 256-token tile with a ragged last tile, compared with the oracle
+    import oracle as orc
+    wl = configs.TINY
+    T, E, k = 1000, 64, 4
+    rng = np.random.default_rng(5)
+    idx_h = np.sort(np.stack([rng.choice(E, k, replace=False) for _ in range(T)]), axis=1).astype(np.int32)
+    ref = orc.permute(idx_h, E)
+    stack_b = MoEStack(wl.with_(T=T), layers=1)
+    b = stack_b.buffers(T)
+    idx = torch.from_numpy(idx_h.ravel()).cuda()
+    b.status.zero_()
+    native.permute(idx, T, k, E, b.counts, b.offsets, b.sorted_tok, b.sorted_j, b.inv, b.active, b.perm_ws,
+                   b.perm_ws.numel(), b.status)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    for key, buf in (("counts", b.counts), ("offsets", b.offsets), ("sorted_tok", b.sorted_tok),
+                     ("sorted_j", b.sorted_j), ("inv", b.inv)):
+        np.testing.assert_array_equal(buf[: ref[key].shape[0]].cpu().numpy(), ref[key], err_msg=key)
