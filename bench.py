@@ -1,0 +1,339 @@
+"""Throughput of one sparse-MoE FFN layer on B200 (C ABI, CUDA kernels).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole layer -- router + top-k, permutation, cache
+lookup, routed experts, shared expert, combine -- over one batch of T synthetic
+tokens, each step on fresh tokens already resident in HBM. Default workload:
+one decode token through a layer of d=2048, 512 experts, top-10 + shared,
+f=768, Q2 weights, Zipf-skewed routing, all experts resident.
+
+Timing: CUDA events on the launching stream around every step; a 512 MiB write
+between steps evicts the 126 MB L2, so every step reads its weights from HBM.
+With N > 1 (torchrun), every rank runs an independent replica on its own
+tokens (no collective on the data path); the reported time is the max over
+ranks. The expert FFN calls are timed separately for the roofline line.
+
+--impl reference times the CPU oracle (plain C, fp64) on a bounded sample of
+the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s (decode T=1/4, 8K prefill); % of HBM / tensor roofline"
+FLUSH_BYTES = 512 << 20
+
+
+def _env_int(name, default):
+    v = os.environ.get(name)
+    return int(v) if v not in (None, "") else default
+
+
+def _measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "50"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) < 9:
+                    continue
+                try:
+                    sm.append(float(c[1]))
+                    mx = float(c[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, c[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ reference arm (CPU oracle)
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return 0
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import oracle as orc
+    from bit_expert_ffn_fp32_b200 import synth
+    from bit_expert_ffn_fp32_b200.configs import ZIPF_ALPHA
+
+    Wr = synth.gen_router(wl.seed, 0, wl.E, wl.d)
+    rank_p = synth.gen_rank_perm(wl.seed, 0, wl.E)
+    bias = synth.zipf_bias(rank_p, ZIPF_ALPHA) if wl.zipf else None
+    shared = synth.gen_expert(wl.seed, 0, wl.E, wl.fmt, wl.d, wl.f)
+    get = lambda e: synth.gen_expert(wl.seed, 0, e, wl.fmt, wl.d, wl.f)  # noqa: E731
+    # Each step is one oracle layer call on a bounded token sample; the run stops
+    # after the requested steps or a ~120 s budget, whichever comes first.
+    T_s = min(wl.T, 4)
+    times = []
+    t_start = time.perf_counter()
+    for step in range(min(args.warmup, 1) + args.steps):
+        x = synth.gen_x(wl.seed, 0, T_s, wl.d, stream=10_000 + step)
+        t0 = time.perf_counter()
+        orc.layer(x, Wr, bias, get, shared, wl.k, wl.fmt)
+        if step >= min(args.warmup, 1):
+            times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_start > 120.0 and times:
+            break
+    tot = sum(times)
+    value = T_s * len(times) / tot
+    sample = (f"{len(times)} of {args.steps} steps run (120 s budget), {T_s} token(s) of {wl.name} per step, "
+              f"oracle layer incl. dequantisation, single thread")
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "tokens_per_step": T_s},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    """The oracle as it stands, on a bounded sample of the workload (rank 0, N=1)."""
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import oracle as orc
+    from bit_expert_ffn_fp32_b200 import synth
+    from bit_expert_ffn_fp32_b200.configs import ZIPF_ALPHA
+
+    Wr = synth.gen_router(wl.seed, 0, wl.E, wl.d)
+    bias = synth.zipf_bias(synth.gen_rank_perm(wl.seed, 0, wl.E), ZIPF_ALPHA) if wl.zipf else None
+    shared = synth.gen_expert(wl.seed, 0, wl.E, wl.fmt, wl.d, wl.f)
+    get = lambda e: synth.gen_expert(wl.seed, 0, e, wl.fmt, wl.d, wl.f)  # noqa: E731
+    T_s = min(wl.T, 4)
+    n_tok, t_tot, it = 0, 0.0, 0
+    while t_tot < budget_s and it < 64:
+        x = synth.gen_x(wl.seed, 0, T_s, wl.d, stream=20_000 + it)
+        t0 = time.perf_counter()
+        orc.layer(x, Wr, bias, get, shared, wl.k, wl.fmt)
+        t_tot += time.perf_counter() - t0
+        n_tok += T_s
+        it += 1
+    return {"value": n_tok / t_tot, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{it} oracle layer calls x {T_s} token(s) of {wl.name} ({t_tot:.1f} s, single thread, "
+                      f"dequantisation included)"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from bit_expert_ffn_fp32_b200 import configs, native, synth
+    from bit_expert_ffn_fp32_b200.layer import MoEStack, x_tensor
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stack = MoEStack(wl, device=dev, layers=1)
+    T = wl.T
+    b = stack.buffers(T)
+    stream = torch.cuda.current_stream()
+    n_steps = args.warmup + args.steps
+    # every step gets its own tokens, generated up front and resident in HBM
+    xs_host = [synth.gen_x(wl.seed, 0, T, wl.d, stream=rank * 1_000_003 + s) for s in range(n_steps)]
+    xs = torch.stack([x_tensor(x, dev) for x in xs_host])
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def layer_step(x, evs=None):
+        k, E, d, f = wl.k, wl.E, wl.d, wl.f
+        native.route(x, stack.Wr[0], stack.bias[0], T, d, E, k, b.logits, b.idx, b.w, b.status)
+        native.permute(b.idx, T, k, E, b.counts, b.offsets, b.sorted_tok, b.sorted_j, b.inv, b.active, b.perm_ws,
+                       0 if b.perm_ws is None else b.perm_ws.numel(), b.status)
+        native.cache_lookup(stack.slot_of[0], stack.num_slots, 0, b.idx, b.w, b.offsets, b.sorted_tok,
+                            b.sorted_j, T, k, E, b.sop, b.miss, b.miss_count, b.idx.numel(), b.status)
+        if evs:
+            evs[1].record(stream)
+        native.expert_ffn(stack.qpool, stack.slot_of[0], x, T, d, f, E, k, b.offsets, b.sorted_tok, b.sorted_j,
+                          b.active, None, b.y_perm, b.h_ws, b.h_ws.numel(), b.status)
+        native.expert_ffn(stack.qpool, stack.shared_slot[0], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
+                          b.sh_sorted_j, b.sh_active, None, b.y_sh, b.h_sh, b.h_sh.numel(), b.status)
+        if evs:
+            evs[2].record(stream)
+        native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y)
+
+    launches_per_step = 2 + (1 if T <= 256 else 3) + 1 + 2 + 2 + 1
+
+    # distinct routed experts per step (for the algorithmic bytes), from a warm-up pass
+    for s in range(args.warmup):
+        flush.fill_(1.0)
+        layer_step(xs[s])
+    torch.cuda.synchronize()
+    b.status.zero_()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.2)
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        layer_step(xs[args.warmup + i], ev[i])
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)]
+    ffn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    total_ms = sum(step_ms)
+    status = int(b.status.item())
+
+    # distinct experts of each step's routing (re-run routing only; not timed)
+    n_act = []
+    for i in range(min(args.steps, 256)):
+        layer_step(xs[args.warmup + i])
+        na = int(b.active[0].item())
+        ids = b.active[1:1 + na].cpu().numpy()
+        res = stack.slot_of_host[0][ids] >= 0
+        n_act.append(int(res.sum()))
+    mean_act = float(np.mean(n_act))
+
+    t = torch.tensor([total_ms, sum(ffn_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, ffn_total = float(t[0]), float(t[1])
+
+    # ---- e2e: pinned host tokens in, layer, result out, every step
+    e2e_ms = None
+    x_pin = torch.from_numpy(np.stack(xs_host[: args.steps]).view(np.int16)).pin_memory()
+    y_pin = torch.empty((args.steps, T, wl.d), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty((T, wl.d), dtype=torch.int16, device=dev)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        e2e_ev[i][0].record(stream)
+        x_dev.copy_(x_pin[i], non_blocking=True)
+        layer_step(x_dev)
+        y_pin[i].copy_(b.y[:T], non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(e2e_ev[i][0].elapsed_time(e2e_ev[i][1]) for i in range(args.steps))
+    t2 = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = float(t2[0])
+
+    if rank != 0:
+        return 0
+    hbm_peak, _, peak_kind = _measured_peaks()
+    eb = native.expert_bytes(wl.fmt, wl.d, wl.f)
+    ffn_bytes = (mean_act + 1) * eb            # routed resident experts + the shared expert, read once
+    ffn_avg_s = ffn_total / args.steps / 1e3
+    achieved = ffn_bytes / ffn_avg_s / 1e9
+    layer_bytes = wl.E * wl.d * 4 + ffn_bytes
+    tokens = world * T * args.steps
+    value = tokens / (total_ms / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "q2xf16->f32" if wl.fmt == 2 else "q3xf16->f32", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens_per_step": T, "l2": "512 MiB write between steps (flushed)",
+                   "parallelism": f"replicas x{world}", "layer_algorithmic_bytes": layer_bytes,
+                   "layer_GBps": layer_bytes / (total_ms / args.steps / 1e3) / 1e9,
+                   "mean_distinct_resident_experts": mean_act},
+        "roofline": {"bound": "hbm", "kernel": "moe_expert_ffn_q%d (gate/up + down, routed + shared)" % wl.fmt,
+                     "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "bytes_per_launch": ffn_bytes,
+                     "avg_launch_us": ffn_avg_s * 1e6},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * wl.d * 2,
+                "d2h_bytes_per_step": T * wl.d * 4},
+        "clocks": clocks, "gpu_launches": launches_per_step * args.steps, "dev_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_T1_d2048_E512_k10_f768_q2")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from bit_expert_ffn_fp32_b200.configs import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    rank = _env_int("RANK", 0)
+    world = _env_int("WORLD_SIZE", 1)
+    local_rank = _env_int("LOCAL_RANK", 0)
+    if args.impl == "reference":
+        return run_reference(args, wl, rank)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())
