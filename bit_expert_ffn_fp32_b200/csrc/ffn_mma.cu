@@ -18,6 +18,7 @@
 #include <cuda_fp16.h>
 #include <algorithm>
 #include <math.h>
+#include <mutex>
 
 #include "common.cuh"
 #include "layout.h"
@@ -413,4 +414,61 @@ MOE_API moe_status moe_expert_ffn_q3(const moe_qpool *W, const int32_t *slot_of,
                                      void *ws, size_t ws_bytes, int32_t *dev_status, moe_stream_t stream) {
     return ffn_launch<3>(W, slot_of, x, T, d, f, E, k, offsets, sorted_tok, sorted_j, active, topk_w, out, ws,
                          ws_bytes, dev_status, stream);
+}
+
+// ---------------------------------------------------------------------------
+// moe_expert_ffn_q2_noalloc: the same kernels with their h scratch in a fixed
+// array inside the library, for callers that cannot allocate device memory.
+namespace moe {
+namespace {
+constexpr size_t kNoAllocBytes = size_t(4) << 20;  // 4 MiB: T*k*f floats of h
+constexpr int kNoAllocMaxDevices = 64;
+}  // namespace
+}  // namespace moe
+
+// One copy per GPU that loads the library, kept until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[moe::kNoAllocBytes];
+
+namespace moe {
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (host code only sees a host-side stand-in under that name).
+moe_status noalloc_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MOE_OK;
+}
+}  // namespace
+}  // namespace moe
+
+MOE_API moe_status moe_expert_ffn_q2_noalloc(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T,
+                                             int d, int f, int E, int k, const int32_t *offsets,
+                                             const int32_t *sorted_tok, const int32_t *sorted_j,
+                                             const int32_t *active, const float *topk_w, float *out,
+                                             int32_t *dev_status, moe_stream_t stream) {
+    if (T > 0 && k > 0 && f > 0 && moe_expert_ffn_workspace_bytes(T, k, f) > kNoAllocBytes) return MOE_ERR_WORKSPACE;
+    void *ws = nullptr;
+    if (T > 0) {
+        const moe_status st = noalloc_scratch(&ws);
+        if (st != MOE_OK) return st;
+    }
+    return ffn_launch<2>(W, slot_of, x, T, d, f, E, k, offsets, sorted_tok, sorted_j, active, topk_w, out, ws,
+                         kNoAllocBytes, dev_status, stream);
 }

@@ -59,6 +59,8 @@ SIGNATURES = {
                                _P]),
     "moe_expert_ffn_q3": (_I, [C.POINTER(QPool), _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P,
                                _P]),
+    "moe_expert_ffn_q2_noalloc": (_I, [C.POINTER(QPool), _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
+                                       _P]),
     "moe_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
 }
 
@@ -166,6 +168,15 @@ def expert_ffn(pool: QPool, slot_of, x, T, d, f, E, k, offsets, sorted_tok, sort
     check(name, fn(C.byref(pool), ptr(slot_of), ptr(x), T, d, f, E, k, ptr(offsets), ptr(sorted_tok),
                    ptr(sorted_j), ptr(active), ptr(topk_w), ptr(out), ptr(ws), ws_bytes, ptr(dev_status),
                    stream_handle(stream)))
+
+
+def expert_ffn_q2_noalloc(pool: QPool, slot_of, x, T, d, f, E, k, offsets, sorted_tok, sorted_j, active, topk_w,
+                          out, dev_status=None, stream=None) -> None:
+    """moe_expert_ffn_q2 with the library's built-in scratch instead of a workspace."""
+    check("moe_expert_ffn_q2_noalloc",
+          lib.moe_expert_ffn_q2_noalloc(C.byref(pool), ptr(slot_of), ptr(x), T, d, f, E, k, ptr(offsets),
+                                        ptr(sorted_tok), ptr(sorted_j), ptr(active), ptr(topk_w), ptr(out),
+                                        ptr(dev_status), stream_handle(stream)))
 
 
 def combine(y_perm, inv, topk_w, slot_of_pair, y_shared, T, k, d, y, stream=None) -> None:

@@ -230,6 +230,33 @@ moe_status moe_expert_ffn_q3(const moe_qpool *W, const int32_t *slot_of, const u
                              int32_t *dev_status, moe_stream_t stream);
 
 /*
+ * moe_expert_ffn_q2 without a caller-supplied workspace. The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory -- for example a plugin inside a host framework that owns every device
+ * buffer and hands the plugin only its inputs and outputs, or a serving loop
+ * that allocates nothing after start-up so its memory footprint is fixed and no
+ * request can fail on an out-of-memory error. Arguments and results are those of
+ * moe_expert_ffn_q2; the caller still passes every input and output.
+ *   Scratch: the hidden activations (T*k*f floats) go to one 4 MiB array built
+ *   into the library; each GPU that loads the library holds its own copy until
+ *   the process exits. T*k*f*4 > 4 MiB returns MOE_ERR_WORKSPACE (for f = 768:
+ *   T*k <= 1365), before anything is enqueued.
+ *   Set-up: the first call on a device looks up that device's copy of the
+ *   array (cudaGetSymbolAddress, with the device current); make that first call
+ *   before any stream capture. Lookup failures return MOE_ERR_CUDA.
+ *   Sharing: every call on a device uses the same array, which keeps whatever
+ *   the last call wrote (nothing in it needs to start at zero: each call writes
+ *   every entry it reads). Calls that can overlap on the GPU -- on different
+ *   streams without ordering between them -- race on the array and corrupt each
+ *   other's results; order them on one stream or use moe_expert_ffn_q2.
+ *   It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+moe_status moe_expert_ffn_q2_noalloc(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d,
+                                     int f, int E, int k, const int32_t *offsets, const int32_t *sorted_tok,
+                                     const int32_t *sorted_j, const int32_t *active, const float *topk_w, float *out,
+                                     int32_t *dev_status, moe_stream_t stream);
+
+/*
  * Gate-weighted combine plus the shared expert:
  *   y[t] = y_shared[t] + sum_{j=0..k-1, slot_of_pair[t*k+j] >= 0} topk_w[t*k+j] * y_perm[inv[t*k+j]]
  *   y_perm fp32 [T*k][d]; inv, topk_w, slot_of_pair [T*k] (slot_of_pair may be
