@@ -185,8 +185,17 @@ def run_ours(args, wl, rank, world, local_rank):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
+    fused = args.path == "fused" or (args.path == "auto" and T <= 8)
+
     def layer_step(x, evs=None):
         k, E, d, f = wl.k, wl.E, wl.d, wl.f
+        if fused:
+            if evs:
+                evs[1].record(stream)
+            stack.forward_fused(0, x, b)
+            if evs:
+                evs[2].record(stream)
+            return
         native.route(x, stack.Wr[0], stack.bias[0], T, d, E, k, b.logits, b.idx, b.w, b.status)
         native.permute(b.idx, T, k, E, b.counts, b.offsets, b.sorted_tok, b.sorted_j, b.inv, b.active, b.perm_ws,
                        0 if b.perm_ws is None else b.perm_ws.numel(), b.status)
@@ -202,7 +211,7 @@ def run_ours(args, wl, rank, world, local_rank):
             evs[2].record(stream)
         native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y)
 
-    launches_per_step = 2 + (1 if T <= 256 else 3) + 1 + 2 + 2 + 1
+    launches_per_step = 1 if fused else 2 + (1 if T <= 256 else 3) + 1 + 2 + 2 + 1
 
     # distinct routed experts per step (for the algorithmic bytes), from a warm-up pass
     for s in range(args.warmup):
@@ -274,9 +283,10 @@ def run_ours(args, wl, rank, world, local_rank):
     hbm_peak, _, peak_kind = _measured_peaks()
     eb = native.expert_bytes(wl.fmt, wl.d, wl.f)
     ffn_bytes = (mean_act + 1) * eb            # routed resident experts + the shared expert, read once
+    layer_bytes = wl.E * wl.d * 4 + ffn_bytes  # + the fp32 router weights
+    kern_bytes = layer_bytes if fused else ffn_bytes
     ffn_avg_s = ffn_total / args.steps / 1e3
-    achieved = ffn_bytes / ffn_avg_s / 1e9
-    layer_bytes = wl.E * wl.d * 4 + ffn_bytes
+    achieved = kern_bytes / ffn_avg_s / 1e9
     tokens = world * T * args.steps
     value = tokens / (total_ms / 1e3)
     line = {
@@ -284,12 +294,15 @@ def run_ours(args, wl, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "q2xf16->f32" if wl.fmt == 2 else "q3xf16->f32", "data": "synthetic",
         "config": {"workload": wl.name, "tokens_per_step": T, "l2": "512 MiB write between steps (flushed)",
+                   "path": "moe_layer_decode (one launch)" if fused else "step-by-step calls",
                    "parallelism": f"replicas x{world}", "layer_algorithmic_bytes": layer_bytes,
                    "layer_GBps": layer_bytes / (total_ms / args.steps / 1e3) / 1e9,
                    "mean_distinct_resident_experts": mean_act},
-        "roofline": {"bound": "hbm", "kernel": "moe_expert_ffn_q%d (gate/up + down, routed + shared)" % wl.fmt,
+        "roofline": {"bound": "hbm",
+                     "kernel": ("decode_layer_kernel (moe_layer_decode: whole layer, one launch)" if fused else
+                                "moe_expert_ffn_q%d (gate/up + down, routed + shared)" % wl.fmt),
                      "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None, "bytes_per_launch": ffn_bytes,
+                     "frac": achieved / hbm_peak, "traffic": None, "bytes_per_launch": kern_bytes,
                      "avg_launch_us": ffn_avg_s * 1e6},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * wl.d * 2,
                 "d2h_bytes_per_step": T * wl.d * 4},
@@ -309,6 +322,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_T1_d2048_E512_k10_f768_q2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["auto", "fused", "steps"], default="auto",
+                    help="auto: one-launch layer for T <= 8 tokens, step-by-step calls otherwise")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

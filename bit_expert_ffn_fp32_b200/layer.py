@@ -104,6 +104,7 @@ class MoEStack:
                     self._pack(l, e, int(slot[e]))
             self._pack(l, wl.E, sh)
         self._bufs: dict[int, Buffers] = {}
+        self._ws: dict = {}
 
     # expert e == E is the layer's shared expert
     def canonical_expert(self, layer: int, e: int) -> dict:
@@ -157,6 +158,35 @@ class MoEStack:
         native.expert_ffn(self.qpool, self.shared_slot[layer], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
                           b.sh_sorted_j, b.sh_active, None, b.y_sh, b.h_sh, b.h_sh.numel(), b.status, stream)
         native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y, stream)
+        return b
+
+    def decode_workspace(self, T: int) -> torch.Tensor:
+        """Zero-filled workspace of moe_layer_decode for T tokens (kept per T)."""
+        key = ("dec", T)
+        if key not in self._ws:
+            n = native.layer_decode_workspace_bytes(T, self.wl.k, self.wl.f, self.wl.E)
+            self._ws[key] = torch.zeros(max(n, 256), dtype=torch.uint8, device=self.device)
+        return self._ws[key]
+
+    def forward_fused(self, layer: int, x: torch.Tensor, b: Buffers | None = None, stream=None,
+                      outputs: bool = True) -> Buffers:
+        """Enqueue one layer as a single moe_layer_decode launch (T <= 8).
+        outputs=False skips the routing/permutation side outputs (only y)."""
+        wl = self.wl
+        T = x.shape[0]
+        b = b or self.buffers(T)
+        ws = self.decode_workspace(T)
+        o = outputs
+        native.layer_decode(self.qpool, self.slot_of[layer], self.L * self.R + layer, layer, x, self.Wr[layer],
+                            self.bias[layer], T, wl.d, wl.f, wl.E, wl.k,
+                            logits=b.logits if o else None, topk_idx=b.idx if o else None,
+                            topk_w=b.w if o else None, counts=b.counts if o else None,
+                            offsets=b.offsets if o else None, sorted_tok=b.sorted_tok if o else None,
+                            sorted_j=b.sorted_j if o else None, inv=b.inv if o else None,
+                            active=b.active if o else None, slot_of_pair=b.sop if o else None,
+                            miss=b.miss if o else None, miss_count=b.miss_count if o else None,
+                            miss_cap=b.idx.numel() if o else 0, y=b.y, ws=ws, ws_bytes=ws.numel(),
+                            dev_status=b.status, stream=stream)
         return b
 
     def misses(self, b: Buffers) -> list:

@@ -62,6 +62,9 @@ SIGNATURES = {
     "moe_expert_ffn_q2_noalloc": (_I, [C.POINTER(QPool), _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
                                        _P]),
     "moe_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "moe_layer_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "moe_layer_decode": (_I, [C.POINTER(QPool), _P, _I32, _I32, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                              _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _SZ, _P, _P]),
 }
 
 
@@ -182,3 +185,19 @@ def expert_ffn_q2_noalloc(pool: QPool, slot_of, x, T, d, f, E, k, offsets, sorte
 def combine(y_perm, inv, topk_w, slot_of_pair, y_shared, T, k, d, y, stream=None) -> None:
     check("moe_combine", lib.moe_combine(ptr(y_perm), ptr(inv), ptr(topk_w), ptr(slot_of_pair), ptr(y_shared), T,
                                          k, d, ptr(y), stream_handle(stream)))
+
+
+def layer_decode_workspace_bytes(T, k, f, E) -> int:
+    return int(lib.moe_layer_decode_workspace_bytes(T, k, f, E))
+
+
+def layer_decode(pool: QPool, slot_of, shared_slot: int, layer: int, x, Wr, bias, T, d, f, E, k, logits=None,
+                 topk_idx=None, topk_w=None, counts=None, offsets=None, sorted_tok=None, sorted_j=None, inv=None,
+                 active=None, slot_of_pair=None, miss=None, miss_count=None, miss_cap=0, y=None, ws=None,
+                 ws_bytes=0, dev_status=None, stream=None) -> None:
+    check("moe_layer_decode",
+          lib.moe_layer_decode(C.byref(pool), ptr(slot_of), shared_slot, layer, ptr(x), ptr(Wr), ptr(bias), T, d, f,
+                               E, k, ptr(logits), ptr(topk_idx), ptr(topk_w), ptr(counts), ptr(offsets),
+                               ptr(sorted_tok), ptr(sorted_j), ptr(inv), ptr(active), ptr(slot_of_pair), ptr(miss),
+                               ptr(miss_count), miss_cap, ptr(y), ptr(ws), ws_bytes, ptr(dev_status),
+                               stream_handle(stream)))

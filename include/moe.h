@@ -229,6 +229,37 @@ moe_status moe_expert_ffn_q3(const moe_qpool *W, const int32_t *slot_of, const u
                              const int32_t *active, const float *topk_w, float *out, void *ws, size_t ws_bytes,
                              int32_t *dev_status, moe_stream_t stream);
 
+/* Workspace bytes moe_layer_decode needs for (T, k, f, E). */
+size_t moe_layer_decode_workspace_bytes(int T, int k, int f, int E);
+
+/*
+ * The whole layer for a few tokens (decode, or an MTP verify batch of one token
+ * plus drafts -- [SAITO] "命中率七成，代价是答案会变" verifies three drafts at once) in
+ * one cooperative launch: router + top-k gates, permutation, cache lookup,
+ * routed experts, shared expert and gate-weighted combine, as defined by
+ * moe_route, moe_permute, moe_cache_lookup, moe_expert_ffn_q2/q3 and
+ * moe_combine. Routing, permutation, slots and misses are identical to those
+ * calls; y agrees with them up to the order of its fp32 additions (the experts'
+ * contributions are added with atomics).
+ *   W, slot_of   pool and this layer's expert -> slot table (W->fmt 2 or 3)
+ *   shared_slot  pool slot of the layer's shared expert
+ *   layer        copied into miss records
+ *   x, Wr, bias  as moe_route; T <= 8, E <= 512, d <= 2048, f <= 1024
+ *   logits .. miss_count  outputs of the step-by-step calls, each may be NULL
+ *   y            fp32 [T][d] (output, overwritten)
+ *   ws           moe_layer_decode_workspace_bytes() bytes, 256-byte aligned,
+ *                zero-filled before first use; each launch leaves its counters
+ *                zeroed again (zero it again after a MOE_DEV_TIMEOUT)
+ * The launch uses every SM (cooperative); two launches on different streams
+ * must not share a workspace.
+ */
+moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t shared_slot, int32_t layer,
+                            const uint16_t *x, const float *Wr, const float *bias, int T, int d, int f, int E, int k,
+                            float *logits, int32_t *topk_idx, float *topk_w, int32_t *counts, int32_t *offsets,
+                            int32_t *sorted_tok, int32_t *sorted_j, int32_t *inv, int32_t *active,
+                            int32_t *slot_of_pair, moe_miss *miss, int32_t *miss_count, int32_t miss_cap, float *y,
+                            void *ws, size_t ws_bytes, int32_t *dev_status, moe_stream_t stream);
+
 /*
  * moe_expert_ffn_q2 without a caller-supplied workspace. The pages have no
  * counterpart to this call; it exists for callers that cannot allocate device
