@@ -1,9 +1,11 @@
 """Build libmoe.so (the CUDA library) in-tree for sm_100a.
 
-    python -m bit_expert_ffn_fp32_b200.build [--force]
+    python -m bit_expert_ffn_fp32_b200.build [--force] [--trace]
 
 Every csrc/*.cu file is compiled with nvcc for sm_100a into _build/ and linked
-into bit_expert_ffn_fp32_b200/libmoe.so next to this file.
+into bit_expert_ffn_fp32_b200/libmoe.so next to this file. --trace builds
+libmoe_trace.so instead: the same library with the one-launch decode kernel
+recording per-phase timestamps (see trace_decode.py).
 """
 from __future__ import annotations
 
@@ -18,6 +20,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build", "obj")
 LIB = os.path.join(PKG, "libmoe.so")
+TRACE_OBJ = os.path.join(ROOT, "_build", "obj_trace")
+TRACE_LIB = os.path.join(PKG, "libmoe_trace.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -36,30 +40,32 @@ def _stale(target: str, sources: list[str]) -> bool:
     return any(os.path.getmtime(s) > t for s in sources)
 
 
-def _compile(src: str, force: bool) -> str:
-    obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, force: bool, objdir: str = OBJ, extra=()) -> str:
+    obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
     if force or _stale(obj, [src] + _deps()):
-        cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
     return obj
 
 
-def build(force: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+def build(force: bool = False, trace: bool = False) -> str:
+    objdir, lib = (TRACE_OBJ, TRACE_LIB) if trace else (OBJ, LIB)
+    extra = ("-DMOE_DECODE_TRACE",) if trace else ()
+    os.makedirs(objdir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force), srcs))
-    if force or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, force, objdir, extra), srcs))
+    if force or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv))
+    print(build(force="--force" in sys.argv, trace="--trace" in sys.argv))

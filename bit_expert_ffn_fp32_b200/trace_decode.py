@@ -1,0 +1,76 @@
+"""Phase timeline of the one-launch decode layer (moe_layer_decode).
+
+    python -m bit_expert_ffn_fp32_b200.build --trace
+    python -m bit_expert_ffn_fp32_b200.trace_decode [WORKLOAD] [--launches N] [--warm]
+
+Loads libmoe_trace.so (the library built with -DMOE_DECODE_TRACE), runs the
+layer N times on fresh tokens with the L2 evicted before each launch (unless
+--warm), and prints, for each phase boundary, the median over launches of the
+median and the slowest CTA, in microseconds since the first CTA started.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes as C
+import os
+
+import numpy as np
+import torch
+
+from . import configs, native, synth
+from .layer import MoEStack, x_tensor
+
+POINTS = {8: "x staged", 10: "router rows (warp 0)", 1: "phase A done", 2: "all logits counted",
+          11: "top-k loads", 12: "top-k candidates", 13: "top-k selected", 6: "top-k + gates",
+          5: "routing tables", 3: "prefetch issued", 7: "phase C done", 4: "kernel end"}
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("workload", nargs="?", default="decode_T1_d2048_E512_k10_f768_q2")
+    ap.add_argument("--launches", type=int, default=40)
+    ap.add_argument("--warm", action="store_true")
+    args = ap.parse_args()
+    path = os.path.join(native.PKG, "libmoe_trace.so")
+    if not os.path.exists(path):
+        raise SystemExit("libmoe_trace.so missing: python -m bit_expert_ffn_fp32_b200.build --trace")
+    tl = C.CDLL(path)
+    for name, (res, argt) in native.SIGNATURES.items():
+        fn = getattr(tl, name)
+        fn.restype = res
+        fn.argtypes = argt
+    native.lib = tl
+    wl = configs.WORKLOADS[args.workload]
+    stack = MoEStack(wl)
+    b = stack.buffers(wl.T)
+    flush = torch.empty(512 << 18, dtype=torch.float32, device="cuda")
+    buf = np.zeros(4096 * 32, np.uint64)
+    acc = {k: [] for k in POINTS}
+    skip = 10
+    for it in range(args.launches + skip):
+        x = x_tensor(synth.gen_x(wl.seed, 0, wl.T, wl.d, stream=0 if args.warm else it))
+        if not args.warm:
+            flush.fill_(1.0)
+        stack.forward_fused(0, x, b)
+        torch.cuda.synchronize()
+        tl.moe_decode_trace_read(buf.ctypes.data)
+        if it < skip:
+            continue
+        tr = buf.reshape(4096, 32)
+        G = int((tr[:, 0] > 0).sum())
+        ns = tr[:G, :16].astype(np.int64)
+        rel = np.where(ns > 0, (ns - ns[:, 0].min()) / 1000.0, np.nan)
+        for k in POINTS:
+            if np.isfinite(rel[:, k]).any():
+                acc[k].append((np.nanmedian(rel[:, k]), np.nanmax(rel[:, k])))
+    print(f"{wl.name}: {G} CTAs, {'warm' if args.warm else 'L2 evicted before each launch'}, "
+          f"status {int(b.status.item())}")
+    print(f"{'point':24s} {'median CTA':>11s} {'slowest CTA':>12s}  (us since first CTA start)")
+    for k, nm in POINTS.items():
+        if acc[k]:
+            a = np.array(acc[k])
+            print(f"{nm:24s} {np.median(a[:, 0]):11.2f} {np.median(a[:, 1]):12.2f}")
+
+
+if __name__ == "__main__":
+    main()
