@@ -7,6 +7,8 @@
 // misses of a non-resident expert are exactly its segment of the sorted
 // permutation; the miss list is those segments, experts ascending, which is
 // (expert, token) order.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -31,7 +33,7 @@ __global__ void __launch_bounds__(kThreads)
         if (e < E) {
             const int sl = slot_of[e];
             const bool bad = sl < -1 || sl >= num_slots;
-            if (bad) flag(status, MOE_DEV_BAD_SLOT);
+            if (bad && blockIdx.x == 0) flag(status, MOE_DEV_BAD_SLOT);
             const int m = (sl < 0 || bad) ? offsets[e + 1] - offsets[e] : 0;
             s_mbase[e] = m;
             sum += m;
@@ -66,13 +68,13 @@ __global__ void __launch_bounds__(kThreads)
             base += m;
         }
     }
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
         *miss_count = total;
         if (total > miss_cap) flag(status, MOE_DEV_MISS_OVERFLOW);
     }
     __syncthreads();
     const int n = T * k;
-    for (int s = threadIdx.x; s < n; s += kThreads) {
+    for (int s = blockIdx.x * kThreads + threadIdx.x; s < n; s += gridDim.x * kThreads) {
         const int t = sorted_tok[s], j = sorted_j[s];
         const int p = t * k + j;
         const int e = topk_idx[p];
@@ -114,7 +116,9 @@ MOE_API moe_status moe_cache_lookup(const int32_t *slot_of, int32_t num_slots, i
     if (int64_t(T) * k >= (int64_t(1) << 31)) return MOE_ERR_OVERFLOW;
     if (!slot_of || !offsets || !miss_count || (miss_cap > 0 && !miss)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!topk_idx || !topk_w || !sorted_tok || !sorted_j || !slot_of_pair)) return MOE_ERR_INVALID_ARG;
-    cache_lookup_kernel<<<1, kThreads, 0, as_cuda(stream)>>>(slot_of, num_slots, layer, topk_idx, topk_w, offsets,
+    // every CTA scans the per-expert miss bases (E values), then handles its pairs
+    const int grid = int(std::min<int64_t>((int64_t(T) * k + kThreads - 1) / kThreads, 148));
+    cache_lookup_kernel<<<std::max(grid, 1), kThreads, 0, as_cuda(stream)>>>(slot_of, num_slots, layer, topk_idx, topk_w, offsets,
                                                              sorted_tok, sorted_j, T, k, E, slot_of_pair, miss,
                                                              miss_count, miss_cap, dev_status);
     return launch_status();

@@ -73,13 +73,13 @@ __device__ void counts_to_offsets(const int *s_cnt, int E, int32_t *counts, int3
 }
 
 // Places the pairs of tokens [t0, t1) in token order; s_base[e] = next position of e.
-// Runs on warp 0 only.
-__device__ void place_tokens(const int32_t *idx, int t0, int t1, int k, int E, int *s_base, int32_t *sorted_tok,
+// Runs on warp 0 only; idx_tile holds the tile's expert ids (shared memory).
+__device__ void place_tokens(const int32_t *idx_tile, int t0, int t1, int k, int E, int *s_base, int32_t *sorted_tok,
                              int32_t *sorted_j, int32_t *inv, int32_t *status) {
     const int lane = threadIdx.x & 31;
     for (int t = t0; t < t1; ++t) {
         const bool on = lane < k;
-        int e = on ? idx[size_t(t) * k + lane] : -1;
+        int e = on ? idx_tile[(t - t0) * k + lane] : -1;
         const bool valid = on && e >= 0 && e < E;
         if (on && !valid) flag(status, MOE_DEV_BAD_INDEX);
         const unsigned vmask = __ballot_sync(0xffffffffu, valid);
@@ -118,8 +118,10 @@ __global__ void __launch_bounds__(kThreads)
     counts_to_offsets(s_cnt, E, counts, offsets, active, s_warp);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += kThreads) s_cnt[e] = offsets[e];
+    __shared__ int s_idx[kTile * kMaxK];
+    for (int i = threadIdx.x; i < T * k; i += kThreads) s_idx[i] = idx[i];
     __syncthreads();
-    if (threadIdx.x < 32) place_tokens(idx, 0, T, k, E, s_cnt, sorted_tok, sorted_j, inv, status);
+    if (threadIdx.x < 32) place_tokens(s_idx, 0, T, k, E, s_cnt, sorted_tok, sorted_j, inv, status);
 }
 
 // Multi-tile path, step 1: per-tile histograms into ws[tile][E].
@@ -160,10 +162,12 @@ __global__ void __launch_bounds__(128)
     permute_scatter_kernel(const int32_t *idx, int T, int k, int E, const int32_t *ws, const int32_t *offsets,
                            int32_t *sorted_tok, int32_t *sorted_j, int32_t *inv, int32_t *status) {
     __shared__ int s_base[kMaxE];
+    __shared__ int s_idx[kTile * kMaxK];
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_base[e] = offsets[e] + ws[size_t(blockIdx.x) * E + e];
-    __syncthreads();
     const int t0 = blockIdx.x * kTile, t1 = min(T, t0 + kTile);
-    if (threadIdx.x < 32) place_tokens(idx, t0, t1, k, E, s_base, sorted_tok, sorted_j, inv, status);
+    for (int i = threadIdx.x; i < (t1 - t0) * k; i += blockDim.x) s_idx[i] = idx[size_t(t0) * k + i];
+    __syncthreads();
+    if (threadIdx.x < 32) place_tokens(s_idx, t0, t1, k, E, s_base, sorted_tok, sorted_j, inv, status);
 }
 
 }  // namespace

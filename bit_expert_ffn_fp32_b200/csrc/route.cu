@@ -63,6 +63,69 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
     }
 }
 
+// Many tokens: one warp = 8 tokens x 8 experts (64 logits), each lane keeping
+// the 64 accumulators of its element class, so every loaded chunk feeds 256
+// fused multiply-adds. The operation order per logit is the same as above.
+constexpr int kTileE = 8, kTileT = 8;
+
+__global__ void __launch_bounds__(256, 2)
+    router_tiled_kernel(const uint16_t *__restrict__ x, const float *__restrict__ Wr, const float *__restrict__ bias,
+                        int T, int d, int E, float *__restrict__ logits, int32_t *status) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e0 = blockIdx.x * (8 * kTileE) + warp * kTileE;
+    const int t0 = blockIdx.y * kTileT;
+    if (e0 >= E) return;
+    float acc[kTileT][kTileE];
+#pragma unroll
+    for (int v = 0; v < kTileT; ++v)
+#pragma unroll
+        for (int u = 0; u < kTileE; ++u) acc[v][u] = 0.f;
+    const int nchunk = d / 128;
+    for (int i = 0; i < nchunk; ++i) {
+        float4 w[kTileE];
+        uint2 xv[kTileT];
+#pragma unroll
+        for (int u = 0; u < kTileE; ++u)
+            w[u] = e0 + u < E ? __ldg(reinterpret_cast<const float4 *>(Wr + size_t(e0 + u) * d + 128 * i + 4 * lane))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int v = 0; v < kTileT; ++v)
+            xv[v] = t0 + v < T ? __ldg(reinterpret_cast<const uint2 *>(x + size_t(t0 + v) * d + 128 * i + 4 * lane))
+                               : make_uint2(0u, 0u);
+#pragma unroll
+        for (int v = 0; v < kTileT; ++v) {
+            const float x0 = bf16_lo(xv[v].x), x1 = bf16_hi(xv[v].x), x2 = bf16_lo(xv[v].y), x3 = bf16_hi(xv[v].y);
+#pragma unroll
+            for (int u = 0; u < kTileE; ++u) {
+                float a = acc[v][u];
+                a = __fmaf_rn(x0, w[u].x, a);
+                a = __fmaf_rn(x1, w[u].y, a);
+                a = __fmaf_rn(x2, w[u].z, a);
+                a = __fmaf_rn(x3, w[u].w, a);
+                acc[v][u] = a;
+            }
+        }
+    }
+#pragma unroll
+    for (int v = 0; v < kTileT; ++v)
+#pragma unroll
+        for (int u = 0; u < kTileE; ++u)
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) acc[v][u] = __fadd_rn(acc[v][u], __shfl_xor_sync(0xffffffffu, acc[v][u], o));
+    if (lane == 0) {
+#pragma unroll
+        for (int v = 0; v < kTileT; ++v)
+#pragma unroll
+            for (int u = 0; u < kTileE; ++u) {
+                if (t0 + v < T && e0 + u < E) {
+                    const float r = bias ? __fadd_rn(acc[v][u], bias[e0 + u]) : acc[v][u];
+                    if (!isfinite(r)) flag(status, MOE_DEV_NONFINITE);
+                    logits[size_t(t0 + v) * E + e0 + u] = r;
+                }
+            }
+    }
+}
+
 // (v1, i1) comes before (v2, i2): larger logit first, then lower id. NaN never wins.
 __device__ __forceinline__ bool before(float v1, int i1, float v2, int i2) {
     return v1 > v2 || (v1 == v2 && i1 < i2);
@@ -164,8 +227,13 @@ MOE_API moe_status moe_route(const uint16_t *x, const float *Wr, const float *bi
     if (T == 0) return MOE_OK;
     if (!x || !Wr || !logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = as_cuda(stream);
-    dim3 g1((E + kWarpsPerCta - 1) / kWarpsPerCta, (T + kTokTile - 1) / kTokTile);
-    router_logits_kernel<<<g1, kWarpsPerCta * 32, 0, s>>>(x, Wr, bias, T, d, E, logits, dev_status);
+    if (T >= 64) {
+        dim3 g((E + 8 * kTileE - 1) / (8 * kTileE), (T + kTileT - 1) / kTileT);
+        router_tiled_kernel<<<g, 256, 0, s>>>(x, Wr, bias, T, d, E, logits, dev_status);
+    } else {
+        dim3 g1((E + kWarpsPerCta - 1) / kWarpsPerCta, (T + kTokTile - 1) / kTokTile);
+        router_logits_kernel<<<g1, kWarpsPerCta * 32, 0, s>>>(x, Wr, bias, T, d, E, logits, dev_status);
+    }
     const int wpb = 8;
     topk_kernel<<<(T + wpb - 1) / wpb, wpb * 32, 0, s>>>(logits, T, E, k, topk_idx, topk_w, dev_status);
     return launch_status();

@@ -219,6 +219,11 @@ size_t moe_expert_ffn_workspace_bytes(int T, int k, int f);
  * sorted_tok[t] = t, sorted_j[t] = 0, active = {1, 0}, slot_of = {its slot}.
  * Activations are staged as fp16 for the tensor cores; |x| or |h| beyond
  * 65504 sets MOE_DEV_NONFINITE.
+ * Paths: with T*k < 512 a weight-streaming kernel reads each expert's packed
+ * codes once per 8 tokens (mma.sync fragments built from the codes); with
+ * T*k >= 512 and E <= 2048 (prefill) the Q2 call runs grouped GEMMs on the tcgen05 tensor
+ * cores, dequantising each 128-row weight tile to fp16 in shared memory
+ * (fp16 rounding of w = s*q + m); the workspace then holds h as fp16.
  */
 moe_status moe_expert_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f,
                              int E, int k, const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j,

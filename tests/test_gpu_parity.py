@@ -200,3 +200,39 @@ def test_multi_tile_permutation():
     for key, buf in (("counts", b.counts), ("offsets", b.offsets), ("sorted_tok", b.sorted_tok),
                      ("sorted_j", b.sorted_j), ("inv", b.inv)):
         np.testing.assert_array_equal(buf[: ref[key].shape[0]].cpu().numpy(), ref[key], err_msg=key)
+
+
+# ---------------------------------------------------------------- tensor-core (prefill) path
+@pytest.mark.parametrize("T", [256, 300, 777])
+def test_tc05_path_tiny_shapes(tiny, T):
+    """T*k >= 512 routes the Q2 expert calls to the tcgen05 grouped GEMMs
+    (ragged N tiles, several M tiles, d=512 K loop)."""
+    x = synth.gen_x(0, 0, T, configs.TINY.d, stream=900 + T)
+    _full_check(tiny, 0, x)            # every token
+
+
+def test_tc05_path_decode_shapes(decode):
+    T = 1000
+    x = synth.gen_x(0, 0, T, configs.DECODE.d, stream=950)
+    _full_check(decode, 0, x, tokens=list(range(0, T, 61)) + [T - 1])
+
+
+def test_tc05_every_pair_written_and_deterministic(decode):
+    """Every routed pair's y_e row is produced (no tile skipped or doubled by the
+    persistent schedule) and two runs give identical bits (no atomics in y_perm mode)."""
+    wl = configs.DECODE
+    T = 1500
+    x = x_tensor(synth.gen_x(0, 0, T, wl.d, stream=951))
+    b = decode.buffers(T)
+    outs = []
+    for fill in (12345.0, -777.0):
+        b.y_perm.fill_(fill)
+        b.h_ws.fill_(0xFF)            # NaN pattern in fp16 / fp32
+        decode.forward(0, x, b)
+        torch.cuda.synchronize()
+        n = T * wl.k
+        yp = b.y_perm[:n].clone()
+        assert not bool(torch.isnan(yp).any())
+        assert not bool((yp == fill).all(dim=1).any())
+        outs.append(yp)
+    assert torch.equal(outs[0], outs[1])
