@@ -168,7 +168,7 @@ def run_ours(args, wl, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
-    from bit_expert_ffn_fp32_b200 import configs, native, synth
+    from bit_expert_ffn_fp32_b200 import configs, native, replicas, synth
     from bit_expert_ffn_fp32_b200.layer import MoEStack, x_tensor
 
     torch.cuda.set_device(local_rank)
@@ -181,7 +181,7 @@ def run_ours(args, wl, rank, world, local_rank):
     # steps get their own tokens, generated up front and resident in HBM (at most
     # 256 MiB of distinct inputs, cycled; the L2 is evicted between steps anyway)
     n_x = max(1, min(n_steps, (256 << 20) // (T * wl.d * 2)))
-    xs_host = [synth.gen_x(wl.seed, 0, T, wl.d, stream=rank * 1_000_003 + s) for s in range(n_x)]
+    xs_host = [synth.gen_x(wl.seed, 0, T, wl.d, stream=s) for s in replicas.token_streams(rank, n_x)]
     xs_dev = torch.stack([x_tensor(x, dev) for x in xs_host])
 
     class _Cycle:
@@ -260,10 +260,7 @@ def run_ours(args, wl, rank, world, local_rank):
     mean_act = float(np.mean(n_act))
     res_pairs_mean = float(np.mean(n_pairs))
 
-    t = torch.tensor([total_ms, sum(ffn_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, ffn_total = float(t[0]), float(t[1])
+    total_ms, ffn_total = replicas.max_over_ranks([total_ms, sum(ffn_ms)], device=dev)
 
     # ---- e2e: pinned host tokens in, layer, result out, every step
     e2e_ms = None
@@ -283,11 +280,9 @@ def run_ours(args, wl, rank, world, local_rank):
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = sum(e2e_ev[i][0].elapsed_time(e2e_ev[i][1]) for i in range(args.steps))
-    t2 = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    (e2e_ms,) = replicas.max_over_ranks([e2e_ms], device=dev)
     if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_ms = float(t2[0])
 
     if rank != 0:
         return 0
@@ -301,7 +296,7 @@ def run_ours(args, wl, rank, world, local_rank):
     tensor_bound = not fused and T * wl.k >= 512 and wl.fmt == 2
     ffn_flops = 2.0 * 3 * wl.d * wl.f * (res_pairs_mean + T)   # routed resident pairs + shared, per step
     tokens = world * T * args.steps
-    value = tokens / (total_ms / 1e3)
+    value = replicas.job_throughput(T * args.steps, world, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -323,7 +318,7 @@ def run_ours(args, wl, rank, world, local_rank):
                       "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                       "frac": achieved / hbm_peak, "traffic": None, "bytes_per_launch": kern_bytes,
                       "avg_launch_us": ffn_avg_s * 1e6}),
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * wl.d * 2,
+        "e2e": {"value": replicas.job_throughput(T * args.steps, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": T * wl.d * 2,
                 "d2h_bytes_per_step": T * wl.d * 4},
         "clocks": clocks, "gpu_launches": launches_per_step * args.steps, "dev_status": status,
     }
