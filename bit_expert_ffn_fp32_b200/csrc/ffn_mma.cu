@@ -206,7 +206,7 @@ moe_status ffn_launch(const moe_qpool *W, const int32_t *slot_of, const uint16_t
     if (W->num_slots <= 0 || W->slot_bytes < int64_t(eg.bytes) || W->slot_bytes % 256 ||
         reinterpret_cast<uintptr_t>(W->base) % 256)
         return MOE_ERR_INVALID_ARG;
-    if (!ws || ws_bytes < moe_expert_ffn_workspace_bytes(T, k, f)) return MOE_ERR_WORKSPACE;
+    if (!ws || ws_bytes < moe_expert_ffn_workspace_bytes(T, k, d, f)) return MOE_ERR_WORKSPACE;
     FfnParams p;
     p.pool = static_cast<const uint8_t *>(W->base);
     p.slot_bytes = W->slot_bytes;
@@ -244,9 +244,11 @@ moe_status ffn_launch(const moe_qpool *W, const int32_t *slot_of, const uint16_t
 
 using namespace moe;
 
-MOE_API size_t moe_expert_ffn_workspace_bytes(int T, int k, int f) {
-    if (T <= 0 || k <= 0 || f <= 0) return 0;
-    return size_t(T) * size_t(k) * size_t(f) * sizeof(float);
+MOE_API size_t moe_expert_ffn_workspace_bytes(int T, int k, int d, int f) {
+    if (T <= 0 || k <= 0 || f <= 0 || d <= 0) return 0;
+    const size_t h32 = size_t(T) * size_t(k) * size_t(f) * sizeof(float);
+    const size_t tc = tc05_x16_offset(T, k, f) + size_t(T) * size_t(d) * 2;
+    return std::max(h32, tc);
 }
 
 MOE_API moe_status moe_expert_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d,
@@ -312,7 +314,7 @@ MOE_API moe_status moe_expert_ffn_q2_noalloc(const moe_qpool *W, const int32_t *
                                              const int32_t *sorted_tok, const int32_t *sorted_j,
                                              const int32_t *active, const float *topk_w, float *out,
                                              int32_t *dev_status, moe_stream_t stream) {
-    if (T > 0 && k > 0 && f > 0 && moe_expert_ffn_workspace_bytes(T, k, f) > kNoAllocBytes) return MOE_ERR_WORKSPACE;
+    if (T > 0 && k > 0 && f > 0 && moe_expert_ffn_workspace_bytes(T, k, d, f) > kNoAllocBytes) return MOE_ERR_WORKSPACE;
     void *ws = nullptr;
     if (T > 0) {
         const moe_status st = noalloc_scratch(&ws);

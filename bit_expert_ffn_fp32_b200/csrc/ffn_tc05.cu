@@ -4,16 +4,19 @@
 // Prompt chunks of up to 8192 tokens ("个人开发者用 AI 十天写出 Strata 引擎，让 12GB 显存跑起
 // 1250 亿参数的 Qwen 3.8 Flash Next", section "等最久的，是它读完你的代码") route ~160 tokens
 // to each of 512 experts, so each expert is a GEMM with the weights as M (128
-// rows per tile) and the expert's tokens as N (up to 128 per tile, padded to 16).
+// rows per tile) and the expert's tokens as N (up to 256 per tile, padded to 16).
 //
 // One persistent CTA per SM walks the (expert, M-tile, N-tile) list; warps are
 // specialised:
-//   producers (4 warps)  dequantise the packed Q2 codes of the tile's weight
-//                        rows straight into 128-byte-swizzled fp16 shared memory
-//                        (w = s*q + m, one fp16 rounding) and gather/convert the
-//                        token rows (bf16 -> fp16, exact for normal values);
+//   producers (8 warps)  copy each K stage's token rows (fp16) into
+//                        128-byte-swizzled shared memory and the stage's packed
+//                        Q2 codes and scales into a staging area, both with
+//                        asynchronous cp.async copies issued two or three stages
+//                        ahead; when a stage has landed they dequantise its codes
+//                        into the fp16 A tile (w = s*q + m, one fp16 rounding);
+//                        the next tile's weights are prefetched into L2;
 //   MMA (1 thread)       issues tcgen05.mma per 16-wide K step into a TMEM
-//                        accumulator (double-buffered across tiles);
+//                        accumulator;
 //   epilogue (4 warps)   drains TMEM: h = silu(g) * u (gate/up kernel), or
 //                        y_e / gate-weighted atomics (down kernel).
 // Stages hand over through mbarriers; every wait is bounded and sets
@@ -40,15 +43,16 @@ constexpr int kTcThreads = kProd + kEpi + 32;  // + MMA warp (12)
 constexpr int kTileN = 256;  // tokens per tile (MMA N, padded to 16)
 constexpr int kSub = 16384;  // 128 rows x 64 cols fp16, SW128
 constexpr int kSubB = 32768;  // 256 rows x 64 cols fp16, SW128
+constexpr int kRawMat = kProd * 16;  // packed codes + scales of one matrix, one stage
 constexpr unsigned long long kTcWaitNs = 200ull * 1000 * 1000;
-constexpr int kMaxActive = 2048;  // experts per call on this path (E <= 2048)
+constexpr int kMaxActive = kTcMaxE;  // experts per call on this path
 
 struct TcParams {
     const uint8_t *pool;
     int64_t slot_bytes;
     int num_slots;
     const int32_t *slot_of;
-    const uint16_t *x;
+    const __half *x16;  // [T][d] fp16 copy of the activations
     int T, d, f, E, k;
     const int32_t *offsets, *sorted_tok, *sorted_j, *active;
     const float *topk_w;
@@ -70,18 +74,17 @@ struct TcSmem {
     int full_prefix[kMaxActive + 1];  // full tiles before active expert a (x MT)
     uint16_t part_list[kMaxActive];   // active experts with a partial tile, largest first
     uint8_t bucket[kMaxActive];       // 16-token size class of each active expert's partial tile (0 = none)
-    int tok[kTileN];                  // token ids of the producers' current tile
     int npart;
     int bucket_start[18];
     int bucket_run[18];
 };
 
-// Whole CTA: build the tile order; returns the tile count.
-__device__ int build_schedule(const TcParams &p, TcSmem &s, int MT) {
+// Whole CTA: build the tile order; returns the tile count. scratch holds
+// blockDim.x ints (the stage buffers, not yet in use).
+__device__ int build_schedule(const TcParams &p, TcSmem &s, int MT, int *part) {
     const int na = p.active[0];
     const int tid = threadIdx.x, nthr = blockDim.x;
     __shared__ int bucket_cnt[17];
-    __shared__ int part[kTcThreads];
     if (tid < 17) bucket_cnt[tid] = 0;
     const int per = (na + nthr - 1) / nthr;
     const int a0 = tid * per;
@@ -180,19 +183,11 @@ __device__ __forceinline__ TileInfo tile_info(const TcParams &p, const TcSmem &s
     return t;
 }
 
-// Half of a 16-byte Q2 lane chunk: block bb (0/1) of the pair, rows g, g+8,
-// plus that block's (s_g, s_g8, m_g, m_g8).
+// The packed codes (8 B) and scale entry (8 B) of one block of one lane chunk:
+// block bb of the pair, rows g and g+8, {s(g), s(g+8), m(g), m(g+8)}.
 struct HalfQ2 {
     uint2 cw, sc;
 };
-
-__device__ __forceinline__ HalfQ2 load_half_q2(const uint8_t *rec, const MatGeom &m, int rg, int blk, int L) {
-    HalfQ2 c;
-    const int pair = blk >> 1, bb = blk & 1;
-    c.cw = __ldg(reinterpret_cast<const uint2 *>(rec + q2_chunk_off(m, rg, pair, L) + 8 * bb));
-    c.sc = __ldg(reinterpret_cast<const uint2 *>(rec + scale_off(m, 2, rg, pair, L >> 2) + 8 * bb));
-    return c;
-}
 
 // Dequantise into a 128-row x 64-col SW128 sub-tile: w = s*q + m in fp16
 // (q made exact in fp16 by the 1024-offset trick, then one fused multiply-add).
@@ -224,21 +219,126 @@ __device__ __forceinline__ void set_abort(TcSmem &s, int32_t *status) {
     if (atomicExch(&s.abort, 1) == 0) flag(status, MOE_DEV_TIMEOUT);
 }
 
-// Copy 8 fp16 (or 8 bf16 converted) values into a B sub-tile row chunk.
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
+// Ask the L2 for the weight rows of tile tau (codes and scales of each of the
+// NMAT matrices, one contiguous range each) and, for the down GEMM, the hidden
+// rows of the tile.
+template <int NMAT, bool GATHER>
+__device__ __forceinline__ void prefetch_tile(const TcParams &p, const TcSmem &s, int tau, int MT,
+                                              const MatGeom *const *mats, int K) {
+    const TileInfo t = tile_info(p, s, tau, MT);
+    const uint8_t *rec = p.pool + int64_t(t.slot) * p.slot_bytes;
+    const int npair = K / 128;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const __half2 hh = __floats2half2_rn(bf16_lo(u[q]), bf16_hi(u[q]));
-        o[q] = *reinterpret_cast<const uint32_t *>(&hh);
+    for (int i = 0; i < NMAT; ++i) {
+        const MatGeom &m = *mats[i];
+        tc::prefetch_l2(rec + q2_chunk_off(m, 8 * t.mi, 0, 0), uint32_t(8 * npair * 512));
+        tc::prefetch_l2(rec + scale_off(m, 2, 8 * t.mi, 0, 0), uint32_t(8 * npair * 128));
     }
-    return make_uint4(o[0], o[1], o[2], o[3]);
+    if (!GATHER && t.rows > 0) tc::prefetch_l2(p.h + int64_t(t.beg) * p.f, uint32_t(t.rows) * uint32_t(p.f) * 2u);
+}
+
+// Producer warps. Stage it lives in slot it % S: NMAT fp16 A sub-tiles, the B
+// sub-tile (256 rows), and a staging area for the packed A bytes. A stage is
+// issued L = S-1 stages ahead (wait until the MMA released the slot, then
+// cp.async of B rows and packed A bytes, one commit group per stage and
+// thread) and finished when its group has landed (dequantise the thread's own
+// packed bytes into A, fence for the tensor core, arrive on full[slot]).
+// GATHER: B row r is the fp16 activation row of token sorted_tok[beg + r]
+// (K = d); otherwise the hidden row beg + r (K = f).
+template <int NMAT, int S, bool GATHER>
+__device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int KS,
+                        const MatGeom *const *mats) {
+    constexpr int L = S - 1;
+    constexpr int kStageBytes = NMAT * kSub + kSubB;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sub_row = lane >> 3, chunk = lane & 7;
+    const int K = GATHER ? p.d : p.f;
+    const int mine = blockIdx.x < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+    const int nstages = mine * KS;
+    unsigned char *raw_base = dyn + S * kStageBytes;
+
+    // issue cursor
+    int i_tau = blockIdx.x, i_ks = 0;
+    const uint8_t *i_rec = nullptr;
+    int i_mi = 0;
+    const __half *brow[8];
+    auto enter_tile = [&]() {
+        const TileInfo t = tile_info(p, s, i_tau, MT);
+        i_rec = p.pool + int64_t(t.slot) * p.slot_bytes;
+        i_mi = t.mi;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = 32 * j + 4 * warp + sub_row;
+            brow[j] = nullptr;
+            if (r < t.rows) {
+                const int64_t row = GATHER ? int64_t(p.sorted_tok[t.beg + r]) : int64_t(t.beg + r);
+                brow[j] = (GATHER ? p.x16 : p.h) + row * K + 8 * chunk;
+            }
+        }
+        if (tid == 0 && i_tau + int(gridDim.x) < total)
+            prefetch_tile<NMAT, GATHER>(p, s, i_tau + gridDim.x, MT, mats, K);
+    };
+    if (mine > 0) enter_tile();
+
+    auto issue = [&](int it) -> bool {
+        const int st = it % S;
+        if (!tc::mbar_wait(&s.empty[st], ((it / S) & 1) ^ 1, kTcWaitNs)) return false;
+        unsigned char *stage = dyn + st * kStageBytes;
+        unsigned char *bsub = stage + NMAT * kSub;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (brow[j])
+                tc::cp_async16(bsub + tc::sw128_off(32 * j + 4 * warp + sub_row, chunk * 8), brow[j] + 64 * i_ks);
+        unsigned char *raw = raw_base + st * (NMAT * kRawMat) + tid * 16;
+        const int pair = i_ks >> 1, bb = i_ks & 1;
+#pragma unroll
+        for (int i = 0; i < NMAT; ++i) {
+            const MatGeom &m = *mats[i];
+            tc::cp_async8(raw + i * kRawMat, i_rec + q2_chunk_off(m, 8 * i_mi + warp, pair, lane) + 8 * bb);
+            tc::cp_async8(raw + i * kRawMat + 8, i_rec + scale_off(m, 2, 8 * i_mi + warp, pair, lane >> 2) + 8 * bb);
+        }
+        if (++i_ks == KS) {
+            i_ks = 0;
+            i_tau += gridDim.x;
+            if (i_tau < total) enter_tile();
+        }
+        return true;
+    };
+
+    bool ok = true;
+#pragma unroll 1
+    for (int q = 0; q < L; ++q) {
+        if (ok && q < nstages) ok = issue(q);
+        tc::cp_async_commit();
+    }
+#pragma unroll 1
+    for (int it = 0; it < nstages && ok; ++it) {
+        tc::cp_async_wait<L - 1>();  // this thread's copies of stage it have landed
+        const int st = it % S;
+        unsigned char *stage = dyn + st * kStageBytes;
+        const unsigned char *raw = raw_base + st * (NMAT * kRawMat) + tid * 16;
+#pragma unroll
+        for (int i = 0; i < NMAT; ++i) {
+            HalfQ2 c;
+            const uint4 v = *reinterpret_cast<const uint4 *>(raw + i * kRawMat);
+            c.cw = make_uint2(v.x, v.y);
+            c.sc = make_uint2(v.z, v.w);
+            store_half_q2(c, warp, lane, stage + i * kSub);
+        }
+        tc::fence_proxy_async();
+        tc::mbar_arrive(&s.full[st]);
+        if (it + L < nstages) ok = issue(it + L);
+        tc::cp_async_commit();
+        if (s.abort) break;
+    }
+    if (!ok) set_abort(s, p.status);
+    tc::cp_async_wait_all();
 }
 
 // -------------------------------------------------------------------- gate/up
-// Stage (64 of K): A_gate 16 KB, A_up 16 KB, B (256 tokens) 32 KB. TMEM: D_g
-// columns 0..255, D_u 256..511 (one accumulator pair; the epilogue is short).
+// Stage (64 of K): A_gate 16 KB, A_up 16 KB, B (256 tokens) 32 KB, plus 8 KB of
+// packed codes. TMEM: D_g columns 0..255, D_u 256..511 (one accumulator pair;
+// the epilogue is short).
 constexpr int kGuStages = 3;
 constexpr int kGuStageBytes = 2 * kSub + kSubB;
 
@@ -260,71 +360,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gateup_q2_kernel(TcParams p)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kMmaWarp) tc::tmem_alloc(&s.tmem_base, 512);
-    const int total = build_schedule(p, s, MT);
+    const int total = build_schedule(p, s, MT, reinterpret_cast<int *>(dyn));
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = s.tmem_base;
 
     if (warp < kProdWarps) {  // --------------------------------------- producers
-        // Per stage a thread loads 2 weight half-chunks and 8 token-row chunks
-        // (8 lanes per 128-byte row piece); loads of stage ks+1 are issued
-        // before stage ks is written, so they overlap the MMAs.
-        int it = 0;
-        const int sub_row = lane >> 3, chunk = lane & 7;
-        for (int tau = blockIdx.x; tau < total && !s.abort; tau += gridDim.x) {
-            const TileInfo ti = tile_info(p, s, tau, MT);
-            const uint8_t *rec = p.pool + int64_t(ti.slot) * p.slot_bytes;
-            asm volatile("bar.sync 1, %0;" ::"r"(kProd));  // previous tile's token list no longer read
-            for (int r = tid; r < kTileN; r += kProd) s.tok[r] = r < ti.rows ? p.sorted_tok[ti.beg + r] : -1;
-            asm volatile("bar.sync 1, %0;" ::"r"(kProd));
-            int rows_tok[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) rows_tok[j] = s.tok[32 * j + 4 * warp + sub_row];
-            HalfQ2 ch[2], chn[2];
-            uint4 xv[8], xvn[8];
-            auto load_stage = [&](int ks, HalfQ2 (&c)[2], uint4 (&v)[8]) {
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int cidx = tid + kProd * i;  // 2 matrices x 8 row groups x 32 lanes
-                    c[i] = load_half_q2(rec, (cidx >> 8) ? p.up : p.gate, 8 * ti.mi + ((cidx >> 5) & 7), ks,
-                                        cidx & 31);
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (rows_tok[j] >= 0)
-                        v[j] = __ldg(reinterpret_cast<const uint4 *>(p.x + int64_t(rows_tok[j]) * p.d + 64 * ks) +
-                                     chunk);
-            };
-            load_stage(0, ch, xv);
-            for (int ks = 0; ks < KS; ++ks, ++it) {
-                const int st = it % kGuStages;
-                const uint32_t ph = (it / kGuStages) & 1;
-                if (ks + 1 < KS) load_stage(ks + 1, chn, xvn);
-                if (!tc::mbar_wait(&s.empty[st], ph ^ 1, kTcWaitNs)) {
-                    set_abort(s, p.status);
-                    break;
-                }
-                unsigned char *stage = dyn + st * kGuStageBytes;
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int cidx = tid + kProd * i;
-                    store_half_q2(ch[i], (cidx >> 5) & 7, cidx & 31, stage + ((cidx >> 8) ? kSub : 0));
-                }
-                unsigned char *bsub = stage + 2 * kSub;
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (rows_tok[j] >= 0)
-                        *reinterpret_cast<uint4 *>(bsub + tc::sw128_off(32 * j + 4 * warp + sub_row, chunk * 8)) =
-                            bf16x8_to_f16x8(xv[j]);
-                tc::fence_proxy_async();
-                tc::mbar_arrive(&s.full[st]);
-#pragma unroll
-                for (int i = 0; i < 2; ++i) ch[i] = chn[i];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) xv[j] = xvn[j];
-            }
-        }
+        const MatGeom *mats[2] = {&p.gate, &p.up};
+        produce<2, kGuStages, true>(p, s, dyn, total, MT, KS, mats);
     } else if (warp < kMmaWarp) {  // ---------------------------------- epilogue
         const int q = warp - kEpiWarp0;  // TMEM lane quadrant (warp % 4)
         int tcount = 0;
@@ -397,8 +441,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gateup_q2_kernel(TcParams p)
 }
 
 // ----------------------------------------------------------------------- down
-// Stage (64 of K): A 16 KB + B (256 hidden rows) 32 KB. TMEM: two 256-column
-// accumulators (the epilogue of one tile overlaps the MMAs of the next).
+// Stage (64 of K): A 16 KB + B (256 hidden rows) 32 KB, plus 4 KB of packed
+// codes. TMEM: two 256-column accumulators (the epilogue of one tile overlaps
+// the MMAs of the next).
 constexpr int kDnStages = 4;
 constexpr int kDnStageBytes = kSub + kSubB;
 
@@ -422,53 +467,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_down_q2_kernel(TcParams p) {
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kMmaWarp) tc::tmem_alloc(&s.tmem_base, 512);
-    const int total = build_schedule(p, s, MT);
+    const int total = build_schedule(p, s, MT, reinterpret_cast<int *>(dyn));
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = s.tmem_base;
 
     if (warp < kProdWarps) {  // --------------------------------------- producers
-        int it = 0;
-        const int sub_row = lane >> 3, chunk = lane & 7;
-        for (int tau = blockIdx.x; tau < total && !s.abort; tau += gridDim.x) {
-            const TileInfo ti = tile_info(p, s, tau, MT);
-            const uint8_t *rec = p.pool + int64_t(ti.slot) * p.slot_bytes;
-            HalfQ2 ch, chn;
-            uint4 hv[8], hvn[8];
-            auto load_stage = [&](int ks, HalfQ2 &c, uint4 (&v)[8]) {
-                c = load_half_q2(rec, p.down, 8 * ti.mi + (tid >> 5), ks, lane);  // 8 row groups x 32 lanes
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int r = 32 * j + 4 * warp + sub_row;
-                    if (r < ti.rows)
-                        v[j] = __ldcg(reinterpret_cast<const uint4 *>(p.h + int64_t(ti.beg + r) * p.f + 64 * ks) + chunk);
-                }
-            };
-            load_stage(0, ch, hv);
-            for (int ks = 0; ks < KS; ++ks, ++it) {
-                const int st = it % kDnStages;
-                const uint32_t ph = (it / kDnStages) & 1;
-                if (ks + 1 < KS) load_stage(ks + 1, chn, hvn);
-                if (!tc::mbar_wait(&s.empty[st], ph ^ 1, kTcWaitNs)) {
-                    set_abort(s, p.status);
-                    break;
-                }
-                unsigned char *stage = dyn + st * kDnStageBytes;
-                store_half_q2(ch, tid >> 5, lane, stage);
-                unsigned char *bsub = stage + kSub;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int r = 32 * j + 4 * warp + sub_row;
-                    if (r < ti.rows) *reinterpret_cast<uint4 *>(bsub + tc::sw128_off(r, chunk * 8)) = hv[j];
-                }
-                tc::fence_proxy_async();
-                tc::mbar_arrive(&s.full[st]);
-                ch = chn;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) hv[j] = hvn[j];
-            }
-        }
+        const MatGeom *mats[1] = {&p.down};
+        produce<1, kDnStages, false>(p, s, dyn, total, MT, KS, mats);
     } else if (warp < kMmaWarp) {  // ---------------------------------- epilogue
         const int q = warp - kEpiWarp0;
         int tcount = 0;
@@ -542,12 +549,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_down_q2_kernel(TcParams p) {
     }
 }
 
+// fp16 copy of the activations for the tensor cores (bf16 -> fp16 is exact for
+// normal values); |x| beyond 65504 sets MOE_DEV_NONFINITE.
+__global__ void __launch_bounds__(256) to_f16_kernel(const uint16_t *__restrict__ x, __half *__restrict__ y, int64_t n8,
+                                                      int32_t *status) {
+    bool bad = false;
+    for (int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x; i < n8; i += int64_t(gridDim.x) * 256) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x) + i);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float lo = bf16_lo(u[q]), hi = bf16_hi(u[q]);
+            bad |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+            const __half2 hh = __floats2half2_rn(lo, hi);
+            o[q] = *reinterpret_cast<const uint32_t *>(&hh);
+        }
+        reinterpret_cast<uint4 *>(y)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (bad) flag(status, MOE_DEV_NONFINITE);
+}
+
 std::mutex g_tc_mu;
 bool g_tc_ready[64] = {};
 int g_tc_sms[64] = {};
 
-constexpr size_t kGuSmem = size_t(kGuStages) * kGuStageBytes + 1024;
-constexpr size_t kDnSmem = size_t(kDnStages) * kDnStageBytes + 1024;
+constexpr size_t kGuSmem = size_t(kGuStages) * (kGuStageBytes + 2 * kRawMat) + 1024;
+constexpr size_t kDnSmem = size_t(kDnStages) * (kDnStageBytes + kRawMat) + 1024;
 
 }  // namespace
 
@@ -555,6 +583,7 @@ constexpr size_t kDnSmem = size_t(kDnStages) * kDnStageBytes + 1024;
 moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f, int E, int k,
                        const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j, const int32_t *active,
                        const float *topk_w, float *out, void *ws, int32_t *dev_status, cudaStream_t stream) {
+    if (reinterpret_cast<uintptr_t>(ws) % 256 || reinterpret_cast<uintptr_t>(x) % 16) return MOE_ERR_INVALID_ARG;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
@@ -580,7 +609,7 @@ moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_
     p.slot_bytes = W->slot_bytes;
     p.num_slots = W->num_slots;
     p.slot_of = slot_of;
-    p.x = x;
+    p.x16 = reinterpret_cast<const __half *>(static_cast<unsigned char *>(ws) + tc05_x16_offset(T, k, f));
     p.T = T;
     p.d = d;
     p.f = f;
@@ -598,6 +627,9 @@ moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_
     p.up = eg.m[1];
     p.down = eg.m[2];
     const int grid = g_tc_sms[dev];
+    const int64_t n8 = int64_t(T) * d / 8;
+    to_f16_kernel<<<int(std::min<int64_t>((n8 + 255) / 256, int64_t(grid) * 8)), 256, 0, stream>>>(
+        x, const_cast<__half *>(p.x16), n8, dev_status);
     tc_gateup_q2_kernel<<<grid, kTcThreads, kGuSmem, stream>>>(p);
     tc_down_q2_kernel<<<grid, kTcThreads, kDnSmem, stream>>>(p);
     return launch_status();

@@ -132,8 +132,8 @@ class MoEStack:
             sop=torch.empty(max(n, 1), **i32), miss=torch.empty(max(n, 1) * native.MISS_BYTES, dtype=torch.uint8,
                                                                 device=dev),
             miss_count=torch.zeros(1, **i32),
-            h_ws=torch.empty(max(native.expert_ffn_workspace_bytes(T, wl.k, wl.f), 4), dtype=torch.uint8, device=dev),
-            h_sh=torch.empty(max(native.expert_ffn_workspace_bytes(T, 1, wl.f), 4), dtype=torch.uint8, device=dev),
+            h_ws=torch.empty(max(native.expert_ffn_workspace_bytes(T, wl.k, wl.d, wl.f), 4), dtype=torch.uint8, device=dev),
+            h_sh=torch.empty(max(native.expert_ffn_workspace_bytes(T, 1, wl.d, wl.f), 4), dtype=torch.uint8, device=dev),
             y_perm=torch.zeros(max(n, 1), wl.d, **f32), y_sh=torch.empty(max(T, 1), wl.d, **f32),
             y=torch.empty(max(T, 1), wl.d, **f32), status=torch.zeros(1, **i32),
             sh_offsets=torch.tensor([0, T], **i32), sh_sorted_tok=torch.arange(max(T, 1), **i32),

@@ -54,7 +54,7 @@ SIGNATURES = {
     "moe_permute_workspace_bytes": (_SZ, [_I, _I, _I]),
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "moe_cache_lookup": (_I, [_P, _I32, _I32, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I32, _P, _P]),
-    "moe_expert_ffn_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "moe_expert_ffn_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "moe_expert_ffn_q2": (_I, [C.POINTER(QPool), _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P,
                                _P]),
     "moe_expert_ffn_q3": (_I, [C.POINTER(QPool), _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P,
@@ -160,8 +160,8 @@ def cache_lookup(slot_of, num_slots, layer, topk_idx, topk_w, offsets, sorted_to
                                                    ptr(dev_status), stream_handle(stream)))
 
 
-def expert_ffn_workspace_bytes(T, k, f) -> int:
-    return int(lib.moe_expert_ffn_workspace_bytes(T, k, f))
+def expert_ffn_workspace_bytes(T, k, d, f) -> int:
+    return int(lib.moe_expert_ffn_workspace_bytes(T, k, d, f))
 
 
 def expert_ffn(pool: QPool, slot_of, x, T, d, f, E, k, offsets, sorted_tok, sorted_j, active, topk_w, out, ws,

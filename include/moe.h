@@ -199,8 +199,10 @@ moe_status moe_cache_lookup(const int32_t *slot_of, int32_t num_slots, int32_t l
                             const int32_t *sorted_j, int T, int k, int E, int32_t *slot_of_pair, moe_miss *miss,
                             int32_t *miss_count, int32_t miss_cap, int32_t *dev_status, moe_stream_t stream);
 
-/* Workspace bytes moe_expert_ffn_q2/q3 need for (T, k, f). */
-size_t moe_expert_ffn_workspace_bytes(int T, int k, int f);
+/* Workspace bytes moe_expert_ffn_q2/q3 need for (T, k, d, f): the larger of
+ * T*k*f fp32 (h, weight-streaming path) and T*k*f fp16 (h) + T*d fp16 (x),
+ * rounded to 256 B (tensor-core path). */
+size_t moe_expert_ffn_workspace_bytes(int T, int k, int d, int f);
 
 /*
  * SwiGLU experts on the packed pool: for every active expert e that has a slot
@@ -221,9 +223,11 @@ size_t moe_expert_ffn_workspace_bytes(int T, int k, int f);
  * 65504 sets MOE_DEV_NONFINITE.
  * Paths: with T*k < 512 a weight-streaming kernel reads each expert's packed
  * codes once per 8 tokens (mma.sync fragments built from the codes); with
- * T*k >= 512 and E <= 2048 (prefill) the Q2 call runs grouped GEMMs on the tcgen05 tensor
+ * T*k >= 512 and E <= 1024 (prefill) the Q2 call runs grouped GEMMs on the tcgen05 tensor
  * cores, dequantising each 128-row weight tile to fp16 in shared memory
- * (fp16 rounding of w = s*q + m); the workspace then holds h as fp16.
+ * (fp16 rounding of w = s*q + m); the workspace then holds h as fp16 [T*k][f]
+ * followed by an fp16 copy of x [T][d]; ws must then be 256-byte and x
+ * 16-byte aligned (else MOE_ERR_INVALID_ARG).
  */
 moe_status moe_expert_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f,
                              int E, int k, const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j,
@@ -273,10 +277,12 @@ moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t 
  * that allocates nothing after start-up so its memory footprint is fixed and no
  * request can fail on an out-of-memory error. Arguments and results are those of
  * moe_expert_ffn_q2; the caller still passes every input and output.
- *   Scratch: the hidden activations (T*k*f floats) go to one 4 MiB array built
- *   into the library; each GPU that loads the library holds its own copy until
- *   the process exits. T*k*f*4 > 4 MiB returns MOE_ERR_WORKSPACE (for f = 768:
- *   T*k <= 1365), before anything is enqueued.
+ *   Scratch: the workspace moe_expert_ffn_q2 would need (hidden activations,
+ *   plus an fp16 copy of x on the tensor-core path) goes to one 4 MiB array
+ *   built into the library; each GPU that loads the library holds its own copy
+ *   until the process exits. moe_expert_ffn_workspace_bytes(T, k, d, f) > 4 MiB
+ *   returns MOE_ERR_WORKSPACE (for d = 2048, f = 768, k = 10: T*k <= 1365),
+ *   before anything is enqueued.
  *   Set-up: the first call on a device looks up that device's copy of the
  *   array (cudaGetSymbolAddress, with the device current); make that first call
  *   before any stream capture. Lookup failures return MOE_ERR_CUDA.
