@@ -5,7 +5,8 @@
 Every csrc/*.cu file is compiled with nvcc for sm_100a into _build/ and linked
 into bit_expert_ffn_fp32_b200/libmoe.so next to this file. --trace builds
 libmoe_trace.so instead: the same library with the one-launch decode kernel
-recording per-phase timestamps (see trace_decode.py).
+recording per-phase timestamps (see trace_decode.py) and the tensor-core
+expert GEMMs summing the cycles each role waits (see trace_prefill.py).
 """
 from __future__ import annotations
 
@@ -52,7 +53,7 @@ def _compile(src: str, force: bool, objdir: str = OBJ, extra=()) -> str:
 
 def build(force: bool = False, trace: bool = False) -> str:
     objdir, lib = (TRACE_OBJ, TRACE_LIB) if trace else (OBJ, LIB)
-    extra = ("-DMOE_DECODE_TRACE",) if trace else ()
+    extra = ("-DMOE_DECODE_TRACE", "-DMOE_TC_TRACE") if trace else ()
     os.makedirs(objdir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:

@@ -41,9 +41,9 @@ inline bool dims_ok(int d, int f) {
 // moe_expert_ffn_q2 when T*k >= kTcMinPairs; the caller has validated arguments.
 constexpr int kTcMinPairs = 512;
 constexpr int kTcMaxE = 1024;
-// Byte offset of the fp16 copy of x inside the tensor-core path's workspace
-// (after h, fp16 [T*k][f], rounded up to 256 B).
-inline size_t tc05_x16_offset(int T, int k, int f) {
+// Byte offset of the permuted fp16 activations (fp16 [T*k][d]) inside the
+// tensor-core path's workspace (after h, fp16 [T*k][f], rounded up to 256 B).
+inline size_t tc05_xperm_offset(int T, int k, int f) {
     return (size_t(T) * size_t(k) * size_t(f) * 2 + 255) & ~size_t(255);
 }
 moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f, int E, int k,

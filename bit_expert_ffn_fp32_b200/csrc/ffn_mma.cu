@@ -247,7 +247,7 @@ using namespace moe;
 MOE_API size_t moe_expert_ffn_workspace_bytes(int T, int k, int d, int f) {
     if (T <= 0 || k <= 0 || f <= 0 || d <= 0) return 0;
     const size_t h32 = size_t(T) * size_t(k) * size_t(f) * sizeof(float);
-    const size_t tc = tc05_x16_offset(T, k, f) + size_t(T) * size_t(d) * 2;
+    const size_t tc = tc05_xperm_offset(T, k, f) + size_t(T) * size_t(k) * size_t(d) * 2;
     return std::max(h32, tc);
 }
 

@@ -8,19 +8,21 @@
 //
 // One persistent CTA per SM walks the (expert, M-tile, N-tile) list; warps are
 // specialised:
-//   producers (8 warps)  copy each K stage's token rows (fp16) into
-//                        128-byte-swizzled shared memory and the stage's packed
-//                        Q2 codes and scales into a staging area, both with
-//                        asynchronous cp.async copies issued two or three stages
-//                        ahead; when a stage has landed they dequantise its codes
-//                        into the fp16 A tile (w = s*q + m, one fp16 rounding);
-//                        the next tile's weights are prefetched into L2;
+//   producers (8 warps)  dequantise each K stage's packed Q2 codes (staged in
+//                        shared memory by the TMA thread) into the fp16 A tile
+//                        in 128-byte-swizzled shared memory (w = s*q + m, one
+//                        fp16 rounding); the B rows (fp16 activation rows in
+//                        sorted order, or hidden rows) come straight from TMA;
 //   MMA (1 thread)       issues tcgen05.mma per 16-wide K step into a TMEM
 //                        accumulator;
-//   epilogue (4 warps)   drains TMEM: h = silu(g) * u (gate/up kernel), or
+//   TMA (2 threads)      issue the tensor-memory-accelerator loads of the
+//                        packed codes and of the B rows, a few stages ahead;
+//   epilogue (8 warps)   drains TMEM: h = silu(g) * u (gate/up kernel), or
 //                        y_e / gate-weighted atomics (down kernel).
 // Stages hand over through mbarriers; every wait is bounded and sets
 // MOE_DEV_TIMEOUT instead of hanging.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -36,23 +38,59 @@ namespace {
 
 constexpr int kProdWarps = 8;
 constexpr int kProd = 32 * kProdWarps;  // producer threads (warps 0-7)
-constexpr int kEpi = 128;               // epilogue threads (warps 8-11)
+constexpr int kEpiWarps = 8;           // epilogue warps 8-15: TMEM lane quadrant warp % 4,
+constexpr int kEpi = 32 * kEpiWarps;    //   column half (warp - 8) / 4
 constexpr int kEpiWarp0 = kProdWarps;
-constexpr int kMmaWarp = kProdWarps + 4;
-constexpr int kTcThreads = kProd + kEpi + 32;  // + MMA warp (12)
+constexpr int kMmaWarp = kProdWarps + kEpiWarps;       // 16
+constexpr int kTmaWarp = kMmaWarp + 1;                 // 17: TMA loads of the packed codes
+constexpr int kTmaBWarp = kMmaWarp + 2;                // 18: TMA loads of the B rows, L2 prefetch
+constexpr int kTcThreads = kProd + kEpi + 96;
 constexpr int kTileN = 256;  // tokens per tile (MMA N, padded to 16)
 constexpr int kSub = 16384;  // 128 rows x 64 cols fp16, SW128
 constexpr int kSubB = 32768;  // 256 rows x 64 cols fp16, SW128
-constexpr int kRawMat = kProd * 16;  // packed codes + scales of one matrix, one stage
 constexpr unsigned long long kTcWaitNs = 200ull * 1000 * 1000;
 constexpr int kMaxActive = kTcMaxE;  // experts per call on this path
+
+// Optional wait accounting (build with -DMOE_TC_TRACE): the first thread of
+// each role (producer warp 0, epilogue warp 8, the MMA thread, the TMA
+// thread) sums the clock64 cycles it spends in each kind of wait and writes
+// the sums per CTA.
+// Slots per role: 0 total, 1..5 waits (see the call sites), 6 stages/tiles.
+#ifdef MOE_TC_TRACE
+constexpr int kTraceCtas = 256;
+__device__ unsigned long long g_tc_trace[2][kTraceCtas][4][8];
+struct TcClock {
+    long long v[8];
+    long long t_start;
+    __device__ void start() {
+        for (int i = 0; i < 8; ++i) v[i] = 0;
+        t_start = clock64();
+    }
+    __device__ long long now() const { return clock64(); }
+    __device__ void add(int i, long long t0) { v[i] += clock64() - t0; }
+    __device__ void count(int i) { v[i] += 1; }
+    __device__ void store(int kernel, int role, bool writer) {
+        v[0] = clock64() - t_start;
+        if (writer && blockIdx.x < kTraceCtas)
+            for (int i = 0; i < 8; ++i) g_tc_trace[kernel][blockIdx.x][role][i] = (unsigned long long)v[i];
+    }
+};
+#else
+struct TcClock {
+    __device__ void start() {}
+    __device__ long long now() const { return 0; }
+    __device__ void add(int, long long) {}
+    __device__ void count(int) {}
+    __device__ void store(int, int, bool) {}
+};
+#endif
 
 struct TcParams {
     const uint8_t *pool;
     int64_t slot_bytes;
     int num_slots;
     const int32_t *slot_of;
-    const __half *x16;  // [T][d] fp16 copy of the activations
+    const __half *xperm;  // [T*k][d] fp16 activation rows in sorted pair order
     int T, d, f, E, k;
     const int32_t *offsets, *sorted_tok, *sorted_j, *active;
     const float *topk_w;
@@ -62,124 +100,134 @@ struct TcParams {
     MatGeom gate, up, down;
 };
 
-// Tile order: every full 256-token tile of every expert first, then the
-// experts' last (partial) tiles from largest to smallest, so the long tiles
-// start early and the short ones fill the end.
+constexpr int kMaxSB = 4;    // B stage slots (max over the two kernels)
+constexpr int kMaxSRP = 4;   // packed-code slots
+constexpr int kKeys = 512;   // schedule sort keys
+
+// Tile order: experts from the largest to the smallest (number of 256-token
+// tiles, then the size of the last tile), each expert's tiles together (N-tile
+// outer, M-tile inner). Long experts start first, short ones fill the end, and
+// the tiles that read the same weights run at the same time, so the weights
+// come from DRAM once.
 struct TcSmem {
-    uint64_t full[4], empty[4], tfull[2], tempty[2];
+    uint64_t fullA[2], emptyA[2], fullB[kMaxSB], emptyB[kMaxSB], fullR[kMaxSRP], emptyR[kMaxSRP], tfull[2], tempty[2];
     uint32_t tmem_base;
     int abort;
-    int nfull_tiles;                 // full tiles (all M-tiles included)
-    int nact;
-    int full_prefix[kMaxActive + 1];  // full tiles before active expert a (x MT)
-    uint16_t part_list[kMaxActive];   // active experts with a partial tile, largest first
-    uint8_t bucket[kMaxActive];       // 16-token size class of each active expert's partial tile (0 = none)
-    int npart;
-    int bucket_start[18];
-    int bucket_run[18];
+    int nexp;                          // experts with at least one tile
+    int tiles_prefix[kMaxActive + 1];  // tiles before sorted expert i
+    int ebeg[kMaxActive];              // sorted expert i: first sorted pair,
+    int erows[kMaxActive];             //   its pair count,
+    int eslot[kMaxActive];             //   its pool slot
 };
 
-// Whole CTA: build the tile order; returns the tile count. scratch holds
-// blockDim.x ints (the stage buffers, not yet in use).
-__device__ int build_schedule(const TcParams &p, TcSmem &s, int MT, int *part) {
-    const int na = p.active[0];
-    const int tid = threadIdx.x, nthr = blockDim.x;
-    __shared__ int bucket_cnt[17];
-    if (tid < 17) bucket_cnt[tid] = 0;
-    const int per = (na + nthr - 1) / nthr;
-    const int a0 = tid * per;
-    int local = 0;
+// Tokens routed to active expert a that this call computes (0 if not resident).
+__device__ __forceinline__ int expert_rows(const TcParams &p, int e) {
+    const bool ok = e >= 0 && e < p.E;
+    const int sl = ok ? p.slot_of[e] : -1;
+    return (ok && sl >= 0 && sl < p.num_slots) ? p.offsets[e + 1] - p.offsets[e] : 0;
+}
+
+// Sort key (larger first): tiles (capped at 32), then the 16-token size class
+// of the last tile; -1 for an expert without tokens.
+__device__ __forceinline__ int sched_key(int n) {
+    if (n <= 0) return -1;
+    const int nt = (n + kTileN - 1) / kTileN;
+    const int last = n - kTileN * (nt - 1);
+    return (min(nt, 32) - 1) * 16 + ((last + 15) >> 4) - 1;
+}
+
+// Whole CTA: build the tile order; returns the tile count. scratch is the
+// (not yet used) stage memory: kKeys + 2 * kMaxActive ints.
+__device__ int build_schedule(const TcParams &p, TcSmem &s, int MT, int *scratch) {
+    const int na = min(p.active[0], kMaxActive);
+    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31;
+    int *hist = scratch;                       // per key: count, then first position
+    int *akey = scratch + kKeys;               // per active expert: key
+    int *ord = scratch + kKeys + kMaxActive;   // sorted position -> expert id
+    for (int i = tid; i < kKeys; i += nthr) hist[i] = 0;
     __syncthreads();
-    for (int i = 0; i < per; ++i) {
-        const int a = a0 + i;
-        if (a < na) {
-            const int e = p.active[1 + a];
-            const bool ok = e >= 0 && e < p.E;
-            const int sl = ok ? p.slot_of[e] : -1;
-            const int n = (ok && sl >= 0 && sl < p.num_slots) ? p.offsets[e + 1] - p.offsets[e] : 0;
-            s.full_prefix[a + 1] = MT * (n / kTileN);
-            local += MT * (n / kTileN);
-            const int rem = n % kTileN;
-            s.bucket[a] = uint8_t(rem ? (rem + 15) >> 4 : 0);  // 1..16
-            if (rem) atomicAdd(&bucket_cnt[(rem + 15) >> 4], 1);
-        }
-    }
-    part[tid] = local;
-    __syncthreads();
-    if (tid == 0) {
-        int run = 0;
-        for (int i = 0; i < nthr; ++i) {
-            const int v = part[i];
-            part[i] = run;
-            run += v;
-        }
-        s.full_prefix[0] = 0;
-        s.nfull_tiles = run;
-        int pos = 0;  // buckets from largest (16) down
-        for (int bk = 16; bk >= 1; --bk) {
-            s.bucket_start[bk] = pos;
-            s.bucket_run[bk] = 0;
-            pos += bucket_cnt[bk];
-        }
-        s.npart = pos;
-        s.nact = na;
+    for (int a = tid; a < na; a += nthr) {
+        const int key = sched_key(expert_rows(p, p.active[1 + a]));
+        akey[a] = key;
+        if (key >= 0) atomicAdd(&hist[key], 1);
     }
     __syncthreads();
-    int run = part[tid];
-    for (int i = 0; i < per; ++i) {
-        const int a = a0 + i;
-        if (a < na) {
-            run += s.full_prefix[a + 1];
-            s.full_prefix[a + 1] = run;
+    if (tid < 32) {  // descending exclusive scan over keys: lane owns keys 16*lane .. 16*lane+15
+        int blk = 0;
+        for (int i = 0; i < 16; ++i) blk += hist[16 * lane + i];
+        int above = 0;  // experts whose key lies in a higher lane's block
+        for (int l = 31; l >= 1; --l) {
+            const int v = __shfl_sync(0xffffffffu, blk, l);
+            if (l > lane) above += v;
         }
-    }
-    // Partial tiles: within a size class, ascending active index, so every CTA
-    // derives the same order (one warp, 32 experts at a time).
-    if (tid < 32) {
+        int run = above;
+        for (int i = 15; i >= 0; --i) {
+            const int c = hist[16 * lane + i];
+            hist[16 * lane + i] = run;
+            run += c;
+        }
+        if (lane == 0) s.nexp = run;
+        __syncwarp();
+        // stable placement in active-index order
         for (int g0 = 0; g0 < na; g0 += 32) {
-            const int a = g0 + tid;
-            const int bk = a < na ? s.bucket[a] : 0;
-            const unsigned peers = __match_any_sync(0xffffffffu, bk);
-            const int rank = __popc(peers & ((1u << tid) - 1));
-            if (bk) s.part_list[s.bucket_start[bk] + s.bucket_run[bk] + rank] = uint16_t(a);
+            const int a = g0 + lane;
+            const int key = a < na ? akey[a] : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, key);
+            const int rank = __popc(peers & ((1u << lane) - 1));
+            if (key >= 0) ord[hist[key] + rank] = p.active[1 + a];
             __syncwarp();
-            if (bk && rank == 0) s.bucket_run[bk] += __popc(peers);
+            if (key >= 0 && rank == 0) hist[key] += __popc(peers);
             __syncwarp();
         }
     }
     __syncthreads();
-    return s.nfull_tiles + MT * s.npart;
+    const int nexp = s.nexp;
+    for (int i = tid; i < nexp; i += nthr) {  // per sorted expert: rows, first pair, slot
+        const int e = ord[i];
+        s.erows[i] = expert_rows(p, e);
+        s.ebeg[i] = p.offsets[e];
+        s.eslot[i] = p.slot_of[e];
+    }
+    __syncthreads();
+    if (tid < 32) {  // tile prefix over the sorted experts: lane owns a contiguous run
+        const int per = (nexp + 31) / 32;
+        const int i0 = min(nexp, lane * per), i1 = min(nexp, i0 + per);
+        int sum = 0;
+        for (int i = i0; i < i1; ++i) sum += MT * ((s.erows[i] + kTileN - 1) / kTileN);
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int acc = incl - sum;
+        for (int i = i0; i < i1; ++i) {
+            s.tiles_prefix[i] = acc;
+            acc += MT * ((s.erows[i] + kTileN - 1) / kTileN);
+        }
+        if (lane == 31) s.tiles_prefix[nexp] = incl;
+    }
+    __syncthreads();
+    return s.tiles_prefix[s.nexp];
 }
 
 struct TileInfo {
-    int e, slot, beg, rows, mi;
+    int slot, beg, rows, mi;
 };
 
 __device__ __forceinline__ TileInfo tile_info(const TcParams &p, const TcSmem &s, int tau, int MT) {
-    int a, ni, local;
-    if (tau < s.nfull_tiles) {
-        int lo = 0, hi = s.nact;  // last a with full_prefix[a] <= tau
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (s.full_prefix[mid] <= tau) lo = mid; else hi = mid;
-        }
-        a = lo;
-        local = tau - s.full_prefix[a];
-        ni = local / MT;
-    } else {
-        const int q = tau - s.nfull_tiles;
-        a = s.part_list[q / MT];
-        local = q;
-        ni = -1;  // the partial tile
+    int lo = 0, hi = s.nexp;  // last i with tiles_prefix[i] <= tau
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s.tiles_prefix[mid] <= tau) lo = mid; else hi = mid;
     }
+    const int local = tau - s.tiles_prefix[lo];
+    const int ni = local / MT;
     TileInfo t;
-    t.e = p.active[1 + a];
-    t.slot = p.slot_of[t.e];
-    t.mi = local % MT;
-    const int beg = p.offsets[t.e], n = p.offsets[t.e + 1] - beg;
-    if (ni < 0) ni = n / kTileN;
-    t.beg = beg + kTileN * ni;
-    t.rows = min(kTileN, n - kTileN * ni);
+    t.slot = s.eslot[lo];
+    t.mi = local - ni * MT;
+    t.beg = s.ebeg[lo] + kTileN * ni;
+    t.rows = min(kTileN, s.erows[lo] - kTileN * ni);
     return t;
 }
 
@@ -219,146 +267,252 @@ __device__ __forceinline__ void set_abort(TcSmem &s, int32_t *status) {
     if (atomicExch(&s.abort, 1) == 0) flag(status, MOE_DEV_TIMEOUT);
 }
 
-// Ask the L2 for the weight rows of tile tau (codes and scales of each of the
-// NMAT matrices, one contiguous range each) and, for the down GEMM, the hidden
-// rows of the tile.
-template <int NMAT, bool GATHER>
-__device__ __forceinline__ void prefetch_tile(const TcParams &p, const TcSmem &s, int tau, int MT,
-                                              const MatGeom *const *mats, int K) {
+// Ask the L2 for tile tau's packed weight rows (codes and scales, one
+// contiguous range per matrix and region) and its B rows (K fp16 each).
+template <int NMAT>
+__device__ __forceinline__ void prefetch_tile(const TcParams &p, const TcSmem &s, int tau, int MT, int K,
+                                              const __half *bsrc) {
     const TileInfo t = tile_info(p, s, tau, MT);
     const uint8_t *rec = p.pool + int64_t(t.slot) * p.slot_bytes;
-    const int npair = K / 128;
+    const MatGeom *mats[2] = {NMAT == 2 ? &p.gate : &p.down, &p.up};
 #pragma unroll
     for (int i = 0; i < NMAT; ++i) {
-        const MatGeom &m = *mats[i];
-        tc::prefetch_l2(rec + q2_chunk_off(m, 8 * t.mi, 0, 0), uint32_t(8 * npair * 512));
-        tc::prefetch_l2(rec + scale_off(m, 2, 8 * t.mi, 0, 0), uint32_t(8 * npair * 128));
+        tc::prefetch_l2(rec + q2_chunk_off(*mats[i], 8 * t.mi, 0, 0), uint32_t(8 * (K / 128) * 512));
+        tc::prefetch_l2(rec + scale_off(*mats[i], 2, 8 * t.mi, 0, 0), uint32_t(8 * (K / 128) * 128));
     }
-    if (!GATHER && t.rows > 0) tc::prefetch_l2(p.h + int64_t(t.beg) * p.f, uint32_t(t.rows) * uint32_t(p.f) * 2u);
+    tc::prefetch_l2(bsrc + int64_t(t.beg) * K, uint32_t(t.rows) * uint32_t(K) * 2u);
 }
 
-// Producer warps. Stage it lives in slot it % S: NMAT fp16 A sub-tiles, the B
-// sub-tile (256 rows), and a staging area for the packed A bytes. A stage is
-// issued L = S-1 stages ahead (wait until the MMA released the slot, then
-// cp.async of B rows and packed A bytes, one commit group per stage and
-// thread) and finished when its group has landed (dequantise the thread's own
-// packed bytes into A, fence for the tensor core, arrive on full[slot]).
-// GATHER: B row r is the fp16 activation row of token sorted_tok[beg + r]
-// (K = d); otherwise the hidden row beg + r (K = f).
-template <int NMAT, int S, bool GATHER>
-__device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int KS,
-                        const MatGeom *const *mats) {
-    constexpr int L = S - 1;
-    constexpr int kStageBytes = NMAT * kSub + kSubB;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int sub_row = lane >> 3, chunk = lane & 7;
-    const int K = GATHER ? p.d : p.f;
+// Packed bytes of one block pair (two K stages) of a 128-row tile, per matrix:
+// 8 row groups x 32 lanes x 16 B of codes, then 8 row groups x 8 x 16 B of scales.
+constexpr int kRawCodes = 8 * 512;
+constexpr int kRawPairMat = kRawCodes + 8 * 128;
+
+// Shared-memory rings of a kernel: SA dequantised A stages (NMAT 128x64 fp16
+// sub-tiles each), SB B stages (256 rows x 64 fp16), SRP slots of packed A
+// bytes (one block pair each).
+template <int NMAT, int SA, int SB, int SRP>
+struct Rings {
+    static constexpr int kA = NMAT * kSub;
+    static constexpr int kRaw = NMAT * kRawPairMat;
+    static constexpr int kBytes = SA * kA + SB * kSubB + SRP * kRaw;
+    __device__ static unsigned char *a(unsigned char *dyn, int it) { return dyn + (it % SA) * kA; }
+    __device__ static unsigned char *b(unsigned char *dyn, int it) { return dyn + SA * kA + (it % SB) * kSubB; }
+    __device__ static unsigned char *raw(unsigned char *dyn, int pp) {
+        return dyn + SA * kA + SB * kSubB + (pp % SRP) * kRaw;
+    }
+};
+
+// Tensor maps of the packed weights, per matrix: codes as uint32 [slot][row
+// group][pair * 128 words], scales as [slot][row group][pair * 32 words].
+struct RawMaps {
+    CUtensorMap code[2], scale[2];
+};
+
+// Walks this CTA's (tile, step) sequence; tau advances by the grid size.
+struct StageCursor {
+    int tau, ks;
+};
+
+// TMA threads (lane 0 of warps 17 and 18), each walking this CTA's stages in
+// order and blocking only on the slot it refills next:
+//   A codes  (warp 17) one load of codes and one of scales per matrix and
+//            block pair (two stages) into slot pp % SRP once every producer
+//            is done with it (emptyR); complete on fullR;
+//   B rows   (warp 18) TMA loads of the tile's rows, 64 per box, into B slot
+//            it % SB once the MMA has released it (emptyB); complete on
+//            fullB. On entering a tile it asks the L2 for the next tile.
+template <int NMAT, int SA, int SB, int SRP>
+__device__ __forceinline__ void issue_codes(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int KS,
+                                            const RawMaps &rm) {
+    using R = Rings<NMAT, SA, SB, SRP>;
+    const int PS = KS / 2;
     const int mine = blockIdx.x < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
-    const int nstages = mine * KS;
-    unsigned char *raw_base = dyn + S * kStageBytes;
-
-    // issue cursor
-    int i_tau = blockIdx.x, i_ks = 0;
-    const uint8_t *i_rec = nullptr;
-    int i_mi = 0;
-    const __half *brow[8];
-    auto enter_tile = [&]() {
-        const TileInfo t = tile_info(p, s, i_tau, MT);
-        i_rec = p.pool + int64_t(t.slot) * p.slot_bytes;
-        i_mi = t.mi;
+    const int npairs = mine * PS;
+    TcClock ck;
+    ck.start();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int r = 32 * j + 4 * warp + sub_row;
-            brow[j] = nullptr;
-            if (r < t.rows) {
-                const int64_t row = GATHER ? int64_t(p.sorted_tok[t.beg + r]) : int64_t(t.beg + r);
-                brow[j] = (GATHER ? p.x16 : p.h) + row * K + 8 * chunk;
-            }
-        }
-        if (tid == 0 && i_tau + int(gridDim.x) < total)
-            prefetch_tile<NMAT, GATHER>(p, s, i_tau + gridDim.x, MT, mats, K);
-    };
-    if (mine > 0) enter_tile();
-
-    auto issue = [&](int it) -> bool {
-        const int st = it % S;
-        if (!tc::mbar_wait(&s.empty[st], ((it / S) & 1) ^ 1, kTcWaitNs)) return false;
-        unsigned char *stage = dyn + st * kStageBytes;
-        unsigned char *bsub = stage + NMAT * kSub;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (brow[j])
-                tc::cp_async16(bsub + tc::sw128_off(32 * j + 4 * warp + sub_row, chunk * 8), brow[j] + 64 * i_ks);
-        unsigned char *raw = raw_base + st * (NMAT * kRawMat) + tid * 16;
-        const int pair = i_ks >> 1, bb = i_ks & 1;
-#pragma unroll
-        for (int i = 0; i < NMAT; ++i) {
-            const MatGeom &m = *mats[i];
-            tc::cp_async8(raw + i * kRawMat, i_rec + q2_chunk_off(m, 8 * i_mi + warp, pair, lane) + 8 * bb);
-            tc::cp_async8(raw + i * kRawMat + 8, i_rec + scale_off(m, 2, 8 * i_mi + warp, pair, lane >> 2) + 8 * bb);
-        }
-        if (++i_ks == KS) {
-            i_ks = 0;
-            i_tau += gridDim.x;
-            if (i_tau < total) enter_tile();
-        }
-        return true;
-    };
-
+    for (int i = 0; i < NMAT; ++i) {
+        tc::prefetch_tensormap(&rm.code[i]);
+        tc::prefetch_tensormap(&rm.scale[i]);
+    }
+    int tau = blockIdx.x, pk = 0;
+    TileInfo t{};
+    if (mine > 0) t = tile_info(p, s, tau, MT);
     bool ok = true;
 #pragma unroll 1
-    for (int q = 0; q < L; ++q) {
-        if (ok && q < nstages) ok = issue(q);
-        tc::cp_async_commit();
+    for (int pr = 0; pr < npairs && !s.abort; ++pr) {
+        const long long t0 = ck.now();
+        if (!tc::mbar_wait(&s.emptyR[pr % SRP], ((pr / SRP) & 1) ^ 1, kTcWaitNs)) {
+            ok = false;
+            break;
+        }
+        ck.add(1, t0);
+        const long long t1 = ck.now();
+        unsigned char *raw = R::raw(dyn, pr);
+        uint64_t *bar = &s.fullR[pr % SRP];
+        tc::mbar_arrive_expect_tx(bar, uint32_t(NMAT * kRawPairMat));
+#pragma unroll
+        for (int i = 0; i < NMAT; ++i) {
+            tc::tma_load_3d(raw + i * kRawPairMat, &rm.code[i], 128 * pk, 8 * t.mi, t.slot, bar);
+            tc::tma_load_3d(raw + i * kRawPairMat + kRawCodes, &rm.scale[i], 32 * pk, 8 * t.mi, t.slot, bar);
+        }
+        ck.add(3, t1);
+        ck.count(6);
+        if (++pk == PS) {
+            pk = 0;
+            tau += gridDim.x;
+            if (tau < total) t = tile_info(p, s, tau, MT);
+        }
     }
+    if (!ok) set_abort(s, p.status);
+    ck.store(NMAT == 2 ? 0 : 1, 3, true);
+}
+
+template <int NMAT, int SA, int SB, int SRP>
+__device__ __forceinline__ void issue_rows(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int KS,
+                                           const void *tmap_b, const __half *bsrc) {
+    using R = Rings<NMAT, SA, SB, SRP>;
+    const int mine = blockIdx.x < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+    const int nstages = mine * KS;
+    tc::prefetch_tensormap(tmap_b);
+    int tau = blockIdx.x, ks = 0;
+    TileInfo t{};
+    if (mine > 0) t = tile_info(p, s, tau, MT);
+    if (mine > 1) prefetch_tile<NMAT>(p, s, tau + gridDim.x, MT, 64 * KS, bsrc);
+    bool ok = true;
 #pragma unroll 1
-    for (int it = 0; it < nstages && ok; ++it) {
-        tc::cp_async_wait<L - 1>();  // this thread's copies of stage it have landed
-        const int st = it % S;
-        unsigned char *stage = dyn + st * kStageBytes;
-        const unsigned char *raw = raw_base + st * (NMAT * kRawMat) + tid * 16;
+    for (int pb = 0; pb < nstages && !s.abort; ++pb) {
+        if (!tc::mbar_wait(&s.emptyB[pb % SB], ((pb / SB) & 1) ^ 1, kTcWaitNs)) {
+            ok = false;
+            break;
+        }
+        unsigned char *bsub = R::b(dyn, pb);
+        uint64_t *bar = &s.fullB[pb % SB];
+        const int nbox = (t.rows + 63) >> 6;
+        tc::mbar_arrive_expect_tx(bar, uint32_t(nbox) * 8192u);
+        for (int j = 0; j < nbox; ++j) tc::tma_load_2d(bsub + j * 8192, tmap_b, 64 * ks, t.beg + 64 * j, bar);
+        if (++ks == KS) {
+            ks = 0;
+            tau += gridDim.x;
+            if (tau < total) t = tile_info(p, s, tau, MT);
+            if (tau + int(gridDim.x) < total) prefetch_tile<NMAT>(p, s, tau + gridDim.x, MT, 64 * KS, bsrc);
+        }
+    }
+    if (!ok) set_abort(s, p.status);
+}
+
+// Producer warps (0-7): for each stage, once its block pair's packed bytes have
+// landed (fullR) and the MMA has released the A slot (emptyA), dequantise the
+// thread's lane chunk into the A ring, then arrive on fullA (and on emptyR
+// after the pair's second block).
+template <int NMAT, int SA, int SB, int SRP>
+__device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int KS) {
+    using R = Rings<NMAT, SA, SB, SRP>;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int mine = blockIdx.x < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+    const int nstages = mine * KS;
+    TcClock ck;
+    ck.start();
+    bool ok = true;
+#pragma unroll 1
+    for (int it = 0; it < nstages; ++it) {
+        const int pp = it >> 1, bb = it & 1;
+        long long t0 = ck.now();
+        if (bb == 0 && !tc::mbar_wait(&s.fullR[pp % SRP], (pp / SRP) & 1, kTcWaitNs)) {
+            ok = false;
+            break;
+        }
+        ck.add(1, t0);
+        t0 = ck.now();
+        if (!tc::mbar_wait(&s.emptyA[it % SA], ((it / SA) & 1) ^ 1, kTcWaitNs)) {
+            ok = false;
+            break;
+        }
+        ck.add(2, t0);
+        t0 = ck.now();
+        unsigned char *atile = R::a(dyn, it);
+        const unsigned char *raw = R::raw(dyn, pp);
 #pragma unroll
         for (int i = 0; i < NMAT; ++i) {
             HalfQ2 c;
-            const uint4 v = *reinterpret_cast<const uint4 *>(raw + i * kRawMat);
-            c.cw = make_uint2(v.x, v.y);
-            c.sc = make_uint2(v.z, v.w);
-            store_half_q2(c, warp, lane, stage + i * kSub);
+            c.cw = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + warp * 512 + lane * 16 + 8 * bb);
+            c.sc = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + kRawCodes + warp * 128 + (lane >> 2) * 16 +
+                                                    8 * bb);
+            store_half_q2(c, warp, lane, atile + i * kSub);
         }
         tc::fence_proxy_async();
-        tc::mbar_arrive(&s.full[st]);
-        if (it + L < nstages) ok = issue(it + L);
-        tc::cp_async_commit();
+        tc::mbar_arrive(&s.fullA[it % SA]);
+        if (bb) tc::mbar_arrive(&s.emptyR[pp % SRP]);
+        ck.add(4, t0);
+        ck.count(6);
         if (s.abort) break;
     }
     if (!ok) set_abort(s, p.status);
-    tc::cp_async_wait_all();
+    ck.store(NMAT == 2 ? 0 : 1, 0, tid == 0);
+}
+
+// Barrier set-up shared by both kernels (thread 0), then TMEM allocation
+// (MMA warp) and the schedule (whole CTA).
+template <int SA, int SB, int SRP>
+__device__ __forceinline__ void init_barriers(TcSmem &s, int acc_bufs) {
+    for (int i = 0; i < SRP; ++i) {
+        tc::mbar_init(&s.fullR[i], 1);
+        tc::mbar_init(&s.emptyR[i], kProd);
+    }
+    for (int i = 0; i < SA; ++i) {
+        tc::mbar_init(&s.fullA[i], kProd);
+        tc::mbar_init(&s.emptyA[i], 1);
+    }
+    for (int i = 0; i < SB; ++i) {
+        tc::mbar_init(&s.fullB[i], 1);
+        tc::mbar_init(&s.emptyB[i], 1);
+    }
+    for (int i = 0; i < acc_bufs; ++i) {
+        tc::mbar_init(&s.tfull[i], 1);
+        tc::mbar_init(&s.tempty[i], kEpi);
+    }
+    s.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// MMA thread: wait for stage it's A and B, then hand both slots back when the
+// MMAs that read them have completed.
+template <int SA, int SB>
+__device__ __forceinline__ bool mma_wait_stage(TcSmem &s, int it, TcClock &ck) {
+    long long t0 = ck.now();
+    if (!tc::mbar_wait(&s.fullA[it % SA], (it / SA) & 1, kTcWaitNs)) return false;
+    ck.add(1, t0);
+    t0 = ck.now();
+    if (!tc::mbar_wait(&s.fullB[it % SB], (it / SB) & 1, kTcWaitNs)) return false;
+    ck.add(2, t0);
+    ck.count(6);
+    tc::fence_after();
+    return true;
+}
+template <int SA, int SB>
+__device__ __forceinline__ void mma_release_stage(TcSmem &s, int it) {
+    tc::mma_commit(&s.emptyA[it % SA]);
+    tc::mma_commit(&s.emptyB[it % SB]);
 }
 
 // -------------------------------------------------------------------- gate/up
-// Stage (64 of K): A_gate 16 KB, A_up 16 KB, B (256 tokens) 32 KB, plus 8 KB of
-// packed codes. TMEM: D_g columns 0..255, D_u 256..511 (one accumulator pair;
-// the epilogue is short).
-constexpr int kGuStages = 3;
-constexpr int kGuStageBytes = 2 * kSub + kSubB;
+// Rings: 2 A stages (gate + up, 32 KB each), 3 B stages (256 tokens, 32 KB
+// each), 4 packed-code slots (one block pair, 10 KB each). TMEM: D_g columns 0..255, D_u
+// 256..511 (one accumulator pair; the epilogue is short).
+constexpr int kGuSA = 2, kGuSB = 3, kGuSR = 4;
+using GuRings = Rings<2, kGuSA, kGuSB, kGuSR>;
 
-__global__ void __launch_bounds__(kTcThreads, 1) tc_gateup_q2_kernel(TcParams p) {
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gateup_q2_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmap_b,
+                        const __grid_constant__ RawMaps rm) {
     extern __shared__ __align__(1024) unsigned char dyn_raw[];
     unsigned char *dyn =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
     __shared__ TcSmem s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int MT = p.f / 128, KS = p.d / 64;
-    if (tid == 0) {
-        for (int i = 0; i < kGuStages; ++i) {
-            tc::mbar_init(&s.full[i], kProd);
-            tc::mbar_init(&s.empty[i], 1);
-        }
-        tc::mbar_init(&s.tfull[0], 1);
-        tc::mbar_init(&s.tempty[0], kEpi);
-        s.abort = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
+    if (tid == 0) init_barriers<kGuSA, kGuSB, kGuSR>(s, 1);
     if (warp == kMmaWarp) tc::tmem_alloc(&s.tmem_base, 512);
     const int total = build_schedule(p, s, MT, reinterpret_cast<int *>(dyn));
     tc::fence_before();
@@ -367,29 +521,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gateup_q2_kernel(TcParams p)
     const uint32_t tmem = s.tmem_base;
 
     if (warp < kProdWarps) {  // --------------------------------------- producers
-        const MatGeom *mats[2] = {&p.gate, &p.up};
-        produce<2, kGuStages, true>(p, s, dyn, total, MT, KS, mats);
+        produce<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, KS);
     } else if (warp < kMmaWarp) {  // ---------------------------------- epilogue
-        const int q = warp - kEpiWarp0;  // TMEM lane quadrant (warp % 4)
+        const int q = warp & 3, half = (warp - kEpiWarp0) >> 2;  // TMEM lane quadrant, column half
         int tcount = 0;
         bool too_big = false;
+        TcClock ck;
+        ck.start();
         for (int tau = blockIdx.x; tau < total && !s.abort; tau += gridDim.x, ++tcount) {
             const TileInfo ti = tile_info(p, s, tau, MT);
-            if (!tc::mbar_wait(&s.tfull[0], tcount & 1, kTcWaitNs)) {
+            const long long t0 = ck.now();
+            if (!tc::mbar_wait_sleep(&s.tfull[0], tcount & 1, kTcWaitNs, 128)) {
                 set_abort(s, p.status);
                 break;
             }
+            ck.add(1, t0);
+            ck.count(6);
             tc::fence_after();
             const int frow = 128 * ti.mi + 32 * q + lane;
             const uint32_t tg = tmem + (uint32_t(32 * q) << 16);
-            for (int c0 = 0; c0 < ti.rows; c0 += 16) {
+            for (int c0 = 16 * half; c0 < ti.rows; c0 += 32) {
                 float g[16], u[16];
+                const long long t1 = ck.now();
                 tc::tmem_ld16(tg + c0, g);
                 tc::tmem_ld16(tg + 256 + c0, u);
+                ck.add(2, t1);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     if (c0 + j < ti.rows) {
-                        const float hv = g[j] / (1.0f + __expf(-g[j])) * u[j];
+                        const float hv = __fdividef(g[j], 1.0f + __expf(-g[j])) * u[j];
                         too_big |= !(fabsf(hv) <= 65504.f);
                         p.h[int64_t(ti.beg + c0 + j) * p.f + frow] = __float2half_rn(hv);
                     }
@@ -399,38 +559,48 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gateup_q2_kernel(TcParams p)
             tc::mbar_arrive(&s.tempty[0]);
         }
         if (too_big) flag(p.status, MOE_DEV_NONFINITE);
+        ck.store(0, 1, warp == kEpiWarp0 && lane == 0);
+    } else if (warp == kTmaWarp) {  // -------------------------------------- TMA
+        if (lane == 0) issue_codes<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, KS, rm);
+    } else if (warp == kTmaBWarp) {
+        if (lane == 0) issue_rows<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, KS, &tmap_b, p.xperm);
     } else if (lane == 0) {  // --------------------------------------------- MMA
         int it = 0, tcount = 0;
-        for (int tau = blockIdx.x; tau < total && !s.abort; tau += gridDim.x, ++tcount) {
+        bool ok = true;
+        TcClock ck;
+        ck.start();
+        for (int tau = blockIdx.x; tau < total && ok && !s.abort; tau += gridDim.x, ++tcount) {
             const TileInfo ti = tile_info(p, s, tau, MT);
             const int npad = (ti.rows + 15) & ~15;
             const uint32_t idesc = tc::idesc_f16(128, npad);
+            const long long t0 = ck.now();
             if (!tc::mbar_wait(&s.tempty[0], (tcount & 1) ^ 1, kTcWaitNs)) {
-                set_abort(s, p.status);
+                ok = false;
                 break;
             }
+            ck.add(3, t0);
             tc::fence_after();
             const uint32_t dg = tmem, du = tmem + 256;
             for (int ks = 0; ks < KS; ++ks, ++it) {
-                const int st = it % kGuStages;
-                const uint32_t ph = (it / kGuStages) & 1;
-                if (!tc::mbar_wait(&s.full[st], ph, kTcWaitNs)) {
-                    set_abort(s, p.status);
+                if (!mma_wait_stage<kGuSA, kGuSB>(s, it, ck)) {
+                    ok = false;
                     break;
                 }
-                tc::fence_after();
-                const uint32_t base = tc::smem_u32(dyn + st * kGuStageBytes);
+                const uint32_t a = tc::smem_u32(GuRings::a(dyn, it));
+                const uint32_t b = tc::smem_u32(GuRings::b(dyn, it));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bd = tc::desc_sw128(base + 2 * kSub + 32 * kk);
+                    const uint64_t bd = tc::desc_sw128(b + 32 * kk);
                     const uint32_t acc = (ks | kk) ? 1u : 0u;
-                    tc::mma_f16(dg, tc::desc_sw128(base + 32 * kk), bd, idesc, acc);
-                    tc::mma_f16(du, tc::desc_sw128(base + kSub + 32 * kk), bd, idesc, acc);
+                    tc::mma_f16(dg, tc::desc_sw128(a + 32 * kk), bd, idesc, acc);
+                    tc::mma_f16(du, tc::desc_sw128(a + kSub + 32 * kk), bd, idesc, acc);
                 }
-                tc::mma_commit(&s.empty[st]);
+                mma_release_stage<kGuSA, kGuSB>(s, it);
             }
-            tc::mma_commit(&s.tfull[0]);
+            if (ok) tc::mma_commit(&s.tfull[0]);
         }
+        if (!ok) set_abort(s, p.status);
+        ck.store(0, 2, true);
     }
     tc::fence_before();
     __syncthreads();
@@ -441,31 +611,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gateup_q2_kernel(TcParams p)
 }
 
 // ----------------------------------------------------------------------- down
-// Stage (64 of K): A 16 KB + B (256 hidden rows) 32 KB, plus 4 KB of packed
-// codes. TMEM: two 256-column accumulators (the epilogue of one tile overlaps
-// the MMAs of the next).
-constexpr int kDnStages = 4;
-constexpr int kDnStageBytes = kSub + kSubB;
+// Rings: 2 A stages (16 KB each), 4 B stages (256 hidden rows, 32 KB each), 4
+// packed-code slots (one block pair, 5 KB each). TMEM: two 256-column accumulators (the
+// epilogue of one tile overlaps the MMAs of the next).
+constexpr int kDnSA = 2, kDnSB = 4, kDnSR = 4;
+using DnRings = Rings<1, kDnSA, kDnSB, kDnSR>;
 
-__global__ void __launch_bounds__(kTcThreads, 1) tc_down_q2_kernel(TcParams p) {
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_down_q2_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ RawMaps rm) {
     extern __shared__ __align__(1024) unsigned char dyn_raw[];
     unsigned char *dyn =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
     __shared__ TcSmem s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int MT = p.d / 128, KS = p.f / 64;
-    if (tid == 0) {
-        for (int i = 0; i < kDnStages; ++i) {
-            tc::mbar_init(&s.full[i], kProd);
-            tc::mbar_init(&s.empty[i], 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&s.tfull[i], 1);
-            tc::mbar_init(&s.tempty[i], kEpi);
-        }
-        s.abort = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
+    if (tid == 0) init_barriers<kDnSA, kDnSB, kDnSR>(s, 2);
     if (warp == kMmaWarp) tc::tmem_alloc(&s.tmem_base, 512);
     const int total = build_schedule(p, s, MT, reinterpret_cast<int *>(dyn));
     tc::fence_before();
@@ -474,23 +635,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_down_q2_kernel(TcParams p) {
     const uint32_t tmem = s.tmem_base;
 
     if (warp < kProdWarps) {  // --------------------------------------- producers
-        const MatGeom *mats[1] = {&p.down};
-        produce<1, kDnStages, false>(p, s, dyn, total, MT, KS, mats);
+        produce<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, KS);
     } else if (warp < kMmaWarp) {  // ---------------------------------- epilogue
-        const int q = warp - kEpiWarp0;
+        const int q = warp & 3, half = (warp - kEpiWarp0) >> 2;
         int tcount = 0;
+        TcClock ck;
+        ck.start();
         for (int tau = blockIdx.x; tau < total && !s.abort; tau += gridDim.x, ++tcount) {
             const TileInfo ti = tile_info(p, s, tau, MT);
             const int b = tcount & 1;
             const uint32_t ph = (tcount >> 1) & 1;
-            if (!tc::mbar_wait(&s.tfull[b], ph, kTcWaitNs)) {
+            const long long t0 = ck.now();
+            if (!tc::mbar_wait_sleep(&s.tfull[b], ph, kTcWaitNs, 128)) {
                 set_abort(s, p.status);
                 break;
             }
+            ck.add(1, t0);
+            ck.count(6);
             tc::fence_after();
             const int drow = 128 * ti.mi + 32 * q + lane;
             const uint32_t td = tmem + (uint32_t(32 * q) << 16) + uint32_t(b * 256);
-            for (int c0 = 0; c0 < ti.rows; c0 += 16) {
+            for (int c0 = 16 * half; c0 < ti.rows; c0 += 32) {
                 float v[16];
                 tc::tmem_ld16(td + c0, v);
 #pragma unroll
@@ -509,37 +674,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_down_q2_kernel(TcParams p) {
             tc::fence_before();
             tc::mbar_arrive(&s.tempty[b]);
         }
+        ck.store(1, 1, warp == kEpiWarp0 && lane == 0);
+    } else if (warp == kTmaWarp) {  // -------------------------------------- TMA
+        if (lane == 0) issue_codes<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, KS, rm);
+    } else if (warp == kTmaBWarp) {
+        if (lane == 0) issue_rows<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, KS, &tmap_b, p.h);
     } else if (lane == 0) {  // --------------------------------------------- MMA
         int it = 0, tcount = 0;
-        for (int tau = blockIdx.x; tau < total && !s.abort; tau += gridDim.x, ++tcount) {
+        bool ok = true;
+        TcClock ck;
+        ck.start();
+        for (int tau = blockIdx.x; tau < total && ok && !s.abort; tau += gridDim.x, ++tcount) {
             const TileInfo ti = tile_info(p, s, tau, MT);
             const int npad = (ti.rows + 15) & ~15;
             const uint32_t idesc = tc::idesc_f16(128, npad);
             const int b = tcount & 1;
             const uint32_t phb = (tcount >> 1) & 1;
+            const long long t0 = ck.now();
             if (!tc::mbar_wait(&s.tempty[b], phb ^ 1, kTcWaitNs)) {
-                set_abort(s, p.status);
+                ok = false;
                 break;
             }
+            ck.add(3, t0);
             tc::fence_after();
             const uint32_t dd = tmem + uint32_t(b * 256);
             for (int ks = 0; ks < KS; ++ks, ++it) {
-                const int st = it % kDnStages;
-                const uint32_t ph = (it / kDnStages) & 1;
-                if (!tc::mbar_wait(&s.full[st], ph, kTcWaitNs)) {
-                    set_abort(s, p.status);
+                if (!mma_wait_stage<kDnSA, kDnSB>(s, it, ck)) {
+                    ok = false;
                     break;
                 }
-                tc::fence_after();
-                const uint32_t base = tc::smem_u32(dyn + st * kDnStageBytes);
+                const uint32_t a = tc::smem_u32(DnRings::a(dyn, it));
+                const uint32_t bb = tc::smem_u32(DnRings::b(dyn, it));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_f16(dd, tc::desc_sw128(base + 32 * kk), tc::desc_sw128(base + kSub + 32 * kk), idesc,
+                    tc::mma_f16(dd, tc::desc_sw128(a + 32 * kk), tc::desc_sw128(bb + 32 * kk), idesc,
                                 (ks | kk) ? 1u : 0u);
-                tc::mma_commit(&s.empty[st]);
+                mma_release_stage<kDnSA, kDnSB>(s, it);
             }
-            tc::mma_commit(&s.tfull[b]);
+            if (ok) tc::mma_commit(&s.tfull[b]);
         }
+        if (!ok) set_abort(s, p.status);
+        ck.store(1, 2, true);
     }
     tc::fence_before();
     __syncthreads();
@@ -549,23 +724,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_down_q2_kernel(TcParams p) {
     }
 }
 
-// fp16 copy of the activations for the tensor cores (bf16 -> fp16 is exact for
-// normal values); |x| beyond 65504 sets MOE_DEV_NONFINITE.
-__global__ void __launch_bounds__(256) to_f16_kernel(const uint16_t *__restrict__ x, __half *__restrict__ y, int64_t n8,
-                                                      int32_t *status) {
+// Activation rows in sorted pair order, as fp16 for the tensor cores:
+// xperm[s] = x[sorted_tok[s]] (bf16 -> fp16 is exact for normal values);
+// |x| beyond 65504 sets MOE_DEV_NONFINITE. One CTA per row at a time.
+__global__ void __launch_bounds__(256) gather_f16_kernel(const uint16_t *__restrict__ x,
+                                                          const int32_t *__restrict__ sorted_tok, int d, int64_t rows,
+                                                          __half *__restrict__ y, int32_t *status) {
     bool bad = false;
-    for (int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x; i < n8; i += int64_t(gridDim.x) * 256) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x) + i);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-        uint32_t o[4];
+    const int n8 = d / 8;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int64_t t = sorted_tok[r];
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * d);
+        uint4 *dst = reinterpret_cast<uint4 *>(y + r * d);
+        for (int c = threadIdx.x; c < n8; c += blockDim.x) {
+            const uint4 v = __ldg(src + c);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float lo = bf16_lo(u[q]), hi = bf16_hi(u[q]);
-            bad |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
-            const __half2 hh = __floats2half2_rn(lo, hi);
-            o[q] = *reinterpret_cast<const uint32_t *>(&hh);
+            for (int q = 0; q < 4; ++q) {
+                const float lo = bf16_lo(u[q]), hi = bf16_hi(u[q]);
+                bad |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+                const __half2 hh = __floats2half2_rn(lo, hi);
+                o[q] = *reinterpret_cast<const uint32_t *>(&hh);
+            }
+            dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        reinterpret_cast<uint4 *>(y)[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (bad) flag(status, MOE_DEV_NONFINITE);
 }
@@ -573,9 +756,52 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const uint16_t *__restrict_
 std::mutex g_tc_mu;
 bool g_tc_ready[64] = {};
 int g_tc_sms[64] = {};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 
-constexpr size_t kGuSmem = size_t(kGuStages) * (kGuStageBytes + 2 * kRawMat) + 1024;
-constexpr size_t kDnSmem = size_t(kDnStages) * (kDnStageBytes + kRawMat) + 1024;
+// 2D fp16 tensor [rows][inner] (row pitch inner * 2 bytes) read in boxes of
+// box_rows x 64 with the 128-byte swizzle the MMA descriptors expect.
+bool f16_map(CUtensorMap *m, const void *base, int64_t inner, int64_t rows, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(inner) * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return g_encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D uint32 view [slots][row groups][words] of one region (codes or scales) of
+// matrix m in every pool slot, read in boxes of 8 row groups x box_words.
+bool raw_map(CUtensorMap *map, const uint8_t *pool, int64_t slot_bytes, int num_slots, uint64_t region_off,
+             int64_t words_per_group, int groups, uint32_t box_words) {
+    const cuuint64_t dims[3] = {cuuint64_t(words_per_group), cuuint64_t(groups), cuuint64_t(num_slots)};
+    const cuuint64_t strides[2] = {cuuint64_t(words_per_group) * 4, cuuint64_t(slot_bytes)};
+    const cuuint32_t box[3] = {box_words, 8, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t *>(pool + region_off), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool raw_maps(RawMaps *rm, const TcParams &p, const MatGeom *const *mats, int nmat) {
+    for (int i = 0; i < nmat; ++i) {
+        const MatGeom &m = *mats[i];
+        if (!raw_map(&rm->code[i], p.pool, p.slot_bytes, p.num_slots, m.codes_off, int64_t(m.NB / 2) * 128, m.NG,
+                     128) ||
+            !raw_map(&rm->scale[i], p.pool, p.slot_bytes, p.num_slots, m.scales_off, int64_t(m.NB / 2) * 32, m.NG,
+                     32))
+            return false;
+    }
+    return true;
+}
+
+constexpr size_t kGuSmem = size_t(GuRings::kBytes) + 1024;
+constexpr size_t kDnSmem = size_t(DnRings::kBytes) + 1024;
+static_assert(kDnSB <= kMaxSB && kGuSB <= kMaxSB && kDnSR <= kMaxSRP && kGuSR <= kMaxSRP,
+              "ring larger than its barrier array");
+static_assert(size_t(kKeys + 2 * kMaxActive) * 4 <= size_t(GuRings::kBytes) &&
+                  size_t(kKeys + 2 * kMaxActive) * 4 <= size_t(DnRings::kBytes),
+              "schedule scratch does not fit the stage memory");
 
 }  // namespace
 
@@ -600,6 +826,17 @@ moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_
                 cudaGetLastError();
                 return MOE_ERR_CUDA;
             }
+            if (!g_encode_tiled) {
+                void *fn = nullptr;
+                cudaDriverEntryPointQueryResult q;
+                if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                        cudaSuccess ||
+                    q != cudaDriverEntryPointSuccess || !fn) {
+                    cudaGetLastError();
+                    return MOE_ERR_CUDA;
+                }
+                g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            }
             g_tc_ready[dev] = true;
         }
     }
@@ -609,7 +846,7 @@ moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_
     p.slot_bytes = W->slot_bytes;
     p.num_slots = W->num_slots;
     p.slot_of = slot_of;
-    p.x16 = reinterpret_cast<const __half *>(static_cast<unsigned char *>(ws) + tc05_x16_offset(T, k, f));
+    p.xperm = reinterpret_cast<const __half *>(static_cast<unsigned char *>(ws) + tc05_xperm_offset(T, k, f));
     p.T = T;
     p.d = d;
     p.f = f;
@@ -627,12 +864,30 @@ moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_
     p.up = eg.m[1];
     p.down = eg.m[2];
     const int grid = g_tc_sms[dev];
-    const int64_t n8 = int64_t(T) * d / 8;
-    to_f16_kernel<<<int(std::min<int64_t>((n8 + 255) / 256, int64_t(grid) * 8)), 256, 0, stream>>>(
-        x, const_cast<__half *>(p.x16), n8, dev_status);
-    tc_gateup_q2_kernel<<<grid, kTcThreads, kGuSmem, stream>>>(p);
-    tc_down_q2_kernel<<<grid, kTcThreads, kDnSmem, stream>>>(p);
+    const int64_t pairs = int64_t(T) * k;
+    gather_f16_kernel<<<int(std::min<int64_t>(pairs, int64_t(grid) * 8)), 256, 0, stream>>>(
+        x, sorted_tok, d, pairs, const_cast<__half *>(p.xperm), dev_status);
+    CUtensorMap map_x, map_h;  // B operands: activation rows (gate/up), hidden rows (down)
+    RawMaps rm_gu, rm_dn;
+    const MatGeom *gu[2] = {&p.gate, &p.up}, *dn[1] = {&p.down};
+    if (!f16_map(&map_x, p.xperm, d, pairs, 64) || !f16_map(&map_h, p.h, f, pairs, 64) || !raw_maps(&rm_gu, p, gu, 2) ||
+        !raw_maps(&rm_dn, p, dn, 1))
+        return MOE_ERR_CUDA;
+    tc_gateup_q2_kernel<<<grid, kTcThreads, kGuSmem, stream>>>(p, map_x, rm_gu);
+    tc_down_q2_kernel<<<grid, kTcThreads, kDnSmem, stream>>>(p, map_h, rm_dn);
     return launch_status();
 }
 
 }  // namespace moe
+
+#ifdef MOE_TC_TRACE
+// Copies the wait accounting of the last tensor-core calls (uint64
+// [2 kernels][256 CTAs][4 roles][8]) to host memory and clears it.
+MOE_API int moe_tc_trace_read(unsigned long long *host) {
+    constexpr size_t kWords = size_t(2) * moe::kTraceCtas * 4 * 8;
+    static unsigned long long zeros[kWords];
+    if (cudaMemcpyFromSymbol(host, moe::g_tc_trace, kWords * 8) != cudaSuccess) return -1;
+    if (cudaMemcpyToSymbol(moe::g_tc_trace, zeros, kWords * 8) != cudaSuccess) return -1;
+    return 0;
+}
+#endif

@@ -200,8 +200,8 @@ moe_status moe_cache_lookup(const int32_t *slot_of, int32_t num_slots, int32_t l
                             int32_t *miss_count, int32_t miss_cap, int32_t *dev_status, moe_stream_t stream);
 
 /* Workspace bytes moe_expert_ffn_q2/q3 need for (T, k, d, f): the larger of
- * T*k*f fp32 (h, weight-streaming path) and T*k*f fp16 (h) + T*d fp16 (x),
- * rounded to 256 B (tensor-core path). */
+ * T*k*f fp32 (h, weight-streaming path) and T*k*f fp16 (h, rounded up to
+ * 256 B) + T*k*d fp16 (activation rows in sorted order) (tensor-core path). */
 size_t moe_expert_ffn_workspace_bytes(int T, int k, int d, int f);
 
 /*
@@ -226,8 +226,8 @@ size_t moe_expert_ffn_workspace_bytes(int T, int k, int d, int f);
  * T*k >= 512 and E <= 1024 (prefill) the Q2 call runs grouped GEMMs on the tcgen05 tensor
  * cores, dequantising each 128-row weight tile to fp16 in shared memory
  * (fp16 rounding of w = s*q + m); the workspace then holds h as fp16 [T*k][f]
- * followed by an fp16 copy of x [T][d]; ws must then be 256-byte and x
- * 16-byte aligned (else MOE_ERR_INVALID_ARG).
+ * followed by the activation rows in sorted pair order as fp16 [T*k][d]; ws
+ * must then be 256-byte and x 16-byte aligned (else MOE_ERR_INVALID_ARG).
  */
 moe_status moe_expert_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f,
                              int E, int k, const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j,
