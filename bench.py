@@ -237,15 +237,25 @@ def run_ours(args, wl, rank, world, local_rank):
     for i in range(args.steps):
         flush.fill_(float(i))
         ev[i][0].record(stream)
-        layer_step(xs[args.warmup + i], ev[i])
+        layer_step(xs[args.warmup + i])
         ev[i][3].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
     step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)]
-    ffn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
     total_ms = sum(step_ms)
+    # The dominant kernel's own time, for the roofline line: the same steps again
+    # with events around it (kept out of the timed steps above, whose value they
+    # would inflate). With one launch per step it is the step itself.
+    if fused:
+        ffn_ms = step_ms
+    else:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            layer_step(xs[args.warmup + i], ev[i])
+        torch.cuda.synchronize()
+        ffn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
     status = int(b.status.item())
 
     # distinct resident experts and resident pairs of each step's routing (not timed)

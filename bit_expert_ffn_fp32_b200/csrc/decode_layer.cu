@@ -474,6 +474,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
                 }
             }
         }
+    }
+    if (warp < T) {
         __syncwarp();
         if (warp == 0) TRACEW(13);
         const int sel_id = lane < k ? s.sel_id[warp][lane] : 0;
@@ -579,40 +581,124 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
     }
     __syncthreads();
     TRACE(5);
-    {  // L2 prefetch of the expert rows this CTA's later tasks read, one region per lane
+    {  // L2 prefetch of every selected expert, spread over the grid: the
+        // concatenation of all resident experts' gate/up parts, then their down
+        // parts and the shared expert's, is cut into G equal slices and the
+        // threads of CTA c ask the L2 for the lines of slice c
         const int nres = s.nres;
-        const int ndt = (nres + 1) * (d / 128);  // down CTA-tasks: (expert, 8 row groups)
-        if (warp == 0) {  // gate/up: 4 regions per task, 8 tasks per pass
-            for (int base = (G - 1 - cta) + G * (lane >> 2); base < nres * NG; base += 8 * G) {
-                const int a = s.res[base / NG], rg = base % NG;
-                const uint8_t *rec = p.pool + int64_t(s.act_slot[a]) * p.slot_bytes;
-                const int r = lane & 3;
-                const MatGeom &m = (r & 1) ? p.up : p.gate;
-                if (r < 2) prefetch_l2(rec + m.codes_off + uint64_t(rg) * gu_codes, gu_codes);
-                else prefetch_l2(rec + m.scales_off + uint64_t(rg) * gu_scales, gu_scales);
+        const uint32_t GU = uint32_t(p.down.codes_off);  // gate + up of one record
+        const uint32_t DN = uint32_t(p.down.bytes);      // down of one record
+        const uint32_t gu_all = uint32_t(nres) * GU;     // < 2^32: at most 128 records of < 8 MB
+        const uint32_t total = gu_all + uint32_t(nres + 1) * DN;
+        const uint32_t lo = uint32_t((uint64_t(total) * uint32_t(cta) / uint32_t(G))) & ~127u;
+        const uint32_t hi = cta == G - 1 ? total : uint32_t((uint64_t(total) * uint32_t(cta + 1) / uint32_t(G))) & ~127u;
+        // one 128-byte line per thread and step (GU and DN are multiples of 256)
+        int r = -1;          // region of the current line and its start
+        uint32_t r0 = 0, r1 = 0;
+        const uint8_t *rsrc = nullptr;
+        for (uint32_t o = lo + uint32_t(tid) * 128u; o < hi; o += uint32_t(kThreads) * 128u) {
+            while (o >= r1) {  // advance to the region holding o (regions in order, each >= 1 step)
+                ++r;
+                r0 = r1;
+                if (r < nres) {
+                    r1 = r0 + GU;
+                    rsrc = p.pool + int64_t(s.act_slot[s.res[r]]) * p.slot_bytes;
+                } else {
+                    const int q = r - nres;
+                    r1 = r0 + DN;
+                    const int slot = q < nres ? s.act_slot[s.res[q]] : p.shared_slot;
+                    rsrc = p.pool + int64_t(slot) * p.slot_bytes + p.down.codes_off;
+                }
             }
-        } else if (warp == 1) {  // down: 2 regions per task, 16 tasks per pass
-            for (int task = cta + G * (lane >> 1); task < ndt; task += 16 * G) {
-                const int ar = task / (d / 128), blk = task % (d / 128);
-                const int slot = ar < nres ? s.act_slot[s.res[ar]] : p.shared_slot;
-                const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
-                if (lane & 1) prefetch_l2(rec + p.down.scales_off + uint64_t(8 * blk) * dn_scales, 8u * dn_scales);
-                else prefetch_l2(rec + p.down.codes_off + uint64_t(8 * blk) * dn_codes, 8u * dn_codes);
-            }
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(rsrc + (o - r0)));
         }
     }
     TRACE(3);
     // ------------------------------------------------------------ phase C
-    for (int task = G - 1 - cta; task < s.nres * NG; task += G) {  // busy phase-A CTAs last
-        const int ar = task / NG, rg = task % NG;
-        const int a = s.res[ar];
-        const uint8_t *rec = p.pool + int64_t(s.act_slot[a]) * p.slot_bytes;
-        gateup_task<FMT>(p, s, sx, rec, rg, s.act_cnt[a], s.s_tok + s.act_beg[a], s.act_beg[a]);
-        __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            atomicAdd(p.done + ar, 1u);
+    {  // busy phase-A CTAs last; warp w handles K quads w, w+8, ... of every task,
+        // and loads the next task's tiles before computing the current one
+        const int ntasks = s.nres * NG;
+        const int NQ = d / 256;
+        const int g = lane >> 2, t = lane & 3;
+        int task = G - 1 - cta;
+        QuadRegs<FMT> ng, nu;  // tiles of the next task (quad = warp)
+        auto load_task = [&](int tk, QuadRegs<FMT> &qg, QuadRegs<FMT> &qu) {
+            const int ar = tk / NG, rg = tk % NG;
+            const uint8_t *rec = p.pool + int64_t(s.act_slot[s.res[ar]]) * p.slot_bytes;
+            quad_load<FMT>(rec, p.gate, rg, warp, lane, qg);
+            quad_load<FMT>(rec, p.up, rg, warp, lane, qu);
+        };
+        const bool one_quad = NQ == kWarps;  // every warp owns exactly one quad
+        if (one_quad && task < ntasks) load_task(task, ng, nu);
+        uint32_t B1[4][8];     // one token: fragments of quad `warp`, built once
+        float xs1[4][2];
+        if (NT == 1 && one_quad) {
+            build_b_bf16<FMT>(g == 0 ? sx : nullptr, warp, t, B1);
+#pragma unroll
+            for (int bq = 0; bq < 4; ++bq) {
+                xs1[bq][0] = t == 0 ? s.xs[4 * warp + bq][0] : 0.f;
+                xs1[bq][1] = 0.f;
+            }
         }
+        int nth = 0;
+        for (; task < ntasks; task += G, ++nth) {
+            const int ar = task / NG, rg = task % NG;
+            const int a = s.res[ar];
+            const int ntok = s.act_cnt[a];
+            const int *tok = s.s_tok + s.act_beg[a];
+            if (!one_quad) {  // general d: tiles loaded inside the task
+                const uint8_t *rec = p.pool + int64_t(s.act_slot[a]) * p.slot_bytes;
+                gateup_task<FMT>(p, s, sx, rec, rg, ntok, tok, s.act_beg[a]);
+                __syncthreads();
+                continue;
+            }
+            const QuadRegs<FMT> cg = ng, cu = nu;
+            if (task + G < ntasks) load_task(task + G, ng, nu);
+            float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
+            if (NT == 1) {
+                quad_compute<FMT>(cg, B1, xs1, ag);
+                quad_compute<FMT>(cu, B1, xs1, au);
+            } else {
+                const uint16_t *xrow = g < ntok ? sx + size_t(tok[g]) * d : nullptr;
+                const int t0 = 2 * t < ntok ? tok[2 * t] : -1, t1 = 2 * t + 1 < ntok ? tok[2 * t + 1] : -1;
+                uint32_t B[4][8];
+                build_b_bf16<FMT>(xrow, warp, t, B);
+                float xs[4][2];
+#pragma unroll
+                for (int bq = 0; bq < 4; ++bq) {
+                    xs[bq][0] = t0 >= 0 ? s.xs[4 * warp + bq][t0] : 0.f;
+                    xs[bq][1] = t1 >= 0 ? s.xs[4 * warp + bq][t1] : 0.f;
+                }
+                quad_compute<FMT>(cg, B, xs, ag);
+                quad_compute<FMT>(cu, B, xs, au);
+            }
+            if (nth < 2 && warp == 0) TRACEW(nth == 0 ? 9 : 15);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                s.red[warp][0][r][lane] = ag[r];
+                s.red[warp][1][r][lane] = au[r];
+            }
+            __syncthreads();
+            if (tid < 128) {
+                const int L = tid >> 2, r = tid & 3;
+                float A = 0.f, U = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) {
+                    A += s.red[w][0][r][L];
+                    U += s.red[w][1][r][L];
+                }
+                const int row = (L >> 2) + ((r & 2) ? 8 : 0);
+                const int n = 2 * (L & 3) + (r & 1);
+                if (n < ntok) p.h[size_t(s.act_beg[a] + n) * f + 16 * rg + row] = A / (1.0f + expf(-A)) * U;
+            }
+            __syncthreads();
+            if (nth == 0) TRACE(14);
+        }
+    }
+    // publish this CTA's h rows once (one fence), then count its tasks per expert
+    if (tid == 0) {
+        __threadfence();
+        for (int task = G - 1 - cta; task < s.nres * NG; task += G) atomicAdd(p.done + task / NG, 1u);
     }
 
     TRACE(7);

@@ -22,7 +22,8 @@ from .layer import MoEStack, x_tensor
 
 POINTS = {8: "x staged", 10: "router rows (warp 0)", 1: "phase A done", 2: "all logits counted",
           11: "top-k loads", 12: "top-k candidates", 13: "top-k selected", 6: "top-k + gates",
-          5: "routing tables", 3: "prefetch issued", 7: "phase C done", 4: "kernel end"}
+          5: "routing tables", 3: "prefetch issued", 9: "C task 1 computed (warp 0)",
+          14: "C task 1 done", 15: "C task 2 computed (warp 0)", 7: "phase C done", 4: "kernel end"}
 
 
 def main() -> None:
