@@ -45,9 +45,12 @@ constexpr int kMmaWarp = kProdWarps + kEpiWarps;       // 16
 constexpr int kTmaWarp = kMmaWarp + 1;                 // 17: TMA loads of the packed codes
 constexpr int kTmaBWarp = kMmaWarp + 2;                // 18: TMA loads of the B rows, L2 prefetch
 constexpr int kTcThreads = kProd + kEpi + 96;
-constexpr int kTileN = 256;  // tokens per tile (MMA N, padded to 16)
-constexpr int kSub = 16384;  // 128 rows x 64 cols fp16, SW128
-constexpr int kSubB = 32768;  // 256 rows x 64 cols fp16, SW128
+// Tokens per tile (MMA N, padded to 16), bounded by tensor memory: gate/up
+// keeps D_gate and D_up (2 x 192 columns) plus two 64-column A stages, down
+// two 192-column accumulators plus two 32-column A stages (of 512 columns).
+constexpr int kTileGu = 192;
+constexpr int kTileDn = 192;
+constexpr int kSubB = 24576;  // B stage: 192 rows x 64 cols fp16, SW128
 constexpr unsigned long long kTcWaitNs = 200ull * 1000 * 1000;
 constexpr int kMaxActive = kTcMaxE;  // experts per call on this path
 
@@ -100,7 +103,7 @@ struct TcParams {
     MatGeom gate, up, down;
 };
 
-constexpr int kMaxSB = 4;    // B stage slots (max over the two kernels)
+constexpr int kMaxSB = 7;    // B stage slots (max over the two kernels)
 constexpr int kMaxSRP = 4;   // packed-code slots
 constexpr int kKeys = 512;   // schedule sort keys
 
@@ -129,16 +132,16 @@ __device__ __forceinline__ int expert_rows(const TcParams &p, int e) {
 
 // Sort key (larger first): tiles (capped at 32), then the 16-token size class
 // of the last tile; -1 for an expert without tokens.
-__device__ __forceinline__ int sched_key(int n) {
+__device__ __forceinline__ int sched_key(int n, int TN) {
     if (n <= 0) return -1;
-    const int nt = (n + kTileN - 1) / kTileN;
-    const int last = n - kTileN * (nt - 1);
+    const int nt = (n + TN - 1) / TN;
+    const int last = n - TN * (nt - 1);
     return (min(nt, 32) - 1) * 16 + ((last + 15) >> 4) - 1;
 }
 
 // Whole CTA: build the tile order; returns the tile count. scratch is the
 // (not yet used) stage memory: kKeys + 2 * kMaxActive ints.
-__device__ int build_schedule(const TcParams &p, TcSmem &s, int MT, int *scratch) {
+__device__ int build_schedule(const TcParams &p, TcSmem &s, int MT, int TN, int *scratch) {
     const int na = min(p.active[0], kMaxActive);
     const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31;
     int *hist = scratch;                       // per key: count, then first position
@@ -147,7 +150,7 @@ __device__ int build_schedule(const TcParams &p, TcSmem &s, int MT, int *scratch
     for (int i = tid; i < kKeys; i += nthr) hist[i] = 0;
     __syncthreads();
     for (int a = tid; a < na; a += nthr) {
-        const int key = sched_key(expert_rows(p, p.active[1 + a]));
+        const int key = sched_key(expert_rows(p, p.active[1 + a]), TN);
         akey[a] = key;
         if (key >= 0) atomicAdd(&hist[key], 1);
     }
@@ -193,7 +196,7 @@ __device__ int build_schedule(const TcParams &p, TcSmem &s, int MT, int *scratch
         const int per = (nexp + 31) / 32;
         const int i0 = min(nexp, lane * per), i1 = min(nexp, i0 + per);
         int sum = 0;
-        for (int i = i0; i < i1; ++i) sum += MT * ((s.erows[i] + kTileN - 1) / kTileN);
+        for (int i = i0; i < i1; ++i) sum += MT * ((s.erows[i] + TN - 1) / TN);
         int incl = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -203,7 +206,7 @@ __device__ int build_schedule(const TcParams &p, TcSmem &s, int MT, int *scratch
         int acc = incl - sum;
         for (int i = i0; i < i1; ++i) {
             s.tiles_prefix[i] = acc;
-            acc += MT * ((s.erows[i] + kTileN - 1) / kTileN);
+            acc += MT * ((s.erows[i] + TN - 1) / TN);
         }
         if (lane == 31) s.tiles_prefix[nexp] = incl;
     }
@@ -215,7 +218,7 @@ struct TileInfo {
     int slot, beg, rows, mi;
 };
 
-__device__ __forceinline__ TileInfo tile_info(const TcParams &p, const TcSmem &s, int tau, int MT) {
+__device__ __forceinline__ TileInfo tile_info(const TcParams &p, const TcSmem &s, int tau, int MT, int TN) {
     int lo = 0, hi = s.nexp;  // last i with tiles_prefix[i] <= tau
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -226,8 +229,8 @@ __device__ __forceinline__ TileInfo tile_info(const TcParams &p, const TcSmem &s
     TileInfo t;
     t.slot = s.eslot[lo];
     t.mi = local - ni * MT;
-    t.beg = s.ebeg[lo] + kTileN * ni;
-    t.rows = min(kTileN, s.erows[lo] - kTileN * ni);
+    t.beg = s.ebeg[lo] + TN * ni;
+    t.rows = min(TN, s.erows[lo] - TN * ni);
     return t;
 }
 
@@ -237,28 +240,25 @@ struct HalfQ2 {
     uint2 cw, sc;
 };
 
-// Dequantise into a 128-row x 64-col SW128 sub-tile: w = s*q + m in fp16
-// (q made exact in fp16 by the 1024-offset trick, then one fused multiply-add).
-__device__ __forceinline__ void store_half_q2(const HalfQ2 &c, int rgl, int L, unsigned char *sub) {
-    const int g = L >> 2, t = L & 3;
+// Dequantise one block of a lane chunk (rows g and g+8, k = 16i + 8s + 2t + h
+// for register slot rho = 2i + s) into fp16 pairs: v[2*rho] row g, v[2*rho+1]
+// row g+8; w = s*q + m (q made exact in fp16 by the 1024-offset trick, then
+// one fused multiply-add).
+__device__ __forceinline__ void dequant_half_q2(const HalfQ2 &c, uint32_t (&v)[16]) {
     const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));
     const __half2 s01 = *reinterpret_cast<const __half2 *>(&c.sc.x);
     const __half2 m01 = *reinterpret_cast<const __half2 *>(&c.sc.y);
-    // rows g and g+8 share (row & 7) = g, so their chunk order is the same
-    unsigned char *row0 = sub + (2 * rgl) * 1024 + g * 128 + 4 * t;  // row 16rgl+g (8-row group 2rgl)
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         const uint32_t w = r ? c.cw.y : c.cw.x;
         const __half2 s2 = r ? __high2half2(s01) : __low2half2(s01);
         const __half2 m2 = r ? __high2half2(m01) : __low2half2(m01);
-        unsigned char *rowp = row0 + r * 1024;  // row g+8 is in the next 8-row group
 #pragma unroll
         for (int rho = 0; rho < 8; ++rho) {
             const uint32_t qbits = ((w >> (2 * rho)) & 0x00030003u) | 0x64006400u;
             const __half2 q = __hsub2(*reinterpret_cast<const __half2 *>(&qbits), k1024);
             const __half2 wv = __hfma2(s2, q, m2);
-            const int j = 2 * (rho >> 1) + (rho & 1);  // 16-byte chunk of the row
-            *reinterpret_cast<__half2 *>(rowp + ((j ^ g) << 4)) = wv;
+            v[2 * rho + r] = *reinterpret_cast<const uint32_t *>(&wv);
         }
     }
 }
@@ -270,9 +270,9 @@ __device__ __forceinline__ void set_abort(TcSmem &s, int32_t *status) {
 // Ask the L2 for tile tau's packed weight rows (codes and scales, one
 // contiguous range per matrix and region) and its B rows (K fp16 each).
 template <int NMAT>
-__device__ __forceinline__ void prefetch_tile(const TcParams &p, const TcSmem &s, int tau, int MT, int K,
+__device__ __forceinline__ void prefetch_tile(const TcParams &p, const TcSmem &s, int tau, int MT, int TN, int K,
                                               const __half *bsrc) {
-    const TileInfo t = tile_info(p, s, tau, MT);
+    const TileInfo t = tile_info(p, s, tau, MT, TN);
     const uint8_t *rec = p.pool + int64_t(t.slot) * p.slot_bytes;
     const MatGeom *mats[2] = {NMAT == 2 ? &p.gate : &p.down, &p.up};
 #pragma unroll
@@ -288,19 +288,15 @@ __device__ __forceinline__ void prefetch_tile(const TcParams &p, const TcSmem &s
 constexpr int kRawCodes = 8 * 512;
 constexpr int kRawPairMat = kRawCodes + 8 * 128;
 
-// Shared-memory rings of a kernel: SA dequantised A stages (NMAT 128x64 fp16
-// sub-tiles each), SB B stages (256 rows x 64 fp16), SRP slots of packed A
-// bytes (one block pair each).
-template <int NMAT, int SA, int SB, int SRP>
+// Shared-memory rings of a kernel: SB B stages (256 rows x 64 fp16) and SRP
+// slots of packed A bytes (one block pair each). The dequantised A stages live
+// in tensor memory.
+template <int NMAT, int SB, int SRP>
 struct Rings {
-    static constexpr int kA = NMAT * kSub;
     static constexpr int kRaw = NMAT * kRawPairMat;
-    static constexpr int kBytes = SA * kA + SB * kSubB + SRP * kRaw;
-    __device__ static unsigned char *a(unsigned char *dyn, int it) { return dyn + (it % SA) * kA; }
-    __device__ static unsigned char *b(unsigned char *dyn, int it) { return dyn + SA * kA + (it % SB) * kSubB; }
-    __device__ static unsigned char *raw(unsigned char *dyn, int pp) {
-        return dyn + SA * kA + SB * kSubB + (pp % SRP) * kRaw;
-    }
+    static constexpr int kBytes = SB * kSubB + SRP * kRaw;
+    __device__ static unsigned char *b(unsigned char *dyn, int it) { return dyn + (it % SB) * kSubB; }
+    __device__ static unsigned char *raw(unsigned char *dyn, int pp) { return dyn + SB * kSubB + (pp % SRP) * kRaw; }
 };
 
 // Tensor maps of the packed weights, per matrix: codes as uint32 [slot][row
@@ -323,9 +319,9 @@ struct StageCursor {
 //            it % SB once the MMA has released it (emptyB); complete on
 //            fullB. On entering a tile it asks the L2 for the next tile.
 template <int NMAT, int SA, int SB, int SRP>
-__device__ __forceinline__ void issue_codes(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int KS,
-                                            const RawMaps &rm) {
-    using R = Rings<NMAT, SA, SB, SRP>;
+__device__ __forceinline__ void issue_codes(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int TN,
+                                            int KS, const RawMaps &rm) {
+    using R = Rings<NMAT, SB, SRP>;
     const int PS = KS / 2;
     const int mine = blockIdx.x < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
     const int npairs = mine * PS;
@@ -338,7 +334,7 @@ __device__ __forceinline__ void issue_codes(const TcParams &p, TcSmem &s, unsign
     }
     int tau = blockIdx.x, pk = 0;
     TileInfo t{};
-    if (mine > 0) t = tile_info(p, s, tau, MT);
+    if (mine > 0) t = tile_info(p, s, tau, MT, TN);
     bool ok = true;
 #pragma unroll 1
     for (int pr = 0; pr < npairs && !s.abort; ++pr) {
@@ -362,7 +358,7 @@ __device__ __forceinline__ void issue_codes(const TcParams &p, TcSmem &s, unsign
         if (++pk == PS) {
             pk = 0;
             tau += gridDim.x;
-            if (tau < total) t = tile_info(p, s, tau, MT);
+            if (tau < total) t = tile_info(p, s, tau, MT, TN);
         }
     }
     if (!ok) set_abort(s, p.status);
@@ -370,16 +366,15 @@ __device__ __forceinline__ void issue_codes(const TcParams &p, TcSmem &s, unsign
 }
 
 template <int NMAT, int SA, int SB, int SRP>
-__device__ __forceinline__ void issue_rows(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int KS,
-                                           const void *tmap_b, const __half *bsrc) {
-    using R = Rings<NMAT, SA, SB, SRP>;
+__device__ __forceinline__ void issue_rows(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int TN,
+                                           int KS, const void *tmap_b, const __half *bsrc) {
+    using R = Rings<NMAT, SB, SRP>;
     const int mine = blockIdx.x < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
     const int nstages = mine * KS;
     tc::prefetch_tensormap(tmap_b);
     int tau = blockIdx.x, ks = 0;
     TileInfo t{};
-    if (mine > 0) t = tile_info(p, s, tau, MT);
-    if (mine > 1) prefetch_tile<NMAT>(p, s, tau + gridDim.x, MT, 64 * KS, bsrc);
+    if (mine > 0) t = tile_info(p, s, tau, MT, TN);
     bool ok = true;
 #pragma unroll 1
     for (int pb = 0; pb < nstages && !s.abort; ++pb) {
@@ -395,21 +390,27 @@ __device__ __forceinline__ void issue_rows(const TcParams &p, TcSmem &s, unsigne
         if (++ks == KS) {
             ks = 0;
             tau += gridDim.x;
-            if (tau < total) t = tile_info(p, s, tau, MT);
-            if (tau + int(gridDim.x) < total) prefetch_tile<NMAT>(p, s, tau + gridDim.x, MT, 64 * KS, bsrc);
+            if (tau < total) t = tile_info(p, s, tau, MT, TN);
         }
     }
     if (!ok) set_abort(s, p.status);
 }
 
-// Producer warps (0-7): for each stage, once its block pair's packed bytes have
-// landed (fullR) and the MMA has released the A slot (emptyA), dequantise the
-// thread's lane chunk into the A ring, then arrive on fullA (and on emptyR
-// after the pair's second block).
+// Producer warps (0-7): warp w owns row group rgl = 2(w%4) + w/4 of the
+// 128-row tile (its tensor-memory lane quadrant is w%4). For each stage, once
+// the block pair's packed bytes have landed (fullR) and the MMA has released
+// the A stage (emptyA), each thread dequantises its lane chunk (rows g, g+8 of
+// the row group; k-slots of t) into registers and stores it to the stage's
+// TMEM columns (lane g / g+8, column 4*rho + t = k/2), then arrives on fullA
+// (and on emptyR after the pair's second block). a_col0: TMEM column of A
+// stage 0, matrix 0; stages are 32*NMAT columns apart.
 template <int NMAT, int SA, int SB, int SRP>
-__device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int KS) {
-    using R = Rings<NMAT, SA, SB, SRP>;
+__device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int KS,
+                                        uint32_t tmem, int a_col0) {
+    using R = Rings<NMAT, SB, SRP>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rgl = 2 * (warp & 3) + (warp >> 2);
+    const uint32_t ta = tmem + (uint32_t(16 * rgl) << 16) + uint32_t(a_col0);
     const int mine = blockIdx.x < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
     const int nstages = mine * KS;
     TcClock ck;
@@ -429,19 +430,22 @@ __device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned c
             ok = false;
             break;
         }
+        tc::fence_after();
         ck.add(2, t0);
         t0 = ck.now();
-        unsigned char *atile = R::a(dyn, it);
         const unsigned char *raw = R::raw(dyn, pp);
 #pragma unroll
         for (int i = 0; i < NMAT; ++i) {
             HalfQ2 c;
-            c.cw = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + warp * 512 + lane * 16 + 8 * bb);
-            c.sc = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + kRawCodes + warp * 128 + (lane >> 2) * 16 +
+            c.cw = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + rgl * 512 + lane * 16 + 8 * bb);
+            c.sc = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + kRawCodes + rgl * 128 + (lane >> 2) * 16 +
                                                     8 * bb);
-            store_half_q2(c, warp, lane, atile + i * kSub);
+            uint32_t v[16];
+            dequant_half_q2(c, v);
+            tc::tmem_st16x128_x8(ta + uint32_t((it % SA) * 32 * NMAT + 32 * i), v);
         }
-        tc::fence_proxy_async();
+        tc::tmem_st_wait();
+        tc::fence_before();
         tc::mbar_arrive(&s.fullA[it % SA]);
         if (bb) tc::mbar_arrive(&s.emptyR[pp % SRP]);
         ck.add(4, t0);
@@ -497,11 +501,14 @@ __device__ __forceinline__ void mma_release_stage(TcSmem &s, int it) {
 }
 
 // -------------------------------------------------------------------- gate/up
-// Rings: 2 A stages (gate + up, 32 KB each), 3 B stages (256 tokens, 32 KB
-// each), 4 packed-code slots (one block pair, 10 KB each). TMEM: D_g columns 0..255, D_u
-// 256..511 (one accumulator pair; the epilogue is short).
-constexpr int kGuSA = 2, kGuSB = 3, kGuSR = 4;
-using GuRings = Rings<2, kGuSA, kGuSB, kGuSR>;
+// Shared memory: 5 B stages (up to 192 tokens, 24 KB each), 4 packed-code
+// slots (one block pair, 10 KB each), 1 KB of h staging per epilogue warp.
+// TMEM: D_gate columns 0..191, D_up 192..383 (one accumulator pair), A stages
+// at 384 and 448 (gate 32 columns, then up 32 columns).
+constexpr int kGuSA = 2, kGuSB = 5, kGuSR = 4;
+constexpr int kHStage = 1024;  // per epilogue warp: 16 tokens x 32 rows of h (fp16)
+constexpr int kGuColU = kTileGu, kGuColA = 2 * kTileGu;
+using GuRings = Rings<2, kGuSB, kGuSR>;
 
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gateup_q2_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmap_b,
@@ -511,17 +518,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
     __shared__ TcSmem s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int MT = p.f / 128, KS = p.d / 64;
+    const int MT = p.f / 128, KS = p.d / 64, TN = kTileGu;
+    unsigned char *hstage = dyn + GuRings::kBytes;  // epilogue staging of h
     if (tid == 0) init_barriers<kGuSA, kGuSB, kGuSR>(s, 1);
     if (warp == kMmaWarp) tc::tmem_alloc(&s.tmem_base, 512);
-    const int total = build_schedule(p, s, MT, reinterpret_cast<int *>(dyn));
+    const int total = build_schedule(p, s, MT, TN, reinterpret_cast<int *>(dyn));
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = s.tmem_base;
 
     if (warp < kProdWarps) {  // --------------------------------------- producers
-        produce<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, KS);
+        produce<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, KS, tmem, kGuColA);
     } else if (warp < kMmaWarp) {  // ---------------------------------- epilogue
         const int q = warp & 3, half = (warp - kEpiWarp0) >> 2;  // TMEM lane quadrant, column half
         int tcount = 0;
@@ -529,7 +537,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         TcClock ck;
         ck.start();
         for (int tau = blockIdx.x; tau < total && !s.abort; tau += gridDim.x, ++tcount) {
-            const TileInfo ti = tile_info(p, s, tau, MT);
+            const TileInfo ti = tile_info(p, s, tau, MT, TN);
             const long long t0 = ck.now();
             if (!tc::mbar_wait_sleep(&s.tfull[0], tcount & 1, kTcWaitNs, 128)) {
                 set_abort(s, p.status);
@@ -538,22 +546,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ck.add(1, t0);
             ck.count(6);
             tc::fence_after();
-            const int frow = 128 * ti.mi + 32 * q + lane;
+            // rows 128mi + 32q + lane of h for 16 tokens at a time: staged in this
+            // warp's 1 KB ([token][32 rows] fp16), then written as 64-byte pieces
+            // (16 bytes per lane) of the tokens' h rows
             const uint32_t tg = tmem + (uint32_t(32 * q) << 16);
+            __half *hs = reinterpret_cast<__half *>(hstage + (warp - kEpiWarp0) * kHStage);
+            __half *hrow0 = p.h + int64_t(ti.beg) * p.f + 128 * ti.mi + 32 * q;
             for (int c0 = 16 * half; c0 < ti.rows; c0 += 32) {
                 float g[16], u[16];
                 const long long t1 = ck.now();
                 tc::tmem_ld16(tg + c0, g);
-                tc::tmem_ld16(tg + 256 + c0, u);
+                tc::tmem_ld16(tg + kGuColU + c0, u);
                 ck.add(2, t1);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    if (c0 + j < ti.rows) {
-                        const float hv = __fdividef(g[j], 1.0f + __expf(-g[j])) * u[j];
-                        too_big |= !(fabsf(hv) <= 65504.f);
-                        p.h[int64_t(ti.beg + c0 + j) * p.f + frow] = __float2half_rn(hv);
-                    }
+                    const float hv = __fdividef(g[j], 1.0f + __expf(-g[j])) * u[j];
+                    too_big |= c0 + j < ti.rows && !(fabsf(hv) <= 65504.f);
+                    hs[j * 32 + lane] = __float2half_rn(hv);
                 }
+                __syncwarp();
+#pragma unroll
+                for (int pass = 0; pass < 2; ++pass) {
+                    const int j = 8 * pass + (lane >> 2), ch = lane & 3;
+                    if (c0 + j < ti.rows)
+                        *reinterpret_cast<uint4 *>(hrow0 + int64_t(c0 + j) * p.f + 8 * ch) =
+                            *reinterpret_cast<const uint4 *>(hs + j * 32 + 8 * ch);
+                }
+                __syncwarp();
             }
             tc::fence_before();
             tc::mbar_arrive(&s.tempty[0]);
@@ -561,16 +580,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (too_big) flag(p.status, MOE_DEV_NONFINITE);
         ck.store(0, 1, warp == kEpiWarp0 && lane == 0);
     } else if (warp == kTmaWarp) {  // -------------------------------------- TMA
-        if (lane == 0) issue_codes<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, KS, rm);
+        if (lane == 0) issue_codes<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, TN, KS, rm);
     } else if (warp == kTmaBWarp) {
-        if (lane == 0) issue_rows<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, KS, &tmap_b, p.xperm);
+        if (lane == 0) issue_rows<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, TN, KS, &tmap_b, p.xperm);
     } else if (lane == 0) {  // --------------------------------------------- MMA
         int it = 0, tcount = 0;
         bool ok = true;
         TcClock ck;
         ck.start();
         for (int tau = blockIdx.x; tau < total && ok && !s.abort; tau += gridDim.x, ++tcount) {
-            const TileInfo ti = tile_info(p, s, tau, MT);
+            const TileInfo ti = tile_info(p, s, tau, MT, TN);
             const int npad = (ti.rows + 15) & ~15;
             const uint32_t idesc = tc::idesc_f16(128, npad);
             const long long t0 = ck.now();
@@ -580,20 +599,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             ck.add(3, t0);
             tc::fence_after();
-            const uint32_t dg = tmem, du = tmem + 256;
+            const uint32_t dg = tmem, du = tmem + kGuColU;
             for (int ks = 0; ks < KS; ++ks, ++it) {
                 if (!mma_wait_stage<kGuSA, kGuSB>(s, it, ck)) {
                     ok = false;
                     break;
                 }
-                const uint32_t a = tc::smem_u32(GuRings::a(dyn, it));
+                const uint32_t a = tmem + uint32_t(kGuColA + (it % kGuSA) * 64);  // gate, then up at +32
                 const uint32_t b = tc::smem_u32(GuRings::b(dyn, it));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t bd = tc::desc_sw128(b + 32 * kk);
                     const uint32_t acc = (ks | kk) ? 1u : 0u;
-                    tc::mma_f16(dg, tc::desc_sw128(a + 32 * kk), bd, idesc, acc);
-                    tc::mma_f16(du, tc::desc_sw128(a + kSub + 32 * kk), bd, idesc, acc);
+                    tc::mma_f16_ta(dg, a + 8 * kk, bd, idesc, acc);
+                    tc::mma_f16_ta(du, a + 32 + 8 * kk, bd, idesc, acc);
                 }
                 mma_release_stage<kGuSA, kGuSB>(s, it);
             }
@@ -611,11 +630,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ----------------------------------------------------------------------- down
-// Rings: 2 A stages (16 KB each), 4 B stages (256 hidden rows, 32 KB each), 4
-// packed-code slots (one block pair, 5 KB each). TMEM: two 256-column accumulators (the
-// epilogue of one tile overlaps the MMAs of the next).
-constexpr int kDnSA = 2, kDnSB = 4, kDnSR = 4;
-using DnRings = Rings<1, kDnSA, kDnSB, kDnSR>;
+// Shared memory: 7 B stages (up to 192 hidden rows, 24 KB each), 4
+// packed-code slots (one block pair, 5 KB each). TMEM: two 192-column
+// accumulators at 0 and 192 (the epilogue of one tile overlaps the MMAs of the
+// next), A stages at 384 and 416.
+constexpr int kDnSA = 2, kDnSB = 7, kDnSR = 4;
+constexpr int kDnColA = 2 * kTileDn;
+using DnRings = Rings<1, kDnSB, kDnSR>;
 
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_down_q2_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmap_b,
@@ -625,24 +646,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
     __shared__ TcSmem s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int MT = p.d / 128, KS = p.f / 64;
+    const int MT = p.d / 128, KS = p.f / 64, TN = kTileDn;
     if (tid == 0) init_barriers<kDnSA, kDnSB, kDnSR>(s, 2);
     if (warp == kMmaWarp) tc::tmem_alloc(&s.tmem_base, 512);
-    const int total = build_schedule(p, s, MT, reinterpret_cast<int *>(dyn));
+    const int total = build_schedule(p, s, MT, TN, reinterpret_cast<int *>(dyn));
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = s.tmem_base;
 
     if (warp < kProdWarps) {  // --------------------------------------- producers
-        produce<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, KS);
+        produce<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, KS, tmem, kDnColA);
     } else if (warp < kMmaWarp) {  // ---------------------------------- epilogue
         const int q = warp & 3, half = (warp - kEpiWarp0) >> 2;
         int tcount = 0;
         TcClock ck;
         ck.start();
         for (int tau = blockIdx.x; tau < total && !s.abort; tau += gridDim.x, ++tcount) {
-            const TileInfo ti = tile_info(p, s, tau, MT);
+            const TileInfo ti = tile_info(p, s, tau, MT, TN);
             const int b = tcount & 1;
             const uint32_t ph = (tcount >> 1) & 1;
             const long long t0 = ck.now();
@@ -654,7 +675,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ck.count(6);
             tc::fence_after();
             const int drow = 128 * ti.mi + 32 * q + lane;
-            const uint32_t td = tmem + (uint32_t(32 * q) << 16) + uint32_t(b * 256);
+            const uint32_t td = tmem + (uint32_t(32 * q) << 16) + uint32_t(b * kTileDn);
             for (int c0 = 16 * half; c0 < ti.rows; c0 += 32) {
                 float v[16];
                 tc::tmem_ld16(td + c0, v);
@@ -676,16 +697,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         ck.store(1, 1, warp == kEpiWarp0 && lane == 0);
     } else if (warp == kTmaWarp) {  // -------------------------------------- TMA
-        if (lane == 0) issue_codes<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, KS, rm);
+        if (lane == 0) issue_codes<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, TN, KS, rm);
     } else if (warp == kTmaBWarp) {
-        if (lane == 0) issue_rows<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, KS, &tmap_b, p.h);
+        if (lane == 0) issue_rows<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, TN, KS, &tmap_b, p.h);
     } else if (lane == 0) {  // --------------------------------------------- MMA
         int it = 0, tcount = 0;
         bool ok = true;
         TcClock ck;
         ck.start();
         for (int tau = blockIdx.x; tau < total && ok && !s.abort; tau += gridDim.x, ++tcount) {
-            const TileInfo ti = tile_info(p, s, tau, MT);
+            const TileInfo ti = tile_info(p, s, tau, MT, TN);
             const int npad = (ti.rows + 15) & ~15;
             const uint32_t idesc = tc::idesc_f16(128, npad);
             const int b = tcount & 1;
@@ -697,18 +718,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             ck.add(3, t0);
             tc::fence_after();
-            const uint32_t dd = tmem + uint32_t(b * 256);
+            const uint32_t dd = tmem + uint32_t(b * kTileDn);
             for (int ks = 0; ks < KS; ++ks, ++it) {
                 if (!mma_wait_stage<kDnSA, kDnSB>(s, it, ck)) {
                     ok = false;
                     break;
                 }
-                const uint32_t a = tc::smem_u32(DnRings::a(dyn, it));
+                const uint32_t a = tmem + uint32_t(kDnColA + (it % kDnSA) * 32);
                 const uint32_t bb = tc::smem_u32(DnRings::b(dyn, it));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_f16(dd, tc::desc_sw128(a + 32 * kk), tc::desc_sw128(bb + 32 * kk), idesc,
-                                (ks | kk) ? 1u : 0u);
+                    tc::mma_f16_ta(dd, a + 8 * kk, tc::desc_sw128(bb + 32 * kk), idesc, (ks | kk) ? 1u : 0u);
                 mma_release_stage<kDnSA, kDnSB>(s, it);
             }
             if (ok) tc::mma_commit(&s.tfull[b]);
@@ -795,7 +815,7 @@ bool raw_maps(RawMaps *rm, const TcParams &p, const MatGeom *const *mats, int nm
     return true;
 }
 
-constexpr size_t kGuSmem = size_t(GuRings::kBytes) + 1024;
+constexpr size_t kGuSmem = size_t(GuRings::kBytes) + size_t(kEpiWarps) * kHStage + 1024;
 constexpr size_t kDnSmem = size_t(DnRings::kBytes) + 1024;
 static_assert(kDnSB <= kMaxSB && kGuSB <= kMaxSB && kDnSR <= kMaxSRP && kGuSR <= kMaxSRP,
               "ring larger than its barrier array");
