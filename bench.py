@@ -41,6 +41,33 @@ def _env_int(name, default):
     return int(v) if v not in (None, "") else default
 
 
+# DRAM bytes (read + written) per step of the roofline kernel(s), from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum; see profiles/),
+# valid only while the sources it was captured on are unchanged.
+PROFILED_TRAFFIC = {
+    # fused decode layer kernel, one launch per step
+    "decode_T1_d2048_E512_k10_f768_q2": (("decode_layer.cu", "mma_q.cuh", "layout.h", "common.cuh"),
+                                         "dcd7d8b103ec6b4e", 20.54e6),
+    # expert FFN launches of one step: fp16 gathers, tcgen05 gate/up and down, routed and shared
+    "prefill_T8192_d2048_E512_k10_f768_q2": (("ffn_tc05.cu", "tc05.cuh", "layout.h", "common.cuh", "ffn_mma.cu"),
+                                             "805ae12cb68d914d", 2511e6),
+}
+
+
+def _profiled_traffic(workload: str):
+    import hashlib
+
+    entry = PROFILED_TRAFFIC.get(workload)
+    if entry is None:
+        return None
+    files, digest, nbytes = entry
+    m = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "bit_expert_ffn_fp32_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    return nbytes if m.hexdigest()[:16] == digest else None
+
+
 def _measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -320,13 +347,15 @@ def run_ours(args, wl, rank, world, local_rank):
         "roofline": ({"bound": "tensor",
                       "kernel": "moe_expert_ffn_q2 tcgen05 grouped GEMMs (gate/up + down, routed + shared)",
                       "achieved": ffn_flops / ffn_avg_s / 1e12, "peak": tc_peak, "peak_kind": peak_kind + " bf16 burst",
-                      "unit": "TFLOP/s", "frac": ffn_flops / ffn_avg_s / 1e12 / tc_peak, "traffic": None,
+                      "unit": "TFLOP/s", "frac": ffn_flops / ffn_avg_s / 1e12 / tc_peak,
+                      "traffic": _profiled_traffic(wl.name),
                       "flops_per_launch": ffn_flops, "avg_launch_us": ffn_avg_s * 1e6} if tensor_bound else
                      {"bound": "hbm",
                       "kernel": ("decode_layer_kernel (moe_layer_decode: whole layer, one launch)" if fused else
                                  "moe_expert_ffn_q%d (gate/up + down, routed + shared)" % wl.fmt),
                       "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                      "frac": achieved / hbm_peak, "traffic": None, "bytes_per_launch": kern_bytes,
+                      "frac": achieved / hbm_peak, "traffic": _profiled_traffic(wl.name) if fused else None,
+                      "bytes_per_launch": kern_bytes,
                       "avg_launch_us": ffn_avg_s * 1e6}),
         "e2e": {"value": replicas.job_throughput(T * args.steps, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": T * wl.d * 2,
                 "d2h_bytes_per_step": T * wl.d * 4},
