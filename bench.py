@@ -151,10 +151,11 @@ def run_reference(args, wl, rank):
             times.append(time.perf_counter() - t0)
         if time.perf_counter() - t_start > 120.0 and times:
             break
-    tot = sum(times)
+    tot = sum(times) * wl.layers  # a step of a stacked workload is wl.layers layer calls
     value = T_s * len(times) / tot
     sample = (f"{len(times)} of {args.steps} steps run (120 s budget), {T_s} token(s) of {wl.name} per step, "
-              f"oracle layer incl. dequantisation, single thread")
+              f"oracle layer incl. dequantisation, single thread"
+              + (f"; one layer call timed per step, x{wl.layers} for the {wl.layers} layers" if wl.layers > 1 else ""))
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
@@ -185,9 +186,10 @@ def cpu_baseline(wl, budget_s=12.0):
         t_tot += time.perf_counter() - t0
         n_tok += T_s
         it += 1
-    return {"value": n_tok / t_tot, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+    return {"value": n_tok / (t_tot * wl.layers), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{it} oracle layer calls x {T_s} token(s) of {wl.name} ({t_tot:.1f} s, single thread, "
-                      f"dequantisation included)"}
+                      f"dequantisation included"
+                      + (f"; x{wl.layers} layers per token" if wl.layers > 1 else "") + ")"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -200,16 +202,21 @@ def run_ours(args, wl, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    stack = MoEStack(wl, device=dev, layers=1)
+    # L > 1 (the stacked-layer workload): a step takes the T tokens through all
+    # L layers, each layer with its own seeded input and its own outputs
+    L = wl.layers
+    stack = MoEStack(wl, device=dev)
     T = wl.T
-    b = stack.buffers(T)
+    bufs = [stack.buffers(T) for _ in range(L)]
+    b = bufs[0]
     stream = torch.cuda.current_stream()
     n_steps = args.warmup + args.steps
     # steps get their own tokens, generated up front and resident in HBM (at most
     # 256 MiB of distinct inputs, cycled; the L2 is evicted between steps anyway)
-    n_x = max(1, min(n_steps, (256 << 20) // (T * wl.d * 2)))
-    xs_host = [synth.gen_x(wl.seed, 0, T, wl.d, stream=s) for s in replicas.token_streams(rank, n_x)]
-    xs_dev = torch.stack([x_tensor(x, dev) for x in xs_host])
+    n_x = max(1, min(n_steps, (256 << 20) // (L * T * wl.d * 2)))
+    xs_host = [np.stack([synth.gen_x(wl.seed, l, T, wl.d, stream=s) for l in range(L)])
+               for s in replicas.token_streams(rank, n_x)]
+    xs_dev = torch.stack([torch.stack([x_tensor(xl, dev) for xl in x]) for x in xs_host])
 
     class _Cycle:
         def __getitem__(self, i):
@@ -221,16 +228,20 @@ def run_ours(args, wl, rank, world, local_rank):
            torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
     fused = args.path == "fused" or (args.path == "auto" and T <= 8)
+    if L > 1 and not fused:
+        raise SystemExit("a multi-layer workload runs the one-launch decode path (T <= 8)")
 
-    def layer_step(x, evs=None):
+    def layer_step(xset, evs=None):
         k, E, d, f = wl.k, wl.E, wl.d, wl.f
         if fused:
             if evs:
                 evs[1].record(stream)
-            stack.forward_fused(0, x, b)
+            for l in range(L):
+                stack.forward_fused(l, xset[l], bufs[l])
             if evs:
                 evs[2].record(stream)
             return
+        x = xset[0]
         native.route(x, stack.Wr[0], stack.bias[0], T, d, E, k, b.logits, b.idx, b.w, b.status)
         native.permute(b.idx, T, k, E, b.counts, b.offsets, b.sorted_tok, b.sorted_j, b.inv, b.active, b.perm_ws,
                        0 if b.perm_ws is None else b.perm_ws.numel(), b.status)
@@ -246,14 +257,15 @@ def run_ours(args, wl, rank, world, local_rank):
             evs[2].record(stream)
         native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y)
 
-    launches_per_step = 1 if fused else 2 + (1 if T <= 256 else 3) + 1 + 2 + 2 + 1
+    launches_per_step = L if fused else 2 + (1 if T <= 256 else 3) + 1 + 2 + 2 + 1
 
     # distinct routed experts per step (for the algorithmic bytes), from a warm-up pass
     for s in range(args.warmup):
         flush.fill_(1.0)
         layer_step(xs[s])
     torch.cuda.synchronize()
-    b.status.zero_()
+    for bl in bufs:
+        bl.status.zero_()
 
     if world > 1:
         dist.barrier()
@@ -283,28 +295,37 @@ def run_ours(args, wl, rank, world, local_rank):
             layer_step(xs[args.warmup + i], ev[i])
         torch.cuda.synchronize()
         ffn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
-    status = int(b.status.item())
+    status = 0
+    for bl in bufs:
+        status |= int(bl.status.item())
 
-    # distinct resident experts and resident pairs of each step's routing (not timed)
-    n_act, n_pairs = [], []
-    for i in range(min(args.steps, 256 if T <= 64 else 4)):
+    # distinct resident experts, resident pairs and misses of each step's routing,
+    # summed over the layers (not timed)
+    n_act, n_pairs, n_miss = [], [], []
+    for i in range(min(args.steps, (256 if T <= 64 else 4) if L == 1 else 8)):
         layer_step(xs[args.warmup + i])
-        na = int(b.active[0].item())
-        ids = b.active[1:1 + na].cpu().numpy()
-        res = stack.slot_of_host[0][ids] >= 0
-        n_act.append(int(res.sum()))
-        n_pairs.append(int((b.sop[: T * wl.k] >= 0).sum().item()) if not fused else T * wl.k)
+        a_sum = p_sum = m_sum = 0
+        for l, bl in enumerate(bufs):
+            na = int(bl.active[0].item())
+            ids = bl.active[1:1 + na].cpu().numpy()
+            a_sum += int((stack.slot_of_host[l][ids] >= 0).sum())
+            p_sum += int((bl.sop[: T * wl.k] >= 0).sum().item())
+            m_sum += int(bl.miss_count.item())
+        n_act.append(a_sum)
+        n_pairs.append(p_sum)
+        n_miss.append(m_sum)
     mean_act = float(np.mean(n_act))
     res_pairs_mean = float(np.mean(n_pairs))
+    hit_rate = res_pairs_mean / (L * T * wl.k)
 
     total_ms, ffn_total = replicas.max_over_ranks([total_ms, sum(ffn_ms)], device=dev)
 
     # ---- e2e: pinned host tokens in, layer, result out, every step
     e2e_ms = None
-    x_pin = torch.from_numpy(np.stack(xs_host).view(np.int16)).pin_memory()
-    n_y = min(args.steps, max(2, (256 << 20) // (T * wl.d * 4)))
-    y_pin = torch.empty((n_y, T, wl.d), dtype=torch.float32).pin_memory()
-    x_dev = torch.empty((T, wl.d), dtype=torch.int16, device=dev)
+    x_pin = torch.from_numpy(np.stack(xs_host).view(np.int16)).pin_memory()  # [n_x][L][T][d]
+    n_y = min(args.steps, max(2, (256 << 20) // (L * T * wl.d * 4)))
+    y_pin = torch.empty((n_y, L, T, wl.d), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty((L, T, wl.d), dtype=torch.int16, device=dev)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
@@ -313,7 +334,8 @@ def run_ours(args, wl, rank, world, local_rank):
         e2e_ev[i][0].record(stream)
         x_dev.copy_(x_pin[i % n_x], non_blocking=True)
         layer_step(x_dev)
-        y_pin[i % n_y].copy_(b.y[:T], non_blocking=True)
+        for l in range(L):
+            y_pin[i % n_y, l].copy_(bufs[l].y[:T], non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = sum(e2e_ev[i][0].elapsed_time(e2e_ev[i][1]) for i in range(args.steps))
@@ -325,8 +347,8 @@ def run_ours(args, wl, rank, world, local_rank):
         return 0
     hbm_peak, tc_peak, peak_kind = _measured_peaks()
     eb = native.expert_bytes(wl.fmt, wl.d, wl.f)
-    ffn_bytes = (mean_act + 1) * eb            # routed resident experts + the shared expert, read once
-    layer_bytes = wl.E * wl.d * 4 + ffn_bytes  # + the fp32 router weights
+    ffn_bytes = (mean_act + L) * eb                # routed resident experts + the shared experts, read once
+    layer_bytes = L * wl.E * wl.d * 4 + ffn_bytes  # + the fp32 router weights (all L layers of a step)
     kern_bytes = layer_bytes if fused else ffn_bytes
     ffn_avg_s = ffn_total / args.steps / 1e3
     achieved = kern_bytes / ffn_avg_s / 1e9
@@ -341,9 +363,11 @@ def run_ours(args, wl, rank, world, local_rank):
                   else "q2xf16->f32" if wl.fmt == 2 else "q3xf16->f32"), "data": "synthetic",
         "config": {"workload": wl.name, "tokens_per_step": T, "l2": "512 MiB write between steps (flushed)",
                    "path": "moe_layer_decode (one launch)" if fused else "step-by-step calls",
-                   "parallelism": f"replicas x{world}", "layer_algorithmic_bytes": layer_bytes,
-                   "layer_GBps": layer_bytes / (total_ms / args.steps / 1e3) / 1e9,
-                   "mean_distinct_resident_experts": mean_act},
+                   "parallelism": f"replicas x{world}", "layers_per_step": L,
+                   "step_algorithmic_bytes": layer_bytes,
+                   "step_GBps": layer_bytes / (total_ms / args.steps / 1e3) / 1e9,
+                   "mean_distinct_resident_experts": mean_act, "hit_rate": hit_rate,
+                   "misses_per_step": float(np.mean(n_miss))},
         "roofline": ({"bound": "tensor",
                       "kernel": "moe_expert_ffn_q2 tcgen05 grouped GEMMs (gate/up + down, routed + shared)",
                       "achieved": ffn_flops / ffn_avg_s / 1e12, "peak": tc_peak, "peak_kind": peak_kind + " bf16 burst",
@@ -351,14 +375,14 @@ def run_ours(args, wl, rank, world, local_rank):
                       "traffic": _profiled_traffic(wl.name),
                       "flops_per_launch": ffn_flops, "avg_launch_us": ffn_avg_s * 1e6} if tensor_bound else
                      {"bound": "hbm",
-                      "kernel": ("decode_layer_kernel (moe_layer_decode: whole layer, one launch)" if fused else
+                      "kernel": ("decode_layer_kernel (moe_layer_decode: whole layer, one launch per layer)" if fused else
                                  "moe_expert_ffn_q%d (gate/up + down, routed + shared)" % wl.fmt),
                       "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                       "frac": achieved / hbm_peak, "traffic": _profiled_traffic(wl.name) if fused else None,
                       "bytes_per_launch": kern_bytes,
                       "avg_launch_us": ffn_avg_s * 1e6}),
-        "e2e": {"value": replicas.job_throughput(T * args.steps, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": T * wl.d * 2,
-                "d2h_bytes_per_step": T * wl.d * 4},
+        "e2e": {"value": replicas.job_throughput(T * args.steps, world, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": L * T * wl.d * 2, "d2h_bytes_per_step": L * T * wl.d * 4},
         "clocks": clocks, "gpu_launches": launches_per_step * args.steps, "dev_status": status,
     }
     if world == 1 and not args.no_cpu_baseline:
