@@ -228,6 +228,8 @@ def run_ours(args, wl, rank, world, local_rank):
            torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
     fused = args.path == "fused" or (args.path == "auto" and T <= 8)
+    # many tokens: gate-weighted accumulation inside the expert call, no y_perm/combine
+    atomic = not fused and args.combine == "atomic"
     if L > 1 and not fused:
         raise SystemExit("a multi-layer workload runs the one-launch decode path (T <= 8)")
 
@@ -249,6 +251,14 @@ def run_ours(args, wl, rank, world, local_rank):
                             b.sorted_j, T, k, E, b.sop, b.miss, b.miss_count, b.idx.numel(), b.status)
         if evs:
             evs[1].record(stream)
+        if atomic:  # shared expert writes y, routed experts add gate * y_e into it
+            native.expert_ffn(stack.qpool, stack.shared_slot[0], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
+                              b.sh_sorted_j, b.sh_active, None, b.y, b.h_sh, b.h_sh.numel(), b.status)
+            native.expert_ffn(stack.qpool, stack.slot_of[0], x, T, d, f, E, k, b.offsets, b.sorted_tok,
+                              b.sorted_j, b.active, b.w, b.y, b.h_ws, b.h_ws.numel(), b.status)
+            if evs:
+                evs[2].record(stream)
+            return
         native.expert_ffn(stack.qpool, stack.slot_of[0], x, T, d, f, E, k, b.offsets, b.sorted_tok, b.sorted_j,
                           b.active, None, b.y_perm, b.h_ws, b.h_ws.numel(), b.status)
         native.expert_ffn(stack.qpool, stack.shared_slot[0], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
@@ -257,7 +267,8 @@ def run_ours(args, wl, rank, world, local_rank):
             evs[2].record(stream)
         native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y)
 
-    launches_per_step = L if fused else 2 + (1 if T <= 256 else 3) + 1 + 2 + 2 + 1
+    ffn_launches = 3 if T * wl.k >= 512 and wl.fmt == 2 else 2  # (+ gather on the tensor-core path)
+    launches_per_step = L if fused else 2 + (1 if T <= 256 else 3) + 1 + 2 * ffn_launches + (0 if atomic else 1)
 
     # distinct routed experts per step (for the algorithmic bytes), from a warm-up pass
     for s in range(args.warmup):
@@ -362,7 +373,9 @@ def run_ours(args, wl, rank, world, local_rank):
         "vs_baseline": None, "dtype": ("f16 (dequantised q2) x f16 -> f32" if (not fused and T * wl.k >= 512 and wl.fmt == 2)
                   else "q2xf16->f32" if wl.fmt == 2 else "q3xf16->f32"), "data": "synthetic",
         "config": {"workload": wl.name, "tokens_per_step": T, "l2": "512 MiB write between steps (flushed)",
-                   "path": "moe_layer_decode (one launch)" if fused else "step-by-step calls",
+                   "path": "moe_layer_decode (one launch)" if fused else
+                   "step-by-step calls" + (", gate-weighted accumulation in the routed expert call" if atomic else
+                                           ", y_perm + moe_combine"),
                    "parallelism": f"replicas x{world}", "layers_per_step": L,
                    "step_algorithmic_bytes": layer_bytes,
                    "step_GBps": layer_bytes / (total_ms / args.steps / 1e3) / 1e9,
@@ -399,6 +412,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_T1_d2048_E512_k10_f768_q2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--combine", choices=["atomic", "kernel"], default="kernel",
+                    help="steps path: gate-weighted atomics in the routed expert call (atomic) or y_perm + moe_combine")
     ap.add_argument("--path", choices=["auto", "fused", "steps"], default="auto",
                     help="auto: one-launch layer for T <= 8 tokens, step-by-step calls otherwise")
     args = ap.parse_args()

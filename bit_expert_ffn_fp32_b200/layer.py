@@ -142,8 +142,14 @@ class MoEStack:
         self._bufs[T] = b
         return b
 
-    def forward(self, layer: int, x: torch.Tensor, b: Buffers | None = None, stream=None) -> Buffers:
-        """Enqueue one layer on x (bf16 bits as int16/uint16-sized tensor [T][d])."""
+    def forward(self, layer: int, x: torch.Tensor, b: Buffers | None = None, stream=None,
+                combine: str = "kernel") -> Buffers:
+        """Enqueue one layer on x (bf16 bits as int16/uint16-sized tensor [T][d]).
+
+        combine="kernel": routed experts write y_e rows (y_perm), the shared
+        expert y_sh, and moe_combine forms y. combine="atomic": the shared
+        expert writes y directly and the routed call adds gate * y_e into it
+        (moe_expert_ffn with topk_w), with no y_perm and no combine pass."""
         wl = self.wl
         T = x.shape[0]
         b = b or self.buffers(T)
@@ -153,6 +159,12 @@ class MoEStack:
                        0 if b.perm_ws is None else b.perm_ws.numel(), b.status, stream)
         native.cache_lookup(self.slot_of[layer], self.num_slots, layer, b.idx, b.w, b.offsets, b.sorted_tok,
                             b.sorted_j, T, k, E, b.sop, b.miss, b.miss_count, b.idx.numel(), b.status, stream)
+        if combine == "atomic":
+            native.expert_ffn(self.qpool, self.shared_slot[layer], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
+                              b.sh_sorted_j, b.sh_active, None, b.y, b.h_sh, b.h_sh.numel(), b.status, stream)
+            native.expert_ffn(self.qpool, self.slot_of[layer], x, T, d, f, E, k, b.offsets, b.sorted_tok,
+                              b.sorted_j, b.active, b.w, b.y, b.h_ws, b.h_ws.numel(), b.status, stream)
+            return b
         native.expert_ffn(self.qpool, self.slot_of[layer], x, T, d, f, E, k, b.offsets, b.sorted_tok, b.sorted_j,
                           b.active, None, b.y_perm, b.h_ws, b.h_ws.numel(), b.status, stream)
         native.expert_ffn(self.qpool, self.shared_slot[layer], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,

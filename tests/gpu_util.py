@@ -12,11 +12,11 @@ OUT_TOL = 2e-3      # max|y - y_ref| / max|y_ref| per layer
 GATE_RTOL = 1e-5
 
 
-def run_layer(stack: MoEStack, layer: int, x_bits: np.ndarray):
+def run_layer(stack: MoEStack, layer: int, x_bits: np.ndarray, combine: str = "kernel"):
     x = x_tensor(x_bits, stack.device)
     b = stack.buffers(x.shape[0])
     b.status.zero_()
-    stack.forward(layer, x, b)
+    stack.forward(layer, x, b, combine=combine)
     torch.cuda.synchronize()
     return b
 

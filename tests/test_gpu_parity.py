@@ -15,10 +15,10 @@ from gpu_util import OUT_TOL, check_routing, oracle_layer, rel_err, run_layer
 pytestmark = pytest.mark.gpu
 
 
-def _full_check(stack, layer, x_bits, tokens=None):
+def _full_check(stack, layer, x_bits, tokens=None, combine="kernel"):
     wl = stack.wl
     T = x_bits.shape[0]
-    b = run_layer(stack, layer, x_bits)
+    b = run_layer(stack, layer, x_bits, combine)
     ref = oracle_layer(stack, layer, x_bits, tokens=tokens)
     assert int(b.status.item()) == 0
     check_routing(b, ref, T, wl.k, wl.E)
@@ -236,3 +236,27 @@ def test_tc05_every_pair_written_and_deterministic(decode):
         assert not bool((yp == fill).all(dim=1).any())
         outs.append(yp)
     assert torch.equal(outs[0], outs[1])
+
+
+# ---------------------------------------------------------------- gate-weighted accumulation mode
+@pytest.mark.parametrize("T", [5, 300])
+def test_atomic_combine_tiny(tiny, T):
+    """Shared expert written into y, routed experts added with gate-weighted
+    atomics inside the expert call (mma.sync path at T=5, tcgen05 at T=300)."""
+    x = synth.gen_x(0, 0, T, configs.TINY.d, stream=960 + T)
+    _full_check(tiny, 0, x, combine="atomic")
+
+
+def test_atomic_combine_decode_shapes(decode):
+    T = 1000
+    x = synth.gen_x(0, 0, T, configs.DECODE.d, stream=961)
+    _full_check(decode, 0, x, tokens=list(range(0, T, 97)) + [T - 1], combine="atomic")
+
+
+def test_atomic_combine_with_misses():
+    """Residency by Zipf rank (stack workload shapes): misses are left out of y."""
+    wl = configs.STACK48.with_(layers=1, T=600)
+    stack = MoEStack(wl)
+    x = synth.gen_x(0, 0, wl.T, wl.d, stream=962)
+    b, ref, _ = _full_check(stack, 0, x, tokens=[0, 1, 299, 599], combine="atomic")
+    assert 0 < int(b.miss_count.item()) < wl.T * wl.k
