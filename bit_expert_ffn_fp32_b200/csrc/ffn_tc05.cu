@@ -434,17 +434,23 @@ __device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned c
         ck.add(2, t0);
         t0 = ck.now();
         const unsigned char *raw = R::raw(dyn, pp);
+        HalfQ2 c[NMAT];  // both matrices' bytes first, then both dequantised together
 #pragma unroll
         for (int i = 0; i < NMAT; ++i) {
-            HalfQ2 c;
-            c.cw = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + rgl * 512 + lane * 16 + 8 * bb);
-            c.sc = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + kRawCodes + rgl * 128 + (lane >> 2) * 16 +
-                                                    8 * bb);
-            uint32_t v[16];
-            dequant_half_q2(c, v);
-            tc::tmem_st16x128_x8(ta + uint32_t((it % SA) * 32 * NMAT + 32 * i), v);
+            c[i].cw = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + rgl * 512 + lane * 16 + 8 * bb);
+            c[i].sc = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + kRawCodes + rgl * 128 +
+                                                       (lane >> 2) * 16 + 8 * bb);
         }
+        uint32_t v[NMAT][16];
+#pragma unroll
+        for (int i = 0; i < NMAT; ++i) dequant_half_q2(c[i], v[i]);
+        const long long t2 = ck.now();
+#pragma unroll
+        for (int i = 0; i < NMAT; ++i) tc::tmem_st16x128_x8(ta + uint32_t((it % SA) * 32 * NMAT + 32 * i), v[i]);
+        ck.add(3, t2);
+        const long long t3 = ck.now();
         tc::tmem_st_wait();
+        ck.add(5, t3);
         tc::fence_before();
         tc::mbar_arrive(&s.fullA[it % SA]);
         if (bb) tc::mbar_arrive(&s.emptyR[pp % SRP]);

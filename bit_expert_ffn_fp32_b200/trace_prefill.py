@@ -23,7 +23,8 @@ from .layer import MoEStack, x_tensor
 
 ROLES = ("producer", "epilogue", "mma", "tma")
 SLOTS = {  # role -> slot -> meaning
-    "producer": {1: "packed codes landed", 2: "A slot free (MMA done)", 4: "dequantise + arrive"},
+    "producer": {1: "packed codes landed", 2: "A slot free (MMA done)", 4: "dequantise + TMEM store + arrive",
+                 3: "of which tcgen05.st issue", 5: "of which tcgen05.wait::st"},
     "epilogue": {1: "accumulator full (tfull)", 2: "TMEM loads (gate/up)"},
     "mma": {1: "A stage full", 2: "B stage full", 3: "accumulator free (tempty)"},
     "tma": {1: "code slot free (producers done)", 3: "issuing code loads"},
