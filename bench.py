@@ -268,7 +268,8 @@ def run_ours(args, wl, rank, world, local_rank):
         native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y)
 
     ffn_launches = 3 if T * wl.k >= 512 and wl.fmt == 2 else 2  # (+ gather on the tensor-core path)
-    launches_per_step = L if fused else 2 + (1 if T <= 256 else 3) + 1 + 2 * ffn_launches + (0 if atomic else 1)
+    perm_launches = 1 if native.permute_workspace_bytes(T, wl.k, wl.E) == 0 else 3
+    launches_per_step = L if fused else 2 + perm_launches + 1 + 2 * ffn_launches + (0 if atomic else 1)
 
     # distinct routed experts per step (for the algorithmic bytes), from a warm-up pass
     for s in range(args.warmup):

@@ -10,7 +10,7 @@
 namespace moe {
 namespace {
 
-constexpr int kTile = 256;     // tokens per tile
+constexpr int kTile = 64;      // tokens per tile
 constexpr int kThreads = 1024;
 
 // Block-wide exclusive scan of one value per thread (kThreads threads).
