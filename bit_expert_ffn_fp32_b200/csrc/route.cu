@@ -213,6 +213,79 @@ __global__ void topk_kernel(const float *__restrict__ logits, int T, int E, int 
     }
 }
 
+// Order-preserving 32-bit key of an fp32 logit: larger logit -> larger key; +0
+// and -0 share a key; 0 marks NaN (never above a number).
+__device__ __forceinline__ uint32_t logit_key32(float v) {
+    if (v != v) return 0u;
+    if (v == 0.f) v = 0.f;
+    const uint32_t u = __float_as_uint(v);
+    const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return k == 0u ? 1u : k;
+}
+
+// E <= 512: one warp per token with the token's logits in registers as 64-bit
+// candidates (logit key << 32 | ~id: larger = larger logit, then lower id).
+// Round r takes the warp-wide maximum (it is unique) into lane r; then the k
+// selections are ranked by id and the gates computed exactly as topk_kernel
+// does (maximum first, normaliser summed in ascending id, one reciprocal).
+__global__ void __launch_bounds__(256)
+    topk_reg_kernel(const float *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ idx,
+                    float *__restrict__ gate, int32_t *status) {
+    constexpr int M = 512 / 32;
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float *row = logits + size_t(t) * E;
+    uint64_t c[M];
+    bool nan = false;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        const int e = lane + 32 * m;
+        if (e < E) {
+            const float v = row[e];
+            nan |= v != v;
+            c[m] = (uint64_t(logit_key32(v)) << 32) | uint64_t(~uint32_t(e));
+        } else {
+            c[m] = 0ull;
+        }
+    }
+    if (__any_sync(0xffffffffu, nan) && lane == 0) flag(status, MOE_DEV_NONFINITE);
+    uint64_t mine = 0ull;
+    for (int r = 0; r < k; ++r) {
+        uint64_t mx = 0ull;
+#pragma unroll
+        for (int m = 0; m < M; ++m) mx = c[m] > mx ? c[m] : mx;
+        const uint32_t hk = __reduce_max_sync(0xffffffffu, uint32_t(mx >> 32));
+        const uint32_t lk = __reduce_max_sync(0xffffffffu, uint32_t(mx >> 32) == hk ? uint32_t(mx) : 0u);
+        const uint64_t win = (uint64_t(hk) << 32) | lk;
+        if (lane == r) mine = win;
+        if (mx == win) {
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+                if (c[m] == win) c[m] = 0ull;
+        }
+    }
+    // a round that found only NaN left takes expert 0 with logit -inf, as topk_kernel does
+    const uint32_t key = uint32_t(mine >> 32);
+    const int my_id = key ? int(~uint32_t(mine)) : 0;
+    const float my_v = key ? __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key) : -INFINITY;
+    const bool sel = lane < k;
+    int rank = 0;  // position of this selection in ascending id order
+    for (int q = 0; q < k; ++q) rank += __shfl_sync(0xffffffffu, my_id, q) < my_id;
+    const float mx = __shfl_sync(0xffffffffu, my_v, 0);
+    const float ex = sel ? expf(my_v - mx) : 0.f;
+    float z = 0.0f;
+    for (int a = 0; a < k; ++a) {
+        const unsigned who = __ballot_sync(0xffffffffu, sel && rank == a);
+        z += __shfl_sync(0xffffffffu, ex, __ffs(who) - 1);
+    }
+    const float inv = 1.0f / z;
+    if (sel) {
+        idx[size_t(t) * k + rank] = my_id;
+        gate[size_t(t) * k + rank] = ex * inv;
+    }
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -235,6 +308,9 @@ MOE_API moe_status moe_route(const uint16_t *x, const float *Wr, const float *bi
         router_logits_kernel<<<g1, kWarpsPerCta * 32, 0, s>>>(x, Wr, bias, T, d, E, logits, dev_status);
     }
     const int wpb = 8;
-    topk_kernel<<<(T + wpb - 1) / wpb, wpb * 32, 0, s>>>(logits, T, E, k, topk_idx, topk_w, dev_status);
+    if (E <= 512)
+        topk_reg_kernel<<<(T + wpb - 1) / wpb, wpb * 32, 0, s>>>(logits, T, E, k, topk_idx, topk_w, dev_status);
+    else
+        topk_kernel<<<(T + wpb - 1) / wpb, wpb * 32, 0, s>>>(logits, T, E, k, topk_idx, topk_w, dev_status);
     return launch_status();
 }
