@@ -63,40 +63,78 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
     }
 }
 
-// Many tokens: one warp = 8 tokens x 8 experts (64 logits), each lane keeping
-// the 64 accumulators of its element class, so every loaded chunk feeds 256
-// fused multiply-adds. The operation order per logit is the same as above.
-constexpr int kTileE = 8, kTileT = 8;
+// Many tokens, shared-memory staging: a CTA of 16 warps owns 32 tokens x 32
+// experts; every 128-element chunk of the tile (32 Wr rows fp32, 32 x rows bf16,
+// 24 KiB) is brought into a ring of shared-memory stages by cp.async, and each warp
+// computes 8 tokens x 8 experts from it with lane l holding the 64 partial sums of
+// element class l (elements 128i+4l+j). Rows past T or E are clamped to the last
+// row (valid memory, results not stored), so the inner loop has no bounds tests.
+// The lane partials are combined by a reduce-scatter that adds exactly the pairs
+// the butterfly adds (lane l and lane l^o, o = 16..1), each sum formed once.
+constexpr int kRsTok = 32, kRsExp = 32, kRsThreads = 512, kRsStages = 4;
+constexpr int kRsWBytes = kRsExp * 128 * 4, kRsXBytes = kRsTok * 128 * 2;
+constexpr int kRsStageBytes = kRsWBytes + kRsXBytes;
+constexpr int kRsSmem = kRsStages * kRsStageBytes;
 
-__global__ void __launch_bounds__(256, 2)
-    router_tiled_kernel(const uint16_t *__restrict__ x, const float *__restrict__ Wr, const float *__restrict__ bias,
-                        int T, int d, int E, float *__restrict__ logits, int32_t *status) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int e0 = blockIdx.x * (8 * kTileE) + warp * kTileE;
-    const int t0 = blockIdx.y * kTileT;
-    if (e0 >= E) return;
-    float acc[kTileT][kTileE];
-#pragma unroll
-    for (int v = 0; v < kTileT; ++v)
-#pragma unroll
-        for (int u = 0; u < kTileE; ++u) acc[v][u] = 0.f;
+__device__ __forceinline__ void rs_cp16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void rs_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void rs_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__global__ void __launch_bounds__(kRsThreads, 1)
+    router_smem_kernel(const uint16_t *__restrict__ x, const float *__restrict__ Wr, const float *__restrict__ bias,
+                       int T, int d, int E, float *__restrict__ logits, int32_t *status) {
+    extern __shared__ __align__(128) uint8_t rs_smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = blockIdx.y * kRsTok, e0 = blockIdx.x * kRsExp;
+    const uint32_t sbase = uint32_t(__cvta_generic_to_shared(rs_smem));
+    // copy assignment: Wr pieces tid and tid + 512 (32 per 512-byte row), x piece tid (16 per row)
+    const int wr0 = tid >> 5, wr1 = (tid + kRsThreads) >> 5, wc = tid & 31;
+    const int xr = tid >> 4, xc = tid & 15;
+    const float *wsrc0 = Wr + size_t(min(e0 + wr0, E - 1)) * d + 4 * wc;
+    const float *wsrc1 = Wr + size_t(min(e0 + wr1, E - 1)) * d + 4 * wc;
+    const uint16_t *xsrc = x + size_t(min(t0 + xr, T - 1)) * d + 8 * xc;
+    const uint32_t wdst0 = wr0 * 512 + wc * 16, wdst1 = wr1 * 512 + wc * 16;
+    const uint32_t xdst = kRsWBytes + xr * 256 + xc * 16;
     const int nchunk = d / 128;
+    auto load = [&](int chunk) {
+        const uint32_t st = sbase + (chunk % kRsStages) * kRsStageBytes;
+        rs_cp16(st + wdst0, wsrc0 + 128 * chunk);
+        rs_cp16(st + wdst1, wsrc1 + 128 * chunk);
+        rs_cp16(st + xdst, xsrc + 128 * chunk);
+    };
+#pragma unroll
+    for (int c = 0; c < kRsStages - 1; ++c) {
+        if (c < nchunk) load(c);
+        rs_commit();
+    }
+    const int wt = warp >> 2, we = warp & 3;  // warp's 8-token and 8-expert group
+    float acc[8][8];
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[v][u] = 0.f;
     for (int i = 0; i < nchunk; ++i) {
-        float4 w[kTileE];
-        uint2 xv[kTileT];
+        rs_wait<kRsStages - 2>();
+        __syncthreads();
+        if (i + kRsStages - 1 < nchunk) load(i + kRsStages - 1);
+        rs_commit();
+        const uint8_t *st = rs_smem + (i % kRsStages) * kRsStageBytes;
+        const float4 *ws = reinterpret_cast<const float4 *>(st) + (we * 8) * 32 + lane;
+        const uint2 *xs = reinterpret_cast<const uint2 *>(st + kRsWBytes) + (wt * 8) * 32 + lane;
+        float4 w[8];
 #pragma unroll
-        for (int u = 0; u < kTileE; ++u)
-            w[u] = e0 + u < E ? __ldg(reinterpret_cast<const float4 *>(Wr + size_t(e0 + u) * d + 128 * i + 4 * lane))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < 8; ++u) w[u] = ws[u * 32];
 #pragma unroll
-        for (int v = 0; v < kTileT; ++v)
-            xv[v] = t0 + v < T ? __ldg(reinterpret_cast<const uint2 *>(x + size_t(t0 + v) * d + 128 * i + 4 * lane))
-                               : make_uint2(0u, 0u);
+        for (int v = 0; v < 8; ++v) {
+            const uint2 xv = xs[v * 32];
+            const float x0 = bf16_lo(xv.x), x1 = bf16_hi(xv.x), x2 = bf16_lo(xv.y), x3 = bf16_hi(xv.y);
 #pragma unroll
-        for (int v = 0; v < kTileT; ++v) {
-            const float x0 = bf16_lo(xv[v].x), x1 = bf16_hi(xv[v].x), x2 = bf16_lo(xv[v].y), x3 = bf16_hi(xv[v].y);
-#pragma unroll
-            for (int u = 0; u < kTileE; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 float a = acc[v][u];
                 a = __fmaf_rn(x0, w[u].x, a);
                 a = __fmaf_rn(x1, w[u].y, a);
@@ -106,23 +144,37 @@ __global__ void __launch_bounds__(256, 2)
             }
         }
     }
+    rs_wait<0>();
+    // reduce-scatter over the 64 logits n = 8v + u: at offset o the lane with bit o
+    // set keeps the upper half of its current values, its partner the lower half
+    float r[64];
 #pragma unroll
-    for (int v = 0; v < kTileT; ++v)
+    for (int v = 0; v < 8; ++v)
 #pragma unroll
-        for (int u = 0; u < kTileE; ++u)
+        for (int u = 0; u < 8; ++u) r[8 * v + u] = acc[v][u];
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) acc[v][u] = __fadd_rn(acc[v][u], __shfl_xor_sync(0xffffffffu, acc[v][u], o));
-    if (lane == 0) {
+    for (int lv = 0; lv < 5; ++lv) {
+        const int o = 16 >> lv, m = 64 >> lv, hm = m >> 1;
+        const bool up = lane & o;
 #pragma unroll
-        for (int v = 0; v < kTileT; ++v)
+        for (int j = 0; j < hm; ++j) {
+            const float keep = up ? r[j + hm] : r[j];
+            const float send = up ? r[j] : r[j + hm];
+            r[j] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, o));
+        }
+    }
+    // lane l now holds logits n = 2l, 2l+1: token 8wt + (l >> 2), experts 8we + 2(l & 3) + {0,1}
+    const int t = t0 + wt * 8 + (lane >> 2);
+    const int e = e0 + we * 8 + 2 * (lane & 3);
+    if (t < T) {
 #pragma unroll
-            for (int u = 0; u < kTileE; ++u) {
-                if (t0 + v < T && e0 + u < E) {
-                    const float r = bias ? __fadd_rn(acc[v][u], bias[e0 + u]) : acc[v][u];
-                    if (!isfinite(r)) flag(status, MOE_DEV_NONFINITE);
-                    logits[size_t(t0 + v) * E + e0 + u] = r;
-                }
+        for (int j = 0; j < 2; ++j) {
+            if (e + j < E) {
+                const float v = bias ? __fadd_rn(r[j], bias[e + j]) : r[j];
+                if (!isfinite(v)) flag(status, MOE_DEV_NONFINITE);
+                logits[size_t(t) * E + e + j] = v;
             }
+        }
     }
 }
 
@@ -299,10 +351,16 @@ MOE_API moe_status moe_route(const uint16_t *x, const float *Wr, const float *bi
     if (int64_t(T) * E >= (int64_t(1) << 31) || int64_t(T) * k >= (int64_t(1) << 31)) return MOE_ERR_OVERFLOW;
     if (T == 0) return MOE_OK;
     if (!x || !Wr || !logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(Wr)) & 15) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = as_cuda(stream);
     if (T >= 64) {
-        dim3 g((E + 8 * kTileE - 1) / (8 * kTileE), (T + kTileT - 1) / kTileT);
-        router_tiled_kernel<<<g, 256, 0, s>>>(x, Wr, bias, T, d, E, logits, dev_status);
+        static bool attr = false;
+        if (!attr) {
+            cudaFuncSetAttribute(router_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRsSmem);
+            attr = true;
+        }
+        dim3 g((E + kRsExp - 1) / kRsExp, (T + kRsTok - 1) / kRsTok);
+        router_smem_kernel<<<g, kRsThreads, kRsSmem, s>>>(x, Wr, bias, T, d, E, logits, dev_status);
     } else {
         dim3 g1((E + kWarpsPerCta - 1) / kWarpsPerCta, (T + kTokTile - 1) / kTokTile);
         router_logits_kernel<<<g1, kWarpsPerCta * 32, 0, s>>>(x, Wr, bias, T, d, E, logits, dev_status);

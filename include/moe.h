@@ -156,7 +156,8 @@ moe_status moe_unpack_expert_host(int fmt, int d, int f, const void *record_host
  *           order (logit desc, id asc), listed in ascending id.
  *   topk_w  fp32 [T][k] (output): softmax of the k selected logits (equal to
  *           a full softmax renormalised over the selected experts).
- * A NaN logit sets MOE_DEV_NONFINITE and is never selected.
+ * A NaN logit sets MOE_DEV_NONFINITE and is never selected. x and Wr must be
+ * 16-byte aligned (else MOE_ERR_INVALID_ARG).
  */
 moe_status moe_route(const uint16_t *x, const float *Wr, const float *bias, int T, int d, int E, int k,
                      float *logits, int32_t *topk_idx, float *topk_w, int32_t *dev_status,

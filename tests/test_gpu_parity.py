@@ -182,7 +182,7 @@ def test_all_misses_gives_shared_only(tiny):
 
 
 def test_multi_tile_permutation():
-    # T above one 256-token tile with a ragged last tile, compared with the oracle
+    # T spanning many 64-token tiles with a ragged last tile, compared with the oracle
     import oracle as orc
     wl = configs.TINY
     T, E, k = 1000, 64, 4
@@ -200,6 +200,46 @@ def test_multi_tile_permutation():
     for key, buf in (("counts", b.counts), ("offsets", b.offsets), ("sorted_tok", b.sorted_tok),
                      ("sorted_j", b.sorted_j), ("inv", b.inv)):
         np.testing.assert_array_equal(buf[: ref[key].shape[0]].cpu().numpy(), ref[key], err_msg=key)
+
+
+# ---------------------------------------------------------------- router shapes
+@pytest.mark.parametrize("T,d,E,k,ties", [
+    (5, 256, 100, 7, False),      # few tokens: one warp per expert
+    (64, 128, 200, 10, True),     # E not a multiple of the 32-expert tile, one 128-chunk
+    (100, 384, 33, 4, False),     # ragged tokens and experts
+    (300, 256, 512, 16, True),    # register top-k at its largest E, k = 16
+    (97, 256, 600, 10, False),    # E > 512: the general top-k
+])
+def test_router_shapes(T, d, E, k, ties):
+    """Logits bit for bit in the fixed fp32 order, selections exact, gates within
+    1e-5, for token and expert counts that leave partial tiles; with ties, rows of
+    Wr are duplicated so equal logits must resolve to the lower expert id."""
+    import oracle as orc
+
+    x_h = synth.gen_x(7, 0, T, d, stream=T + E)
+    W_h = synth.gen_router(7, 0, E, d)
+    if ties:
+        W_h[E - 1] = W_h[3]
+        W_h[11] = W_h[2]
+    rng = np.random.default_rng(T * 1000 + E)
+    bias_h = (rng.standard_normal(E) * 0.5).astype(np.float32)
+    if ties:
+        bias_h[E - 1], bias_h[11] = bias_h[3], bias_h[2]
+    l32, _, _ = orc.router(x_h, W_h, bias_h)
+    idx_ref, gate_ref = orc.topk(l32, k)
+    x = torch.from_numpy(x_h.view(np.int16)).cuda()
+    W = torch.from_numpy(W_h).cuda()
+    bias = torch.from_numpy(bias_h).cuda()
+    logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    native.route(x, W, bias, T, d, E, k, logits, idx, w, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    np.testing.assert_array_equal(logits.cpu().numpy().view(np.uint32), l32.view(np.uint32))
+    np.testing.assert_array_equal(idx.cpu().numpy(), idx_ref)
+    np.testing.assert_allclose(w.cpu().numpy(), gate_ref, rtol=1e-5, atol=1e-7)
 
 
 # ---------------------------------------------------------------- tensor-core (prefill) path
