@@ -63,18 +63,22 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
     }
 }
 
-// Many tokens, shared-memory staging: a CTA of 16 warps owns 32 tokens x 32
-// experts; every 128-element chunk of the tile (32 Wr rows fp32, 32 x rows bf16,
-// 24 KiB) is brought into a ring of shared-memory stages by cp.async, and each warp
-// computes 8 tokens x 8 experts from it with lane l holding the 64 partial sums of
-// element class l (elements 128i+4l+j). Rows past T or E are clamped to the last
-// row (valid memory, results not stored), so the inner loop has no bounds tests.
-// The lane partials are combined by a reduce-scatter that adds exactly the pairs
-// the butterfly adds (lane l and lane l^o, o = 16..1), each sum formed once.
-constexpr int kRsTok = 32, kRsExp = 32, kRsThreads = 512, kRsStages = 4;
+// Many tokens, shared-memory staging: a CTA of 8 warps owns 32 tokens x 16
+// experts (two CTAs per SM); every 128-element chunk of the tile (16 Wr rows fp32,
+// 32 x rows bf16, 16 KiB) is brought into a ring of shared-memory stages by
+// cp.async, and each warp computes 8 tokens x 8 experts from it with lane l holding
+// the 64 partial sums of element class l (elements 128i+4l+j), two tokens per
+// packed fp32 fma. Rows past T or E are clamped to the last row (valid memory,
+// results not stored), so the inner loop has no bounds tests. The lane partials
+// are combined by a reduce-scatter that adds exactly the pairs the butterfly adds
+// (lane l and lane l^o, o = 16..1), each sum formed once.
+constexpr int kRsTok = 32, kRsExp = 16, kRsThreads = 256, kRsStages = 4, kRsChunksPerSync = 2;
 constexpr int kRsWBytes = kRsExp * 128 * 4, kRsXBytes = kRsTok * 128 * 2;
 constexpr int kRsStageBytes = kRsWBytes + kRsXBytes;
 constexpr int kRsSmem = kRsStages * kRsStageBytes;
+constexpr int kWP = kRsExp * 32 / kRsThreads, kXP = kRsTok * 16 / kRsThreads;
+static_assert(kWP * kRsThreads == kRsExp * 32 && kXP * kRsThreads == kRsTok * 16, "pieces");
+constexpr int kWE = kRsExp / 8;  // expert groups of warps
 
 __device__ __forceinline__ void rs_cp16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -85,62 +89,89 @@ __device__ __forceinline__ void rs_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__global__ void __launch_bounds__(kRsThreads, 1)
+__global__ void __launch_bounds__(kRsThreads, 2)
     router_smem_kernel(const uint16_t *__restrict__ x, const float *__restrict__ Wr, const float *__restrict__ bias,
                        int T, int d, int E, float *__restrict__ logits, int32_t *status) {
     extern __shared__ __align__(128) uint8_t rs_smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.y * kRsTok, e0 = blockIdx.x * kRsExp;
     const uint32_t sbase = uint32_t(__cvta_generic_to_shared(rs_smem));
-    // copy assignment: Wr pieces tid and tid + 512 (32 per 512-byte row), x piece tid (16 per row)
-    const int wr0 = tid >> 5, wr1 = (tid + kRsThreads) >> 5, wc = tid & 31;
-    const int xr = tid >> 4, xc = tid & 15;
-    const float *wsrc0 = Wr + size_t(min(e0 + wr0, E - 1)) * d + 4 * wc;
-    const float *wsrc1 = Wr + size_t(min(e0 + wr1, E - 1)) * d + 4 * wc;
-    const uint16_t *xsrc = x + size_t(min(t0 + xr, T - 1)) * d + 8 * xc;
-    const uint32_t wdst0 = wr0 * 512 + wc * 16, wdst1 = wr1 * 512 + wc * 16;
-    const uint32_t xdst = kRsWBytes + xr * 256 + xc * 16;
+    // this thread's 16-byte pieces of a chunk: Wr pieces tid + n*256 (32 per row),
+    // x pieces tid + n*256 (16 per row)
+    const float *wsrc[kWP];
+    uint32_t wdst[kWP];
+    const uint16_t *xsrc[kXP];
+    uint32_t xdst[kXP];
+#pragma unroll
+    for (int n = 0; n < kWP; ++n) {
+        const int p = tid + n * kRsThreads, r = p >> 5, c = p & 31;
+        wsrc[n] = Wr + size_t(min(e0 + r, E - 1)) * d + 4 * c;
+        wdst[n] = r * 512 + c * 16;
+    }
+#pragma unroll
+    for (int n = 0; n < kXP; ++n) {
+        const int p = tid + n * kRsThreads, r = p >> 4, c = p & 15;
+        xsrc[n] = x + size_t(min(t0 + r, T - 1)) * d + 8 * c;
+        xdst[n] = kRsWBytes + r * 256 + c * 16;
+    }
     const int nchunk = d / 128;
     auto load = [&](int chunk) {
         const uint32_t st = sbase + (chunk % kRsStages) * kRsStageBytes;
-        rs_cp16(st + wdst0, wsrc0 + 128 * chunk);
-        rs_cp16(st + wdst1, wsrc1 + 128 * chunk);
-        rs_cp16(st + xdst, xsrc + 128 * chunk);
-    };
 #pragma unroll
-    for (int c = 0; c < kRsStages - 1; ++c) {
+        for (int n = 0; n < kWP; ++n) rs_cp16(st + wdst[n], wsrc[n] + 128 * chunk);
+#pragma unroll
+        for (int n = 0; n < kXP; ++n) rs_cp16(st + xdst[n], xsrc[n] + 128 * chunk);
+    };
+    // chunks in flight ahead of the one computed; one barrier per kRsChunksPerSync chunks
+    constexpr int kPre = kRsStages - kRsChunksPerSync;
+#pragma unroll
+    for (int c = 0; c < kPre; ++c) {
         if (c < nchunk) load(c);
         rs_commit();
     }
-    const int wt = warp >> 2, we = warp & 3;  // warp's 8-token and 8-expert group
-    float acc[8][8];
+    const int wt = warp / kWE, we = warp % kWE;  // warp's 8-token and 8-expert group
+    // acc[q][u]: logits of tokens 2q and 2q+1 with expert u, advanced together by
+    // one packed fma per element (each half a single-rounding fp32 fma)
+    float2 acc[4][8];
 #pragma unroll
-    for (int v = 0; v < 8; ++v)
+    for (int q = 0; q < 4; ++q)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) acc[v][u] = 0.f;
+        for (int u = 0; u < 8; ++u) acc[q][u] = make_float2(0.f, 0.f);
     for (int i = 0; i < nchunk; ++i) {
-        rs_wait<kRsStages - 2>();
-        __syncthreads();
-        if (i + kRsStages - 1 < nchunk) load(i + kRsStages - 1);
-        rs_commit();
+        if (i % kRsChunksPerSync == 0) {
+            rs_wait<kPre - kRsChunksPerSync>();
+            __syncthreads();
+#pragma unroll
+            for (int c = 0; c < kRsChunksPerSync; ++c) {
+                if (i + kPre + c < nchunk) load(i + kPre + c);
+                rs_commit();
+            }
+        }
         const uint8_t *st = rs_smem + (i % kRsStages) * kRsStageBytes;
         const float4 *ws = reinterpret_cast<const float4 *>(st) + (we * 8) * 32 + lane;
         const uint2 *xs = reinterpret_cast<const uint2 *>(st + kRsWBytes) + (wt * 8) * 32 + lane;
-        float4 w[8];
+        float2 X[4][4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) w[u] = ws[u * 32];
+        for (int q = 0; q < 4; ++q) {
+            const uint2 xa = xs[(2 * q) * 32], xb = xs[(2 * q + 1) * 32];
+            X[q][0] = make_float2(bf16_lo(xa.x), bf16_lo(xb.x));
+            X[q][1] = make_float2(bf16_hi(xa.x), bf16_hi(xb.x));
+            X[q][2] = make_float2(bf16_lo(xa.y), bf16_lo(xb.y));
+            X[q][3] = make_float2(bf16_hi(xa.y), bf16_hi(xb.y));
+        }
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const uint2 xv = xs[v * 32];
-            const float x0 = bf16_lo(xv.x), x1 = bf16_hi(xv.x), x2 = bf16_lo(xv.y), x3 = bf16_hi(xv.y);
+        for (int u = 0; u < 8; ++u) {
+            const float4 wv = ws[u * 32];
+            const float2 w0 = make_float2(wv.x, wv.x), w1 = make_float2(wv.y, wv.y);
+            const float2 w2 = make_float2(wv.z, wv.z), w3 = make_float2(wv.w, wv.w);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                float a = acc[v][u];
-                a = __fmaf_rn(x0, w[u].x, a);
-                a = __fmaf_rn(x1, w[u].y, a);
-                a = __fmaf_rn(x2, w[u].z, a);
-                a = __fmaf_rn(x3, w[u].w, a);
-                acc[v][u] = a;
+            for (int q = 0; q < 4; ++q) {
+                float2 c = acc[q][u];
+                c = __ffma2_rn(X[q][0], w0, c);
+                c = __ffma2_rn(X[q][1], w1, c);
+                c = __ffma2_rn(X[q][2], w2, c);
+                c = __ffma2_rn(X[q][3], w3, c);
+                acc[q][u] = c;
             }
         }
     }
@@ -149,9 +180,12 @@ __global__ void __launch_bounds__(kRsThreads, 1)
     // set keeps the upper half of its current values, its partner the lower half
     float r[64];
 #pragma unroll
-    for (int v = 0; v < 8; ++v)
+    for (int q = 0; q < 4; ++q)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) r[8 * v + u] = acc[v][u];
+        for (int u = 0; u < 8; ++u) {
+            r[8 * (2 * q) + u] = acc[q][u].x;
+            r[8 * (2 * q + 1) + u] = acc[q][u].y;
+        }
 #pragma unroll
     for (int lv = 0; lv < 5; ++lv) {
         const int o = 16 >> lv, m = 64 >> lv, hm = m >> 1;
