@@ -50,7 +50,7 @@ PROFILED_TRAFFIC = {
                                          "dcd7d8b103ec6b4e", 20.54e6),
     # expert FFN launches of one step: fp16 gathers, tcgen05 gate/up and down, routed and shared
     "prefill_T8192_d2048_E512_k10_f768_q2": (("ffn_tc05.cu", "tc05.cuh", "layout.h", "common.cuh", "ffn_mma.cu"),
-                                             "805ae12cb68d914d", 2511e6),
+                                             "c9ce5905da33cce4", 2505e6),
 }
 
 

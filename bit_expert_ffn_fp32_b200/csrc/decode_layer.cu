@@ -42,7 +42,6 @@ __device__ unsigned long long moe_decode_trace[4096 * 32];
             unsigned long long t_;                                                                    \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                    \
             moe_decode_trace[blockIdx.x * 32 + (i)] = t_;                                             \
-            moe_decode_trace[blockIdx.x * 32 + 16 + (i)] = clock64();                                 \
         }                                                                                             \
     } while (0)
 #define TRACEW(i)                                                                                     \
@@ -51,7 +50,6 @@ __device__ unsigned long long moe_decode_trace[4096 * 32];
             unsigned long long t_;                                                                    \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                    \
             moe_decode_trace[blockIdx.x * 32 + (i)] = t_;                                             \
-            moe_decode_trace[blockIdx.x * 32 + 16 + (i)] = clock64();                                 \
         }                                                                                             \
     } while (0)
 #else
@@ -79,6 +77,17 @@ constexpr int kSharedIdx = kMaxPairs;         // done[] slot of the shared exper
 constexpr int kMaxDimDec = 2048;
 constexpr int kCandMax = 64;  // candidates ranked in shared memory; more take the round-based path
 constexpr unsigned long long kWaitNs = 100ull * 1000 * 1000;
+constexpr int kMaxSlots = 8;  // weight-ring slots at most
+constexpr int kMaxFDec = 1024;  // expert width f (h staging and B fragments)
+constexpr int kCBatch = 4;      // gate/up units computed in one pass (one token)
+static_assert(kCBatch * kWarps * 2 * 16 <= kWarps * 2 * 4 * 32, "batched partials fit in red[]");
+static_assert(kMaxSlots <= kWarps, "one warp announces each initial ring unit");
+
+// Dynamic shared memory: T*d bf16 activations, T rows of h (fp32), then the
+// weight ring from this 128-byte aligned offset.
+__host__ __device__ inline size_t ring_off(int T, int d, int f) {
+    return ((((size_t(T) * d * 2 + 15) & ~size_t(15)) + size_t(T) * f * 4) + 127) & ~size_t(127);
+}
 
 struct DecodeParams {
     const uint8_t *pool;
@@ -104,6 +113,10 @@ struct DecodeParams {
     unsigned *done;  // [kMaxPairs + 1] gate/up tasks finished per resident expert
     float *h;        // [(T*k + T)][f]: sorted pair rows, then shared-expert rows
     MatGeom gate, up, down;
+    // shared-memory weight ring of phases C and D: nslots slots of rslot bytes;
+    // per row group, the codes and scales bytes of gate/up (gu_*) and down (dn_*)
+    int nslots;
+    uint32_t rslot, gu_cb, gu_sb, dn_cb, dn_sb;
 };
 
 struct Smem {
@@ -117,11 +130,15 @@ struct Smem {
     int inv[kMaxPairs];
     int act_e[kMaxPairs], act_beg[kMaxPairs], act_cnt[kMaxPairs], act_slot[kMaxPairs], act_mbase[kMaxPairs];
     int res[kMaxPairs];                     // active index of each resident expert
-    float hsb[1024 / 64][kMaxTokDec];       // block sums of the staged h rows
+    float hsb[kMaxFDec / 64][kMaxTokDec];   // block sums of the staged h rows
     uint64_t cand[kMaxTokDec][kCandMax];    // top-k candidates per token
     float sel_v[kMaxTokDec][kMaxK];
     int sel_id[kMaxTokDec][kMaxK];
     unsigned first_mask[kMaxPairs / 32];    // pair s starts a new expert
+    uint64_t full[kMaxSlots];               // weight ring: slot filled (bulk-copy bytes landed)
+    // B fragments of the staged h rows, built once per down unit and shared by
+    // every warp: quad qd, fragment registers 4*r4..4*r4+3, lane: [qd][r4][lane]
+    uint4 bfrag[kMaxFDec / 256][8][32];
     int nact, nres, nmiss;
     int ok, last;
 };
@@ -153,6 +170,36 @@ __device__ bool wait_geq(const unsigned *p, unsigned target, int32_t *status) {
         }
         __nanosleep(32);
     }
+    return true;
+}
+
+// Weight ring: bulk copies global -> this CTA's shared memory that complete
+// on an mbarrier (transaction bytes), and a bounded wait for a slot's phase.
+__device__ __forceinline__ uint32_t saddr(const void *p) { return uint32_t(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ void ring_expect(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void ring_copy(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     saddr(dst)),
+                 "l"(src), "r"(bytes), "r"(saddr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ bool ring_test(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred q;\nmbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\nselp.u32 %0, 1, 0, q;\n}"
+        : "=r"(done)
+        : "r"(saddr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// false after kWaitNs (the caller flags MOE_DEV_TIMEOUT)
+__device__ bool ring_wait(uint64_t *bar, uint32_t parity) {
+    if (ring_test(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (!ring_test(bar, parity))
+        if (globaltimer() - t0 > kWaitNs) return false;
     return true;
 }
 
@@ -260,6 +307,33 @@ __device__ void gateup_task(const DecodeParams &p, Smem &s, const uint16_t *sx, 
     }
 }
 
+// Packed codes and scales of one 16-row x 256-column tile (columns 256qd..)
+// from a row group's bytes in shared memory, laid out as in the record: codes
+// at cb, scales at sb (the offsets of q2_chunk_off / q3_word_off / scale_off
+// relative to the row group's start).
+template <int FMT>
+__device__ __forceinline__ void quad_load_smem(const uint8_t *cb, const uint8_t *sb, int qd, int lane,
+                                               QuadRegs<FMT> &q) {
+    const int g = lane >> 2;
+    if constexpr (FMT == 2) {
+        q.c0 = *reinterpret_cast<const uint4 *>(cb + ((2 * qd) * 32 + lane) * 16);
+        q.c1 = *reinterpret_cast<const uint4 *>(cb + ((2 * qd + 1) * 32 + lane) * 16);
+        q.s0 = *reinterpret_cast<const uint4 *>(sb + ((2 * qd) * 8 + g) * 16);
+        q.s1 = *reinterpret_cast<const uint4 *>(sb + ((2 * qd + 1) * 8 + g) * 16);
+    } else {
+#pragma unroll
+        for (int w = 0; w < 3; ++w) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(cb + qd * 1536 + w * 512 + lane * 16);
+            q.W[4 * w + 0] = v.x;
+            q.W[4 * w + 1] = v.y;
+            q.W[4 * w + 2] = v.z;
+            q.W[4 * w + 3] = v.w;
+        }
+        q.s0 = *reinterpret_cast<const uint2 *>(sb + ((2 * qd) * 8 + g) * 8);
+        q.s1 = *reinterpret_cast<const uint2 *>(sb + ((2 * qd + 1) * 8 + g) * 8);
+    }
+}
+
 // Block sums of the staged activations, one warp per (64-block, token); whole CTA.
 __device__ __forceinline__ void stage_xsum(Smem &s, const uint16_t *sx, int NB, int T, int d) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -278,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
     extern __shared__ __align__(16) unsigned char dyn[];
     __shared__ Smem s;
     uint16_t *sx = reinterpret_cast<uint16_t *>(dyn);                                        // [T][d] bf16
-    float *sh = reinterpret_cast<float *>(dyn + ((size_t(p.T) * p.d * 2 + 15) & ~size_t(15)));  // [8][f] h
+    float *sh = reinterpret_cast<float *>(dyn + ((size_t(p.T) * p.d * 2 + 15) & ~size_t(15)));  // [T][f] h
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x, cta = blockIdx.x;
     const int T = p.T, k = p.k, E = p.E, d = p.d, f = p.f;
@@ -288,11 +362,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
     const uint8_t *shrec = p.pool + int64_t(p.shared_slot) * p.slot_bytes;
     const uint32_t gu_codes = FMT == 2 ? uint32_t(d / 128) * 512u : uint32_t(d / 256) * 1536u;
     const uint32_t gu_scales = uint32_t(d / 128) * (FMT == 2 ? 128u : 64u);
-    const uint32_t dn_codes = FMT == 2 ? uint32_t(f / 128) * 512u : uint32_t(f / 256) * 1536u;
-    const uint32_t dn_scales = uint32_t(f / 128) * (FMT == 2 ? 128u : 64u);
     bool too_big = false;
+    int ring_issued = 0, ring_used = 0;  // thread 0: weight-ring units copied / consumed
 
     TRACE(0);
+    if (tid == 0) {
+        for (int i = 0; i < kMaxSlots; ++i)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&s.full[i])) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     // ------------------------------------------------------------ phase A
     if (tid == 0) {  // start the HBM reads of this CTA's phase-A task right away
         for (int task = cta; task < NG + nrt; task += G) {
@@ -509,128 +587,177 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
     }
     __syncthreads();
     TRACE(6);
-    if (T == 1 && tid < npairs) {  // one token: its list is already in id order
-        s.pair_e[tid] = s.idx[0][tid];
-        s.s_tok[tid] = 0;
-        s.s_j[tid] = tid;
-        s.inv[tid] = tid;
-    } else if (tid < npairs) {  // stable sort of the pairs by (expert, pair index)
-        const int pp = tid;
-        const int e = s.idx[pp / k][pp % k];
-        int rank = 0;
-        for (int q = 0; q < npairs; ++q) {
-            const int eq = s.idx[q / k][q % k];
-            rank += (eq < e) || (eq == e && q < pp);
-        }
-        s.pair_e[rank] = e;
-        s.s_tok[rank] = pp / k;
-        s.s_j[rank] = pp % k;
-        s.inv[pp] = rank;
-    }
-    __syncthreads();
-    {  // experts with tokens, their segments, slots and miss bases (ballot scans)
-        const bool in = tid < npairs;
-        const bool first = in && (tid == 0 || s.pair_e[tid] != s.pair_e[tid - 1]);
-        const unsigned fm = __ballot_sync(0xffffffffu, first);
-        if (lane == 0 && warp < kMaxPairs / 32) s.first_mask[warp] = fm;
-        __syncthreads();
-        if (first) {
-            int a = __popc(fm & ((1u << lane) - 1));
-            for (int w = 0; w < warp; ++w) a += __popc(s.first_mask[w]);
-            const int e = s.pair_e[tid];
-            const int sl = s.slot[e];
-            const bool bad = sl < -1 || sl >= p.num_slots;
-            if (bad && cta == 0) flag(p.status, MOE_DEV_BAD_SLOT);
-            s.act_e[a] = e;
-            s.act_beg[a] = tid;
-            s.act_slot[a] = bad ? -1 : sl;
-        }
-        if (tid == 0) {
-            int na = 0;
-            for (int w = 0; w < (npairs + 31) / 32; ++w) na += __popc(s.first_mask[w]);
-            s.nact = na;
-        }
-        __syncthreads();
-        const int na = s.nact;
-        if (tid < na) s.act_cnt[tid] = (tid + 1 < na ? s.act_beg[tid + 1] : npairs) - s.act_beg[tid];
-        __syncthreads();
-        if (warp == 0) {  // resident list and miss bases over <= 128 actives, 32 at a time
-            int nr = 0, nm = 0;
-            for (int a0 = 0; a0 < na; a0 += 32) {
-                const int a = a0 + lane;
-                const bool act = a < na;
-                const bool res = act && s.act_slot[a] >= 0;
-                const int cm = act && !res ? s.act_cnt[a] : 0;
-                const unsigned rm = __ballot_sync(0xffffffffu, res);
-                int mpre = cm;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, mpre, o);
-                    if (lane >= o) mpre += v;
-                }
-                if (act) s.act_mbase[a] = nm + mpre - cm;
-                if (res) s.res[nr + __popc(rm & ((1u << lane) - 1))] = a;
-                nr += __popc(rm);
-                nm += __shfl_sync(0xffffffffu, mpre, 31);
+    if (T == 1) {
+        if (warp == 0) {  // one token: its k experts (id order) are the active experts, one pair each
+            const bool in = lane < k;
+            int sl = -1;
+            if (in) {
+                const int e = s.idx[0][lane];
+                s.pair_e[lane] = e;
+                s.s_tok[lane] = 0;
+                s.s_j[lane] = lane;
+                s.inv[lane] = lane;
+                sl = s.slot[e];
+                const bool bad = sl < -1 || sl >= p.num_slots;
+                if (bad && cta == 0) flag(p.status, MOE_DEV_BAD_SLOT);
+                if (bad) sl = -1;
+                s.act_e[lane] = e;
+                s.act_beg[lane] = lane;
+                s.act_cnt[lane] = 1;
+                s.act_slot[lane] = sl;
             }
+            const unsigned rm = __ballot_sync(0xffffffffu, in && sl >= 0);
+            const unsigned mm = __ballot_sync(0xffffffffu, in && sl < 0);
+            const unsigned lt = (1u << lane) - 1u;
+            if (in) s.act_mbase[lane] = __popc(mm & lt);
+            if (in && sl >= 0) s.res[__popc(rm & lt)] = lane;
             if (lane == 0) {
-                s.nres = nr;
-                s.nmiss = nm;
+                s.nact = k;
+                s.nres = __popc(rm);
+                s.nmiss = __popc(mm);
+            }
+        }
+    } else {
+        if (tid < npairs) {  // stable sort of the pairs by (expert, pair index)
+            const int pp = tid;
+            const int e = s.idx[pp / k][pp % k];
+            int rank = 0;
+            for (int q = 0; q < npairs; ++q) {
+                const int eq = s.idx[q / k][q % k];
+                rank += (eq < e) || (eq == e && q < pp);
+            }
+            s.pair_e[rank] = e;
+            s.s_tok[rank] = pp / k;
+            s.s_j[rank] = pp % k;
+            s.inv[pp] = rank;
+        }
+        __syncthreads();
+        {  // experts with tokens, their segments, slots and miss bases (ballot scans)
+            const bool in = tid < npairs;
+            const bool first = in && (tid == 0 || s.pair_e[tid] != s.pair_e[tid - 1]);
+            const unsigned fm = __ballot_sync(0xffffffffu, first);
+            if (lane == 0 && warp < kMaxPairs / 32) s.first_mask[warp] = fm;
+            __syncthreads();
+            if (first) {
+                int a = __popc(fm & ((1u << lane) - 1));
+                for (int w = 0; w < warp; ++w) a += __popc(s.first_mask[w]);
+                const int e = s.pair_e[tid];
+                const int sl = s.slot[e];
+                const bool bad = sl < -1 || sl >= p.num_slots;
+                if (bad && cta == 0) flag(p.status, MOE_DEV_BAD_SLOT);
+                s.act_e[a] = e;
+                s.act_beg[a] = tid;
+                s.act_slot[a] = bad ? -1 : sl;
+            }
+            if (tid == 0) {
+                int na = 0;
+                for (int w = 0; w < (npairs + 31) / 32; ++w) na += __popc(s.first_mask[w]);
+                s.nact = na;
+            }
+            __syncthreads();
+            const int na = s.nact;
+            if (tid < na) s.act_cnt[tid] = (tid + 1 < na ? s.act_beg[tid + 1] : npairs) - s.act_beg[tid];
+            __syncthreads();
+            if (warp == 0) {  // resident list and miss bases over <= 128 actives, 32 at a time
+                int nr = 0, nm = 0;
+                for (int a0 = 0; a0 < na; a0 += 32) {
+                    const int a = a0 + lane;
+                    const bool act = a < na;
+                    const bool res = act && s.act_slot[a] >= 0;
+                    const int cm = act && !res ? s.act_cnt[a] : 0;
+                    const unsigned rm = __ballot_sync(0xffffffffu, res);
+                    int mpre = cm;
+    #pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int v = __shfl_up_sync(0xffffffffu, mpre, o);
+                        if (lane >= o) mpre += v;
+                    }
+                    if (act) s.act_mbase[a] = nm + mpre - cm;
+                    if (res) s.res[nr + __popc(rm & ((1u << lane) - 1))] = a;
+                    nr += __popc(rm);
+                    nm += __shfl_sync(0xffffffffu, mpre, 31);
+                }
+                if (lane == 0) {
+                    s.nres = nr;
+                    s.nmiss = nm;
+                }
             }
         }
     }
     __syncthreads();
     TRACE(5);
-    {  // L2 prefetch of every selected expert, spread over the grid: the
-        // concatenation of all resident experts' gate/up parts, then their down
-        // parts and the shared expert's, is cut into G equal slices and the
-        // threads of CTA c ask the L2 for the lines of slice c
+    {
+        // ------------------------------------------------------------ weight ring
+        // This CTA's units: its gate/up tasks (task = G-1-cta + u*G < nres*NG,
+        // busy phase-A CTAs last), then its down tasks (a contiguous range of
+        // tasks < (nres+1)*nblk; a down task is an expert x 8 row groups of d,
+        // the shared expert last). Thread 0 bulk-copies a unit's packed bytes
+        // (contiguous per row group in the record) into ring slot u % NS as soon
+        // as the routing tables exist, the first NS units at once, and refills a
+        // slot with unit u + NS once unit u has been computed.
+        const int NQ = d / 256, NQf = f / 256, nblk = d / 128;
         const int nres = s.nres;
-        const uint32_t GU = uint32_t(p.down.codes_off);  // gate + up of one record
-        const uint32_t DN = uint32_t(p.down.bytes);      // down of one record
-        const uint32_t gu_all = uint32_t(nres) * GU;     // < 2^32: at most 128 records of < 8 MB
-        const uint32_t total = gu_all + uint32_t(nres + 1) * DN;
-        const uint32_t lo = uint32_t((uint64_t(total) * uint32_t(cta) / uint32_t(G))) & ~127u;
-        const uint32_t hi = cta == G - 1 ? total : uint32_t((uint64_t(total) * uint32_t(cta + 1) / uint32_t(G))) & ~127u;
-        // one 128-byte line per thread and step (GU and DN are multiples of 256)
-        int r = -1;          // region of the current line and its start
-        uint32_t r0 = 0, r1 = 0;
-        const uint8_t *rsrc = nullptr;
-        for (uint32_t o = lo + uint32_t(tid) * 128u; o < hi; o += uint32_t(kThreads) * 128u) {
-            while (o >= r1) {  // advance to the region holding o (regions in order, each >= 1 step)
-                ++r;
-                r0 = r1;
-                if (r < nres) {
-                    r1 = r0 + GU;
-                    rsrc = p.pool + int64_t(s.act_slot[s.res[r]]) * p.slot_bytes;
-                } else {
-                    const int q = r - nres;
-                    r1 = r0 + DN;
-                    const int slot = q < nres ? s.act_slot[s.res[q]] : p.shared_slot;
-                    rsrc = p.pool + int64_t(slot) * p.slot_bytes + p.down.codes_off;
-                }
+        const int ctasks = nres * NG, dtasks = (nres + 1) * nblk;
+        const int cfirst = G - 1 - cta;
+        const int nC = ctasks > cfirst ? (ctasks - cfirst + G - 1) / G : 0;
+        // down tasks: a contiguous range per CTA (consecutive tasks mostly share an
+        // expert, whose staged h and B fragments are then reused)
+        const int dlo = int(int64_t(dtasks) * cta / G), nD = int(int64_t(dtasks) * (cta + 1) / G) - dlo;
+        const int nU = nC + nD, NS = p.nslots;
+        uint8_t *ring = dyn + ring_off(T, d, f);
+        // copy c (0..3 gate/up: gate codes, gate scales, up codes, up scales;
+        // 0..1 down: codes, scales) of unit u; one thread per copy
+        auto issue_copy = [&](int u, int c) {
+            uint8_t *dst = ring + size_t(u % NS) * p.rslot;
+            uint64_t *bar = &s.full[u % NS];
+            if (u < nC) {
+                const int task = cfirst + u * G, ar = task / NG, rg = task % NG;
+                const uint8_t *rec = p.pool + int64_t(s.act_slot[s.res[ar]]) * p.slot_bytes;
+                const MatGeom &m = c < 2 ? p.gate : p.up;
+                const uint32_t off = (c >> 1) * (p.gu_cb + p.gu_sb) + (c & 1) * p.gu_cb;
+                if (c & 1)
+                    ring_copy(dst + off, rec + m.scales_off + uint64_t(rg) * p.gu_sb, p.gu_sb, bar);
+                else
+                    ring_copy(dst + off, rec + m.codes_off + uint64_t(rg) * p.gu_cb, p.gu_cb, bar);
+            } else if (c < 2) {
+                const int task = dlo + (u - nC), ar = task / nblk, blk = task % nblk;
+                const int slot = ar == nres ? p.shared_slot : s.act_slot[s.res[ar]];
+                const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
+                if (c)
+                    ring_copy(dst + 8 * p.dn_cb, rec + p.down.scales_off + uint64_t(8 * blk) * p.dn_sb,
+                              8u * p.dn_sb, bar);
+                else
+                    ring_copy(dst, rec + p.down.codes_off + uint64_t(8 * blk) * p.dn_cb, 8u * p.dn_cb, bar);
             }
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(rsrc + (o - r0)));
-        }
-    }
-    TRACE(3);
-    // ------------------------------------------------------------ phase C
-    {  // busy phase-A CTAs last; warp w handles K quads w, w+8, ... of every task,
-        // and loads the next task's tiles before computing the current one
-        const int ntasks = s.nres * NG;
-        const int NQ = d / 256;
-        const int g = lane >> 2, t = lane & 3;
-        int task = G - 1 - cta;
-        QuadRegs<FMT> ng, nu;  // tiles of the next task (quad = warp)
-        auto load_task = [&](int tk, QuadRegs<FMT> &qg, QuadRegs<FMT> &qu) {
-            const int ar = tk / NG, rg = tk % NG;
-            const uint8_t *rec = p.pool + int64_t(s.act_slot[s.res[ar]]) * p.slot_bytes;
-            quad_load<FMT>(rec, p.gate, rg, warp, lane, qg);
-            quad_load<FMT>(rec, p.up, rg, warp, lane, qu);
         };
+        auto unit_bytes = [&](int u) { return u < nC ? 2u * (p.gu_cb + p.gu_sb) : 8u * (p.dn_cb + p.dn_sb); };
+        auto issue = [&](int u) {  // one thread, all copies of unit u
+            ring_expect(&s.full[u % NS], unit_bytes(u));
+            for (int c = 0; c < 4; ++c) issue_copy(u, c);
+        };
+        {  // the first min(nU, NS) units at once: warp u announces unit u, its lanes 0..3 copy
+            const int n0 = min(nU, NS);
+            if (warp < n0) {
+                if (lane == 0) ring_expect(&s.full[warp], unit_bytes(warp));
+                __syncwarp();
+                if (lane < 4) issue_copy(warp, lane);
+            }
+            ring_issued = n0;  // meaningful in thread 0
+        }
+        TRACE(3);
+        // every thread waits for unit u's bytes itself; false (all threads) on timeout
+        auto await_unit = [&](int u) -> bool {
+            const bool got = ring_wait(&s.full[u % NS], uint32_t(u / NS) & 1u);
+            if (!got && tid == 0) flag(p.status, MOE_DEV_TIMEOUT);
+            const bool all = __syncthreads_and(got) != 0;
+            if (all && tid == 0) ++ring_used;
+            return all;
+        };
+
+        // ------------------------------------------------------------ phase C
+        const int g = lane >> 2, t = lane & 3;
         const bool one_quad = NQ == kWarps;  // every warp owns exactly one quad
-        if (one_quad && task < ntasks) load_task(task, ng, nu);
-        uint32_t B1[4][8];     // one token: fragments of quad `warp`, built once
+        uint32_t B1[4][8];                   // one token: fragments of quad `warp`, built once
         float xs1[4][2];
         if (NT == 1 && one_quad) {
             build_b_bf16<FMT>(g == 0 ? sx : nullptr, warp, t, B1);
@@ -640,45 +767,105 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
                 xs1[bq][1] = 0.f;
             }
         }
-        int nth = 0;
-        for (; task < ntasks; task += G, ++nth) {
-            const int ar = task / NG, rg = task % NG;
+        // One token and all of this CTA's gate/up units in the ring at once: wait
+        // for all of them, compute every unit's quad `warp` back to back (their
+        // MMA chains interleave), then one reduction over warps for all units
+        // (same summation order as the per-unit path below).
+        const bool batch = NT == 1 && one_quad && nC <= min(NS, kCBatch);
+        if (batch) {
+            // every thread waits for each unit itself and computes it at once:
+            // no barrier until all units are done
+            bool got = true;
+            float ag[kCBatch][4], au[kCBatch][4];
+#pragma unroll
+            for (int i = 0; i < kCBatch; ++i) {
+                if (i < nC) {
+                    got = got && ring_wait(&s.full[i], 0u);
+                    if (i == 0) TRACE(16);
+                    const uint8_t *slot = ring + size_t(i) * p.rslot;
+                    QuadRegs<FMT> qg, qu;
+                    quad_load_smem<FMT>(slot, slot + p.gu_cb, warp, lane, qg);
+                    quad_load_smem<FMT>(slot + p.gu_cb + p.gu_sb, slot + 2 * p.gu_cb + p.gu_sb, warp, lane, qu);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) ag[i][r] = au[i][r] = 0.f;
+                    quad_compute<FMT>(qg, B1, xs1, ag[i]);
+                    quad_compute<FMT>(qu, B1, xs1, au[i]);
+                }
+            }
+            if (warp == 0) TRACEW(9);
+            if (!got && tid == 0) flag(p.status, MOE_DEV_TIMEOUT);
+            if (!__syncthreads_and(got)) goto finish;
+            if (tid == 0) ring_used = nC;
+            // token 0 sits in lanes t == 0: rows g (r = 0) and g + 8 (r = 2)
+            float(*red1)[kWarps][2][16] = reinterpret_cast<float(*)[kWarps][2][16]>(&s.red[0][0][0][0]);
+            if (t == 0) {
+#pragma unroll
+                for (int i = 0; i < kCBatch; ++i) {
+                    if (i < nC) {
+                        red1[i][warp][0][g] = ag[i][0];
+                        red1[i][warp][0][g + 8] = ag[i][2];
+                        red1[i][warp][1][g] = au[i][0];
+                        red1[i][warp][1][g + 8] = au[i][2];
+                    }
+                }
+            }
+            __syncthreads();
+            TRACE(17);
+            if (tid < nC * 16) {
+                const int i = tid >> 4, row = tid & 15;
+                const int task = cfirst + i * G, ar = task / NG, rg = task % NG;
+                float A = 0.f, U = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) {
+                    A += red1[i][w][0][row];
+                    U += red1[i][w][1][row];
+                }
+                p.h[size_t(s.act_beg[s.res[ar]]) * f + 16 * rg + row] = A / (1.0f + expf(-A)) * U;
+            }
+            __syncthreads();  // slots and red[] read by everyone
+            if (tid == 0)
+                while (ring_issued < nU && ring_issued < nC + NS) issue(ring_issued++);
+            TRACE(14);
+        }
+        for (int u = 0; !batch && u < nC; ++u) {
+            const int task = cfirst + u * G, ar = task / NG, rg = task % NG;
             const int a = s.res[ar];
             const int ntok = s.act_cnt[a];
             const int *tok = s.s_tok + s.act_beg[a];
-            if (!one_quad) {  // general d: tiles loaded inside the task
-                const uint8_t *rec = p.pool + int64_t(s.act_slot[a]) * p.slot_bytes;
-                gateup_task<FMT>(p, s, sx, rec, rg, ntok, tok, s.act_beg[a]);
-                __syncthreads();
-                continue;
-            }
-            const QuadRegs<FMT> cg = ng, cu = nu;
-            if (task + G < ntasks) load_task(task + G, ng, nu);
+            if (!await_unit(u)) goto finish;
+            if (u == 0) TRACE(16);
+            const uint8_t *slot = ring + size_t(u % NS) * p.rslot;
             float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
-            if (NT == 1) {
-                quad_compute<FMT>(cg, B1, xs1, ag);
-                quad_compute<FMT>(cu, B1, xs1, au);
-            } else {
-                const uint16_t *xrow = g < ntok ? sx + size_t(tok[g]) * d : nullptr;
-                const int t0 = 2 * t < ntok ? tok[2 * t] : -1, t1 = 2 * t + 1 < ntok ? tok[2 * t + 1] : -1;
-                uint32_t B[4][8];
-                build_b_bf16<FMT>(xrow, warp, t, B);
-                float xs[4][2];
+            for (int qd = warp; qd < NQ; qd += kWarps) {
+                QuadRegs<FMT> qg, qu;
+                quad_load_smem<FMT>(slot, slot + p.gu_cb, qd, lane, qg);
+                quad_load_smem<FMT>(slot + p.gu_cb + p.gu_sb, slot + 2 * p.gu_cb + p.gu_sb, qd, lane, qu);
+                if (NT == 1 && one_quad) {
+                    quad_compute<FMT>(qg, B1, xs1, ag);
+                    quad_compute<FMT>(qu, B1, xs1, au);
+                } else {
+                    const uint16_t *xrow = g < ntok ? sx + size_t(tok[g]) * d : nullptr;
+                    const int t0 = 2 * t < ntok ? tok[2 * t] : -1, t1 = 2 * t + 1 < ntok ? tok[2 * t + 1] : -1;
+                    uint32_t B[4][8];
+                    build_b_bf16<FMT>(xrow, qd, t, B);
+                    float xs[4][2];
 #pragma unroll
-                for (int bq = 0; bq < 4; ++bq) {
-                    xs[bq][0] = t0 >= 0 ? s.xs[4 * warp + bq][t0] : 0.f;
-                    xs[bq][1] = t1 >= 0 ? s.xs[4 * warp + bq][t1] : 0.f;
+                    for (int bq = 0; bq < 4; ++bq) {
+                        xs[bq][0] = t0 >= 0 ? s.xs[4 * qd + bq][t0] : 0.f;
+                        xs[bq][1] = t1 >= 0 ? s.xs[4 * qd + bq][t1] : 0.f;
+                    }
+                    quad_compute<FMT>(qg, B, xs, ag);
+                    quad_compute<FMT>(qu, B, xs, au);
                 }
-                quad_compute<FMT>(cg, B, xs, ag);
-                quad_compute<FMT>(cu, B, xs, au);
             }
-            if (nth < 2 && warp == 0) TRACEW(nth == 0 ? 9 : 15);
+            if (u < 2 && warp == 0) TRACEW(u == 0 ? 9 : 15);
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 s.red[warp][0][r][lane] = ag[r];
                 s.red[warp][1][r][lane] = au[r];
             }
             __syncthreads();
+            if (u == 0) TRACE(17);
             if (tid < 128) {
                 const int L = tid >> 2, r = tid & 3;
                 float A = 0.f, U = 0.f;
@@ -691,80 +878,108 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
                 const int n = 2 * (L & 3) + (r & 1);
                 if (n < ntok) p.h[size_t(s.act_beg[a] + n) * f + 16 * rg + row] = A / (1.0f + expf(-A)) * U;
             }
-            __syncthreads();
-            if (nth == 0) TRACE(14);
+            __syncthreads();  // slot and red[] read by everyone
+            if (tid == 0 && ring_issued < nU) issue(ring_issued++);
+            if (u == 0) TRACE(14);
         }
-    }
-    // publish this CTA's h rows once (one fence), then count its tasks per expert
-    if (tid == 0) {
-        __threadfence();
-        for (int task = G - 1 - cta; task < s.nres * NG; task += G) atomicAdd(p.done + task / NG, 1u);
-    }
+        // publish this CTA's h rows (written before the last barrier): one fence
+        // and one count per task, by as many threads
+        for (int u = tid; u < nC; u += kThreads) {
+            __threadfence();
+            atomicAdd(p.done + (cfirst + u * G) / NG, 1u);
+        }
 
-    TRACE(7);
-    // ------------------------------------------------------------ phase D
-    {
-        const int nres = s.nres;
-        const int nblk = d / 128;  // CTA-task = (expert, 8 row groups of d)
-        const int NQf = f / 256;
-        for (int task = cta; task < (nres + 1) * nblk; task += G) {
-            const int ar = task / nblk, blk = task % nblk;
+        TRACE(7);
+        // ------------------------------------------------------------ phase D
+        int staged = -1;  // expert whose h, block sums and B fragments are in shared memory
+        for (int u = nC; u < nU; ++u) {
+            const int task = dlo + (u - nC), ar = task / nblk, blk = task % nblk;
             const bool shared = ar == nres;
             const int a = shared ? 0 : s.res[ar];
             const int ntok = shared ? T : s.act_cnt[a];
             const int beg = shared ? npairs : s.act_beg[a];
-            const int slot = shared ? p.shared_slot : s.act_slot[a];
-            const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
             const int rg = 8 * blk + warp;
-            // this warp's first two weight tiles now (they do not depend on h)
-            QuadRegs<FMT> q0, q1;
-            quad_load<FMT>(rec, p.down, rg, 0, lane, q0);
-            if (NQf > 1) quad_load<FMT>(rec, p.down, rg, 1, lane, q1);
-            __syncthreads();  // previous task's readers of sh are done
-            if (tid == 0) s.ok = wait_geq(p.done + (shared ? kSharedIdx : ar), unsigned(NG), p.status);
-            __syncthreads();
-            if (!s.ok) continue;
-            {
-                constexpr int kHv = NT * 1024 / 4 / kThreads + 1;  // float4 per thread at most
-                const float4 *src = reinterpret_cast<const float4 *>(p.h + size_t(beg) * f);
-                float4 *dst = reinterpret_cast<float4 *>(sh);
-                const int nh = ntok * f / 4;
-                float4 hv[kHv];
-#pragma unroll
-                for (int u = 0; u < kHv; ++u)
-                    if (tid + u * kThreads < nh) hv[u] = __ldcg(src + tid + u * kThreads);
-#pragma unroll
-                for (int u = 0; u < kHv; ++u)
-                    if (tid + u * kThreads < nh) dst[tid + u * kThreads] = hv[u];
+            if (!await_unit(u)) goto finish;
+            if (u == nC) TRACE(18);
+            if (ar != staged) {  // the expert's first unit here: wait for its h, stage it
+                staged = ar;
+                if (tid == 0) s.ok = wait_geq(p.done + (shared ? kSharedIdx : ar), unsigned(NG), p.status);
+                __syncthreads();
+                if (!s.ok) goto finish;
+                if (u == nC) TRACE(19);
+                {  // the expert's h rows (written by other CTAs: read through L2) into shared memory
+                    constexpr int kHv = NT * kMaxFDec / 4 / kThreads + 1;  // float4 per thread at most
+                    const float4 *src = reinterpret_cast<const float4 *>(p.h + size_t(beg) * f);
+                    float4 *dst = reinterpret_cast<float4 *>(sh);
+                    const int nh = ntok * f / 4;
+                    float4 hv[kHv];
+    #pragma unroll
+                    for (int v = 0; v < kHv; ++v)
+                        if (tid + v * kThreads < nh) hv[v] = __ldcg(src + tid + v * kThreads);
+    #pragma unroll
+                    for (int v = 0; v < kHv; ++v)
+                        if (tid + v * kThreads < nh) dst[tid + v * kThreads] = hv[v];
+                }
+                __syncthreads();
+                for (int job = warp; job < (f / 64) * ntok; job += kWarps) {  // block sums of h
+                    const int bb = job / ntok, n = job % ntok;
+                    const float2 v = *reinterpret_cast<const float2 *>(sh + size_t(n) * f + 64 * bb + 2 * lane);
+                    float sum = v.x + v.y;
+    #pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                    if (lane == 0) s.hsb[bb][n] = sum;
+                }
+                // B fragments of every quad of h (element (k, n=gg) of slot rho of
+                // block bq for lane (gg, tt): columns 256qd + 64bq + slot_k(rho, tt),
+                // divided by 2^slot_exp), one 16-byte entry per thread and step
+                for (int e = tid; e < NQf * 256; e += kThreads) {
+                    const int qd = e >> 8, ln = (e >> 3) & 31, r4 = e & 7;
+                    const int gg = ln >> 2, tt = ln & 3, bq = r4 >> 1;
+                    const float *src = gg < ntok ? sh + size_t(gg) * f + 256 * qd + 64 * bq : nullptr;
+                    uint32_t v[4];
+    #pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int rho = (r4 & 1) * 4 + j;
+                        float lo = 0.f, hi = 0.f;
+                        if (src) {
+                            const float2 hv = *reinterpret_cast<const float2 *>(src + slot_k(rho, tt, 0));
+                            lo = hv.x;
+                            hi = hv.y;
+                            too_big |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+                        }
+                        const float sc = __int_as_float((127 - slot_exp<FMT>(bq, rho)) << 23);  // 2^-exp
+                        v[j] = pack_half2(lo * sc, hi * sc);
+                    }
+                    s.bfrag[qd][r4][ln] = make_uint4(v[0], v[1], v[2], v[3]);
+                }
+                __syncthreads();
             }
-            __syncthreads();
-            for (int job = warp; job < (f / 64) * ntok; job += kWarps) {  // block sums of h
-                const int bb = job / ntok, n = job % ntok;
-                const float2 v = *reinterpret_cast<const float2 *>(sh + size_t(n) * f + 64 * bb + 2 * lane);
-                float sum = v.x + v.y;
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                if (lane == 0) s.hsb[bb][n] = sum;
-            }
-            __syncthreads();
-            const int g = lane >> 2, t = lane & 3;
-            const float *hrow = g < ntok ? sh + size_t(g) * f : nullptr;
+            if (u == nC) TRACE(20);
+            const uint8_t *slot = ring + size_t(u % NS) * p.rslot;
+            const uint8_t *cb = slot + warp * p.dn_cb, *sb = slot + 8 * p.dn_cb + warp * p.dn_sb;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-            for (int qd = 0; qd < NQf; ++qd) {  // tile qd computes while tile qd+2 loads
-                QuadRegs<FMT> cur = q0;
-                q0 = q1;
-                if (qd + 2 < NQf) quad_load<FMT>(rec, p.down, rg, qd + 2, lane, q1);
+            for (int qd = 0; qd < NQf; ++qd) {
+                QuadRegs<FMT> q;
+                quad_load_smem<FMT>(cb, sb, qd, lane, q);
                 uint32_t B[4][8];
-                build_b_f32_smem<FMT>(hrow, qd, t, B, too_big);
+#pragma unroll
+                for (int r4 = 0; r4 < 8; ++r4) {
+                    const uint4 v = s.bfrag[qd][r4][lane];
+                    B[r4 >> 1][(r4 & 1) * 4 + 0] = v.x;
+                    B[r4 >> 1][(r4 & 1) * 4 + 1] = v.y;
+                    B[r4 >> 1][(r4 & 1) * 4 + 2] = v.z;
+                    B[r4 >> 1][(r4 & 1) * 4 + 3] = v.w;
+                }
                 float xs[4][2];
 #pragma unroll
                 for (int bq = 0; bq < 4; ++bq) {
                     xs[bq][0] = 2 * t < ntok ? s.hsb[4 * qd + bq][2 * t] : 0.f;
                     xs[bq][1] = 2 * t + 1 < ntok ? s.hsb[4 * qd + bq][2 * t + 1] : 0.f;
                 }
-                quad_compute<FMT>(cur, B, xs, acc);
+                quad_compute<FMT>(q, B, xs, acc);
             }
+            if (u == nC && warp == 0) TRACEW(21);
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 const int n = 2 * t + (r & 1);
@@ -776,6 +991,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
                     atomicAdd(p.y + size_t(tk) * d + row, gw * acc[r]);
                 }
             }
+            __syncthreads();  // slot, sh, bfrag and hsb read by everyone
+            if (u == nC) TRACE(22);
+            if (tid == 0 && ring_issued < nU) issue(ring_issued++);
         }
     }
 
@@ -829,6 +1047,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
     }
 
 finish:
+    if (tid == 0)  // copies still in flight (error paths only) land before the CTA leaves
+        for (int u = ring_used; u < ring_issued; ++u)
+            if (!ring_wait(&s.full[u % p.nslots], uint32_t(u / p.nslots) & 1u)) break;
     if (too_big) flag(p.status, MOE_DEV_NONFINITE);
     __syncthreads();
     TRACE(4);
@@ -849,47 +1070,56 @@ finish:
     }
 }
 
-// Dynamic shared memory: T*d bf16 activations, then up to 8 rows of h (fp32).
-constexpr size_t kDynSmemMax = size_t(kMaxTokDec) * kMaxDimDec * 2 + size_t(kMaxTokDec) * 1024 * 4;
-
-size_t dyn_smem(int T, int d, int f) { return ((size_t(T) * d * 2 + 15) & ~size_t(15)) + size_t(T) * f * 4; }
-
 struct LaunchCache {
     int grid[8][64] = {};
+    int avail[8][64] = {};  // dynamic shared memory a CTA can have
     bool ready[8][64] = {};
 };
 std::mutex g_mu;
 LaunchCache g_cache;
 
 template <int FMT, int NT>
-moe_status launch(const DecodeParams &p, size_t smem, cudaStream_t stream) {
+moe_status launch(DecodeParams p, cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
     constexpr int ci = (FMT - 2) * 4 + (NT == 1 ? 0 : NT == 2 ? 1 : NT == 4 ? 2 : 3);
-    int grid;
+    int grid, avail;
     {
         std::lock_guard<std::mutex> lock(g_mu);
         if (!g_cache.ready[ci][dev]) {
-            int sms = 0, per = 0;
-            if (cudaFuncSetAttribute(decode_layer_kernel<FMT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     int(kDynSmemMax)) != cudaSuccess ||
-                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_layer_kernel<FMT, NT>, kThreads,
-                                                              kDynSmemMax) != cudaSuccess ||
+            int sms = 0, per = 0, optin = 0;
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, decode_layer_kernel<FMT, NT>) != cudaSuccess ||
+                cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+                cudaGetLastError();
+                return MOE_ERR_CUDA;
+            }
+            const int av = optin - int(fa.sharedSizeBytes);
+            if (av <= 0 ||
+                cudaFuncSetAttribute(decode_layer_kernel<FMT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, av) !=
+                    cudaSuccess ||
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_layer_kernel<FMT, NT>, kThreads, av) !=
+                    cudaSuccess ||
                 per < 1) {
                 cudaGetLastError();
                 return MOE_ERR_CUDA;
             }
             g_cache.grid[ci][dev] = sms * std::min(per, kCtasPerSm);
+            g_cache.avail[ci][dev] = av;
             g_cache.ready[ci][dev] = true;
         }
         grid = g_cache.grid[ci][dev];
+        avail = g_cache.avail[ci][dev];
     }
-    DecodeParams pp = p;
-    void *args[] = {&pp};
+    const size_t base = ring_off(p.T, p.d, p.f);
+    if (size_t(avail) < base + 2 * size_t(p.rslot)) return MOE_ERR_UNSUPPORTED;
+    p.nslots = int(std::min<size_t>(kMaxSlots, (size_t(avail) - base) / p.rslot));
+    const size_t smem = base + size_t(p.nslots) * p.rslot;
+    void *args[] = {&p};
     if (cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(decode_layer_kernel<FMT, NT>), dim3(grid),
                                     dim3(kThreads), args, smem, stream) != cudaSuccess) {
         cudaGetLastError();
@@ -899,11 +1129,11 @@ moe_status launch(const DecodeParams &p, size_t smem, cudaStream_t stream) {
 }
 
 template <int FMT>
-moe_status launch_fmt(const DecodeParams &p, size_t smem, cudaStream_t stream) {
-    if (p.T <= 1) return launch<FMT, 1>(p, smem, stream);
-    if (p.T <= 2) return launch<FMT, 2>(p, smem, stream);
-    if (p.T <= 4) return launch<FMT, 4>(p, smem, stream);
-    return launch<FMT, 8>(p, smem, stream);
+moe_status launch_fmt(const DecodeParams &p, cudaStream_t stream) {
+    if (p.T <= 1) return launch<FMT, 1>(p, stream);
+    if (p.T <= 2) return launch<FMT, 2>(p, stream);
+    if (p.T <= 4) return launch<FMT, 4>(p, stream);
+    return launch<FMT, 8>(p, stream);
 }
 
 size_t ws_align(size_t x) { return (x + 255) & ~size_t(255); }
@@ -930,7 +1160,7 @@ MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, 
     if (!W || T < 0 || E <= 0 || k <= 0 || miss_cap < 0) return MOE_ERR_INVALID_ARG;
     if (W->fmt != 2 && W->fmt != 3) return MOE_ERR_INVALID_ARG;
     if (W->d != d || W->f != f) return MOE_ERR_INVALID_ARG;
-    if (!dims_ok(d, f) || d > kMaxDimDec || T > kMaxTokDec || E > kMaxEDec || k > kMaxK || k > E)
+    if (!dims_ok(d, f) || d > kMaxDimDec || f > kMaxFDec || T > kMaxTokDec || E > kMaxEDec || k > kMaxK || k > E)
         return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!slot_of || !x || !Wr || !y) return MOE_ERR_INVALID_ARG;
@@ -982,14 +1212,31 @@ MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, 
     p.gate = eg.m[0];
     p.up = eg.m[1];
     p.down = eg.m[2];
-    if (dyn_smem(T, d, f) > kDynSmemMax) return MOE_ERR_UNSUPPORTED;
-    const size_t smem = dyn_smem(T, d, f);
-    return W->fmt == 2 ? launch_fmt<2>(p, smem, as_cuda(stream)) : launch_fmt<3>(p, smem, as_cuda(stream));
+    // bytes of one row group's codes and scales (contiguous in the record), and
+    // the ring slot: a gate/up task (both matrices) or a down task (8 row groups)
+    const int fmt = W->fmt;
+    auto cbytes = [&](const MatGeom &m) {
+        return uint32_t(fmt == 2 ? q2_chunk_off(m, 1, 0, 0) - q2_chunk_off(m, 0, 0, 0)
+                                 : q3_word_off(m, 1, 0, 0, 0) - q3_word_off(m, 0, 0, 0, 0));
+    };
+    auto sbytes = [&](const MatGeom &m) { return uint32_t(scale_off(m, fmt, 1, 0, 0) - scale_off(m, fmt, 0, 0, 0)); };
+    p.gu_cb = cbytes(p.gate);
+    p.gu_sb = sbytes(p.gate);
+    p.dn_cb = cbytes(p.down);
+    p.dn_sb = sbytes(p.down);
+    if ((p.gu_cb | p.gu_sb | p.dn_cb | p.dn_sb) % 16 ||
+        (p.gate.codes_off | p.gate.scales_off | p.up.codes_off | p.up.scales_off | p.down.codes_off |
+         p.down.scales_off) % 16 ||
+        cbytes(p.up) != p.gu_cb || sbytes(p.up) != p.gu_sb)
+        return MOE_ERR_UNSUPPORTED;
+    p.rslot = (std::max(2u * (p.gu_cb + p.gu_sb), 8u * (p.dn_cb + p.dn_sb)) + 127u) & ~127u;
+    p.nslots = 0;
+    return fmt == 2 ? launch_fmt<2>(p, as_cuda(stream)) : launch_fmt<3>(p, as_cuda(stream));
 }
 
 #ifdef MOE_DECODE_TRACE
 // Trace builds only: copy the phase timestamps to host memory.
-MOE_API int moe_decode_trace_read(void *dst) {  // 4096 CTAs x (16 timestamps, 16 clocks)
+MOE_API int moe_decode_trace_read(void *dst) {  // 4096 CTAs x 32 timestamps
     return int(cudaMemcpyFromSymbol(dst, moe_decode_trace, sizeof(moe_decode_trace)));
 }
 #endif

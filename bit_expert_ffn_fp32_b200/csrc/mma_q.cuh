@@ -41,6 +41,16 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// c = A * B  (m16n8k16 with a zero accumulator input: no zeroed registers needed)
+__device__ __forceinline__ void mma16816_zc(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
@@ -142,9 +152,11 @@ __device__ __forceinline__ void quad_compute(const QuadRegs<FMT> &q, const uint3
         const uint32_t mn[4] = {q.s0.y, q.s0.w, q.s1.y, q.s1.w};
 #pragma unroll
         for (int bq = 0; bq < 4; ++bq) {
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            float c[4];
+            mma16816_zc(c, q2_reg(wg[bq], 0), q2_reg(wg8[bq], 0), q2_reg(wg[bq], 1), q2_reg(wg8[bq], 1), B[bq][0],
+                        B[bq][1]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 1; i < 4; ++i)
                 mma16816(c, q2_reg(wg[bq], 2 * i), q2_reg(wg8[bq], 2 * i), q2_reg(wg[bq], 2 * i + 1),
                          q2_reg(wg8[bq], 2 * i + 1), B[bq][2 * i], B[bq][2 * i + 1]);
             block_epilogue<2>(c, sc[bq], mn[bq], xs[bq][0], xs[bq][1], acc);
@@ -153,9 +165,11 @@ __device__ __forceinline__ void quad_compute(const QuadRegs<FMT> &q, const uint3
         const uint32_t sc[4] = {q.s0.x, q.s0.y, q.s1.x, q.s1.y};
 #pragma unroll
         for (int bq = 0; bq < 4; ++bq) {
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            float c[4];
+            mma16816_zc(c, q3_reg(q.W, 8 * bq, 0), q3_reg(q.W, 8 * bq, 1), q3_reg(q.W, 8 * bq + 1, 0),
+                        q3_reg(q.W, 8 * bq + 1, 1), B[bq][0], B[bq][1]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 1; i < 4; ++i) {
                 const int u0 = 8 * bq + 2 * i, u1 = u0 + 1;
                 mma16816(c, q3_reg(q.W, u0, 0), q3_reg(q.W, u0, 1), q3_reg(q.W, u1, 0), q3_reg(q.W, u1, 1),
                          B[bq][2 * i], B[bq][2 * i + 1]);

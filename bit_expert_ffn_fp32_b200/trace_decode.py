@@ -22,8 +22,11 @@ from .layer import MoEStack, x_tensor
 
 POINTS = {8: "x staged", 10: "router rows (warp 0)", 1: "phase A done", 2: "all logits counted",
           11: "top-k loads", 12: "top-k candidates", 13: "top-k selected", 6: "top-k + gates",
-          5: "routing tables", 3: "prefetch issued", 9: "C task 1 computed (warp 0)",
-          14: "C task 1 done", 15: "C task 2 computed (warp 0)", 7: "phase C done", 4: "kernel end"}
+          5: "routing tables", 3: "ring copies issued", 9: "C task 1 computed (warp 0)",
+          16: "C task 1 bytes landed", 17: "C task 1 partials synced", 14: "C task 1 done",
+          15: "C task 2 computed (warp 0)", 7: "phase C done", 18: "D unit 1 bytes landed",
+          19: "D unit 1 expert ready", 20: "D unit 1 h staged", 21: "D unit 1 computed (warp 0)",
+          22: "D unit 1 done", 4: "kernel end"}
 
 
 def main() -> None:
@@ -59,7 +62,7 @@ def main() -> None:
             continue
         tr = buf.reshape(4096, 32)
         G = int((tr[:, 0] > 0).sum())
-        ns = tr[:G, :16].astype(np.int64)
+        ns = tr[:G, :].astype(np.int64)
         rel = np.where(ns > 0, (ns - ns[:, 0].min()) / 1000.0, np.nan)
         for k in POINTS:
             if np.isfinite(rel[:, k]).any():
