@@ -47,7 +47,7 @@ def _env_int(name, default):
 PROFILED_TRAFFIC = {
     # fused decode layer kernel, one launch per step
     "decode_T1_d2048_E512_k10_f768_q2": (("decode_layer.cu", "mma_q.cuh", "layout.h", "common.cuh"),
-                                         "dcd7d8b103ec6b4e", 20.54e6),
+                                         "866ff83c958ad8d0", 20.56e6),
     # expert FFN launches of one step: fp16 gathers, tcgen05 gate/up and down, routed and shared
     "prefill_T8192_d2048_E512_k10_f768_q2": (("ffn_tc05.cu", "tc05.cuh", "layout.h", "common.cuh", "ffn_mma.cu"),
                                              "c9ce5905da33cce4", 2505e6),
