@@ -50,7 +50,7 @@ PROFILED_TRAFFIC = {
                                          "866ff83c958ad8d0", 20.56e6),
     # expert FFN launches of one step: fp16 gathers, tcgen05 gate/up and down, routed and shared
     "prefill_T8192_d2048_E512_k10_f768_q2": (("ffn_tc05.cu", "tc05.cuh", "layout.h", "common.cuh", "ffn_mma.cu"),
-                                             "c9ce5905da33cce4", 2505e6),
+                                             "60d411ce6b0a09e6", 2506e6),
 }
 
 

@@ -398,11 +398,11 @@ __device__ __forceinline__ void issue_rows(const TcParams &p, TcSmem &s, unsigne
 
 // Producer warps (0-7): warp w owns row group rgl = 2(w%4) + w/4 of the
 // 128-row tile (its tensor-memory lane quadrant is w%4). For each stage, once
-// the block pair's packed bytes have landed (fullR) and the MMA has released
-// the A stage (emptyA), each thread dequantises its lane chunk (rows g, g+8 of
-// the row group; k-slots of t) into registers and stores it to the stage's
-// TMEM columns (lane g / g+8, column 4*rho + t = k/2), then arrives on fullA
-// (and on emptyR after the pair's second block). a_col0: TMEM column of A
+// the block pair's packed bytes have landed (fullR), each thread loads its lane
+// chunk (rows g, g+8 of the row group; k-slots of t), releases the code slot
+// after the pair's second block (emptyR) and dequantises into registers; once
+// the MMA has released the A stage (emptyA) it stores the chunk to the stage's
+// TMEM columns (lane g / g+8, column 4*rho + t = k/2) and arrives on fullA. a_col0: TMEM column of A
 // stage 0, matrix 0; stages are 32*NMAT columns apart.
 template <int NMAT, int SA, int SB, int SRP>
 __device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int KS,
@@ -426,13 +426,6 @@ __device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned c
         }
         ck.add(1, t0);
         t0 = ck.now();
-        if (!tc::mbar_wait(&s.emptyA[it % SA], ((it / SA) & 1) ^ 1, kTcWaitNs)) {
-            ok = false;
-            break;
-        }
-        tc::fence_after();
-        ck.add(2, t0);
-        t0 = ck.now();
         const unsigned char *raw = R::raw(dyn, pp);
         HalfQ2 c[NMAT];  // both matrices' bytes first, then both dequantised together
 #pragma unroll
@@ -441,9 +434,20 @@ __device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned c
             c[i].sc = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + kRawCodes + rgl * 128 +
                                                        (lane >> 2) * 16 + 8 * bb);
         }
+        if (bb) tc::mbar_arrive(&s.emptyR[pp % SRP]);  // both blocks of the pair are in registers
+        // dequantise into registers while the MMA may still be reading this A stage
         uint32_t v[NMAT][16];
 #pragma unroll
         for (int i = 0; i < NMAT; ++i) dequant_half_q2(c[i], v[i]);
+        ck.add(4, t0);
+        t0 = ck.now();
+        if (!tc::mbar_wait(&s.emptyA[it % SA], ((it / SA) & 1) ^ 1, kTcWaitNs)) {
+            ok = false;
+            break;
+        }
+        tc::fence_after();
+        ck.add(2, t0);
+        t0 = ck.now();
         const long long t2 = ck.now();
 #pragma unroll
         for (int i = 0; i < NMAT; ++i) tc::tmem_st16x128_x8(ta + uint32_t((it % SA) * 32 * NMAT + 32 * i), v[i]);
@@ -453,7 +457,6 @@ __device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned c
         ck.add(5, t3);
         tc::fence_before();
         tc::mbar_arrive(&s.fullA[it % SA]);
-        if (bb) tc::mbar_arrive(&s.emptyR[pp % SRP]);
         ck.add(4, t0);
         ck.count(6);
         if (s.abort) break;
