@@ -144,12 +144,18 @@ __global__ void __launch_bounds__(kThreads)
     permute_scan_kernel(int ntiles, int E, int32_t *ws, int32_t *counts, int32_t *offsets, int32_t *active) {
     __shared__ int s_cnt[kMaxE];
     __shared__ int s_warp[32];
+    constexpr int kBatch = 16;  // tiles whose counts are loaded together (one L2 round trip)
     for (int e = threadIdx.x; e < E; e += kThreads) {
         int run = 0;
-        for (int tile = 0; tile < ntiles; ++tile) {
-            const int h = ws[size_t(tile) * E + e];
-            ws[size_t(tile) * E + e] = run;
-            run += h;
+        for (int t0 = 0; t0 < ntiles; t0 += kBatch) {
+            int h[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) h[j] = t0 + j < ntiles ? ws[size_t(t0 + j) * E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                if (t0 + j < ntiles) ws[size_t(t0 + j) * E + e] = run;
+                run += h[j];
+            }
         }
         s_cnt[e] = run;
     }
