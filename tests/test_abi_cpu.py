@@ -56,6 +56,9 @@ def test_host_validation_rejects_before_launch():
     assert L.moe_route(dummy, dummy, None, 1 << 30, 2048, 512, 10, dummy, dummy, dummy, None, None) == 5
     # T == 0 is a no-op
     assert L.moe_route(None, None, None, 0, 2048, 512, 10, None, None, None, None, None) == 0
+    # x or Wr not 16-byte aligned
+    assert L.moe_route(dummy + 8, dummy, None, 4, 2048, 512, 10, dummy, dummy, dummy, None, None) == 1
+    assert L.moe_route(dummy, dummy + 4, None, 4, 2048, 512, 10, dummy, dummy, dummy, None, None) == 1
     # permute: too small workspace for a multi-tile input
     need = native.permute_workspace_bytes(8192, 10, 512)
     assert need > 0
@@ -76,6 +79,14 @@ def test_host_validation_rejects_before_launch():
     assert L.moe_expert_ffn_q2(C.byref(pool), *small) == 3
     pool.slot_bytes = 1000
     assert L.moe_expert_ffn_q2(C.byref(pool), *args) == 1
+    # one-launch decode layer: f above the 1024 it stages, T above 8
+    wide = native.QPool(dummy * 256, 1 << 22, 10, 2, 2048, 2048)
+    dec = [dummy, 0, 0, dummy, dummy, None, 1, 2048, 2048, 512, 10] + [None] * 12 + [0, dummy, dummy, 1 << 24,
+                                                                                   None, None]
+    assert L.moe_layer_decode(C.byref(wide), *dec) == 2
+    dec9 = list(dec)
+    dec9[6], dec9[8] = 9, 768
+    assert L.moe_layer_decode(C.byref(pool), *dec9) == 2
     # combine: d not a multiple of 4
     assert L.moe_combine(dummy, dummy, dummy, None, None, 2, 10, 2046, dummy, None) == 2
     # pack: missing hi plane for Q3
