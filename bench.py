@@ -84,10 +84,14 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, out_dir: str | None = None):
+        """The raw samples go to <out_dir>/clocks_gpu<i>.csv (default: a temporary directory)."""
+        import tempfile
+
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        d = out_dir or tempfile.mkdtemp(prefix="moe_clocks_")
+        self.path = os.path.join(d, f"clocks_gpu{gpu_index}.csv")
 
     def start(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
@@ -282,7 +286,7 @@ def run_ours(args, wl, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(local_rank)
+    sampler = ClockSampler(local_rank, args.clocks_dir)
     sampler.start()
     time.sleep(0.2)
     for i in range(args.steps):
@@ -413,6 +417,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_T1_d2048_E512_k10_f768_q2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-dir", default=None,
+                    help="keep the raw nvidia-smi clock samples of the timed region in this directory")
     ap.add_argument("--combine", choices=["atomic", "kernel"], default="kernel",
                     help="steps path: gate-weighted atomics in the routed expert call (atomic) or y_perm + moe_combine")
     ap.add_argument("--path", choices=["auto", "fused", "steps"], default="auto",
