@@ -196,6 +196,49 @@ def cpu_baseline(wl, budget_s=12.0):
                       + (f"; x{wl.layers} layers per token" if wl.layers > 1 else "") + ")"}
 
 
+# ------------------------------------------------------------------ host completion of misses
+MISS_DTYPE = [("layer", "<i4"), ("expert", "<i4"), ("token", "<i4"), ("j", "<i4"), ("gate", "<f4")]
+
+
+def _time_host_misses(stack, wl, bufs, x_step):
+    """moe_complete_misses_host over one step's miss lists (all layers): each
+    layer's missed experts are packed into a host pool first (not timed), then
+    the completion of every layer is timed on the host clock with all threads."""
+    import time
+
+    from bit_expert_ffn_fp32_b200 import native
+
+    L, T = wl.layers, wl.T
+    stride = (native.expert_bytes(wl.fmt, wl.d, wl.f) + 255) // 256 * 256
+    work, n_rec, n_exp = [], 0, 0
+    for l in range(L):
+        recs = np.array(stack.misses(bufs[l]), dtype=MISS_DTYPE)
+        if len(recs) == 0:
+            continue
+        y = np.ascontiguousarray(bufs[l].y[:T].cpu().numpy())
+        experts = sorted(set(recs["expert"].tolist()))
+        buf = np.zeros(stride * len(experts) + 256, np.uint8)
+        base = buf.ctypes.data + (-buf.ctypes.data) % 256
+        slot_of = np.full(wl.E, -1, np.int32)
+        for s_, e in enumerate(experts):
+            ex = stack.canonical_expert(l, e)
+            q = [native.qmatrix(ex[m]["codes"], ex[m]["scale"], ex[m]["min"], ex[m]["hi"]) for m in ("gate", "up", "down")]
+            native.pack_expert_host(wl.fmt, wl.d, wl.f, *q, base + s_ * stride)
+            slot_of[e] = s_
+        pool = native.QPool(base, stride, len(experts), wl.fmt, wl.d, wl.f)
+        work.append((l, recs, y, buf, pool, slot_of, np.ascontiguousarray(x_step[l])))
+        n_rec += len(recs)
+        n_exp += len(experts)
+    threads = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    for l, recs, y, _buf, pool, slot_of, xl in work:
+        native.complete_misses_host(pool, slot_of, wl.E, recs, len(recs), l, xl, T, y, 0)
+    dt = time.perf_counter() - t0
+    return {"ms_per_step": dt * 1e3, "misses_per_step": n_rec, "distinct_experts_per_step": n_exp,
+            "threads": threads, "call": "moe_complete_misses_host (host C++, fp32), one call per layer",
+            "sample": "the misses of the last end-to-end step"}
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args, wl, rank, world, local_rank):
     import torch
@@ -361,6 +404,10 @@ def run_ours(args, wl, rank, world, local_rank):
 
     if rank != 0:
         return 0
+    # stacked layers: the host completion of the last e2e step's misses, on this machine's cores
+    host_leg = None
+    if L > 1 and not args.no_host_misses:
+        host_leg = _time_host_misses(stack, wl, bufs, xs_host[(args.steps - 1) % n_x])
     hbm_peak, tc_peak, peak_kind = _measured_peaks()
     eb = native.expert_bytes(wl.fmt, wl.d, wl.f)
     ffn_bytes = (mean_act + L) * eb                # routed resident experts + the shared experts, read once
@@ -405,6 +452,8 @@ def run_ours(args, wl, rank, world, local_rank):
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
+    if host_leg is not None:
+        line["host_miss_completion"] = host_leg
     print(json.dumps(line), flush=True)
     return 0
 
@@ -417,6 +466,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_T1_d2048_E512_k10_f768_q2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-host-misses", action="store_true",
+                    help="stacked layers: skip timing the host completion of the miss lists")
     ap.add_argument("--clocks-dir", default=None,
                     help="keep the raw nvidia-smi clock samples of the timed region in this directory")
     ap.add_argument("--combine", choices=["atomic", "kernel"], default="kernel",

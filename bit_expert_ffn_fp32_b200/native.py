@@ -65,6 +65,7 @@ SIGNATURES = {
     "moe_layer_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "moe_layer_decode": (_I, [C.POINTER(QPool), _P, _I32, _I32, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                               _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _SZ, _P, _P]),
+    "moe_complete_misses_host": (_I, [C.POINTER(QPool), _P, _I, _P, _I32, _I32, _P, _I, _P, _I]),
 }
 
 
@@ -201,3 +202,12 @@ def layer_decode(pool: QPool, slot_of, shared_slot: int, layer: int, x, Wr, bias
                                ptr(sorted_tok), ptr(sorted_j), ptr(inv), ptr(active), ptr(slot_of_pair), ptr(miss),
                                ptr(miss_count), miss_cap, ptr(y), ptr(ws), ws_bytes, ptr(dev_status),
                                stream_handle(stream)))
+
+
+def complete_misses_host(pool: QPool, slot_of, E: int, miss, n: int, layer: int, x, T: int, y,
+                         nthreads: int = 0) -> None:
+    """Host completion of a layer's miss list (host arrays: slot_of int32 [E],
+    miss records, x uint16 [T][d], y float32 [T][d] accumulated in place)."""
+    check("moe_complete_misses_host",
+          lib.moe_complete_misses_host(C.byref(pool), ptr(slot_of), E, ptr(miss), n, layer, ptr(x), T, ptr(y),
+                                       nthreads))
