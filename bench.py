@@ -254,7 +254,7 @@ def run_ours(args, wl, rank, world, local_rank):
     L = wl.layers
     stack = MoEStack(wl, device=dev)
     T = wl.T
-    bufs = [stack.buffers(T) for _ in range(L)]
+    bufs = [stack.buffers(T)] + [stack.buffers(T, fresh=True) for _ in range(L - 1)]  # one set per layer
     b = bufs[0]
     stream = torch.cuda.current_stream()
     n_steps = args.warmup + args.steps

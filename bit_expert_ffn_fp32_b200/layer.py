@@ -114,8 +114,11 @@ class MoEStack:
         upload_expert(self.canonical_expert(layer, e), self.wl.fmt, self.wl.d, self.wl.f,
                       self.pool.data_ptr() + slot * self.slot_bytes, self.device)
 
-    def buffers(self, T: int) -> Buffers:
-        if T in self._bufs:
+    def buffers(self, T: int, fresh: bool = False) -> Buffers:
+        """Outputs and workspaces for T tokens: one cached set per T, or a new
+        set with fresh=True (e.g. one per layer when several layers' outputs
+        must stay readable)."""
+        if T in self._bufs and not fresh:
             return self._bufs[T]
         wl, dev = self.wl, self.device
         n = T * wl.k
@@ -139,7 +142,8 @@ class MoEStack:
             sh_offsets=torch.tensor([0, T], **i32), sh_sorted_tok=torch.arange(max(T, 1), **i32),
             sh_sorted_j=torch.zeros(max(T, 1), **i32), sh_active=torch.tensor([1, 0], **i32),
         )
-        self._bufs[T] = b
+        if T not in self._bufs:
+            self._bufs[T] = b
         return b
 
     def forward(self, layer: int, x: torch.Tensor, b: Buffers | None = None, stream=None,
