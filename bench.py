@@ -201,42 +201,32 @@ MISS_DTYPE = [("layer", "<i4"), ("expert", "<i4"), ("token", "<i4"), ("j", "<i4"
 
 
 def _time_host_misses(stack, wl, bufs, x_step):
-    """moe_complete_misses_host over one step's miss lists (all layers): each
-    layer's missed experts are packed into a host pool first (not timed), then
-    the completion of every layer is timed on the host clock with all threads."""
+    """moe_complete_misses_host over one step's miss lists (all layers), the
+    missed experts in canonical host storage (generated first, not timed), the
+    completion of every layer timed on the host clock with all threads."""
     import time
 
     from bit_expert_ffn_fp32_b200 import native
 
     L, T = wl.layers, wl.T
-    stride = (native.expert_bytes(wl.fmt, wl.d, wl.f) + 255) // 256 * 256
     work, n_rec, n_exp = [], 0, 0
     for l in range(L):
         recs = np.array(stack.misses(bufs[l]), dtype=MISS_DTYPE)
         if len(recs) == 0:
             continue
         y = np.ascontiguousarray(bufs[l].y[:T].cpu().numpy())
-        experts = sorted(set(recs["expert"].tolist()))
-        buf = np.zeros(stride * len(experts) + 256, np.uint8)
-        base = buf.ctypes.data + (-buf.ctypes.data) % 256
-        slot_of = np.full(wl.E, -1, np.int32)
-        for s_, e in enumerate(experts):
-            ex = stack.canonical_expert(l, e)
-            q = [native.qmatrix(ex[m]["codes"], ex[m]["scale"], ex[m]["min"], ex[m]["hi"]) for m in ("gate", "up", "down")]
-            native.pack_expert_host(wl.fmt, wl.d, wl.f, *q, base + s_ * stride)
-            slot_of[e] = s_
-        pool = native.QPool(base, stride, len(experts), wl.fmt, wl.d, wl.f)
-        work.append((l, recs, y, buf, pool, slot_of, np.ascontiguousarray(x_step[l])))
+        canon = {e: stack.canonical_expert(l, e) for e in sorted(set(recs["expert"].tolist()))}
+        work.append((l, recs, y, canon, native.expert_table(wl.E, canon), np.ascontiguousarray(x_step[l])))
         n_rec += len(recs)
-        n_exp += len(experts)
+        n_exp += len(canon)
     threads = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
-    for l, recs, y, _buf, pool, slot_of, xl in work:
-        native.complete_misses_host(pool, slot_of, wl.E, recs, len(recs), l, xl, T, y, 0)
+    for l, recs, y, _canon, tab, xl in work:
+        native.complete_misses_host(wl.fmt, wl.d, wl.f, tab, wl.E, recs, len(recs), l, xl, T, y, 0)
     dt = time.perf_counter() - t0
     return {"ms_per_step": dt * 1e3, "misses_per_step": n_rec, "distinct_experts_per_step": n_exp,
-            "threads": threads, "call": "moe_complete_misses_host (host C++, fp32), one call per layer",
-            "sample": "the misses of the last end-to-end step"}
+            "threads": threads, "call": "moe_complete_misses_host (host C++, fp32 lookup-table dot products), "
+            "one call per layer", "sample": "the misses of the last end-to-end step"}
 
 
 # ------------------------------------------------------------------ our arm

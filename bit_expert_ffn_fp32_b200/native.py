@@ -65,7 +65,7 @@ SIGNATURES = {
     "moe_layer_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "moe_layer_decode": (_I, [C.POINTER(QPool), _P, _I32, _I32, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                               _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _SZ, _P, _P]),
-    "moe_complete_misses_host": (_I, [C.POINTER(QPool), _P, _I, _P, _I32, _I32, _P, _I, _P, _I]),
+    "moe_complete_misses_host": (_I, [_I, _I, _I, _P, _I, _P, _I32, _I32, _P, _I, _P, _I]),
 }
 
 
@@ -204,10 +204,22 @@ def layer_decode(pool: QPool, slot_of, shared_slot: int, layer: int, x, Wr, bias
                                stream_handle(stream)))
 
 
-def complete_misses_host(pool: QPool, slot_of, E: int, miss, n: int, layer: int, x, T: int, y,
+def expert_table(E: int, experts: dict) -> C.Array:
+    """moe_qmatrix [E][3] (gate, up, down) for the experts given as
+    {e: canonical expert dict}; absent experts get NULL matrices. The arrays
+    must stay alive while the table is used."""
+    tab = (QMatrix * (3 * E))()
+    for e, ex in experts.items():
+        for i, m in enumerate(("gate", "up", "down")):
+            tab[3 * e + i] = qmatrix(ex[m]["codes"], ex[m]["scale"], ex[m]["min"], ex[m]["hi"])
+    return tab
+
+
+def complete_misses_host(fmt: int, d: int, f: int, experts: C.Array, E: int, miss, n: int, layer: int, x, T: int, y,
                          nthreads: int = 0) -> None:
-    """Host completion of a layer's miss list (host arrays: slot_of int32 [E],
-    miss records, x uint16 [T][d], y float32 [T][d] accumulated in place)."""
+    """Host completion of a layer's miss list (host arrays: experts from
+    expert_table, miss records, x uint16 [T][d], y float32 [T][d] accumulated
+    in place)."""
     check("moe_complete_misses_host",
-          lib.moe_complete_misses_host(C.byref(pool), ptr(slot_of), E, ptr(miss), n, layer, ptr(x), T, ptr(y),
+          lib.moe_complete_misses_host(fmt, d, f, C.cast(experts, _P), E, ptr(miss), n, layer, ptr(x), T, ptr(y),
                                        nthreads))

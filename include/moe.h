@@ -245,22 +245,24 @@ moe_status moe_expert_ffn_q3(const moe_qpool *W, const int32_t *slot_of, const u
  * 新方案最高90t/s Hermes 调用60t/s" (section "为什么从 18t/s 变成 60-90t/s") does
  * with the experts kept in system RAM. For every record i of miss[0..n):
  *   y[miss[i].token] += miss[i].gate * down(silu(gate_proj x) * up_proj x),
- * x = x[miss[i].token], with the weights dequantised in fp32 from the packed
- * record of expert miss[i].expert in a HOST pool. Results are added in record
- * order, so y does not depend on nthreads.
- *   host_pool  moe_qpool whose base is host memory (records packed with
- *              moe_pack_expert_host); fmt, d, f give the shapes
- *   slot_of    int32 [E] (host): host-pool slot of each expert of this layer
+ * x = x[miss[i].token], in fp32 from the expert's canonical storage (w = s*q+m
+ * or s*(q-4) applied per 64-block to the block's code-weighted sum). Results
+ * are added in record order, so y does not depend on nthreads.
+ *   fmt, d, f  format and shapes (as for the pool)
+ *   experts    moe_qmatrix [E][3] (host): gate [f][d], up [f][d], down [d][f]
+ *              of every expert of this layer in canonical host storage; only
+ *              the experts the records name are read
  *   miss, n    the layer's miss records (host), as moe_cache_lookup or
  *              moe_layer_decode wrote them; every record must name `layer`
  *   x          bf16 bits [T][d] (host), the layer's input
  *   y          fp32 [T][d] (host), accumulated into (e.g. the GPU's partial y)
  *   nthreads   worker threads (0 = the machine's hardware threads)
- * Returns MOE_ERR_INVALID_ARG for a record with another layer, an expert outside
- * [0, E), a token outside [0, T) or an expert without a host slot, before any
- * change to y. Blocking; no GPU involvement.
+ * Returns MOE_ERR_INVALID_ARG, before any change to y, for a record with
+ * another layer, an expert outside [0, E), a token outside [0, T) or an expert
+ * whose matrices are missing (NULL codes/scale, min for Q2, hi for Q3).
+ * Blocking; no GPU involvement.
  */
-moe_status moe_complete_misses_host(const moe_qpool *host_pool, const int32_t *slot_of, int E, const moe_miss *miss,
+moe_status moe_complete_misses_host(int fmt, int d, int f, const moe_qmatrix *experts, int E, const moe_miss *miss,
                                     int32_t n, int32_t layer, const uint16_t *x, int T, float *y, int nthreads);
 
 /* Workspace bytes moe_layer_decode needs for (T, k, f, E). */

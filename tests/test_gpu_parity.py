@@ -136,25 +136,16 @@ def test_stack48_cache_and_misses():
 
 def _complete_on_host(stack, layer, x_bits, b):
     """The GPU's partial y plus moe_complete_misses_host over the layer's miss
-    list, with the missed experts packed into a host pool."""
+    list, the missed experts given in canonical host storage."""
     wl = stack.wl
     recs = np.array(stack.misses(b), dtype=[("layer", "<i4"), ("expert", "<i4"), ("token", "<i4"), ("j", "<i4"),
                                             ("gate", "<f4")])
     y = np.ascontiguousarray(b.y[: x_bits.shape[0]].cpu().numpy())
     if len(recs) == 0:
         return y
-    experts = sorted(set(recs["expert"].tolist()))
-    stride = (native.expert_bytes(wl.fmt, wl.d, wl.f) + 255) // 256 * 256
-    buf = np.zeros(stride * len(experts) + 256, np.uint8)
-    base = buf.ctypes.data + (-buf.ctypes.data) % 256
-    slot_of = np.full(wl.E, -1, np.int32)
-    for s_, e in enumerate(experts):
-        ex = stack.canonical_expert(layer, e)
-        q = [native.qmatrix(ex[m]["codes"], ex[m]["scale"], ex[m]["min"], ex[m]["hi"]) for m in ("gate", "up", "down")]
-        native.pack_expert_host(wl.fmt, wl.d, wl.f, *q, base + s_ * stride)
-        slot_of[e] = s_
-    pool = native.QPool(base, stride, len(experts), wl.fmt, wl.d, wl.f)
-    native.complete_misses_host(pool, slot_of, wl.E, recs, len(recs), layer, np.ascontiguousarray(x_bits),
+    canon = {e: stack.canonical_expert(layer, e) for e in sorted(set(recs["expert"].tolist()))}
+    tab = native.expert_table(wl.E, canon)
+    native.complete_misses_host(wl.fmt, wl.d, wl.f, tab, wl.E, recs, len(recs), layer, np.ascontiguousarray(x_bits),
                                 x_bits.shape[0], y, 0)
     return y
 
