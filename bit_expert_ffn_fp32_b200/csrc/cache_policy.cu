@@ -1,0 +1,126 @@
+// Expert-cache policy: which experts hold the pool's slots.
+//
+// The engine of "个人开发者用 AI 十天写出 Strata 引擎，让 12GB 显存跑起 1250 亿参数的
+// Qwen 3.8 Flash Next" (section "命中率七成，代价是答案会变") fills the GPU's free
+// room with the experts called most often and keeps swapping while the
+// conversation runs, moving an expert in once it starts to be used frequently;
+// it reports a higher hit rate than a fixed frequency curve (72% against 50%).
+// This file is that policy on the host, in integer arithmetic so that its
+// decisions are exactly reproducible:
+//   - every routed (token, expert) pair of a layer adds 1 to count[layer][expert]
+//     (hits and misses alike);
+//   - every `epoch` tokens (counted on layer 0's observations) all counts are
+//     halved (count >>= 1): recent use weighs more than old use;
+//   - a plan first gives free slots to the non-resident experts with the
+//     highest counts (count > 0), then swaps the best non-resident expert for
+//     the worst resident one while best.count > worst.count + margin, at most
+//     max_swaps changes per plan. Order: count descending, then (layer, expert)
+//     ascending for candidates; count ascending, then (layer, expert)
+//     descending for victims; free slots in ascending slot order.
+// The caller applies a plan by copying each admitted expert's record into its
+// slot (e.g. moe_pack_expert or a host-to-device copy of the packed record)
+// and the changed rows of the slot table to the device.
+#include <algorithm>
+#include <cstring>
+#include <vector>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+struct PolicyHeader {
+    uint32_t magic;
+    int32_t L, E, S;
+    int32_t epoch, margin;
+    int64_t clock;  // tokens observed on layer 0 since the last halving
+};
+constexpr uint32_t kPolicyMagic = 0x4d4f4543u;  // "MOEC"
+
+size_t policy_bytes(int L, int E) { return sizeof(PolicyHeader) + size_t(L) * E * sizeof(uint32_t); }
+
+PolicyHeader *header(void *state) { return static_cast<PolicyHeader *>(state); }
+uint32_t *counts(void *state) { return reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(state) + sizeof(PolicyHeader)); }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+MOE_API size_t moe_cache_policy_bytes(int L, int E) {
+    if (L <= 0 || E <= 0 || int64_t(L) * E >= (int64_t(1) << 31)) return 0;
+    return policy_bytes(L, E);
+}
+
+MOE_API moe_status moe_cache_policy_init(void *state, size_t bytes, int L, int E, int S, int epoch, int margin) {
+    if (!state || L <= 0 || E <= 0 || S < 0 || epoch <= 0 || margin < 0) return MOE_ERR_INVALID_ARG;
+    if (int64_t(L) * E >= (int64_t(1) << 31)) return MOE_ERR_OVERFLOW;
+    if (bytes < policy_bytes(L, E)) return MOE_ERR_WORKSPACE;
+    PolicyHeader *h = header(state);
+    h->magic = kPolicyMagic;
+    h->L = L;
+    h->E = E;
+    h->S = S;
+    h->epoch = epoch;
+    h->margin = margin;
+    h->clock = 0;
+    std::memset(counts(state), 0, size_t(L) * E * sizeof(uint32_t));
+    return MOE_OK;
+}
+
+MOE_API moe_status moe_cache_policy_observe(void *state, int layer, const int32_t *topk_idx, int T, int k) {
+    if (!state || header(state)->magic != kPolicyMagic) return MOE_ERR_INVALID_ARG;
+    PolicyHeader *h = header(state);
+    if (layer < 0 || layer >= h->L || T < 0 || k <= 0 || (T > 0 && !topk_idx)) return MOE_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < int64_t(T) * k; ++i)
+        if (topk_idx[i] < 0 || topk_idx[i] >= h->E) return MOE_ERR_INVALID_ARG;
+    uint32_t *c = counts(state);
+    if (layer == 0) {  // the token clock: halve everything once per epoch
+        h->clock += T;
+        while (h->clock >= h->epoch) {
+            h->clock -= h->epoch;
+            for (int64_t i = 0; i < int64_t(h->L) * h->E; ++i) c[i] >>= 1;
+        }
+    }
+    uint32_t *row = c + size_t(layer) * h->E;
+    for (int64_t i = 0; i < int64_t(T) * k; ++i)
+        if (row[topk_idx[i]] < 0xffffffffu) ++row[topk_idx[i]];
+    return MOE_OK;
+}
+
+MOE_API int32_t moe_cache_policy_plan(void *state, int32_t *slot_of, moe_swap *swaps, int32_t max_swaps) {
+    if (!state || header(state)->magic != kPolicyMagic || !slot_of || max_swaps < 0 || (max_swaps > 0 && !swaps))
+        return -int32_t(MOE_ERR_INVALID_ARG);
+    const PolicyHeader *h = header(state);
+    const int64_t LE = int64_t(h->L) * h->E;
+    const uint32_t *c = counts(state);
+    // the slot table must be a partial injection into [0, S)
+    std::vector<int32_t> owner(h->S, -1);  // slot -> layer * E + expert
+    for (int64_t i = 0; i < LE; ++i) {
+        const int32_t s = slot_of[i];
+        if (s < -1 || s >= h->S || (s >= 0 && owner[s] >= 0)) return -int32_t(MOE_ERR_INVALID_ARG);
+        if (s >= 0) owner[s] = int32_t(i);
+    }
+    std::vector<int32_t> cand, vict;  // non-resident with count > 0; resident
+    for (int64_t i = 0; i < LE; ++i) (slot_of[i] >= 0 ? vict : cand).push_back(int32_t(i));
+    cand.erase(std::remove_if(cand.begin(), cand.end(), [&](int32_t i) { return c[i] == 0; }), cand.end());
+    std::sort(cand.begin(), cand.end(), [&](int32_t a, int32_t b) { return c[a] != c[b] ? c[a] > c[b] : a < b; });
+    std::sort(vict.begin(), vict.end(), [&](int32_t a, int32_t b) { return c[a] != c[b] ? c[a] < c[b] : a > b; });
+    int32_t n = 0;
+    size_t ci = 0, vi = 0;
+    for (int32_t s = 0; s < h->S && n < max_swaps && ci < cand.size(); ++s) {  // free slots first
+        if (owner[s] >= 0) continue;
+        const int32_t e = cand[ci++];
+        slot_of[e] = s;
+        swaps[n++] = moe_swap{s, e / h->E, e % h->E, -1, -1};
+    }
+    for (; n < max_swaps && ci < cand.size() && vi < vict.size(); ++ci, ++vi) {
+        const int32_t in = cand[ci], out = vict[vi];
+        if (!(uint64_t(c[in]) > uint64_t(c[out]) + uint64_t(h->margin))) break;
+        const int32_t s = slot_of[out];
+        slot_of[out] = -1;
+        slot_of[in] = s;
+        swaps[n++] = moe_swap{s, in / h->E, in % h->E, out / h->E, out % h->E};
+    }
+    return n;
+}

@@ -36,6 +36,10 @@ class QMatrix(C.Structure):
     _fields_ = [("codes", _P), ("hi", _P), ("scale", _P), ("min", _P)]
 
 
+class Swap(C.Structure):
+    _fields_ = [("slot", _I32), ("layer_in", _I32), ("expert_in", _I32), ("layer_out", _I32), ("expert_out", _I32)]
+
+
 class Miss(C.Structure):
     _fields_ = [("layer", _I32), ("expert", _I32), ("token", _I32), ("j", _I32), ("gate", C.c_float)]
 
@@ -66,6 +70,10 @@ SIGNATURES = {
     "moe_layer_decode": (_I, [C.POINTER(QPool), _P, _I32, _I32, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                               _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _SZ, _P, _P]),
     "moe_complete_misses_host": (_I, [_I, _I, _I, _P, _I, _P, _I32, _I32, _P, _I, _P, _I]),
+    "moe_cache_policy_bytes": (_SZ, [_I, _I]),
+    "moe_cache_policy_init": (_I, [_P, _SZ, _I, _I, _I, _I, _I]),
+    "moe_cache_policy_observe": (_I, [_P, _I, _P, _I, _I]),
+    "moe_cache_policy_plan": (_I32, [_P, _P, _P, _I32]),
 }
 
 
@@ -223,3 +231,36 @@ def complete_misses_host(fmt: int, d: int, f: int, experts: C.Array, E: int, mis
     check("moe_complete_misses_host",
           lib.moe_complete_misses_host(fmt, d, f, C.cast(experts, _P), E, ptr(miss), n, layer, ptr(x), T, ptr(y),
                                        nthreads))
+
+
+class CachePolicy:
+    """Host expert-cache policy (moe_cache_policy_*): counts of routed pairs,
+    halved every `epoch` tokens, and slot plans against an [L][E] slot table."""
+
+    def __init__(self, L: int, E: int, S: int, epoch: int, margin: int = 0):
+        import numpy as np
+
+        n = int(lib.moe_cache_policy_bytes(L, E))
+        if n == 0:
+            raise MoeError("moe_cache_policy_bytes", 2)
+        self.L, self.E, self.S = L, E, S
+        self.state = np.zeros(n, np.uint8)
+        check("moe_cache_policy_init", lib.moe_cache_policy_init(self.state.ctypes.data, n, L, E, S, epoch, margin))
+
+    def observe(self, layer: int, topk_idx) -> None:
+        import numpy as np
+
+        idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+        T, k = idx.shape
+        check("moe_cache_policy_observe", lib.moe_cache_policy_observe(self.state.ctypes.data, layer, idx.ctypes.data,
+                                                                       T, k))
+
+    def plan(self, slot_of, max_swaps: int) -> list:
+        """Update slot_of (int32 [L][E] numpy, in place); the changes as tuples
+        (slot, layer_in, expert_in, layer_out, expert_out)."""
+        buf = (Swap * max(1, max_swaps))()
+        n = int(lib.moe_cache_policy_plan(self.state.ctypes.data, slot_of.ctypes.data, buf, max_swaps))
+        if n < 0:
+            raise MoeError("moe_cache_policy_plan", -n)
+        return [(buf[i].slot, buf[i].layer_in, buf[i].expert_in, buf[i].layer_out, buf[i].expert_out)
+                for i in range(n)]

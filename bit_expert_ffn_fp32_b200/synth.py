@@ -32,7 +32,7 @@ from __future__ import annotations
 import numpy as np
 
 # Tensor ids inside the Philox key.
-_T_X, _T_WR, _T_PERM, _T_EXPERT = 1, 2, 3, 4
+_T_X, _T_WR, _T_PERM, _T_EXPERT, _T_TRACE = 1, 2, 3, 4, 5
 _MAT_ID = {"gate": 0, "up": 1, "down": 2}
 _PART_ID = {"codes": 0, "hi": 1, "scale": 2, "min": 3}
 
@@ -130,3 +130,26 @@ def slot_table_by_rank(rank: np.ndarray, resident: int, first_slot: int) -> np.n
     hot = rank <= resident
     slot[hot] = (first_slot + rank[hot] - 1).astype(np.int32)
     return slot
+
+
+def gen_routing_trace(seed: int, L: int, E: int, k: int, n_tokens: int, s: float = 1.1, drift_every: int = 0,
+                      drift_swaps: int = 0) -> np.ndarray:
+    """Synthetic routing of n_tokens tokens through L layers: int32
+    [n_tokens][L][k], each row k distinct expert ids (ascending) drawn without
+    replacement with probability proportional to rank^-s, where each layer has
+    its own seeded rank permutation. Every drift_every tokens (0 = never), each
+    layer exchanges the ranks of drift_swaps random expert pairs: popularity
+    drifts the way a conversation changes topic."""
+    rng = rng_for(seed, _T_TRACE, L, E, k)
+    rank = np.stack([rng.permutation(E) + 1 for _ in range(L)])  # rank[l][e] in 1..E
+    out = np.empty((n_tokens, L, k), np.int32)
+    for t in range(n_tokens):
+        if drift_every and t and t % drift_every == 0:
+            for l in range(L):
+                for _ in range(drift_swaps):
+                    a, b = rng.integers(0, E, 2)
+                    rank[l, a], rank[l, b] = rank[l, b], rank[l, a]
+        # without replacement: the k largest of log p + Gumbel noise
+        keys = -s * np.log(rank) + rng.gumbel(size=(L, E))
+        out[t] = np.sort(np.argpartition(-keys, k - 1, axis=1)[:, :k], axis=1)
+    return out

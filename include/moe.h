@@ -265,6 +265,42 @@ moe_status moe_expert_ffn_q3(const moe_qpool *W, const int32_t *slot_of, const u
 moe_status moe_complete_misses_host(int fmt, int d, int f, const moe_qmatrix *experts, int E, const moe_miss *miss,
                                     int32_t n, int32_t layer, const uint16_t *x, int T, float *y, int nthreads);
 
+/*
+ * Expert-cache policy ([SAITO] "命中率七成，代价是答案会变": the free GPU room is
+ * filled with the most frequently called experts, swapped while the
+ * conversation runs). Host state in caller-owned memory; integer arithmetic,
+ * so decisions are exactly reproducible:
+ *   - observe: every routed pair of `layer` adds 1 to count[layer][expert];
+ *     every `epoch` tokens (counted on layer 0) all counts are halved;
+ *   - plan: free slots go to the non-resident (layer, expert) with the highest
+ *     counts (> 0); then the best non-resident replaces the worst resident
+ *     while best.count > worst.count + margin; at most max_swaps changes.
+ *     Candidates rank by count desc, then layer*E+expert asc; victims by count
+ *     asc, then layer*E+expert desc; free slots are filled in ascending order.
+ * The slot pool is shared by all L layers: slot_of is int32 [L][E] (host),
+ * -1 = not resident, each slot in [0, S) held at most once; plan updates it in
+ * place and lists the changes. The caller then copies every admitted expert's
+ * record into its slot and the slot table to the device.
+ */
+typedef struct moe_swap {
+    int32_t slot;
+    int32_t layer_in, expert_in;    /* the expert that now holds the slot      */
+    int32_t layer_out, expert_out;  /* its previous holder, -1/-1 if it was free */
+} moe_swap;
+
+/* Bytes of policy state for L layers of E experts (0 if unsupported). */
+size_t moe_cache_policy_bytes(int L, int E);
+
+/* Initialise the state (all counts 0); S slots; epoch > 0 tokens; margin >= 0. */
+moe_status moe_cache_policy_init(void *state, size_t bytes, int L, int E, int S, int epoch, int margin);
+
+/* Count one layer call's routing: topk_idx int32 [T][k] (host). */
+moe_status moe_cache_policy_observe(void *state, int layer, const int32_t *topk_idx, int T, int k);
+
+/* Plan slot changes; returns the number written to swaps (<= max_swaps), or
+ * -(moe_status) on an invalid state or slot table (slot_of then unchanged). */
+int32_t moe_cache_policy_plan(void *state, int32_t *slot_of, moe_swap *swaps, int32_t max_swaps);
+
 /* Workspace bytes moe_layer_decode needs for (T, k, f, E). */
 size_t moe_layer_decode_workspace_bytes(int T, int k, int f, int E);
 
