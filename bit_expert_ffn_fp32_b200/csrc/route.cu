@@ -9,6 +9,8 @@
 // for o = 16..1 is exactly the pairwise combination of the definition.
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -388,10 +390,24 @@ MOE_API moe_status moe_route(const uint16_t *x, const float *Wr, const float *bi
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(Wr)) & 15) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = as_cuda(stream);
     if (T >= 64) {
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(router_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRsSmem);
-            attr = true;
+        // the kernel's shared memory (64 KiB) needs the opt-in, once per device
+        static std::mutex mu;
+        static bool ready[64] = {};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        {
+            std::lock_guard<std::mutex> lock(mu);
+            if (!ready[dev]) {
+                if (cudaFuncSetAttribute(router_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRsSmem) !=
+                    cudaSuccess) {
+                    cudaGetLastError();
+                    return MOE_ERR_CUDA;
+                }
+                ready[dev] = true;
+            }
         }
         dim3 g((E + kRsExp - 1) / kRsExp, (T + kRsTok - 1) / kRsTok);
         router_smem_kernel<<<g, kRsThreads, kRsSmem, s>>>(x, Wr, bias, T, d, E, logits, dev_status);
