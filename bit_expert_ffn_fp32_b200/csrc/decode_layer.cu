@@ -77,6 +77,7 @@ constexpr int kSharedIdx = kMaxPairs;         // done[] slot of the shared exper
 constexpr int kMaxDimDec = 2048;
 constexpr int kCandMax = 64;  // candidates ranked in shared memory; more take the round-based path
 constexpr unsigned long long kWaitNs = 100ull * 1000 * 1000;
+constexpr unsigned long long kWaitSteps = 1ull << 27;  // polls: >= 4 s of 32 ns sleeps
 constexpr int kMaxSlots = 8;  // weight-ring slots at most
 constexpr int kMaxFDec = 1024;  // expert width f (h staging and B fragments)
 constexpr int kCBatch = 4;      // gate/up units computed in one pass (one token)
@@ -163,8 +164,9 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
 __device__ bool wait_geq(const unsigned *p, unsigned target, int32_t *status) {
     if (ld_acquire(p) >= target) return true;
     const unsigned long long t0 = globaltimer();
-    while (ld_acquire(p) < target) {
-        if (globaltimer() - t0 > kWaitNs) {
+    // the iteration cap ends the wait even if the timer stood still (each step sleeps >= 32 ns)
+    for (unsigned long long it = 0; ld_acquire(p) < target; ++it) {
+        if (globaltimer() - t0 > kWaitNs || it > kWaitSteps) {
             flag(status, MOE_DEV_TIMEOUT);
             return false;
         }
@@ -194,13 +196,31 @@ __device__ __forceinline__ bool ring_test(uint64_t *bar, uint32_t parity) {
         : "memory");
     return done != 0;
 }
-// false after kWaitNs (the caller flags MOE_DEV_TIMEOUT)
+// false after kWaitNs, or kWaitSteps polls (the caller flags MOE_DEV_TIMEOUT)
 __device__ bool ring_wait(uint64_t *bar, uint32_t parity) {
     if (ring_test(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
-    while (!ring_test(bar, parity))
-        if (globaltimer() - t0 > kWaitNs) return false;
+    for (unsigned long long it = 0; !ring_test(bar, parity); ++it) {
+        if (globaltimer() - t0 > kWaitNs || it > kWaitSteps) return false;
+        if (it > 1024) __nanosleep(32);
+    }
     return true;
+}
+
+// One CTA runs the two waits above against objects nothing completes (a device
+// counter below target, a fresh mbarrier phase with no arrival): both give up
+// with MOE_DEV_TIMEOUT; elapsed[0..1] receive their durations.
+__global__ void wait_probe_kernel(const unsigned *counter, unsigned target, unsigned long long *elapsed,
+                                  int32_t *status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    const unsigned long long t0 = globaltimer();
+    wait_geq(counter, target, status);
+    const unsigned long long t1 = globaltimer();
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&bar)) : "memory");
+    if (!ring_wait(&bar, 0u)) flag(status, MOE_DEV_TIMEOUT);
+    elapsed[0] = t1 - t0;
+    elapsed[1] = globaltimer() - t1;
 }
 
 // Order-preserving key of an fp32 logit: larger logit -> larger key; +0 and -0
@@ -1232,6 +1252,14 @@ MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, 
     p.rslot = (std::max(2u * (p.gu_cb + p.gu_sb), 8u * (p.dn_cb + p.dn_sb)) + 127u) & ~127u;
     p.nslots = 0;
     return fmt == 2 ? launch_fmt<2>(p, as_cuda(stream)) : launch_fmt<3>(p, as_cuda(stream));
+}
+
+MOE_API moe_status moe_debug_wait_probe(const uint32_t *counter, uint32_t target, uint64_t *elapsed_ns,
+                                        int32_t *dev_status, moe_stream_t stream) {
+    if (!counter || !elapsed_ns || !dev_status) return MOE_ERR_INVALID_ARG;
+    wait_probe_kernel<<<1, 32, 0, as_cuda(stream)>>>(counter, target,
+                                                     reinterpret_cast<unsigned long long *>(elapsed_ns), dev_status);
+    return launch_status();
 }
 
 #ifdef MOE_DECODE_TRACE

@@ -70,6 +70,7 @@ SIGNATURES = {
     "moe_layer_decode": (_I, [C.POINTER(QPool), _P, _I32, _I32, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                               _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _SZ, _P, _P]),
     "moe_complete_misses_host": (_I, [_I, _I, _I, _P, _I, _P, _I32, _I32, _P, _I, _P, _I]),
+    "moe_debug_wait_probe": (_I, [_P, C.c_uint32, _P, _P, _P]),
     "moe_cache_policy_bytes": (_SZ, [_I, _I]),
     "moe_cache_policy_init": (_I, [_P, _SZ, _I, _I, _I, _I, _I]),
     "moe_cache_policy_observe": (_I, [_P, _I, _P, _I, _I]),
@@ -264,3 +265,10 @@ class CachePolicy:
             raise MoeError("moe_cache_policy_plan", -n)
         return [(buf[i].slot, buf[i].layer_in, buf[i].expert_in, buf[i].layer_out, buf[i].expert_out)
                 for i in range(n)]
+
+
+def debug_wait_probe(counter, target: int, elapsed_ns, dev_status, stream=None) -> None:
+    """moe_debug_wait_probe: the library's bounded waits against a counter below
+    target and an mbarrier phase nothing completes (device tensors)."""
+    check("moe_debug_wait_probe", lib.moe_debug_wait_probe(ptr(counter), target, ptr(elapsed_ns), ptr(dev_status),
+                                                           stream_handle(stream)))

@@ -301,6 +301,19 @@ moe_status moe_cache_policy_observe(void *state, int layer, const int32_t *topk_
  * -(moe_status) on an invalid state or slot table (slot_of then unchanged). */
 int32_t moe_cache_policy_plan(void *state, int32_t *slot_of, moe_swap *swaps, int32_t max_swaps);
 
+/*
+ * Diagnostic for the bounded waits: one CTA runs the library's two in-kernel
+ * waits against objects that nothing completes -- the device counter *counter
+ * (read with acquire loads) awaited until >= target, then a fresh shared-memory
+ * mbarrier phase with no arrival. Each gives up after the library's wait limit
+ * (100 ms, or a poll count that bounds it should the timer stand still) and
+ * sets MOE_DEV_TIMEOUT in *dev_status; elapsed_ns (device, uint64 [2]) receives
+ * the two durations. With *counter >= target the first wait returns at once.
+ * All pointers are device pointers; asynchronous on the stream.
+ */
+moe_status moe_debug_wait_probe(const uint32_t *counter, uint32_t target, uint64_t *elapsed_ns,
+                                int32_t *dev_status, moe_stream_t stream);
+
 /* Workspace bytes moe_layer_decode needs for (T, k, f, E). */
 size_t moe_layer_decode_workspace_bytes(int T, int k, int f, int E);
 

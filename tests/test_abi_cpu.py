@@ -87,6 +87,9 @@ def test_host_validation_rejects_before_launch():
     dec9 = list(dec)
     dec9[6], dec9[8] = 9, 768
     assert L.moe_layer_decode(C.byref(pool), *dec9) == 2
+    # wait probe: null pointers
+    assert L.moe_debug_wait_probe(None, 1, dummy, dummy, None) == 1
+    assert L.moe_debug_wait_probe(dummy, 1, None, dummy, None) == 1
     # combine: d not a multiple of 4
     assert L.moe_combine(dummy, dummy, dummy, None, None, 2, 10, 2046, dummy, None) == 2
     # pack: missing hi plane for Q3
