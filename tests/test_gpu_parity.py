@@ -221,28 +221,6 @@ def test_multi_tile_permutation():
         np.testing.assert_array_equal(buf[: ref[key].shape[0]].cpu().numpy(), ref[key], err_msg=key)
 
 
-# ---------------------------------------------------------------- bounded waits
-def test_bounded_waits_time_out_and_leave_the_context_usable(tiny):
-    """The library's in-kernel waits on a counter that nothing raises and on an
-    mbarrier phase that nothing completes give up after their 100 ms limit with
-    MOE_DEV_TIMEOUT (no hang, no fault), and the context runs a layer after."""
-    counter = torch.zeros(1, dtype=torch.int32, device="cuda")
-    el = torch.zeros(2, dtype=torch.int64, device="cuda")
-    st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    native.debug_wait_probe(counter, 1, el, st)
-    torch.cuda.synchronize()
-    assert int(st.item()) & native.DEV_TIMEOUT
-    e = el.cpu().numpy()
-    assert np.all(e >= 90e6) and np.all(e < 10e9), e
-    counter.fill_(3)                       # already at its target: no wait
-    st.zero_()
-    native.debug_wait_probe(counter, 3, el, st)
-    torch.cuda.synchronize()
-    assert int(el[0].item()) < 1e6 and int(st.item()) & native.DEV_TIMEOUT
-    x = synth.gen_x(0, 0, configs.TINY.T, configs.TINY.d)
-    _full_check(tiny, 0, x)
-
-
 # ---------------------------------------------------------------- router shapes
 @pytest.mark.parametrize("T,d,E,k,ties", [
     (5, 256, 100, 7, False),      # few tokens: one warp per expert
