@@ -110,6 +110,24 @@ class MoEStack:
     def canonical_expert(self, layer: int, e: int) -> dict:
         return synth.gen_expert(self.seed, layer, e, self.wl.fmt, self.wl.d, self.wl.f)
 
+    def apply_swaps(self, swaps) -> None:
+        """Carry out a cache-policy plan: every (slot, layer_in, expert_in,
+        layer_out, expert_out) packs expert_in's record into slot (on the
+        current stream, after the work already queued there) and updates the
+        slot tables, host and device."""
+        changed = set()
+        for slot, l_in, e_in, l_out, e_out in swaps:
+            if not 0 <= slot < self.L * self.R:
+                raise ValueError("slot %d outside the routed slots" % slot)
+            if l_out >= 0:
+                self.slot_of_host[l_out][e_out] = -1
+                changed.add(l_out)
+            self.slot_of_host[l_in][e_in] = slot
+            changed.add(l_in)
+            self._pack(l_in, e_in, slot)
+        for l in changed:
+            self.slot_of[l].copy_(torch.from_numpy(np.ascontiguousarray(self.slot_of_host[l], dtype=np.int32)))
+
     def _pack(self, layer: int, e: int, slot: int) -> None:
         upload_expert(self.canonical_expert(layer, e), self.wl.fmt, self.wl.d, self.wl.f,
                       self.pool.data_ptr() + slot * self.slot_bytes, self.device)
