@@ -225,8 +225,9 @@ size_t moe_expert_ffn_workspace_bytes(int T, int k, int d, int f);
  * Paths: with T*k < 512 a weight-streaming kernel reads each expert's packed
  * codes once per 8 tokens (mma.sync fragments built from the codes); with
  * T*k >= 512 and E <= 1024 (prefill) the Q2 call runs grouped GEMMs on the tcgen05 tensor
- * cores, dequantising each 128-row weight tile to fp16 in shared memory
- * (fp16 rounding of w = s*q + m); the workspace then holds h as fp16 [T*k][f]
+ * cores, dequantising each 128-row weight tile to fp16 in registers and storing
+ * it to tensor memory (fp16 rounding of w = s*q + m, one fused multiply-add);
+ * the workspace then holds h as fp16 [T*k][f]
  * followed by the activation rows in sorted pair order as fp16 [T*k][d]; ws
  * must then be 256-byte and x 16-byte aligned (else MOE_ERR_INVALID_ARG).
  */
