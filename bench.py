@@ -411,7 +411,10 @@ def run_ours(args, wl, rank, world, local_rank):
     value = replicas.job_throughput(T * args.steps, world, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "step_ms_quantiles": {"median": float(np.median(step_ms)), "p90": float(np.percentile(step_ms, 90)),
+                              "min": float(np.min(step_ms)), "note": "this rank's per-step CUDA-event times"},
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": ("f16 (dequantised q2) x f16 -> f32" if (not fused and T * wl.k >= 512 and wl.fmt == 2)
                   else "q2xf16->f32" if wl.fmt == 2 else "q3xf16->f32"), "data": "synthetic",
         "config": {"workload": wl.name, "tokens_per_step": T, "l2": "512 MiB write between steps (flushed)",
