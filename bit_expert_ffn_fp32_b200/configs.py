@@ -1,4 +1,4 @@
-"""The five MoE-layer workloads this library is measured and tested on.
+"""The MoE-layer workloads this library is measured and tested on.
 
 Shapes follow the Qwen3.8-Flash-Next MoE block described in "个人开发者用 AI
 十天写出 Strata 引擎，让 12GB 显存跑起 1250 亿参数的 Qwen 3.8 Flash Next"
@@ -47,6 +47,9 @@ WORKLOADS = {
     "tiny_T16_d512_E64_k4_f256_q2": Workload("tiny_T16_d512_E64_k4_f256_q2", 16, 512, 64, 4, 256, 2, zipf=False),
     "decode_T1_d2048_E512_k10_f768_q2": Workload("decode_T1_d2048_E512_k10_f768_q2", 1, 2048, 512, 10, 768, 2),
     "verify_T4_d2048_E512_k10_f768_q3": Workload("verify_T4_d2048_E512_k10_f768_q3", 4, 2048, 512, 10, 768, 3),
+    # wider MTP verify batches (1 token + 1 or 7 drafts), same layer
+    "verify_T2_d2048_E512_k10_f768_q3": Workload("verify_T2_d2048_E512_k10_f768_q3", 2, 2048, 512, 10, 768, 3),
+    "verify_T8_d2048_E512_k10_f768_q3": Workload("verify_T8_d2048_E512_k10_f768_q3", 8, 2048, 512, 10, 768, 3),
     "prefill_T8192_d2048_E512_k10_f768_q2": Workload("prefill_T8192_d2048_E512_k10_f768_q2", 8192, 2048, 512, 10, 768, 2),
     "stack48_T1_d2048_E512_k10_f768_q2_res25": Workload(
         "stack48_T1_d2048_E512_k10_f768_q2_res25", 1, 2048, 512, 10, 768, 2, layers=48, resident=128),
