@@ -235,44 +235,4 @@ __device__ __forceinline__ void build_b_bf16(const uint16_t *src, int qd, int t,
         }
 }
 
-// B fragments of one quad from fp32 activations written earlier by this same
-// grid (read through L2, never the non-coherent path); nullptr = zeros.
-template <int FMT>
-__device__ __forceinline__ void build_b_f32_cg(const float *src, int qd, int t, uint32_t (&B)[4][8], bool &too_big) {
-#pragma unroll
-    for (int bq = 0; bq < 4; ++bq)
-#pragma unroll
-        for (int rho = 0; rho < 8; ++rho) {
-            float lo = 0.f, hi = 0.f;
-            if (src) {
-                const float2 v = __ldcg(reinterpret_cast<const float2 *>(src + 256 * qd + 64 * bq + slot_k(rho, t, 0)));
-                lo = v.x;
-                hi = v.y;
-                too_big |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
-            }
-            const float sc = __int_as_float((127 - slot_exp<FMT>(bq, rho)) << 23);
-            B[bq][rho] = pack_half2(lo * sc, hi * sc);
-        }
-}
-
-// B fragments of one quad from fp32 activations in shared memory; nullptr = zeros.
-template <int FMT>
-__device__ __forceinline__ void build_b_f32_smem(const float *src, int qd, int t, uint32_t (&B)[4][8],
-                                                 bool &too_big) {
-#pragma unroll
-    for (int bq = 0; bq < 4; ++bq)
-#pragma unroll
-        for (int rho = 0; rho < 8; ++rho) {
-            float lo = 0.f, hi = 0.f;
-            if (src) {
-                const float2 v = *reinterpret_cast<const float2 *>(src + 256 * qd + 64 * bq + slot_k(rho, t, 0));
-                lo = v.x;
-                hi = v.y;
-                too_big |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
-            }
-            const float sc = __int_as_float((127 - slot_exp<FMT>(bq, rho)) << 23);
-            B[bq][rho] = pack_half2(lo * sc, hi * sc);
-        }
-}
-
 }  // namespace moe
