@@ -9,6 +9,7 @@ MOE_API const char *moe_status_str(moe_status s) {
         case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or too small";
         case MOE_ERR_CUDA: return "MOE_ERR_CUDA: kernel launch rejected";
         case MOE_ERR_OVERFLOW: return "MOE_ERR_OVERFLOW: size product overflows";
+        case MOE_ERR_HOST: return "MOE_ERR_HOST: host memory or a host thread could not be had";
     }
     return "MOE_ERR_UNKNOWN";
 }

@@ -247,6 +247,8 @@ using namespace moe;
 MOE_API size_t moe_expert_ffn_workspace_bytes(int T, int k, int d, int f) {
     if (T <= 0 || k <= 0 || f <= 0 || d <= 0) return 0;
     const size_t h32 = size_t(T) * size_t(k) * size_t(f) * sizeof(float);
+    if (int64_t(T) * k < kTcMinPairs) return h32;  // only the weight-streaming path can run
+    // the tensor-core path may run (it also needs the fp16 activation rows)
     const size_t tc = tc05_xperm_offset(T, k, f) + size_t(T) * size_t(k) * size_t(d) * 2;
     return std::max(h32, tc);
 }
@@ -284,9 +286,13 @@ namespace moe {
 namespace {
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+void *g_noalloc_ctx[kNoAllocMaxDevices] = {};  // driver context the address belongs to
+using CtxGetCurrentFn = int (*)(void **);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
 
 // Device address of g_noalloc_scratch on the current device, looked up once per
-// device (host code only sees a host-side stand-in under that name).
+// device and driver context (host code only sees a host-side stand-in under
+// that name; after a context is destroyed, its addresses are gone).
 moe_status noalloc_scratch(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -295,13 +301,28 @@ moe_status noalloc_scratch(void **out) {
     }
     if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (!g_ctx_get_current) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 4000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    }
+    void *ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != 0) return MOE_ERR_CUDA;
+    if (!ctx || !g_noalloc_ptr[dev] || g_noalloc_ctx[dev] != ctx) {
+        // (the runtime makes the device's primary context current here if none was)
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
             cudaGetLastError();
             return MOE_ERR_CUDA;
         }
+        if (g_ctx_get_current(&ctx) != 0 || !ctx) return MOE_ERR_CUDA;
         g_noalloc_ptr[dev] = p;
+        g_noalloc_ctx[dev] = ctx;
     }
     *out = g_noalloc_ptr[dev];
     return MOE_OK;

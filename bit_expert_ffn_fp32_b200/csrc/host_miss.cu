@@ -139,6 +139,9 @@ bool matrix_ok(const moe_qmatrix &m, int fmt) {
     return m.codes && m.scale && (fmt == 2 ? m.min != nullptr : m.hi != nullptr);
 }
 
+moe_status complete_misses(int fmt, int d, int f, const moe_qmatrix *experts, const moe_miss *miss, int32_t n,
+                           const uint16_t *x, float *y, int nthreads);
+
 }  // namespace
 }  // namespace moe
 
@@ -160,6 +163,19 @@ MOE_API moe_status moe_complete_misses_host(int fmt, int d, int f, const moe_qma
         const moe_qmatrix *q = experts + size_t(m.expert) * 3;
         if (!matrix_ok(q[0], fmt) || !matrix_ok(q[1], fmt) || !matrix_ok(q[2], fmt)) return MOE_ERR_INVALID_ARG;
     }
+    try {
+        return complete_misses(fmt, d, f, experts, miss, n, x, y, nthreads);
+    } catch (...) {  // host memory or thread creation failed; y is unchanged
+        return MOE_ERR_HOST;
+    }
+}
+
+namespace moe {
+namespace {
+// The validated work of moe_complete_misses_host. May throw (std::bad_alloc,
+// std::system_error) before y is touched; y is written only at the end.
+moe_status complete_misses(int fmt, int d, int f, const moe_qmatrix *experts, const moe_miss *miss, int32_t n,
+                           const uint16_t *x, float *y, int nthreads) {
     // records grouped by expert (stable: record order kept inside a group)
     std::vector<int32_t> order(n);
     for (int32_t i = 0; i < n; ++i) order[i] = i;
@@ -173,7 +189,8 @@ MOE_API moe_status moe_complete_misses_host(int fmt, int d, int f, const moe_qma
 
     std::vector<float> contrib(size_t(n) * d);  // FFN output of record i (without its gate)
     std::atomic<int> next_group{0};
-    auto worker = [&]() {
+    std::atomic<bool> failed{false};
+    auto work = [&]() {
         InputTables tab;
         std::vector<float> xf(d), a(f), u(f), h(f);
         while (true) {
@@ -195,12 +212,25 @@ MOE_API moe_status moe_complete_misses_host(int fmt, int d, int f, const moe_qma
             }
         }
     };
+    auto worker = [&]() {
+        try {
+            work();
+        } catch (...) {
+            failed = true;
+            next_group = ngroups;  // the other workers stop at their next group
+        }
+    };
     const int hw = int(std::max(1u, std::thread::hardware_concurrency()));
     const int nth = std::max(1, std::min(nthreads > 0 ? nthreads : hw, ngroups));
     std::vector<std::thread> pool;
-    for (int t = 1; t < nth; ++t) pool.emplace_back(worker);
+    pool.reserve(nth);
+    try {
+        for (int t = 1; t < nth; ++t) pool.emplace_back(worker);
+    } catch (...) {  // fewer threads than asked: the started ones and this one finish the work
+    }
     worker();
     for (auto &th : pool) th.join();
+    if (failed) return MOE_ERR_HOST;
     for (int32_t i = 0; i < n; ++i) {  // record order: deterministic for any thread count
         float *yr = y + size_t(miss[i].token) * d;
         const float g = miss[i].gate;
@@ -209,3 +239,5 @@ MOE_API moe_status moe_complete_misses_host(int fmt, int d, int f, const moe_qma
     }
     return MOE_OK;
 }
+}  // namespace
+}  // namespace moe

@@ -13,6 +13,8 @@ the host and packed on the device by ``moe_pack_expert``.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
 import numpy as np
@@ -26,8 +28,13 @@ def _t(a, device):
     return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device)
 
 
-def upload_expert(ex: dict, fmt: int, d: int, f: int, dst_ptr: int, device, stream=None) -> None:
-    """Pack one canonical expert (numpy) into the device record at dst_ptr."""
+def upload_expert(ex: dict, fmt: int, d: int, f: int, dst_ptr: int, device, stream=None, sync: bool = True) -> None:
+    """Pack one canonical expert (numpy) into the device record at dst_ptr.
+
+    The canonical arrays are copied to temporary device tensors and packed on
+    the current stream (or ``stream``). With sync=False nothing waits: the
+    temporaries are released to torch's stream-ordered allocator, so later work
+    on the same stream cannot reuse them before the pack kernel has run."""
     keep = []
     mats = []
     for m in ("gate", "up", "down"):
@@ -36,8 +43,11 @@ def upload_expert(ex: dict, fmt: int, d: int, f: int, dst_ptr: int, device, stre
                  _t(None if c["min"] is None else c["min"].view(np.int16), device), _t(c["hi"], device)]
         keep.append(parts)
         mats.append(native.qmatrix(parts[0], parts[1], parts[2], parts[3]))
+    if stream is not None and sync is False:
+        raise ValueError("sync=False packs on the current stream only")
     native.pack_expert(fmt, d, f, mats[0], mats[1], mats[2], dst_ptr, stream)
-    torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+    if sync:
+        torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
     del keep
 
 
@@ -99,10 +109,18 @@ class MoEStack:
             self.slot_of.append(_t(slot, self.device))
             sh = self.L * self.R + l
             self.shared_slot.append(torch.tensor([sh], dtype=torch.int32, device=self.device))
-            for e in range(wl.E):
-                if slot[e] >= 0:
-                    self._pack(l, e, int(slot[e]))
-            self._pack(l, wl.E, sh)
+        # every resident expert and each layer's shared expert: generated on host
+        # threads, packed on the current stream in order, one wait at the end
+        jobs = [(l, e, int(self.slot_of_host[l][e])) for l in range(self.L) for e in range(wl.E)
+                if self.slot_of_host[l][e] >= 0]
+        jobs += [(l, wl.E, self.L * self.R + l) for l in range(self.L)]
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            for c0 in range(0, len(jobs), 64):  # at most 64 generated experts held at once
+                chunk = jobs[c0:c0 + 64]
+                for (l, e, slot), canon in zip(chunk, ex.map(lambda j: self.canonical_expert(j[0], j[1]), chunk)):
+                    upload_expert(canon, wl.fmt, wl.d, wl.f, self.pool.data_ptr() + slot * self.slot_bytes,
+                                  self.device, sync=False)
+        torch.cuda.current_stream().synchronize()
         self._bufs: dict[int, Buffers] = {}
         self._ws: dict = {}
 

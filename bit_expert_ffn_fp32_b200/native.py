@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG, "libmoe.so")
 
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
-                4: "MOE_ERR_CUDA", 5: "MOE_ERR_OVERFLOW"}
+                4: "MOE_ERR_CUDA", 5: "MOE_ERR_OVERFLOW", 6: "MOE_ERR_HOST"}
 DEV_BAD_INDEX, DEV_BAD_SLOT, DEV_NONFINITE, DEV_MISS_OVERFLOW, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
 
 _P = C.c_void_p

@@ -53,7 +53,8 @@ typedef enum moe_status {
     MOE_ERR_UNSUPPORTED = 2, /* shape outside the supported range (see top)   */
     MOE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required    */
     MOE_ERR_CUDA = 4,        /* a kernel launch was rejected by the runtime   */
-    MOE_ERR_OVERFLOW = 5     /* a size product overflows                     */
+    MOE_ERR_OVERFLOW = 5,    /* a size product overflows                     */
+    MOE_ERR_HOST = 6         /* host memory or a host thread could not be had */
 } moe_status;
 
 /* Device-side status bits, OR-ed into *dev_status. */
@@ -200,9 +201,11 @@ moe_status moe_cache_lookup(const int32_t *slot_of, int32_t num_slots, int32_t l
                             const int32_t *sorted_j, int T, int k, int E, int32_t *slot_of_pair, moe_miss *miss,
                             int32_t *miss_count, int32_t miss_cap, int32_t *dev_status, moe_stream_t stream);
 
-/* Workspace bytes moe_expert_ffn_q2/q3 need for (T, k, d, f): the larger of
- * T*k*f fp32 (h, weight-streaming path) and T*k*f fp16 (h, rounded up to
- * 256 B) + T*k*d fp16 (activation rows in sorted order) (tensor-core path). */
+/* Workspace bytes moe_expert_ffn_q2/q3 need for (T, k, d, f). With T*k < 512
+ * only the weight-streaming path can run and the workspace is h as fp32,
+ * T*k*f*4 bytes. With T*k >= 512 the tensor-core path may run, and the size is
+ * the larger of that and T*k*f fp16 (h, rounded up to 256 B) + T*k*d fp16
+ * (activation rows in sorted order). */
 size_t moe_expert_ffn_workspace_bytes(int T, int k, int d, int f);
 
 /*
@@ -260,7 +263,10 @@ moe_status moe_expert_ffn_q3(const moe_qpool *W, const int32_t *slot_of, const u
  *   nthreads   worker threads (0 = the machine's hardware threads)
  * Returns MOE_ERR_INVALID_ARG, before any change to y, for a record with
  * another layer, an expert outside [0, E), a token outside [0, T) or an expert
- * whose matrices are missing (NULL codes/scale, min for Q2, hi for Q3).
+ * whose matrices are missing (NULL codes/scale, min for Q2, hi for Q3), and
+ * MOE_ERR_HOST, with y unchanged, if host memory for the per-record results
+ * cannot be had. If fewer threads than asked can be started, the call finishes
+ * the work on those it has.
  * Blocking; no GPU involvement.
  */
 moe_status moe_complete_misses_host(int fmt, int d, int f, const moe_qmatrix *experts, int E, const moe_miss *miss,
@@ -358,11 +364,15 @@ moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t 
  *   plus an fp16 copy of x on the tensor-core path) goes to one 4 MiB array
  *   built into the library; each GPU that loads the library holds its own copy
  *   until the process exits. moe_expert_ffn_workspace_bytes(T, k, d, f) > 4 MiB
- *   returns MOE_ERR_WORKSPACE (for d = 2048, f = 768, k = 10: T*k <= 1365),
- *   before anything is enqueued.
+ *   returns MOE_ERR_WORKSPACE before anything is enqueued. For d = 2048,
+ *   f = 768 that admits T*k <= 744: below 512 pairs the scratch holds
+ *   T*k*f*4 bytes of h; from 512 pairs on the tensor-core layout needs
+ *   T*k*(2f + 2d) bytes (5,632 per pair), and 744 * 5,632 <= 4 MiB < 745 * 5,632.
  *   Set-up: the first call on a device looks up that device's copy of the
  *   array (cudaGetSymbolAddress, with the device current); make that first call
- *   before any stream capture. Lookup failures return MOE_ERR_CUDA.
+ *   before any stream capture. The address is kept per device and driver
+ *   context and looked up again when a call runs in a context it has not seen
+ *   (for example after cudaDeviceReset). Lookup failures return MOE_ERR_CUDA.
  *   Sharing: every call on a device uses the same array, which keeps whatever
  *   the last call wrote (nothing in it needs to start at zero: each call writes
  *   every entry it reads). Calls that can overlap on the GPU -- on different

@@ -223,20 +223,32 @@ def layer(x: np.ndarray, Wr: np.ndarray, bias, get_expert, shared: dict, k: int,
     if slot_of is None:
         slot_of = np.arange(E, dtype=np.int32)
     sop, misses, nmiss = cache_lookup(slot_of, layer_id, idx, gate, E, miss_cap)
-    toks = range(T) if tokens is None else list(tokens)
+    toks = list(range(T)) if tokens is None else list(tokens)
     xf = bf16_to_f64(x)
     y_part = np.full((T, d), np.nan)
     y_full = np.full((T, d), np.nan)
+    # Every needed FFN_e(x_t) is evaluated once, one expert at a time (so that
+    # only one expert's fp64 matrices are held at once); the per-token sums
+    # below then add them in the definition's order.
+    ffn: dict[tuple[int, int], np.ndarray] = {}
+    need: dict[int, list[int]] = {}
+    for t in toks:
+        for j in range(k):
+            need.setdefault(int(idx[t, j]), []).append(t)
+    for e in sorted(need):
+        W = dequant_expert(get_expert(e), fmt)
+        ts = sorted(set(need[e]))
+        rows = expert_ffn(W, xf[ts])
+        for i, t in enumerate(ts):
+            ffn[(e, t)] = rows[i]
+        del W
     Wsh = dequant_expert(shared, fmt)
-    memo: dict[int, dict] = {}
     for t in toks:
         acc_hit = expert_ffn(Wsh, xf[t])[0]
         acc_all = acc_hit.copy()
         for j in range(k):
             e = int(idx[t, j])
-            if e not in memo:
-                memo[e] = dequant_expert(get_expert(e), fmt)
-            ye = gate[t, j] * expert_ffn(memo[e], xf[t])[0]
+            ye = gate[t, j] * ffn[(e, t)]
             acc_all = acc_all + ye
             if slot_of[e] >= 0:
                 acc_hit = acc_hit + ye

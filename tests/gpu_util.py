@@ -52,3 +52,23 @@ def check_routing(b, ref, T: int, k: int, E: int):
     na = int(p["active"][0])
     np.testing.assert_array_equal(b.active[: na + 1].cpu().numpy(), p["active"][: na + 1])
     np.testing.assert_array_equal(b.sop[: T * k].cpu().numpy(), ref["slot_of_pair"])
+
+
+def oracle_pair_rows(stack: MoEStack, layer: int, x_bits: np.ndarray, perm: dict, positions) -> np.ndarray:
+    """The oracle's y_e row (expert output before the gate) of every sorted pair
+    position in `positions`, from the oracle's own permutation `perm`; each
+    expert is dequantised once (fp64 [len(positions)][d])."""
+    wl = stack.wl
+    xf = orc.bf16_to_f64(x_bits)
+    offs = perm["offsets"]
+    positions = list(positions)
+    out = np.empty((len(positions), wl.d), np.float64)
+    by_e: dict[int, list[int]] = {}
+    for i, s in enumerate(positions):
+        e = int(np.searchsorted(offs, s, side="right") - 1)
+        by_e.setdefault(e, []).append(i)
+    for e, rows in by_e.items():
+        W = orc.dequant_expert(stack.canonical_expert(layer, e), wl.fmt)
+        toks = [int(perm["sorted_tok"][positions[i]]) for i in rows]
+        out[rows] = orc.expert_ffn(W, xf[toks])
+    return out

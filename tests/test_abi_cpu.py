@@ -97,6 +97,24 @@ def test_host_validation_rejects_before_launch():
     assert L.moe_pack_expert(3, 2048, 768, C.byref(q), C.byref(q), C.byref(q), dummy * 256, None) == 1
 
 
+def test_expert_ffn_workspace_per_path_and_noalloc_limit():
+    """Below 512 pairs only the weight-streaming path runs (h as fp32); from 512
+    pairs on the tensor-core layout (fp16 h + fp16 activation rows) is included.
+    The allocation-free call's 4 MiB array therefore takes up to 744 pairs at
+    d=2048, f=768, and 745 pairs are refused before any CUDA call."""
+    d, f = 2048, 768
+    assert native.expert_ffn_workspace_bytes(1, 10, d, f) == 10 * f * 4
+    assert native.expert_ffn_workspace_bytes(51, 10, d, f) == 510 * f * 4
+    assert native.expert_ffn_workspace_bytes(512, 1, d, f) == 512 * (2 * f + 2 * d)
+    lim = 4 << 20
+    assert native.expert_ffn_workspace_bytes(744, 1, d, f) <= lim < native.expert_ffn_workspace_bytes(745, 1, d, f)
+    pool = native.QPool(0x1000 * 256, 1474560, 10, 2, d, f)
+    dummy = 0x1000
+    rc = native.lib.moe_expert_ffn_q2_noalloc(C.byref(pool), dummy, dummy, 745, d, f, 512, 1, dummy, dummy, dummy,
+                                              dummy, None, dummy, None, None)
+    assert rc == 3
+
+
 def _canon(fmt, d, f, seed):
     return synth.gen_expert(seed, 0, 0, fmt, d, f)
 

@@ -107,6 +107,20 @@ def test_fused_verify_q3(verify):
         _check(verify, 0, synth.gen_x(0, 0, 4, configs.VERIFY.d, stream=s))
 
 
+@pytest.mark.parametrize("T", [2, 8])
+def test_fused_verify_q3_wider_batches(verify, T):
+    """MTP verify batches of one token plus 1 or 7 drafts on Q3 experts."""
+    for s in range(2):
+        _check(verify, 0, synth.gen_x(0, 0, T, configs.VERIFY.d, stream=700 + 10 * T + s))
+
+
+@pytest.mark.parametrize("T", [2, 4, 8])
+def test_fused_decode_q2_batches(decode, T):
+    """Q2 layer with 2, 4 and 8 tokens (several tokens per expert), against the oracle."""
+    for s in range(2):
+        _check(decode, 0, synth.gen_x(0, 0, T, configs.DECODE.d, stream=800 + 10 * T + s))
+
+
 def test_fused_with_misses():
     wl = configs.STACK48
     stack = MoEStack(wl, layers=3)

@@ -10,7 +10,7 @@ import torch
 
 from bit_expert_ffn_fp32_b200 import configs, native, synth
 from bit_expert_ffn_fp32_b200.layer import MoEStack, x_tensor
-from gpu_util import OUT_TOL, check_routing, oracle_layer, rel_err, run_layer
+from gpu_util import OUT_TOL, check_routing, oracle_layer, oracle_pair_rows, rel_err, run_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -101,15 +101,40 @@ def test_verify_layer_q3(verify):
         _full_check(verify, 0, x)
 
 
-def test_prefill_chunk_routing_and_sampled_outputs():
+def test_prefill_chunk_every_tile_against_the_oracle():
+    """8192-token prefill chunk (tcgen05 grouped GEMMs). Routing, permutation and
+    slots bit-exact for every token; y against the oracle at 64 tokens; and the
+    routed experts' output rows y_e (before the gate) against the oracle's
+    expert FFN at the first and the last pair of every (expert, 192-token N
+    tile) of the persistent schedule, plus every pair of the most loaded expert."""
     wl = configs.PREFILL
     stack = MoEStack(wl)
     x = synth.gen_x(0, 0, wl.T, wl.d)
     rng = np.random.default_rng(0)
-    toks = sorted(set([0, wl.T - 1] + list(rng.choice(wl.T, 4, replace=False))))
+    toks = sorted(set([0, wl.T - 1] + [int(t) for t in rng.choice(wl.T, 62, replace=False)]))
     b, ref, err = _full_check(stack, 0, x, tokens=toks)
-    counts = b.counts.cpu().numpy()
+    assert len(toks) >= 64
+    perm = ref["perm"]
+    counts, offs = perm["counts"], perm["offsets"]
     assert counts.sum() == wl.T * wl.k and counts.max() > 500     # Zipf skew present
+    tn = 192                                                      # tokens per N tile
+    pos = set()
+    for e in range(wl.E):
+        for i0 in range(0, int(counts[e]), tn):
+            pos.add(int(offs[e]) + i0)
+            pos.add(int(offs[e]) + min(i0 + tn, int(counts[e])) - 1)
+    big = int(np.argmax(counts))
+    pos |= set(range(int(offs[big]), int(offs[big + 1])))
+    pos = sorted(pos)
+    want = oracle_pair_rows(stack, 0, x, perm, pos)
+    got = b.y_perm[torch.tensor(pos, dtype=torch.long, device=b.y_perm.device)].cpu().numpy().astype(np.float64)
+    pos_a = np.array(pos)
+    expert_of = np.searchsorted(offs, pos_a, side="right") - 1
+    worst = 0.0
+    for e in np.unique(expert_of):
+        sel = expert_of == e
+        worst = max(worst, rel_err(got[sel], want[sel]))
+    assert worst <= OUT_TOL, worst
 
 
 def test_stack48_cache_and_misses():

@@ -32,9 +32,23 @@ def _routed(stack, x, T):
     return b
 
 
-@pytest.mark.parametrize("wl,T", [(configs.TINY, 16), (configs.DECODE, 4)], ids=["tiny_T16", "decode_T4"])
+_STACKS = {}
+
+
+def _stack(wl):
+    # one pool per workload for the whole file (building the 512-expert pool takes a while)
+    if wl.name not in _STACKS:
+        _STACKS[wl.name] = MoEStack(wl)
+    return _STACKS[wl.name]
+
+
+@pytest.mark.parametrize("wl,T", [(configs.TINY, 16), (configs.DECODE, 4), (configs.DECODE, 64)],
+                         ids=["tiny_T16", "decode_T4", "decode_T64_tensor_core"])
 def test_noalloc_matches_workspace_call_twice(wl, T):
-    stack = MoEStack(wl)
+    """T*k = 64 and 40 pairs run the weight-streaming kernels; 640 pairs (between
+    512 and the 744-pair limit at d=2048, f=768) run the tensor-core GEMMs with
+    h and the fp16 activation rows in the built-in array."""
+    stack = _stack(wl)
     for call in range(2):
         x = x_tensor(synth.gen_x(wl.seed, 0, T, wl.d, stream=500 + call), stack.device)
         b = _routed(stack, x, T)
@@ -52,11 +66,25 @@ def test_noalloc_matches_workspace_call_twice(wl, T):
         assert np.all(np.isfinite(ref)) and np.all(np.isfinite(got))
         err = np.max(np.abs(got - ref)) / np.max(np.abs(ref))
         assert err <= OUT_TOL, (call, err)
+        if T * wl.k >= 512:  # the tensor-core range also against the oracle, at every 16th sorted pair
+            import oracle as orc
+            from gpu_util import oracle_pair_rows
+
+            x_bits = synth.gen_x(wl.seed, 0, T, wl.d, stream=500 + call)
+            l32, _, _ = orc.router(x_bits, synth.gen_router(wl.seed, 0, wl.E, wl.d),
+                                   None if stack.bias[0] is None else stack.bias[0].cpu().numpy())
+            idx, _ = orc.topk(l32, wl.k)
+            perm = orc.permute(idx, wl.E)
+            np.testing.assert_array_equal(b.sorted_tok[:n].cpu().numpy(), perm["sorted_tok"])
+            pos = sorted(set(range(0, n, 16)) | {n - 1})
+            want = oracle_pair_rows(stack, 0, x_bits, perm, pos)
+            err_o = np.max(np.abs(got[pos] - want)) / np.max(np.abs(want))
+            assert err_o <= OUT_TOL, (call, err_o)
 
 
 def test_noalloc_refuses_more_than_its_scratch():
     wl = configs.DECODE
-    stack = MoEStack(wl.with_(E=16, k=4), layers=1)
+    stack = MoEStack(wl.with_(E=16, k=4, resident=-1), layers=1)
     T = 2048                      # 2048 * 4 * 768 * 4 B = 24 MiB > 4 MiB
     dummy = torch.zeros(8, dtype=torch.int32, device="cuda")
     with pytest.raises(native.MoeError) as ei:
