@@ -290,7 +290,7 @@ class Evictor:
 
     def __call__(self, i):
         self.w.fill_(float(i))
-        self.torch.sum(self.r, dtype=self.torch.float32, out=self.out)
+        self.torch.sum(self.r, 0, out=self.out)
 
 
 def measure(wl, stack, args, rank, world, local_rank, dev, evict):
