@@ -251,7 +251,7 @@ def run_reference(args, wl, rank):
 MISS_DTYPE = [("layer", "<i4"), ("expert", "<i4"), ("token", "<i4"), ("j", "<i4"), ("gate", "<f4")]
 
 
-def _time_host_misses(stack, wl, bufs, x_step):
+def _time_host_misses(stack, wl, sb, x_step):
     """moe_complete_misses_host over one step's miss lists (all layers), the
     missed experts in canonical host storage (generated first, not timed), the
     completion of every layer timed on the host clock with all threads."""
@@ -260,10 +260,10 @@ def _time_host_misses(stack, wl, bufs, x_step):
     L, T = wl.layers, wl.T
     work, n_rec, n_exp = [], 0, 0
     for l in range(L):
-        recs = np.array(stack.misses(bufs[l]), dtype=MISS_DTYPE)
+        recs = np.array(stack.stack_misses(sb, l), dtype=MISS_DTYPE)
         if len(recs) == 0:
             continue
-        y = np.ascontiguousarray(bufs[l].y[:T].cpu().numpy())
+        y = np.ascontiguousarray(sb.y[l, :T].cpu().numpy())
         canon = {e: stack.canonical_expert(l, e) for e in sorted(set(recs["expert"].tolist()))}
         work.append((l, recs, y, canon, native.expert_table(wl.E, canon), np.ascontiguousarray(x_step[l])))
         n_rec += len(recs)
@@ -302,7 +302,7 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
     from bit_expert_ffn_fp32_b200.layer import x_tensor
 
     L, T = wl.layers, wl.T
-    bufs = [stack.buffers(T)] + [stack.buffers(T, fresh=True) for _ in range(L - 1)]
+    bufs = [stack.buffers(T)]
     b = bufs[0]
     stream = torch.cuda.current_stream()
     steps, warmup = args.steps, args.warmup
@@ -316,14 +316,18 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
     xs = lambda i: xs_dev[i % n_x]  # noqa: E731
 
     fused = T <= 8
+    stacked = fused and L > 1  # all layers in one moe_stack_decode launch
+    sb = stack.stack_buffers(T) if stacked else None
     k, E, d, f = wl.k, wl.E, wl.d, wl.f
 
     def layer_step(xset, evs=None):
         if fused:
             if evs:
                 evs[0].record(stream)
-            for l in range(L):
-                stack.forward_fused(l, xset[l], bufs[l])
+            if stacked:
+                stack.forward_stack(xset, sb)
+            else:
+                stack.forward_fused(0, xset[0], b)
             if evs:
                 evs[1].record(stream)
             return
@@ -346,10 +350,11 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
     tc_path = T * wl.k >= 512 and wl.fmt == 2
     ffn_launches = 3 if tc_path else 2  # (+ the fp16 gather on the tensor-core path)
     perm_launches = 1 if native.permute_workspace_bytes(T, wl.k, wl.E) == 0 else 3
-    launches_per_step = L if fused else 2 + perm_launches + 1 + 2 * ffn_launches + 1
+    launches_per_step = 1 if fused else 2 + perm_launches + 1 + 2 * ffn_launches + 1
+    statuses = [sb.status] if stacked else [bl.status for bl in bufs]
 
-    for bl in bufs:
-        bl.status.zero_()
+    for st in statuses:
+        st.zero_()
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     ev = [(mk(), mk()) for _ in range(steps)]
     if world > 1:
@@ -383,8 +388,8 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
         torch.cuda.synchronize()
         kern_ms = [kev[i][0].elapsed_time(kev[i][1]) for i in range(steps)]
     status = 0
-    for bl in bufs:
-        status |= int(bl.status.item())
+    for st in statuses:
+        status |= int(st.item())
 
     # distinct resident experts, resident pairs and misses of each step's routing,
     # summed over the layers (not timed)
@@ -392,7 +397,16 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
     for i in range(min(steps, (64 if T <= 64 else 4) if L == 1 else 4)):
         layer_step(xs(warmup + i))
         a_sum = p_sum = m_sum = 0
-        for l, bl in enumerate(bufs):
+        if stacked:
+            idx_h = sb.idx[:, : T * wl.k].cpu().numpy()
+            sop_h = sb.sop[:, : T * wl.k].cpu().numpy()
+            mc_h = sb.miss_count.cpu().numpy()
+            for l in range(L):
+                ids = np.unique(idx_h[l])
+                a_sum += int((stack.slot_of_host[l][ids] >= 0).sum())
+                p_sum += int((sop_h[l] >= 0).sum())
+                m_sum += int(mc_h[l])
+        for l, bl in enumerate(bufs if not stacked else []):
             na = int(bl.active[0].item())
             ids = bl.active[1:1 + na].cpu().numpy()
             a_sum += int((stack.slot_of_host[l][ids] >= 0).sum())
@@ -419,7 +433,9 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
         e2e_ev[i][0].record(stream)
         x_dev.copy_(x_pin[i % n_x], non_blocking=True)
         layer_step(x_dev)
-        for l in range(L):
+        if stacked:
+            y_pin[i % n_y].copy_(sb.y[:, :T], non_blocking=True)
+        for l in range(L if not stacked else 0):
             y_pin[i % n_y, l].copy_(bufs[l].y[:T], non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
@@ -444,13 +460,13 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
     else:
         kb = layer_bytes if fused else ffn_bytes
         roof = {"bound": "hbm",
-                "kernel": ("decode_layer_kernel (moe_layer_decode: whole layer, one launch per layer"
-                           + (f", {L} launches per step" if L > 1 else "") + ")") if fused else
+                "kernel": ("decode_layer_kernel (moe_stack_decode: %d layers in one launch)" % L if stacked else
+                           "decode_layer_kernel (moe_layer_decode: whole layer, one launch)") if fused else
                           "moe_expert_ffn_q%d (gate/up + down, routed + shared)" % wl.fmt,
                 "achieved": kb / kern_avg_s / 1e9, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                 "frac": kb / kern_avg_s / 1e9 / hbm_peak, "traffic": traffic,
                 "traffic_scope": "DRAM bytes per step (all launches of the step)",
-                "bytes_per_launch": kb / (L if fused else 1), "avg_launch_us": kern_avg_s * 1e6 / (L if fused else 1)}
+                "bytes_per_launch": kb, "avg_launch_us": kern_avg_s * 1e6}
     line = {
         "value": replicas.job_throughput(T * steps, world, total_ms), "unit": "tokens/s",
         "ms_per_step": total_ms / steps,
@@ -461,8 +477,8 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
                   else "q2xf16->f32" if wl.fmt == 2 else "q3xf16->f32"),
         "config": {"workload": wl.name, "tokens_per_step": T,
                    "l2": "512 MiB write + 256 MiB read of other buffers between steps (flushed, clean)",
-                   "path": "moe_layer_decode (one launch per layer)" if fused else
-                   "step-by-step calls, y_perm + moe_combine",
+                   "path": ("moe_stack_decode (all layers, one launch)" if stacked else
+                            "moe_layer_decode (one launch)") if fused else "step-by-step calls, y_perm + moe_combine",
                    "parallelism": f"replicas x{world}", "layers_per_step": L,
                    "step_algorithmic_bytes": layer_bytes,
                    "step_GBps": layer_bytes / (total_ms / steps / 1e3) / 1e9,
@@ -473,8 +489,8 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
                 "h2d_bytes_per_step": L * T * wl.d * 2, "d2h_bytes_per_step": L * T * wl.d * 4},
         "clocks": clocks, "gpu_launches": launches_per_step * steps, "dev_status": status,
     }
-    if L > 1 and not args.no_host_misses and rank == 0:
-        line["host_miss_completion"] = _time_host_misses(stack, wl, bufs, xs_host[(steps - 1) % n_x])
+    if stacked and not args.no_host_misses and rank == 0:
+        line["host_miss_completion"] = _time_host_misses(stack, wl, sb, xs_host[(steps - 1) % n_x])
     return line
 
 

@@ -1,5 +1,6 @@
-// One whole MoE layer for a few tokens (decode, MTP verify) in one
-// cooperative launch.
+// Whole MoE layers for a few tokens (decode, MTP verify) in one cooperative
+// launch of thread-block clusters: one layer (moe_layer_decode) or a stack of
+// layers (moe_stack_decode).
 //
 // Per token the router scores the layer's experts, the top k (10 of 512 in
 // "个人开发者用 AI 十天写出 Strata 引擎，让 12GB 显存跑起 1250 亿参数的 Qwen 3.8 Flash
@@ -7,23 +8,35 @@
 // 2/3-bit weights, hot experts are read from an HBM pool and the rest are
 // reported as misses ("5070ti16g单卡跑qwen 3.8 flash next 新方案最高90t/s Hermes
 // 调用60t/s", section "为什么从 18t/s 变成 60-90t/s"), and the always-on shared expert
-// is added. With T <= 8 tokens the layer reads ~20 MB and does little arithmetic,
-// so it is bound by HBM and by latency; this kernel keeps every SM streaming:
+// is added. With T <= 8 tokens a layer reads ~20 MB and does little
+// arithmetic: it is bound by HBM and by the chain router -> top-k -> expert
+// weights -> hidden -> down. Per layer:
 //
-//  A  (no routing needed)  router logits for all experts, the shared expert's
-//     gate/up, zeroing of y -- all CTAs at once;
-//     grid barrier (logits complete);
-//  B  every CTA computes the top-k, gates and permutation itself from the
-//     logits in L2 (no second barrier), CTA 0 writes them out, and every CTA
-//     issues L2 bulk prefetches for the expert rows its later tasks read, so
-//     HBM streams the selected experts at once;
-//  C  routed gate/up tasks (expert, 16-row group): h = silu(Wg x) * (Wu x) into
-//     scratch, then a per-expert completion counter;
-//  D  down tasks (expert or shared, 16-row group) wait for their expert's
-//     counter, compute Wd h and add gate * y_e into y with atomics.
+//  router  every CTA bulk-copies its ~E/G router rows (and the activations)
+//          into shared memory, computes those logits in the fixed fp32 order
+//          and arrives at a grid barrier; meanwhile the clusters whose first
+//          task is a shared-expert task start copying its weights, and every
+//          CTA asks the L2 for its slice of the next layer's router rows and
+//          shared expert;
+//  top-k   after the barrier every CTA selects the top k of every token from
+//          the logits (a CTA-wide selection, identical in all CTAs) and builds
+//          the routing tables and the task list itself;
+//  tasks   a task is (expert, block of HB hidden rows): HB = 128 for Q2 (one
+//          block pair of the down matrix) and 256 for Q3 (one block quad).
+//          The C CTAs of a cluster split a task: CTA r computes the gate/up
+//          partial sums of the HB rows over its d/C slice of K, the partials
+//          are exchanged through distributed shared memory (one cluster
+//          barrier), every CTA forms h = silu(a) * u for the HB rows, and CTA
+//          r computes down rows [r d/C, (r+1) d/C) over the HB columns and
+//          adds gate * y_e into y with vector atomics. No task waits for
+//          another cluster. The weights of a task stream into per-warp slices
+//          of a shared-memory ring with bulk copies (each warp copies and
+//          waits for its own rows), the next task's copies issued as soon as
+//          a warp's slice is free.
 //
-// Every wait is bounded (MOE_DEV_TIMEOUT after 100 ms) and the last CTA to
-// leave resets the counters, so the workspace stays zeroed between launches.
+// Every wait on another CTA or on a copy is bounded (MOE_DEV_TIMEOUT after
+// 100 ms); the last CTA to leave resets the grid counters, so the workspace
+// stays zeroed between launches.
 #include <algorithm>
 #include <math.h>
 #include <mutex>
@@ -33,20 +46,13 @@
 #include "mma_q.cuh"
 
 // Optional phase timestamps (build with -DMOE_DECODE_TRACE): thread 0 of every
-// CTA records %globaltimer at each phase boundary into moe_decode_trace.
+// CTA records %globaltimer at each phase boundary of the first layer into
+// moe_decode_trace.
 #ifdef MOE_DECODE_TRACE
 __device__ unsigned long long moe_decode_trace[4096 * 32];
 #define TRACE(i)                                                                                      \
     do {                                                                                              \
-        if (threadIdx.x == 0) {                                                                       \
-            unsigned long long t_;                                                                    \
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                    \
-            moe_decode_trace[blockIdx.x * 32 + (i)] = t_;                                             \
-        }                                                                                             \
-    } while (0)
-#define TRACEW(i)                                                                                     \
-    do {                                                                                              \
-        if ((threadIdx.x & 31) == 0) {                                                                \
+        if (threadIdx.x == 0 && l == 0) {                                                             \
             unsigned long long t_;                                                                    \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                    \
             moe_decode_trace[blockIdx.x * 32 + (i)] = t_;                                             \
@@ -56,91 +62,89 @@ __device__ unsigned long long moe_decode_trace[4096 * 32];
 #define TRACE(i) \
     do {         \
     } while (0)
-#define TRACEW(i) \
-    do {          \
-    } while (0)
 #endif
 
 namespace moe {
 namespace {
 
-#ifndef MOE_DECODE_CTAS_PER_SM
-#define MOE_DECODE_CTAS_PER_SM 1
-#endif
-constexpr int kCtasPerSm = MOE_DECODE_CTAS_PER_SM;  // resident CTAs per SM (register budget)
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxTokDec = 8;
 constexpr int kMaxEDec = 512;
 constexpr int kMaxPairs = kMaxTokDec * kMaxK;  // 128
-constexpr int kSharedIdx = kMaxPairs;         // done[] slot of the shared expert
 constexpr int kMaxDimDec = 2048;
-constexpr int kCandMax = 64;  // candidates ranked in shared memory; more take the round-based path
+constexpr int kMaxFDec = 4096;
 constexpr unsigned long long kWaitNs = 100ull * 1000 * 1000;
 constexpr unsigned long long kWaitSteps = 1ull << 27;  // polls: >= 4 s of 32 ns sleeps
-constexpr int kMaxSlots = 8;  // weight-ring slots at most
-constexpr int kMaxFDec = 1024;  // expert width f (h staging and B fragments)
-constexpr int kCBatch = 4;      // gate/up units computed in one pass (one token)
-static_assert(kCBatch * kWarps * 2 * 16 <= kWarps * 2 * 4 * 32, "batched partials fit in red[]");
-static_assert(kMaxSlots <= kWarps, "one warp announces each initial ring unit");
+constexpr int kMaxBuf = 2;                             // task buffers in the weight ring
 
-// Dynamic shared memory: T*d bf16 activations, T rows of h (fp32), then the
-// weight ring from this 128-byte aligned offset.
-__host__ __device__ inline size_t ring_off(int T, int d, int f) {
-    return ((((size_t(T) * d * 2 + 15) & ~size_t(15)) + size_t(T) * f * 4) + 127) & ~size_t(127);
-}
+// Geometry of one launch (host-computed; see plan()).
+struct Geo {
+    int C;        // CTAs per cluster: K of gate/up and the rows of down are split C ways
+    int HB;       // hidden rows per task (128 Q2, 256 Q3)
+    int NHB;      // tasks per expert, f / HB
+    int KR;       // gate/up K columns per CTA, d / C
+    int NQR;      // 256-column quads per CTA, KR / 256
+    int DR;       // down rows per CTA, d / C
+    int NDRW;     // down row groups per warp, DR / 16 / 8
+    int GUW;      // gate/up row groups per warp, HB / 16 / 8
+    uint32_t gu_c, gu_s;  // codes / scales bytes of one gate/up row group (one matrix) over KR
+    uint32_t dn_c, dn_s;  // codes / scales bytes of one down row group over the task's HB columns
+    uint32_t gu_warp, dn_warp, region;  // per-warp slices and one task buffer (8 warps)
+    int nbuf;             // task buffers in the ring
+    uint32_t part_bytes;  // one partial-sum buffer (also the down-result staging)
+    // dynamic shared memory offsets
+    uint32_t off_bfx, off_part, off_h, off_bfh, off_ring, total;
+};
 
 struct DecodeParams {
     const uint8_t *pool;
     int64_t slot_bytes;
     int num_slots;
-    const int32_t *slot_of;
-    int shared_slot;
-    int layer;
-    const uint16_t *x;
-    const float *Wr;
-    const float *bias;
+    int L;                       // layers in this launch
+    const int32_t *slot_of;      // [L][E]
+    const int32_t *shared_slot;  // [L] (device), or NULL: shared_slot0 for the one layer
+    int shared_slot0;
+    int layer0;                  // layer id of the first layer (miss records)
+    const uint16_t *x;           // [L][T][d]
+    const float *Wr;             // [L][E][d]
+    const float *bias;           // [L][E] or NULL
     int T, d, f, E, k;
-    float *logits;
-    int32_t *topk_idx;
+    float *logits;               // [2][T][E] workspace, or [T][E] output for L == 1
+    bool logits_out;
+    int32_t *topk_idx;           // [L][T*k] or NULL
     float *topk_w;
-    int32_t *counts, *offsets, *sorted_tok, *sorted_j, *inv, *active, *slot_of_pair;
-    moe_miss *miss;
-    int32_t *miss_count;
+    int32_t *counts, *offsets, *sorted_tok, *sorted_j, *inv, *active;  // L == 1 only (else NULL)
+    int32_t *slot_of_pair;       // [L][T*k] or NULL
+    moe_miss *miss;              // [L][miss_cap] or NULL
+    int32_t *miss_count;         // [L] or NULL
     int miss_cap;
-    float *y;
+    float *y;                    // [L][T][d]
     int32_t *status;
-    unsigned *ctr;   // [0] barrier arrivals, [1] CTAs finished
-    unsigned *done;  // [kMaxPairs + 1] gate/up tasks finished per resident expert
-    float *h;        // [(T*k + T)][f]: sorted pair rows, then shared-expert rows
+    unsigned *ctr;               // [0] barrier arrivals, [1] CTAs finished
     MatGeom gate, up, down;
-    // shared-memory weight ring of phases C and D: nslots slots of rslot bytes;
-    // per row group, the codes and scales bytes of gate/up (gu_*) and down (dn_*)
-    int nslots;
-    uint32_t rslot, gu_cb, gu_sb, dn_cb, dn_sb;
+    Geo g;
 };
 
 struct Smem {
-    float xs[kMaxDimDec / 64][kMaxTokDec];  // block sums of x per token
-    float red[kWarps][2][4][32];            // split-K partials of gate/up
     int slot[kMaxEDec];                     // this layer's expert -> slot table
     int idx[kMaxTokDec][kMaxK];
     float w[kMaxTokDec][kMaxK];
+    uint64_t wl[kWarps][kMaxK];             // per-warp top-k lists (keys)
+    uint64_t sel[kMaxTokDec][kMaxK];        // merged top-k per token, best first
     int pair_e[kMaxPairs];                  // expert of sorted pair s
     int s_tok[kMaxPairs], s_j[kMaxPairs];   // sorted pairs
     int inv[kMaxPairs];
     int act_e[kMaxPairs], act_beg[kMaxPairs], act_cnt[kMaxPairs], act_slot[kMaxPairs], act_mbase[kMaxPairs];
     int res[kMaxPairs];                     // active index of each resident expert
-    float hsb[kMaxFDec / 64][kMaxTokDec];   // block sums of the staged h rows
-    uint64_t cand[kMaxTokDec][kCandMax];    // top-k candidates per token
-    float sel_v[kMaxTokDec][kMaxK];
-    int sel_id[kMaxTokDec][kMaxK];
-    unsigned first_mask[kMaxPairs / 32];    // pair s starts a new expert
-    uint64_t full[kMaxSlots];               // weight ring: slot filled (bulk-copy bytes landed)
-    // B fragments of the staged h rows, built once per down unit and shared by
-    // every warp: quad qd, fragment registers 4*r4..4*r4+3, lane: [qd][r4][lane]
-    uint4 bfrag[kMaxFDec / 256][8][32];
-    int nact, nres, nmiss;
+    unsigned first_mask[kMaxPairs / 32];
+    float xs[kMaxDimDec / 64][kMaxTokDec];  // block sums of x over this CTA's K slice
+    float hsb[4][kMaxTokDec];               // block sums of the task's h columns
+    float gsel[kMaxTokDec];                 // gate of each token for the current task (0 = not routed)
+    uint64_t rt_bar;                        // router rows landed
+    uint64_t gu_bar[kMaxBuf][kWarps];       // per-warp gate/up slice landed
+    uint64_t dn_bar[kMaxBuf][kWarps];       // per-warp down slice landed
+    int nact, nres, nmiss, ntask;
     int ok, last;
 };
 
@@ -175,19 +179,22 @@ __device__ bool wait_geq(const unsigned *p, unsigned target, int32_t *status) {
     return true;
 }
 
-// Weight ring: bulk copies global -> this CTA's shared memory that complete
-// on an mbarrier (transaction bytes), and a bounded wait for a slot's phase.
+// Bulk copies global -> this CTA's shared memory that complete on an
+// mbarrier (transaction bytes), and a bounded wait for an mbarrier phase.
 __device__ __forceinline__ uint32_t saddr(const void *p) { return uint32_t(__cvta_generic_to_shared(p)); }
-__device__ __forceinline__ void ring_expect(uint64_t *bar, uint32_t bytes) {
+__device__ __forceinline__ void bar_init(uint64_t *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_expect(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void ring_copy(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+__device__ __forceinline__ void bulk_copy(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                      saddr(dst)),
                  "l"(src), "r"(bytes), "r"(saddr(bar))
                  : "memory");
 }
-__device__ __forceinline__ bool ring_test(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool bar_test(uint64_t *bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
         "{\n.reg .pred q;\nmbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\nselp.u32 %0, 1, 0, q;\n}"
@@ -197,14 +204,56 @@ __device__ __forceinline__ bool ring_test(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 // false after kWaitNs, or kWaitSteps polls (the caller flags MOE_DEV_TIMEOUT)
-__device__ bool ring_wait(uint64_t *bar, uint32_t parity) {
-    if (ring_test(bar, parity)) return true;
+__device__ bool bar_wait(uint64_t *bar, uint32_t parity) {
+    if (bar_test(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
-    for (unsigned long long it = 0; !ring_test(bar, parity); ++it) {
+    for (unsigned long long it = 0; !bar_test(bar, parity); ++it) {
         if (globaltimer() - t0 > kWaitNs || it > kWaitSteps) return false;
         if (it > 1024) __nanosleep(32);
     }
     return true;
+}
+
+// Cluster helpers: this CTA's rank, and every thread's arrival + wait at the
+// cluster barrier (hardware; each CTA of a cluster runs the same sequence of
+// cluster barriers on every path, so each one completes).
+__device__ __forceinline__ unsigned cluster_rank() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ unsigned cluster_id() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ unsigned cluster_count() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory object in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t peer_addr(const void *p, unsigned rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_peer(uint32_t a) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ int ld_peer_int(uint32_t a) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_add4(float *p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
 }
 
 // One CTA runs the two waits above against objects nothing completes (a device
@@ -217,8 +266,9 @@ __global__ void wait_probe_kernel(const unsigned *counter, unsigned target, unsi
     const unsigned long long t0 = globaltimer();
     wait_geq(counter, target, status);
     const unsigned long long t1 = globaltimer();
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&bar)) : "memory");
-    if (!ring_wait(&bar, 0u)) flag(status, MOE_DEV_TIMEOUT);
+    bar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!bar_wait(&bar, 0u)) flag(status, MOE_DEV_TIMEOUT);
     elapsed[0] = t1 - t0;
     elapsed[1] = globaltimer() - t1;
 }
@@ -232,36 +282,28 @@ __device__ __forceinline__ uint32_t logit_key(float v) {
     const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
     return k == 0u ? 1u : k;
 }
-
-// Router logits (fixed fp32 order, see moe.h). The 16 chunk loads of a row are
-// issued before the activations are staged, so the two overlap.
-constexpr int kRouterChunks = kMaxDimDec / 128;  // 16
-
-__device__ __forceinline__ void router_load(const DecodeParams &p, int e, int lane, float4 (&wv)[kRouterChunks]) {
-    const float *w = p.Wr + size_t(e) * p.d + 4 * lane;
-#pragma unroll
-    for (int u = 0; u < kRouterChunks; ++u)
-        if (u < p.d / 128) wv[u] = __ldg(reinterpret_cast<const float4 *>(w + 128 * u));
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
 }
 
+// One router row (fixed fp32 order, see moe.h) for NT tokens from shared memory.
 template <int NT>
-__device__ void router_row(const DecodeParams &p, const uint16_t *sx, int e, int lane,
-                           const float4 (&wv)[kRouterChunks]) {
+__device__ void router_row(const float *wrow, const uint16_t *sx, int T, int d, int lane, const float *bias, int e,
+                           float *logits, int E, int32_t *status) {
     float acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-#pragma unroll
-    for (int u = 0; u < kRouterChunks; ++u) {
-        if (u >= p.d / 128) break;
+    for (int u = 0; u < d / 128; ++u) {
+        const float4 wv = *reinterpret_cast<const float4 *>(wrow + 128 * u + 4 * lane);
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-            if (t < p.T) {
-                const uint2 xv = *reinterpret_cast<const uint2 *>(sx + size_t(t) * p.d + 128 * u + 4 * lane);
+            if (t < T) {
+                const uint2 xv = *reinterpret_cast<const uint2 *>(sx + size_t(t) * d + 128 * u + 4 * lane);
                 float a = acc[t];
-                a = __fmaf_rn(bf16_lo(xv.x), wv[u].x, a);
-                a = __fmaf_rn(bf16_hi(xv.x), wv[u].y, a);
-                a = __fmaf_rn(bf16_lo(xv.y), wv[u].z, a);
-                a = __fmaf_rn(bf16_hi(xv.y), wv[u].w, a);
+                a = __fmaf_rn(bf16_lo(xv.x), wv.x, a);
+                a = __fmaf_rn(bf16_hi(xv.x), wv.y, a);
+                a = __fmaf_rn(bf16_lo(xv.y), wv.z, a);
+                a = __fmaf_rn(bf16_hi(xv.y), wv.w, a);
                 acc[t] = a;
             }
         }
@@ -271,763 +313,326 @@ __device__ void router_row(const DecodeParams &p, const uint16_t *sx, int e, int
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) acc[t] = __fadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], o));
     if (lane == 0) {
-        const float b = p.bias ? p.bias[e] : 0.f;
-        for (int t = 0; t < p.T; ++t) {
-            const float v = p.bias ? __fadd_rn(acc[t], b) : acc[t];
-            if (!isfinite(v)) flag(p.status, MOE_DEV_NONFINITE);
-            p.logits[size_t(t) * p.E + e] = v;
+        const float b = bias ? bias[e] : 0.f;
+        for (int t = 0; t < T; ++t) {
+            const float v = bias ? __fadd_rn(acc[t], b) : acc[t];
+            if (!isfinite(v)) flag(status, MOE_DEV_NONFINITE);
+            __stcg(logits + size_t(t) * E + e, v);
         }
     }
 }
 
-// Gate/up of one 16-row group for up to 8 tokens of one expert into h rows.
-// tok[n] = token index (for x and xs), hrow0 + n = scratch row. Whole CTA;
-// every warp loads all of its weight tiles before computing.
-template <int FMT>
-__device__ void gateup_task(const DecodeParams &p, Smem &s, const uint16_t *sx, const uint8_t *rec, int rg,
-                            int ntok, const int *tok, int hrow0) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int NQ = p.d / 256;
-    float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint16_t *xrow = g < ntok ? sx + size_t(tok[g]) * p.d : nullptr;
-    const int t0 = 2 * t < ntok ? tok[2 * t] : -1, t1 = 2 * t + 1 < ntok ? tok[2 * t + 1] : -1;
-    for (int qd = warp; qd < NQ; qd += kWarps) {
-        QuadRegs<FMT> qg, qu;
-        quad_load<FMT>(rec, p.gate, rg, qd, lane, qg);
-        quad_load<FMT>(rec, p.up, rg, qd, lane, qu);
-        uint32_t B[4][8];
-        build_b_bf16<FMT>(xrow, qd, t, B);
-        float xs[4][2];
+// Q2 down tile of one block pair (16 rows x 128 columns): c = the lane's 16
+// code bytes, s = its 16 scale bytes (see layout.h), B / xs for the pair's two
+// blocks.
+__device__ __forceinline__ void pair_compute_q2(uint4 c, uint4 s, const uint32_t (&B)[2][8], const float (&xs)[2][2],
+                                                float (&acc)[4]) {
+    const uint32_t wg[2] = {c.x, c.z}, wg8[2] = {c.y, c.w};
+    const uint32_t sc[2] = {s.x, s.z}, mn[2] = {s.y, s.w};
 #pragma unroll
-        for (int bq = 0; bq < 4; ++bq) {
-            xs[bq][0] = t0 >= 0 ? s.xs[4 * qd + bq][t0] : 0.f;
-            xs[bq][1] = t1 >= 0 ? s.xs[4 * qd + bq][t1] : 0.f;
-        }
-        quad_compute<FMT>(qg, B, xs, ag);
-        quad_compute<FMT>(qu, B, xs, au);
-    }
+    for (int bq = 0; bq < 2; ++bq) {
+        float cc[4];
+        mma16816_zc(cc, q2_reg(wg[bq], 0), q2_reg(wg8[bq], 0), q2_reg(wg[bq], 1), q2_reg(wg8[bq], 1), B[bq][0],
+                    B[bq][1]);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        s.red[warp][0][r][lane] = ag[r];
-        s.red[warp][1][r][lane] = au[r];
-    }
-    __syncthreads();
-    if (threadIdx.x < 128) {
-        const int L = threadIdx.x >> 2, r = threadIdx.x & 3;
-        float A = 0.f, U = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            A += s.red[w][0][r][L];
-            U += s.red[w][1][r][L];
-        }
-        const int row = (L >> 2) + ((r & 2) ? 8 : 0);
-        const int n = 2 * (L & 3) + (r & 1);
-        if (n < ntok) p.h[size_t(hrow0 + n) * p.f + 16 * rg + row] = A / (1.0f + expf(-A)) * U;
+        for (int i = 1; i < 4; ++i)
+            mma16816(cc, q2_reg(wg[bq], 2 * i), q2_reg(wg8[bq], 2 * i), q2_reg(wg[bq], 2 * i + 1),
+                     q2_reg(wg8[bq], 2 * i + 1), B[bq][2 * i], B[bq][2 * i + 1]);
+        block_epilogue<2>(cc, sc[bq], mn[bq], xs[bq][0], xs[bq][1], acc);
     }
 }
 
-// Packed codes and scales of one 16-row x 256-column tile (columns 256qd..)
-// from a row group's bytes in shared memory, laid out as in the record: codes
-// at cb, scales at sb (the offsets of q2_chunk_off / q3_word_off / scale_off
-// relative to the row group's start).
+// Packed codes and scales of one 16-row x 256-column tile from shared memory:
+// cb / sb point at the first quad of a row group's slice as copied from the
+// record (codes contiguous per quad, scales per block pair).
 template <int FMT>
-__device__ __forceinline__ void quad_load_smem(const uint8_t *cb, const uint8_t *sb, int qd, int lane,
-                                               QuadRegs<FMT> &q) {
+__device__ __forceinline__ void quad_smem(const uint8_t *cb, const uint8_t *sb, int qi, int lane, QuadRegs<FMT> &q) {
     const int g = lane >> 2;
     if constexpr (FMT == 2) {
-        q.c0 = *reinterpret_cast<const uint4 *>(cb + ((2 * qd) * 32 + lane) * 16);
-        q.c1 = *reinterpret_cast<const uint4 *>(cb + ((2 * qd + 1) * 32 + lane) * 16);
-        q.s0 = *reinterpret_cast<const uint4 *>(sb + ((2 * qd) * 8 + g) * 16);
-        q.s1 = *reinterpret_cast<const uint4 *>(sb + ((2 * qd + 1) * 8 + g) * 16);
+        q.c0 = *reinterpret_cast<const uint4 *>(cb + ((2 * qi) * 32 + lane) * 16);
+        q.c1 = *reinterpret_cast<const uint4 *>(cb + ((2 * qi + 1) * 32 + lane) * 16);
+        q.s0 = *reinterpret_cast<const uint4 *>(sb + ((2 * qi) * 8 + g) * 16);
+        q.s1 = *reinterpret_cast<const uint4 *>(sb + ((2 * qi + 1) * 8 + g) * 16);
     } else {
 #pragma unroll
         for (int w = 0; w < 3; ++w) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(cb + qd * 1536 + w * 512 + lane * 16);
+            const uint4 v = *reinterpret_cast<const uint4 *>(cb + qi * 1536 + w * 512 + lane * 16);
             q.W[4 * w + 0] = v.x;
             q.W[4 * w + 1] = v.y;
             q.W[4 * w + 2] = v.z;
             q.W[4 * w + 3] = v.w;
         }
-        q.s0 = *reinterpret_cast<const uint2 *>(sb + ((2 * qd) * 8 + g) * 8);
-        q.s1 = *reinterpret_cast<const uint2 *>(sb + ((2 * qd + 1) * 8 + g) * 8);
+        q.s0 = *reinterpret_cast<const uint2 *>(sb + ((2 * qi) * 8 + g) * 8);
+        q.s1 = *reinterpret_cast<const uint2 *>(sb + ((2 * qi + 1) * 8 + g) * 8);
     }
 }
 
-// Block sums of the staged activations, one warp per (64-block, token); whole CTA.
-__device__ __forceinline__ void stage_xsum(Smem &s, const uint16_t *sx, int NB, int T, int d) {
+// Per-layer pointers.
+struct LayerPtrs {
+    const int32_t *slot_of;
+    const uint16_t *x;
+    const float *Wr, *bias;
+    float *y, *logits;
+    int shared_slot;
+};
+__device__ __forceinline__ LayerPtrs layer_ptrs(const DecodeParams &p, int l) {
+    LayerPtrs q;
+    q.slot_of = p.slot_of + size_t(l) * p.E;
+    q.x = p.x + size_t(l) * p.T * p.d;
+    q.Wr = p.Wr + size_t(l) * p.E * p.d;
+    q.bias = p.bias ? p.bias + size_t(l) * p.E : nullptr;
+    q.y = p.y + size_t(l) * p.T * p.d;
+    q.logits = p.logits + (p.logits_out ? 0 : size_t(l & 1) * p.T * p.E);
+    q.shared_slot = p.shared_slot ? __ldg(p.shared_slot + l) : p.shared_slot0;
+    return q;
+}
+
+// Task tau of the layer: the shared expert's blocks first, then the resident
+// routed experts' blocks. Returns the pool slot, sets hb and the active index
+// (-1 for the shared expert).
+__device__ __forceinline__ int task_slot(const DecodeParams &p, const Smem &s, const LayerPtrs &lp, int tau, int &hb,
+                                         int &a) {
+    const int NHB = p.g.NHB;
+    if (tau < NHB) {
+        hb = tau;
+        a = -1;
+        return lp.shared_slot;
+    }
+    const int r = (tau - NHB) / NHB;
+    hb = (tau - NHB) % NHB;
+    a = s.res[r];
+    return s.act_slot[a];
+}
+
+// Lanes of one warp issue the bulk copies of the warp's gate/up slice of task
+// (slot, hb) into buffer b (lane 0 sets the expected bytes first).
+template <int FMT>
+__device__ __forceinline__ void issue_gu(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int warp, int lane,
+                                         unsigned rank, int slot, int hb) {
+    const Geo &g = p.g;
+    uint8_t *dst = ring + size_t(b) * g.region + size_t(warp) * g.gu_warp;
+    const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
+    const int kq0 = int(rank) * g.NQR;  // first quad of this CTA's K slice
+    if (lane == 0) bar_expect(&s.gu_bar[b][warp], g.gu_warp);
+    __syncwarp();
+    // copy c: row group gi = c / 4, matrix (c / 2) % 2, codes (c even) or scales
+    if (lane < 4 * g.GUW) {
+        const int gi = lane >> 2, mi = (lane >> 1) & 1, sc = lane & 1;
+        const MatGeom &m = mi ? p.up : p.gate;
+        const int rg = hb * (g.HB / 16) + warp + 8 * gi;
+        uint8_t *d0 = dst + size_t(gi * 2 + mi) * (g.gu_c + g.gu_s) + (sc ? g.gu_c : 0);
+        uint64_t off;
+        if (sc)
+            off = scale_off(m, FMT, rg, 2 * kq0, 0);
+        else
+            off = FMT == 2 ? q2_chunk_off(m, rg, 2 * kq0, 0) : q3_word_off(m, rg, kq0, 0, 0);
+        bulk_copy(d0, rec + off, sc ? g.gu_s : g.gu_c, &s.gu_bar[b][warp]);
+    }
+}
+
+// The warp's down slice: row groups rank*DR/16 + warp*NDRW + j, the task's HB
+// columns (block pair hb for Q2, block quad hb for Q3).
+template <int FMT>
+__device__ __forceinline__ void issue_dn(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int warp, int lane,
+                                         unsigned rank, int slot, int hb) {
+    const Geo &g = p.g;
+    uint8_t *dst = ring + size_t(b) * g.region + size_t(kWarps) * g.gu_warp + size_t(warp) * g.dn_warp;
+    const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
+    if (lane == 0) bar_expect(&s.dn_bar[b][warp], g.dn_warp);
+    __syncwarp();
+    if (lane < 2 * g.NDRW) {
+        const int j = lane >> 1, sc = lane & 1;
+        const int rg = int(rank) * (g.DR / 16) + warp * g.NDRW + j;
+        uint8_t *d0 = dst + size_t(j) * (g.dn_c + g.dn_s) + (sc ? g.dn_c : 0);
+        uint64_t off;
+        if (sc)
+            off = scale_off(p.down, FMT, rg, FMT == 2 ? hb : 2 * hb, 0);
+        else
+            off = FMT == 2 ? q2_chunk_off(p.down, rg, hb, 0) : q3_word_off(p.down, rg, hb, 0, 0);
+        bulk_copy(d0, rec + off, sc ? g.dn_s : g.dn_c, &s.dn_bar[b][warp]);
+    }
+}
+
+// Top-k of every token from the logits in global memory (written by all CTAs
+// of this launch): WPT = 8 / NT warps per token each find the k best of their
+// share of the experts by k rounds of a warp-wide maximum of 64-bit keys
+// (logit key << 32 | ~id: larger logit first, then lower id); the WPT sorted
+// lists are merged by counting, for every entry, the entries of the other
+// lists above it. Then softmax over the selected logits and ascending-id order
+// (the arithmetic of moe_route).
+template <int NT>
+__device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, int T, int E, int k) {
+    constexpr int WPT = kWarps / NT;       // warps per token
+    constexpr int M = kMaxEDec / 32 / WPT;  // keys per lane
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int job = warp; job < NB * T; job += kWarps) {
-        const int b = job / T, n = job % T;
-        const uint32_t u = *reinterpret_cast<const uint32_t *>(sx + size_t(n) * d + 64 * b + 2 * lane);
-        float v = bf16_lo(u) + bf16_hi(u);
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) s.xs[b][n] = v;
-    }
-}
-
-template <int FMT, int NT>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(DecodeParams p) {
-    extern __shared__ __align__(16) unsigned char dyn[];
-    __shared__ Smem s;
-    uint16_t *sx = reinterpret_cast<uint16_t *>(dyn);                                        // [T][d] bf16
-    float *sh = reinterpret_cast<float *>(dyn + ((size_t(p.T) * p.d * 2 + 15) & ~size_t(15)));  // [T][f] h
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int G = gridDim.x, cta = blockIdx.x;
-    const int T = p.T, k = p.k, E = p.E, d = p.d, f = p.f;
-    const int NG = f / 16, NB = d / 64;
-    const int npairs = T * k;
-    const int nrt = (E + kWarps - 1) / kWarps;  // router CTA-tasks (8 rows each)
-    const uint8_t *shrec = p.pool + int64_t(p.shared_slot) * p.slot_bytes;
-    const uint32_t gu_codes = FMT == 2 ? uint32_t(d / 128) * 512u : uint32_t(d / 256) * 1536u;
-    const uint32_t gu_scales = uint32_t(d / 128) * (FMT == 2 ? 128u : 64u);
-    bool too_big = false;
-    int ring_issued = 0, ring_used = 0;  // thread 0: weight-ring units copied / consumed
-
-    TRACE(0);
-    if (tid == 0) {
-        for (int i = 0; i < kMaxSlots; ++i)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&s.full[i])) : "memory");
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    // ------------------------------------------------------------ phase A
-    if (tid == 0) {  // start the HBM reads of this CTA's phase-A task right away
-        for (int task = cta; task < NG + nrt; task += G) {
-            if (task < NG) {
-                prefetch_l2(shrec + p.gate.codes_off + uint64_t(task) * gu_codes, gu_codes);
-                prefetch_l2(shrec + p.up.codes_off + uint64_t(task) * gu_codes, gu_codes);
-                prefetch_l2(shrec + p.gate.scales_off + uint64_t(task) * gu_scales, gu_scales);
-                prefetch_l2(shrec + p.up.scales_off + uint64_t(task) * gu_scales, gu_scales);
-            } else {
-                const int e0 = kWarps * (task - NG);
-                const int ne = min(kWarps, E - e0);
-                prefetch_l2(p.Wr + size_t(e0) * d, uint32_t(ne) * uint32_t(d) * 4u);
-            }
-        }
-    }
-    // a router CTA-task (8 rows) loads its weights before anything else
-    const int rtask = cta - NG;  // valid when 0 <= rtask < nrt (one phase-A task per CTA when G >= NG + nrt)
-    const bool router_cta = G >= NG + nrt && rtask >= 0 && rtask < nrt;
-    float4 wv[kRouterChunks];
-    if (router_cta && kWarps * rtask + warp < E) router_load(p, kWarps * rtask + warp, lane, wv);
-    {  // stage x and the slot table: every load of a thread is issued before any store
-        constexpr int kXv = NT * kMaxDimDec / 8 / kThreads;  // uint4 per thread at most
-        constexpr int kSv = kMaxEDec / kThreads;
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.x);
-        uint4 *dst = reinterpret_cast<uint4 *>(sx);
-        const int nx = T * d / 8;
-        uint4 xv[kXv];
-        int sv[kSv];
-#pragma unroll
-        for (int u = 0; u < kXv; ++u)
-            if (tid + u * kThreads < nx) xv[u] = __ldg(src + tid + u * kThreads);
-#pragma unroll
-        for (int u = 0; u < kSv; ++u)
-            if (tid + u * kThreads < E) sv[u] = __ldg(p.slot_of + tid + u * kThreads);
-#pragma unroll
-        for (int u = 0; u < kXv; ++u)
-            if (tid + u * kThreads < nx) dst[tid + u * kThreads] = xv[u];
-#pragma unroll
-        for (int u = 0; u < kSv; ++u)
-            if (tid + u * kThreads < E) s.slot[tid + u * kThreads] = sv[u];
-        for (int i = cta * kThreads + tid; i < T * d; i += G * kThreads) p.y[i] = 0.f;
-    }
-    __syncthreads();
-    TRACE(8);
-    if (tid < kMaxTokDec) s.idx[0][tid] = tid;  // identity token list for the shared expert
-    __syncthreads();
-    bool xsum_ready = false;  // the router path does not need the block sums
-    for (int task = cta; task < NG + nrt; task += G) {
-        if (task < NG) {
-            if (!xsum_ready) {
-                stage_xsum(s, sx, NB, T, d);
-                __syncthreads();
-                xsum_ready = true;
-            }
-            gateup_task<FMT>(p, s, sx, shrec, task, T, s.idx[0], npairs);
-            __syncthreads();
-            if (tid == 0) {
-                __threadfence();
-                atomicAdd(p.done + kSharedIdx, 1u);
-            }
-        } else {
-            const int e0 = kWarps * (task - NG);
-            if (e0 + warp < E) {
-                if (!router_cta) router_load(p, e0 + warp, lane, wv);
-                router_row<NT>(p, sx, e0 + warp, lane, wv);
-                if (warp == 0) TRACEW(10);
-            }
-            __syncthreads();
-            if (tid == 0) {  // these router rows are written
-                __threadfence();
-                atomicAdd(p.ctr, unsigned(min(kWarps, E - e0)));
-            }
-        }
-    }
-    if (!xsum_ready) stage_xsum(s, sx, NB, T, d);  // for phase C (synchronised below)
-    TRACE(1);
-    // routing needs every logit: wait for all E router rows (not for the
-    // shared expert's gate/up, which only phase D waits for)
-    if (tid == 0) s.ok = wait_geq(p.ctr, unsigned(E), p.status);
-    __syncthreads();
-    if (!s.ok) goto finish;
-    TRACE(2);
-
-    // ------------------------------------------------------------ phase B
-    if (warp < T) {
-        // Top-k of token `warp` without selection rounds. A candidate is the
-        // 64-bit (logit key << 32 | ~id): larger = larger logit, then lower id,
-        // so the top k are the k largest candidates. The k-th largest lane
-        // maximum L is a lower bound for the k-th largest candidate overall (the
-        // k lanes whose maxima are >= L hold k candidates >= L), so only the
-        // candidates >= L (usually a few more than k) are gathered and ranked.
-        constexpr int M = kMaxEDec / 32;
-        const float *row = p.logits + size_t(warp) * E;
-        float lv[M];
-#pragma unroll
-        for (int m = 0; m < M; ++m) lv[m] = lane + 32 * m < E ? __ldcg(row + lane + 32 * m) : 0.f;
-        if (warp == 0) {
-            float sum_ = 0.f;
-            for (int m = 0; m < M; ++m) sum_ += lv[m];
-            if (sum_ == 12345.f) flag(p.status, 0);
-            TRACEW(11);
-        }
+    const int tt = warp / WPT, sub = warp % WPT;
+    if (tt < T) {
+        const float *row = logits + size_t(tt) * E;
         uint64_t c[M];
-        uint64_t mx = 0ull;
+        bool nan = false;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-            const int e = lane + 32 * m;
-            c[m] = e < E ? (uint64_t(logit_key(lv[m])) << 32) | uint64_t(~uint32_t(e)) : 0ull;
-            mx = c[m] > mx ? c[m] : mx;
+            const int e = sub * 32 + lane + 32 * WPT * m;
+            if (e < E) {
+                const float v = __ldcg(row + e);
+                nan |= v != v;
+                c[m] = (uint64_t(logit_key(v)) << 32) | uint64_t(~uint32_t(e));
+            } else {
+                c[m] = 0ull;
+            }
         }
-        int above = 0;  // lanes whose maximum beats ours
+        if (__any_sync(0xffffffffu, nan) && lane == 0 && blockIdx.x == 0) flag(p.status, MOE_DEV_NONFINITE);
+        uint64_t mine = 0ull;
+        for (int r = 0; r < k; ++r) {
+            uint64_t mx = 0ull;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) above += __shfl_sync(0xffffffffu, mx, q) > mx;
-        const unsigned kth = __ballot_sync(0xffffffffu, above == k - 1);
-        const uint64_t L = __shfl_sync(0xffffffffu, mx, __ffs(kth) - 1);
-        int cnt = 0;
+            for (int m = 0; m < M; ++m) mx = c[m] > mx ? c[m] : mx;
+            const uint32_t hk = __reduce_max_sync(0xffffffffu, uint32_t(mx >> 32));
+            const uint32_t lk = __reduce_max_sync(0xffffffffu, uint32_t(mx >> 32) == hk ? uint32_t(mx) : 0u);
+            const uint64_t win = (uint64_t(hk) << 32) | lk;
+            if (lane == r) mine = win;
+            if (mx == win && win != 0ull) {
 #pragma unroll
-        for (int m = 0; m < M; ++m) cnt += c[m] >= L;
-        int pre = cnt;  // inclusive prefix over lanes
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, pre, o);
-            if (lane >= o) pre += v;
+                for (int m = 0; m < M; ++m)
+                    if (c[m] == win) c[m] = 0ull;
+            }
         }
-        const int ncand = __shfl_sync(0xffffffffu, pre, 31);
-        if (warp == 0) TRACEW(12);
-        uint64_t *cand = s.cand[warp];
-        int pos = pre - cnt;
-#pragma unroll
-        for (int m = 0; m < M; ++m)
-            if (c[m] >= L) {
-                if (pos < kCandMax) cand[pos] = c[m];
-                ++pos;
-            }
-        __syncwarp();
-        if (ncand <= 32) {  // one candidate per lane, ranked with shuffles
-            const uint64_t me = lane < ncand ? cand[lane] : 0ull;
-            int r = 0;
-#pragma unroll
-            for (int q = 0; q < 32; ++q) r += __shfl_sync(0xffffffffu, me, q) > me;
-            if (lane < ncand && r < k) {
-                const uint32_t key = uint32_t(me >> 32);
-                const uint32_t u = (key & 0x80000000u) ? (key ^ 0x80000000u) : ~key;
-                s.sel_v[warp][r] = __uint_as_float(u);
-                s.sel_id[warp][r] = int(~uint32_t(me));
-            }
-        } else if (ncand <= kCandMax) {
-            for (int i = lane; i < ncand; i += 32) {
-                const uint64_t me = cand[i];
-                int r = 0;
-                for (int q = 0; q < ncand; ++q) r += cand[q] > me;
-                if (r < k) {  // selected: keep its value and id (ordered by id below)
-                    const uint32_t key = uint32_t(me >> 32);
-                    const uint32_t u = (key & 0x80000000u) ? (key ^ 0x80000000u) : ~key;
-                    s.sel_v[warp][r] = __uint_as_float(u);
-                    s.sel_id[warp][r] = int(~uint32_t(me));
-                }
-            }
-        } else {  // many near-equal maxima: k rounds of a warp-wide arg-max
-            uint64_t best = 0ull;
-#pragma unroll
-            for (int m = 0; m < M; ++m) best = c[m] > best ? c[m] : best;
-            for (int r = 0; r < k; ++r) {
-                const uint32_t hk = uint32_t(best >> 32), hl = uint32_t(best);
-                const uint32_t mk = __reduce_max_sync(0xffffffffu, hk);
-                const uint32_t ml = __reduce_max_sync(0xffffffffu, hk == mk ? hl : 0u);
-                if (lane == 0) {
-                    const uint32_t u = (mk & 0x80000000u) ? (mk ^ 0x80000000u) : ~mk;
-                    s.sel_v[warp][r] = __uint_as_float(u);
-                    s.sel_id[warp][r] = int(~ml);
-                }
-                if (hk == mk && hl == ml) {
-                    best = 0ull;
-#pragma unroll
-                    for (int m = 0; m < M; ++m) {
-                        if (c[m] == ((uint64_t(mk) << 32) | ml)) c[m] = 0ull;
-                        best = c[m] > best ? c[m] : best;
-                    }
-                }
-            }
+        if (WPT == 1) {
+            if (lane < k) s.sel[tt][lane] = mine;
+        } else if (lane < k) {
+            s.wl[warp][lane] = mine;
         }
     }
-    if (warp < T) {
-        __syncwarp();
-        if (warp == 0) TRACEW(13);
-        const int sel_id = lane < k ? s.sel_id[warp][lane] : 0;
-        const float sel_v = lane < k ? s.sel_v[warp][lane] : 0.f;
-        // sort the k selections by id and apply the softmax (normaliser summed in
-        // ascending expert id, as moe_route does)
-        const float vmax = __shfl_sync(0xffffffffu, sel_v, 0);
-        const float ex = lane < k ? expf(sel_v - vmax) : 0.f;
-        int rank = 0;
-        for (int q = 0; q < k; ++q) rank += (__shfl_sync(0xffffffffu, sel_id, q) < sel_id);
-        // ex of the a-th smallest id sits in the lane whose rank is a
-        const unsigned rank_src = lane < k ? unsigned(rank) : 31u;
-        float ex_by_id[kMaxK];
-        int src_lane[kMaxK];
-#pragma unroll
-        for (int a = 0; a < kMaxK; ++a) {
-            const unsigned hit = __ballot_sync(0xffffffffu, lane < k && rank_src == unsigned(a));
-            src_lane[a] = hit ? __ffs(hit) - 1 : 0;
-        }
-#pragma unroll
-        for (int a = 0; a < kMaxK; ++a) ex_by_id[a] = __shfl_sync(0xffffffffu, ex, src_lane[a]);
-        float z = 0.f;
-#pragma unroll
-        for (int a = 0; a < kMaxK; ++a)
-            if (a < k) z += ex_by_id[a];
-        const float inv_z = 1.0f / z;
-        if (lane < k) {
-            s.idx[warp][rank] = sel_id;
-            s.w[warp][rank] = ex * inv_z;
-        }
-    }
-    __syncthreads();
-    TRACE(6);
-    if (T == 1) {
-        if (warp == 0) {  // one token: its k experts (id order) are the active experts, one pair each
-            const bool in = lane < k;
-            int sl = -1;
-            if (in) {
-                const int e = s.idx[0][lane];
-                s.pair_e[lane] = e;
-                s.s_tok[lane] = 0;
-                s.s_j[lane] = lane;
-                s.inv[lane] = lane;
-                sl = s.slot[e];
-                const bool bad = sl < -1 || sl >= p.num_slots;
-                if (bad && cta == 0) flag(p.status, MOE_DEV_BAD_SLOT);
-                if (bad) sl = -1;
-                s.act_e[lane] = e;
-                s.act_beg[lane] = lane;
-                s.act_cnt[lane] = 1;
-                s.act_slot[lane] = sl;
-            }
-            const unsigned rm = __ballot_sync(0xffffffffu, in && sl >= 0);
-            const unsigned mm = __ballot_sync(0xffffffffu, in && sl < 0);
-            const unsigned lt = (1u << lane) - 1u;
-            if (in) s.act_mbase[lane] = __popc(mm & lt);
-            if (in && sl >= 0) s.res[__popc(rm & lt)] = lane;
-            if (lane == 0) {
-                s.nact = k;
-                s.nres = __popc(rm);
-                s.nmiss = __popc(mm);
-            }
-        }
-    } else {
-        if (tid < npairs) {  // stable sort of the pairs by (expert, pair index)
-            const int pp = tid;
-            const int e = s.idx[pp / k][pp % k];
-            int rank = 0;
-            for (int q = 0; q < npairs; ++q) {
-                const int eq = s.idx[q / k][q % k];
-                rank += (eq < e) || (eq == e && q < pp);
-            }
-            s.pair_e[rank] = e;
-            s.s_tok[rank] = pp / k;
-            s.s_j[rank] = pp % k;
-            s.inv[pp] = rank;
-        }
+    if (WPT > 1) {
         __syncthreads();
-        {  // experts with tokens, their segments, slots and miss bases (ballot scans)
-            const bool in = tid < npairs;
-            const bool first = in && (tid == 0 || s.pair_e[tid] != s.pair_e[tid - 1]);
-            const unsigned fm = __ballot_sync(0xffffffffu, first);
-            if (lane == 0 && warp < kMaxPairs / 32) s.first_mask[warp] = fm;
-            __syncthreads();
-            if (first) {
-                int a = __popc(fm & ((1u << lane) - 1));
-                for (int w = 0; w < warp; ++w) a += __popc(s.first_mask[w]);
-                const int e = s.pair_e[tid];
-                const int sl = s.slot[e];
-                const bool bad = sl < -1 || sl >= p.num_slots;
-                if (bad && cta == 0) flag(p.status, MOE_DEV_BAD_SLOT);
-                s.act_e[a] = e;
-                s.act_beg[a] = tid;
-                s.act_slot[a] = bad ? -1 : sl;
-            }
-            if (tid == 0) {
-                int na = 0;
-                for (int w = 0; w < (npairs + 31) / 32; ++w) na += __popc(s.first_mask[w]);
-                s.nact = na;
-            }
-            __syncthreads();
-            const int na = s.nact;
-            if (tid < na) s.act_cnt[tid] = (tid + 1 < na ? s.act_beg[tid + 1] : npairs) - s.act_beg[tid];
-            __syncthreads();
-            if (warp == 0) {  // resident list and miss bases over <= 128 actives, 32 at a time
-                int nr = 0, nm = 0;
-                for (int a0 = 0; a0 < na; a0 += 32) {
-                    const int a = a0 + lane;
-                    const bool act = a < na;
-                    const bool res = act && s.act_slot[a] >= 0;
-                    const int cm = act && !res ? s.act_cnt[a] : 0;
-                    const unsigned rm = __ballot_sync(0xffffffffu, res);
-                    int mpre = cm;
-    #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int v = __shfl_up_sync(0xffffffffu, mpre, o);
-                        if (lane >= o) mpre += v;
-                    }
-                    if (act) s.act_mbase[a] = nm + mpre - cm;
-                    if (res) s.res[nr + __popc(rm & ((1u << lane) - 1))] = a;
-                    nr += __popc(rm);
-                    nm += __shfl_sync(0xffffffffu, mpre, 31);
+        if (tt < T && lane < k) {
+            const uint64_t me = s.wl[warp][lane];
+            int rank = lane;
+            for (int o = 0; o < WPT; ++o) {
+                if (o == sub) continue;
+                const uint64_t *ol = s.wl[tt * WPT + o];
+                int lo = 0, hi = k;  // entries of list o above me (lists are descending)
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (ol[mid] > me) lo = mid + 1; else hi = mid;
                 }
-                if (lane == 0) {
-                    s.nres = nr;
-                    s.nmiss = nm;
-                }
+                rank += lo;
             }
+            if (rank < k) s.sel[tt][rank] = me;
         }
     }
     __syncthreads();
-    TRACE(5);
-    {
-        // ------------------------------------------------------------ weight ring
-        // This CTA's units: its gate/up tasks (task = G-1-cta + u*G < nres*NG,
-        // busy phase-A CTAs last), then its down tasks (a contiguous range of
-        // tasks < (nres+1)*nblk; a down task is an expert x 8 row groups of d,
-        // the shared expert last). Thread 0 bulk-copies a unit's packed bytes
-        // (contiguous per row group in the record) into ring slot u % NS as soon
-        // as the routing tables exist, the first NS units at once, and refills a
-        // slot with unit u + NS once unit u has been computed.
-        const int NQ = d / 256, NQf = f / 256, nblk = d / 128;
-        const int nres = s.nres;
-        const int ctasks = nres * NG, dtasks = (nres + 1) * nblk;
-        const int cfirst = G - 1 - cta;
-        const int nC = ctasks > cfirst ? (ctasks - cfirst + G - 1) / G : 0;
-        // down tasks: a contiguous range per CTA (consecutive tasks mostly share an
-        // expert, whose staged h and B fragments are then reused)
-        const int dlo = int(int64_t(dtasks) * cta / G), nD = int(int64_t(dtasks) * (cta + 1) / G) - dlo;
-        const int nU = nC + nD, NS = p.nslots;
-        uint8_t *ring = dyn + ring_off(T, d, f);
-        // copy c (0..3 gate/up: gate codes, gate scales, up codes, up scales;
-        // 0..1 down: codes, scales) of unit u; one thread per copy
-        auto issue_copy = [&](int u, int c) {
-            uint8_t *dst = ring + size_t(u % NS) * p.rslot;
-            uint64_t *bar = &s.full[u % NS];
-            if (u < nC) {
-                const int task = cfirst + u * G, ar = task / NG, rg = task % NG;
-                const uint8_t *rec = p.pool + int64_t(s.act_slot[s.res[ar]]) * p.slot_bytes;
-                const MatGeom &m = c < 2 ? p.gate : p.up;
-                const uint32_t off = (c >> 1) * (p.gu_cb + p.gu_sb) + (c & 1) * p.gu_cb;
-                if (c & 1)
-                    ring_copy(dst + off, rec + m.scales_off + uint64_t(rg) * p.gu_sb, p.gu_sb, bar);
-                else
-                    ring_copy(dst + off, rec + m.codes_off + uint64_t(rg) * p.gu_cb, p.gu_cb, bar);
-            } else if (c < 2) {
-                const int task = dlo + (u - nC), ar = task / nblk, blk = task % nblk;
-                const int slot = ar == nres ? p.shared_slot : s.act_slot[s.res[ar]];
-                const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
-                if (c)
-                    ring_copy(dst + 8 * p.dn_cb, rec + p.down.scales_off + uint64_t(8 * blk) * p.dn_sb,
-                              8u * p.dn_sb, bar);
-                else
-                    ring_copy(dst, rec + p.down.codes_off + uint64_t(8 * blk) * p.dn_cb, 8u * p.dn_cb, bar);
-            }
-        };
-        auto unit_bytes = [&](int u) { return u < nC ? 2u * (p.gu_cb + p.gu_sb) : 8u * (p.dn_cb + p.dn_sb); };
-        auto issue = [&](int u) {  // one thread, all copies of unit u
-            ring_expect(&s.full[u % NS], unit_bytes(u));
-            for (int c = 0; c < 4; ++c) issue_copy(u, c);
-        };
-        {  // the first min(nU, NS) units at once: warp u announces unit u, its lanes 0..3 copy
-            const int n0 = min(nU, NS);
-            if (warp < n0) {
-                if (lane == 0) ring_expect(&s.full[warp], unit_bytes(warp));
-                __syncwarp();
-                if (lane < 4) issue_copy(warp, lane);
-            }
-            ring_issued = n0;  // meaningful in thread 0
+    if (warp < T) {  // one warp per token: softmax, ascending id order (as moe_route)
+        const uint64_t mine = lane < k ? s.sel[warp][lane] : 0ull;
+        const uint32_t key = uint32_t(mine >> 32);
+        // a round that found only NaN left takes expert 0 with logit -inf, as moe_route does
+        const int my_id = key ? int(~uint32_t(mine)) : 0;
+        const float my_v = key ? key_value(key) : -INFINITY;
+        const bool sel = lane < k;
+        int rank = 0;
+        for (int q = 0; q < k; ++q) rank += __shfl_sync(0xffffffffu, my_id, q) < my_id;
+        const float mx = __shfl_sync(0xffffffffu, my_v, 0);
+        const float ex = sel ? expf(my_v - mx) : 0.f;
+        float z = 0.0f;
+        for (int a = 0; a < k; ++a) {
+            const unsigned who = __ballot_sync(0xffffffffu, sel && rank == a);
+            z += __shfl_sync(0xffffffffu, ex, __ffs(who) - 1);
         }
-        TRACE(3);
-        // every thread waits for unit u's bytes itself; false (all threads) on timeout
-        auto await_unit = [&](int u) -> bool {
-            const bool got = ring_wait(&s.full[u % NS], uint32_t(u / NS) & 1u);
-            if (!got && tid == 0) flag(p.status, MOE_DEV_TIMEOUT);
-            const bool all = __syncthreads_and(got) != 0;
-            if (all && tid == 0) ++ring_used;
-            return all;
-        };
-
-        // ------------------------------------------------------------ phase C
-        const int g = lane >> 2, t = lane & 3;
-        const bool one_quad = NQ == kWarps;  // every warp owns exactly one quad
-        uint32_t B1[4][8];                   // one token: fragments of quad `warp`, built once
-        float xs1[4][2];
-        if (NT == 1 && one_quad) {
-            build_b_bf16<FMT>(g == 0 ? sx : nullptr, warp, t, B1);
-#pragma unroll
-            for (int bq = 0; bq < 4; ++bq) {
-                xs1[bq][0] = t == 0 ? s.xs[4 * warp + bq][0] : 0.f;
-                xs1[bq][1] = 0.f;
-            }
-        }
-        // One token and all of this CTA's gate/up units in the ring at once: wait
-        // for all of them, compute every unit's quad `warp` back to back (their
-        // MMA chains interleave), then one reduction over warps for all units
-        // (same summation order as the per-unit path below).
-        const bool batch = NT == 1 && one_quad && nC <= min(NS, kCBatch);
-        if (batch) {
-            // every thread waits for each unit itself and computes it at once:
-            // no barrier until all units are done
-            bool got = true;
-            float ag[kCBatch][4], au[kCBatch][4];
-#pragma unroll
-            for (int i = 0; i < kCBatch; ++i) {
-                if (i < nC) {
-                    got = got && ring_wait(&s.full[i], 0u);
-                    if (i == 0) TRACE(16);
-                    const uint8_t *slot = ring + size_t(i) * p.rslot;
-                    QuadRegs<FMT> qg, qu;
-                    quad_load_smem<FMT>(slot, slot + p.gu_cb, warp, lane, qg);
-                    quad_load_smem<FMT>(slot + p.gu_cb + p.gu_sb, slot + 2 * p.gu_cb + p.gu_sb, warp, lane, qu);
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) ag[i][r] = au[i][r] = 0.f;
-                    quad_compute<FMT>(qg, B1, xs1, ag[i]);
-                    quad_compute<FMT>(qu, B1, xs1, au[i]);
-                }
-            }
-            if (warp == 0) TRACEW(9);
-            if (!got && tid == 0) flag(p.status, MOE_DEV_TIMEOUT);
-            if (!__syncthreads_and(got)) goto finish;
-            if (tid == 0) ring_used = nC;
-            // token 0 sits in lanes t == 0: rows g (r = 0) and g + 8 (r = 2)
-            float(*red1)[kWarps][2][16] = reinterpret_cast<float(*)[kWarps][2][16]>(&s.red[0][0][0][0]);
-            if (t == 0) {
-#pragma unroll
-                for (int i = 0; i < kCBatch; ++i) {
-                    if (i < nC) {
-                        red1[i][warp][0][g] = ag[i][0];
-                        red1[i][warp][0][g + 8] = ag[i][2];
-                        red1[i][warp][1][g] = au[i][0];
-                        red1[i][warp][1][g + 8] = au[i][2];
-                    }
-                }
-            }
-            __syncthreads();
-            TRACE(17);
-            if (tid < nC * 16) {
-                const int i = tid >> 4, row = tid & 15;
-                const int task = cfirst + i * G, ar = task / NG, rg = task % NG;
-                float A = 0.f, U = 0.f;
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) {
-                    A += red1[i][w][0][row];
-                    U += red1[i][w][1][row];
-                }
-                p.h[size_t(s.act_beg[s.res[ar]]) * f + 16 * rg + row] = A / (1.0f + expf(-A)) * U;
-            }
-            __syncthreads();  // slots and red[] read by everyone
-            if (tid == 0)
-                while (ring_issued < nU && ring_issued < nC + NS) issue(ring_issued++);
-            TRACE(14);
-        }
-        for (int u = 0; !batch && u < nC; ++u) {
-            const int task = cfirst + u * G, ar = task / NG, rg = task % NG;
-            const int a = s.res[ar];
-            const int ntok = s.act_cnt[a];
-            const int *tok = s.s_tok + s.act_beg[a];
-            if (!await_unit(u)) goto finish;
-            if (u == 0) TRACE(16);
-            const uint8_t *slot = ring + size_t(u % NS) * p.rslot;
-            float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int qd = warp; qd < NQ; qd += kWarps) {
-                QuadRegs<FMT> qg, qu;
-                quad_load_smem<FMT>(slot, slot + p.gu_cb, qd, lane, qg);
-                quad_load_smem<FMT>(slot + p.gu_cb + p.gu_sb, slot + 2 * p.gu_cb + p.gu_sb, qd, lane, qu);
-                if (NT == 1 && one_quad) {
-                    quad_compute<FMT>(qg, B1, xs1, ag);
-                    quad_compute<FMT>(qu, B1, xs1, au);
-                } else {
-                    const uint16_t *xrow = g < ntok ? sx + size_t(tok[g]) * d : nullptr;
-                    const int t0 = 2 * t < ntok ? tok[2 * t] : -1, t1 = 2 * t + 1 < ntok ? tok[2 * t + 1] : -1;
-                    uint32_t B[4][8];
-                    build_b_bf16<FMT>(xrow, qd, t, B);
-                    float xs[4][2];
-#pragma unroll
-                    for (int bq = 0; bq < 4; ++bq) {
-                        xs[bq][0] = t0 >= 0 ? s.xs[4 * qd + bq][t0] : 0.f;
-                        xs[bq][1] = t1 >= 0 ? s.xs[4 * qd + bq][t1] : 0.f;
-                    }
-                    quad_compute<FMT>(qg, B, xs, ag);
-                    quad_compute<FMT>(qu, B, xs, au);
-                }
-            }
-            if (u < 2 && warp == 0) TRACEW(u == 0 ? 9 : 15);
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                s.red[warp][0][r][lane] = ag[r];
-                s.red[warp][1][r][lane] = au[r];
-            }
-            __syncthreads();
-            if (u == 0) TRACE(17);
-            if (tid < 128) {
-                const int L = tid >> 2, r = tid & 3;
-                float A = 0.f, U = 0.f;
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) {
-                    A += s.red[w][0][r][L];
-                    U += s.red[w][1][r][L];
-                }
-                const int row = (L >> 2) + ((r & 2) ? 8 : 0);
-                const int n = 2 * (L & 3) + (r & 1);
-                if (n < ntok) p.h[size_t(s.act_beg[a] + n) * f + 16 * rg + row] = A / (1.0f + expf(-A)) * U;
-            }
-            __syncthreads();  // slot and red[] read by everyone
-            if (tid == 0 && ring_issued < nU) issue(ring_issued++);
-            if (u == 0) TRACE(14);
-        }
-        // publish this CTA's h rows (written before the last barrier): one fence
-        // and one count per task, by as many threads
-        for (int u = tid; u < nC; u += kThreads) {
-            __threadfence();
-            atomicAdd(p.done + (cfirst + u * G) / NG, 1u);
-        }
-
-        TRACE(7);
-        // ------------------------------------------------------------ phase D
-        int staged = -1;  // expert whose h, block sums and B fragments are in shared memory
-        for (int u = nC; u < nU; ++u) {
-            const int task = dlo + (u - nC), ar = task / nblk, blk = task % nblk;
-            const bool shared = ar == nres;
-            const int a = shared ? 0 : s.res[ar];
-            const int ntok = shared ? T : s.act_cnt[a];
-            const int beg = shared ? npairs : s.act_beg[a];
-            const int rg = 8 * blk + warp;
-            if (!await_unit(u)) goto finish;
-            if (u == nC) TRACE(18);
-            if (ar != staged) {  // the expert's first unit here: wait for its h, stage it
-                staged = ar;
-                if (tid == 0) s.ok = wait_geq(p.done + (shared ? kSharedIdx : ar), unsigned(NG), p.status);
-                __syncthreads();
-                if (!s.ok) goto finish;
-                if (u == nC) TRACE(19);
-                {  // the expert's h rows (written by other CTAs: read through L2) into shared memory
-                    constexpr int kHv = NT * kMaxFDec / 4 / kThreads + 1;  // float4 per thread at most
-                    const float4 *src = reinterpret_cast<const float4 *>(p.h + size_t(beg) * f);
-                    float4 *dst = reinterpret_cast<float4 *>(sh);
-                    const int nh = ntok * f / 4;
-                    float4 hv[kHv];
-    #pragma unroll
-                    for (int v = 0; v < kHv; ++v)
-                        if (tid + v * kThreads < nh) hv[v] = __ldcg(src + tid + v * kThreads);
-    #pragma unroll
-                    for (int v = 0; v < kHv; ++v)
-                        if (tid + v * kThreads < nh) dst[tid + v * kThreads] = hv[v];
-                }
-                __syncthreads();
-                for (int job = warp; job < (f / 64) * ntok; job += kWarps) {  // block sums of h
-                    const int bb = job / ntok, n = job % ntok;
-                    const float2 v = *reinterpret_cast<const float2 *>(sh + size_t(n) * f + 64 * bb + 2 * lane);
-                    float sum = v.x + v.y;
-    #pragma unroll
-                    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                    if (lane == 0) s.hsb[bb][n] = sum;
-                }
-                // B fragments of every quad of h (element (k, n=gg) of slot rho of
-                // block bq for lane (gg, tt): columns 256qd + 64bq + slot_k(rho, tt),
-                // divided by 2^slot_exp), one 16-byte entry per thread and step
-                for (int e = tid; e < NQf * 256; e += kThreads) {
-                    const int qd = e >> 8, ln = (e >> 3) & 31, r4 = e & 7;
-                    const int gg = ln >> 2, tt = ln & 3, bq = r4 >> 1;
-                    const float *src = gg < ntok ? sh + size_t(gg) * f + 256 * qd + 64 * bq : nullptr;
-                    uint32_t v[4];
-    #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int rho = (r4 & 1) * 4 + j;
-                        float lo = 0.f, hi = 0.f;
-                        if (src) {
-                            const float2 hv = *reinterpret_cast<const float2 *>(src + slot_k(rho, tt, 0));
-                            lo = hv.x;
-                            hi = hv.y;
-                            too_big |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
-                        }
-                        const float sc = __int_as_float((127 - slot_exp<FMT>(bq, rho)) << 23);  // 2^-exp
-                        v[j] = pack_half2(lo * sc, hi * sc);
-                    }
-                    s.bfrag[qd][r4][ln] = make_uint4(v[0], v[1], v[2], v[3]);
-                }
-                __syncthreads();
-            }
-            if (u == nC) TRACE(20);
-            const uint8_t *slot = ring + size_t(u % NS) * p.rslot;
-            const uint8_t *cb = slot + warp * p.dn_cb, *sb = slot + 8 * p.dn_cb + warp * p.dn_sb;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-            for (int qd = 0; qd < NQf; ++qd) {
-                QuadRegs<FMT> q;
-                quad_load_smem<FMT>(cb, sb, qd, lane, q);
-                uint32_t B[4][8];
-#pragma unroll
-                for (int r4 = 0; r4 < 8; ++r4) {
-                    const uint4 v = s.bfrag[qd][r4][lane];
-                    B[r4 >> 1][(r4 & 1) * 4 + 0] = v.x;
-                    B[r4 >> 1][(r4 & 1) * 4 + 1] = v.y;
-                    B[r4 >> 1][(r4 & 1) * 4 + 2] = v.z;
-                    B[r4 >> 1][(r4 & 1) * 4 + 3] = v.w;
-                }
-                float xs[4][2];
-#pragma unroll
-                for (int bq = 0; bq < 4; ++bq) {
-                    xs[bq][0] = 2 * t < ntok ? s.hsb[4 * qd + bq][2 * t] : 0.f;
-                    xs[bq][1] = 2 * t + 1 < ntok ? s.hsb[4 * qd + bq][2 * t + 1] : 0.f;
-                }
-                quad_compute<FMT>(q, B, xs, acc);
-            }
-            if (u == nC && warp == 0) TRACEW(21);
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int n = 2 * t + (r & 1);
-                if (n < ntok) {
-                    const int row = 16 * rg + g + ((r & 2) ? 8 : 0);
-                    const int sp = beg + n;
-                    const int tk = shared ? n : s.s_tok[sp];
-                    const float gw = shared ? 1.f : s.w[tk][s.s_j[sp]];
-                    atomicAdd(p.y + size_t(tk) * d + row, gw * acc[r]);
-                }
-            }
-            __syncthreads();  // slot, sh, bfrag and hsb read by everyone
-            if (u == nC) TRACE(22);
-            if (tid == 0 && ring_issued < nU) issue(ring_issued++);
+        const float inv = 1.0f / z;
+        if (sel) {
+            s.idx[warp][rank] = my_id;
+            s.w[warp][rank] = ex * inv;
         }
     }
+    __syncthreads();
+}
 
-    // the last CTA publishes routing, permutation, slots and misses (nothing in
-    // this launch reads them, so it happens after the compute)
-    if (cta == G - 1) {
-        for (int i = tid; i < npairs; i += kThreads) {
-            const int t = i / k, j = i % k;
-            if (p.topk_idx) p.topk_idx[i] = s.idx[t][j];
-            if (p.topk_w) p.topk_w[i] = s.w[t][j];
-            if (p.sorted_tok) p.sorted_tok[i] = s.s_tok[i];
-            if (p.sorted_j) p.sorted_j[i] = s.s_j[i];
-            if (p.inv) p.inv[i] = s.inv[i];
+// Routing tables from s.idx: sorted pairs, active experts with their slots,
+// resident list, miss bases, and the task count. Whole CTA.
+__device__ void routing_tables(const DecodeParams &p, Smem &s, int T, int k) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int npairs = T * k;
+    if (tid < npairs) {  // stable sort of the pairs by (expert, pair index)
+        const int pp = tid;
+        const int e = s.idx[pp / k][pp % k];
+        int rank = 0;
+        for (int q = 0; q < npairs; ++q) {
+            const int eq = s.idx[q / k][q % k];
+            rank += (eq < e) || (eq == e && q < pp);
         }
+        s.pair_e[rank] = e;
+        s.s_tok[rank] = pp / k;
+        s.s_j[rank] = pp % k;
+        s.inv[pp] = rank;
+    }
+    __syncthreads();
+    const bool in = tid < npairs;
+    const bool first = in && (tid == 0 || s.pair_e[tid] != s.pair_e[tid - 1]);
+    const unsigned fm = __ballot_sync(0xffffffffu, first);
+    if (lane == 0 && warp < kMaxPairs / 32) s.first_mask[warp] = fm;
+    __syncthreads();
+    if (first) {
+        int a = __popc(fm & ((1u << lane) - 1));
+        for (int w = 0; w < warp; ++w) a += __popc(s.first_mask[w]);
+        const int e = s.pair_e[tid];
+        const int sl = (e >= 0 && e < p.E) ? s.slot[e] : -1;
+        const bool bad = sl < -1 || sl >= p.num_slots;
+        if (bad && blockIdx.x == 0) flag(p.status, MOE_DEV_BAD_SLOT);
+        s.act_e[a] = e;
+        s.act_beg[a] = tid;
+        s.act_slot[a] = bad ? -1 : sl;
+    }
+    if (tid == 0) {
+        int na = 0;
+        for (int w = 0; w < (npairs + 31) / 32; ++w) na += __popc(s.first_mask[w]);
+        s.nact = na;
+    }
+    __syncthreads();
+    const int na = s.nact;
+    if (tid < na) s.act_cnt[tid] = (tid + 1 < na ? s.act_beg[tid + 1] : npairs) - s.act_beg[tid];
+    __syncthreads();
+    if (warp == 0) {  // resident list and miss bases over <= 128 actives, 32 at a time
+        int nr = 0, nm = 0;
+        for (int a0 = 0; a0 < na; a0 += 32) {
+            const int a = a0 + lane;
+            const bool act = a < na;
+            const bool res = act && s.act_slot[a] >= 0;
+            const int cm = act && !res ? s.act_cnt[a] : 0;
+            const unsigned rm = __ballot_sync(0xffffffffu, res);
+            int mpre = cm;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, mpre, o);
+                if (lane >= o) mpre += v;
+            }
+            if (act) s.act_mbase[a] = nm + mpre - cm;
+            if (res) s.res[nr + __popc(rm & ((1u << lane) - 1))] = a;
+            nr += __popc(rm);
+            nm += __shfl_sync(0xffffffffu, mpre, 31);
+        }
+        if (lane == 0) {
+            s.nres = nr;
+            s.nmiss = nm;
+            s.ntask = (nr + 1) * p.g.NHB;
+        }
+    }
+    __syncthreads();
+}
+
+// Routing, permutation, slots and misses of layer l to global memory (one CTA).
+__device__ void publish(const DecodeParams &p, Smem &s, int l, int T, int k, int E) {
+    const int tid = threadIdx.x;
+    const int npairs = T * k;
+    const size_t po = size_t(l) * npairs;
+    for (int i = tid; i < npairs; i += kThreads) {
+        const int t = i / k, j = i % k;
+        if (p.topk_idx) p.topk_idx[po + i] = s.idx[t][j];
+        if (p.topk_w) p.topk_w[po + i] = s.w[t][j];
+        if (p.sorted_tok) p.sorted_tok[i] = s.s_tok[i];
+        if (p.sorted_j) p.sorted_j[i] = s.s_j[i];
+        if (p.inv) p.inv[i] = s.inv[i];
+    }
+    if (p.offsets || p.counts) {
         for (int e = tid; e <= E; e += kThreads) {
             int lo = 0, hi = s.nact;  // first active expert >= e
             while (lo < hi) {
@@ -1037,66 +642,470 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_kernel(Deco
             if (p.offsets) p.offsets[e] = lo < s.nact ? s.act_beg[lo] : npairs;
             if (p.counts && e < E) p.counts[e] = (lo < s.nact && s.act_e[lo] == e) ? s.act_cnt[lo] : 0;
         }
-        if (p.active) {
-            for (int a = tid; a < s.nact; a += kThreads) p.active[1 + a] = s.act_e[a];
-            if (tid == 0) p.active[0] = s.nact;
-        }
-        for (int sp = tid; sp < npairs; sp += kThreads) {
-            int a = 0;
-            while (a + 1 < s.nact && s.act_beg[a + 1] <= sp) ++a;
-            const bool res = s.act_slot[a] >= 0;
-            const int pp = s.s_tok[sp] * k + s.s_j[sp];
-            if (p.slot_of_pair) p.slot_of_pair[pp] = res ? s.act_slot[a] : -1;
-            if (!res && p.miss) {
-                const int mi = s.act_mbase[a] + (sp - s.act_beg[a]);
-                if (mi < p.miss_cap) {
-                    moe_miss m;
-                    m.layer = p.layer;
-                    m.expert = s.act_e[a];
-                    m.token = s.s_tok[sp];
-                    m.j = s.s_j[sp];
-                    m.gate = s.w[m.token][m.j];
-                    p.miss[mi] = m;
-                }
+    }
+    if (p.active) {
+        for (int a = tid; a < s.nact; a += kThreads) p.active[1 + a] = s.act_e[a];
+        if (tid == 0) p.active[0] = s.nact;
+    }
+    moe_miss *miss = p.miss ? p.miss + size_t(l) * p.miss_cap : nullptr;
+    for (int sp = tid; sp < npairs; sp += kThreads) {
+        int a = 0;
+        while (a + 1 < s.nact && s.act_beg[a + 1] <= sp) ++a;
+        const bool res = s.act_slot[a] >= 0;
+        const int pp = s.s_tok[sp] * k + s.s_j[sp];
+        if (p.slot_of_pair) p.slot_of_pair[po + pp] = res ? s.act_slot[a] : -1;
+        if (!res && miss) {
+            const int mi = s.act_mbase[a] + (sp - s.act_beg[a]);
+            if (mi < p.miss_cap) {
+                moe_miss m;
+                m.layer = p.layer0 + l;
+                m.expert = s.act_e[a];
+                m.token = s.s_tok[sp];
+                m.j = s.s_j[sp];
+                m.gate = s.w[m.token][m.j];
+                miss[mi] = m;
             }
         }
-        if (tid == 0) {
-            if (p.miss_count) *p.miss_count = s.nmiss;
-            if (s.nmiss > p.miss_cap && p.miss) flag(p.status, MOE_DEV_MISS_OVERFLOW);
+    }
+    if (tid == 0) {
+        if (p.miss_count) p.miss_count[l] = s.nmiss;
+        if (s.nmiss > p.miss_cap && p.miss) flag(p.status, MOE_DEV_MISS_OVERFLOW);
+    }
+}
+
+template <int FMT, int NT>
+__global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams p) {
+    extern __shared__ __align__(128) unsigned char dyn[];
+    __shared__ Smem s;
+    const Geo &g = p.g;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = gridDim.x, cta = blockIdx.x;
+    const unsigned rank = cluster_rank(), cid = cluster_id(), ncl = cluster_count();
+    const int T = p.T, k = p.k, E = p.E, d = p.d;
+    const int gl = lane >> 2, tl = lane & 3;  // MMA fragment coordinates of this lane
+    uint4 *bfx = reinterpret_cast<uint4 *>(dyn + g.off_bfx);  // x B fragments [NQR][8][32]
+    float *part = reinterpret_cast<float *>(dyn + g.off_part);  // [2][HB/16][32][8] partials
+    float *hs = reinterpret_cast<float *>(dyn + g.off_h);       // [HB][8] h of the task
+    uint32_t *bfh = reinterpret_cast<uint32_t *>(dyn + g.off_bfh);  // [HB/64][8][32] h B fragments
+    uint8_t *ring = dyn + g.off_ring;
+    const int part_floats = int(g.part_bytes / 4);
+    bool too_big = false, ok = true;
+    unsigned bar_target = 0;  // grid barrier arrivals this CTA has waited for
+    // per-warp ring bookkeeping (identical in every lane of a warp)
+    int seq = 0;  // tasks of this CTA started so far, over all layers (buffer = seq % nbuf)
+
+    if (tid == 0) {
+        bar_init(&s.rt_bar, 1);
+        for (int b = 0; b < kMaxBuf; ++b)
+            for (int w = 0; w < kWarps; ++w) {
+                bar_init(&s.gu_bar[b][w], 1);
+                bar_init(&s.dn_bar[b][w], 1);
+            }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    // rows of the router this CTA computes (contiguous, about E/G)
+    const int rb = int(int64_t(E) * cta / G), re = int(int64_t(E) * (cta + 1) / G);
+    const int nrows = re - rb;
+
+    for (int l = 0; l < p.L; ++l) {
+        const LayerPtrs lp = layer_ptrs(p, l);
+        TRACE(0);
+        // ------------------------------------------------ router rows + activations
+        float *rrows = reinterpret_cast<float *>(ring);  // router rows, then x, in the ring
+        uint16_t *sx = reinterpret_cast<uint16_t *>(ring + size_t(nrows) * d * 4);
+        if (tid == 0 && nrows > 0) {
+            bar_expect(&s.rt_bar, uint32_t(nrows) * uint32_t(d) * 4u);
+            bulk_copy(rrows, lp.Wr + size_t(rb) * d, uint32_t(nrows) * uint32_t(d) * 4u, &s.rt_bar);
         }
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(lp.x);
+            uint4 *dst = reinterpret_cast<uint4 *>(sx);
+            for (int i = tid; i < T * d / 8; i += kThreads) dst[i] = __ldg(src + i);
+            for (int e = tid; e < E; e += kThreads) s.slot[e] = __ldg(lp.slot_of + e);
+            // this CTA's slice of y starts at zero (before the grid barrier, so before any atomic)
+            for (int i = cta * kThreads + tid; i < T * d; i += G * kThreads) lp.y[i] = 0.f;
+        }
+        __syncthreads();
+        // block sums of x over this CTA's K slice, and its B fragments (all 8 token columns)
+        const int k0 = int(rank) * g.KR;
+        for (int job = warp; job < (g.KR / 64) * T; job += kWarps) {
+            const int bb = job / T, n = job % T;
+            const uint32_t u = *reinterpret_cast<const uint32_t *>(sx + size_t(n) * d + k0 + 64 * bb + 2 * lane);
+            float v = bf16_lo(u) + bf16_hi(u);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) s.xs[bb][n] = v;
+        }
+        for (int e = tid; e < g.NQR * 256; e += kThreads) {
+            const int qi = e >> 8, ln = (e >> 3) & 31, r4 = e & 7;
+            const int gg = ln >> 2, tt = ln & 3, bq = r4 >> 1;
+            const uint16_t *src = gg < T ? sx + size_t(gg) * d + k0 + 256 * qi + 64 * bq : nullptr;
+            uint32_t v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int rho = (r4 & 1) * 4 + j;
+                float lo = 0.f, hi = 0.f;
+                if (src) {
+                    const uint32_t u = *reinterpret_cast<const uint32_t *>(src + slot_k(rho, tt, 0));
+                    lo = bf16_lo(u);
+                    hi = bf16_hi(u);
+                }
+                const float sc = __int_as_float((127 - slot_exp<FMT>(bq, rho)) << 23);  // 2^-exp
+                v[j] = pack_half2(lo * sc, hi * sc);
+            }
+            bfx[(qi * 8 + r4) * 32 + ln] = make_uint4(v[0], v[1], v[2], v[3]);
+        }
+        if (nrows > 0) {
+            const bool got = bar_wait(&s.rt_bar, uint32_t(l & 1));
+            if (!got && tid == 0) flag(p.status, MOE_DEV_TIMEOUT);
+            ok = ok && got;
+            if (got && warp < nrows)
+                router_row<NT>(rrows + size_t(warp) * d, sx, T, d, lane, lp.bias, rb + warp, lp.logits, E, p.status);
+            for (int r = warp + kWarps; got && r < nrows; r += kWarps)
+                router_row<NT>(rrows + size_t(r) * d, sx, T, d, lane, lp.bias, rb + r, lp.logits, E, p.status);
+        }
+        ok = __syncthreads_and(ok) != 0;  // logits written; router rows and x consumed (the ring is free)
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(p.ctr, 1u);
+        }
+        bar_target += unsigned(G);
+        TRACE(1);
+        // this cluster's tasks known before routing: the shared expert's blocks
+        const int nsh = g.NHB;
+        int known = 0;  // tasks of this cluster whose index is known (its list: cid, cid + ncl, ...)
+        while (int(cid) + known * int(ncl) < nsh) ++known;
+        const int seq0 = seq;  // this layer's first task of this CTA
+        int gu_next = 0, dn_next = 0;  // next task (layer-local) whose slices this warp copies
+        auto issue_upto = [&](int n_known, int gu_done, int dn_done) {
+            while (gu_next < n_known && gu_next < gu_done + g.nbuf) {
+                int hb, a;
+                const int slot = task_slot(p, s, lp, int(cid) + gu_next * int(ncl), hb, a);
+                issue_gu<FMT>(p, s, ring, (seq0 + gu_next) % g.nbuf, warp, lane, rank, slot, hb);
+                ++gu_next;
+            }
+            while (dn_next < n_known && dn_next < dn_done + g.nbuf) {
+                int hb, a;
+                const int slot = task_slot(p, s, lp, int(cid) + dn_next * int(ncl), hb, a);
+                issue_dn<FMT>(p, s, ring, (seq0 + dn_next) % g.nbuf, warp, lane, rank, slot, hb);
+                ++dn_next;
+            }
+        };
+        if (ok) issue_upto(known, 0, 0);
+        // the next layer's router rows and a slice of its shared expert into the L2
+        if (tid == 0 && l + 1 < p.L) {
+            const LayerPtrs np = layer_ptrs(p, l + 1);
+            if (nrows > 0) prefetch_l2(np.Wr + size_t(rb) * d, uint32_t(nrows) * uint32_t(d) * 4u);
+            const uint64_t eb = uint64_t(p.down.codes_off) + p.down.bytes;  // record bytes
+            const uint64_t c0 = (eb * uint64_t(cta) / uint64_t(G)) & ~uint64_t(15);
+            const uint64_t c1 = (eb * uint64_t(cta + 1) / uint64_t(G)) & ~uint64_t(15);
+            if (c1 > c0) prefetch_l2(p.pool + int64_t(np.shared_slot) * p.slot_bytes + c0, uint32_t(c1 - c0));
+            if (cta == 0) prefetch_l2(np.slot_of, uint32_t(E) * 4u);
+        }
+        // ------------------------------------------------ grid barrier: all logits written
+        if (tid == 0) s.ok = wait_geq(p.ctr, bar_target, p.status);
+        __syncthreads();
+        ok = ok && s.ok;
+        TRACE(2);
+        if (ok) {
+            topk_cta<NT>(p, s, lp.logits, T, E, k);
+            TRACE(3);
+            routing_tables(p, s, T, k);
+        }
+        TRACE(4);
+        // every CTA of the cluster runs the same number of tasks (and cluster barriers):
+        // if any of them failed to route, none of them runs a task
+        if (tid == 0) s.last = ok ? s.ntask : -1;
+        cluster_sync();
+        int ntask = s.last;
+        for (int r = 0; r < g.C; ++r)
+            if (unsigned(r) != rank) ntask = min(ntask, ld_peer_int(peer_addr(&s.last, unsigned(r))));
+        cluster_sync();  // the peers' flags are read before anyone changes them
+        if (ntask < 0) {
+            ntask = 0;
+            ok = false;
+        }
+        const int nmine = ntask > int(cid) ? (ntask - int(cid) + int(ncl) - 1) / int(ncl) : 0;
+        if (ok) issue_upto(nmine, 0, 0);
+        // ------------------------------------------------ tasks
+        for (int i = 0; i < nmine; ++i) {
+            const int b = (seq0 + i) % g.nbuf;
+            const uint32_t ph = uint32_t((seq0 + i) / g.nbuf) & 1u;
+            int hb, a;
+            task_slot(p, s, lp, int(cid) + i * int(ncl), hb, a);
+            float *mypart = part + size_t(i & 1) * part_floats;
+            // gate/up partial sums of this warp's row groups over this CTA's K slice
+            bool got = ok && bar_wait(&s.gu_bar[b][warp], ph);
+            if (i == 0) TRACE(5);
+            if (got) {
+                const uint8_t *slice = ring + size_t(b) * g.region + size_t(warp) * g.gu_warp;
+                for (int gi = 0; gi < g.GUW; ++gi) {
+                    float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
+                    const uint8_t *gc = slice + size_t(gi * 2) * (g.gu_c + g.gu_s);
+                    const uint8_t *uc = gc + (g.gu_c + g.gu_s);
+                    for (int qi = 0; qi < g.NQR; ++qi) {
+                        uint32_t B[4][8];
+#pragma unroll
+                        for (int r4 = 0; r4 < 8; ++r4) {
+                            const uint4 v = bfx[(qi * 8 + r4) * 32 + lane];
+                            B[r4 >> 1][(r4 & 1) * 4 + 0] = v.x;
+                            B[r4 >> 1][(r4 & 1) * 4 + 1] = v.y;
+                            B[r4 >> 1][(r4 & 1) * 4 + 2] = v.z;
+                            B[r4 >> 1][(r4 & 1) * 4 + 3] = v.w;
+                        }
+                        float xs[4][2];
+#pragma unroll
+                        for (int bq = 0; bq < 4; ++bq) {
+                            xs[bq][0] = 2 * tl < T ? s.xs[4 * qi + bq][2 * tl] : 0.f;
+                            xs[bq][1] = 2 * tl + 1 < T ? s.xs[4 * qi + bq][2 * tl + 1] : 0.f;
+                        }
+                        QuadRegs<FMT> qg, qu;
+                        quad_smem<FMT>(gc, gc + g.gu_c, qi, lane, qg);
+                        quad_smem<FMT>(uc, uc + g.gu_c, qi, lane, qu);
+                        quad_compute<FMT>(qg, B, xs, ag);
+                        quad_compute<FMT>(qu, B, xs, au);
+                    }
+                    float4 *dst = reinterpret_cast<float4 *>(mypart + (size_t(warp + 8 * gi) * 32 + lane) * 8);
+                    dst[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
+                    dst[1] = make_float4(au[0], au[1], au[2], au[3]);
+                }
+            }
+            if (!got && ok && lane == 0) flag(p.status, MOE_DEV_TIMEOUT);
+            ok = ok && __all_sync(0xffffffffu, got);
+            __syncwarp();
+            // this warp's gate/up slice of buffer b is free: copy ahead
+            if (ok) issue_upto(nmine, i + 1, i);
+            if (i == 0) TRACE(6);
+            // ---- exchange the partials inside the cluster
+            cluster_sync();
+            if (i == 0) TRACE(7);
+            ok = __syncthreads_and(ok) != 0;
+            // h = silu(a) * u for the HB rows x T tokens, partials summed in rank order
+            for (int e = tid; e < g.HB * NT; e += kThreads) {
+                const int row = e / NT, tok = e % NT;
+                const int lrg = row >> 4, rr = row & 15;
+                const int ln = 4 * (rr & 7) + (tok >> 1), ix = 2 * (rr >> 3) + (tok & 1);
+                const float *src = mypart + (size_t(lrg) * 32 + ln) * 8 + ix;
+                float A = 0.f, U = 0.f;
+                for (int r = 0; r < g.C; ++r) {
+                    float av, uv;
+                    if (unsigned(r) == rank) {
+                        av = src[0];
+                        uv = src[4];
+                    } else {
+                        av = ld_peer(peer_addr(src, unsigned(r)));
+                        uv = ld_peer(peer_addr(src + 4, unsigned(r)));
+                    }
+                    A = r == 0 ? av : A + av;
+                    U = r == 0 ? uv : U + uv;
+                }
+                const float h = (ok && tok < T) ? A / (1.0f + expf(-A)) * U : 0.f;
+                too_big |= !(fabsf(h) <= 65504.f);
+                hs[row * 8 + tok] = h;
+            }
+            if (tid < NT) {  // gate of each token for this task
+                float gw = 0.f;
+                if (tid < T) {
+                    if (a < 0) {
+                        gw = 1.f;
+                    } else {
+                        for (int n = 0; n < s.act_cnt[a]; ++n) {
+                            const int sp = s.act_beg[a] + n;
+                            if (s.s_tok[sp] == tid) gw = s.w[tid][s.s_j[sp]];
+                        }
+                    }
+                }
+                s.gsel[tid] = gw;
+            }
+            __syncthreads();
+            // B fragments of h for the task's HB down columns (8 token columns) and block sums
+            const int nbh = g.HB / 64;
+            for (int e = tid; e < nbh * 8 * 32; e += kThreads) {
+                const int bq = e >> 8, rho = (e >> 5) & 7, ln = e & 31;
+                const int gg = ln >> 2, tt = ln & 3;
+                const int kk = 64 * bq + slot_k(rho, tt, 0);
+                const float lo = gg < NT ? hs[kk * 8 + gg] : 0.f, hi = gg < NT ? hs[(kk + 1) * 8 + gg] : 0.f;
+                const float sc = __int_as_float((127 - slot_exp<FMT>(bq, rho)) << 23);
+                bfh[e] = pack_half2(lo * sc, hi * sc);
+            }
+            for (int job = warp; job < nbh * NT; job += kWarps) {
+                const int bq = job / NT, n = job % NT;
+                float v = hs[(64 * bq + lane) * 8 + n] + hs[(64 * bq + 32 + lane) * 8 + n];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0) s.hsb[bq][n] = v;
+            }
+            __syncthreads();
+            // ---- down rows of this CTA over the task's columns
+            float *yst = part + size_t((i + 1) & 1) * part_floats;  // staging [NT][DR] in the other partial buffer
+            got = ok && bar_wait(&s.dn_bar[b][warp], ph);
+            if (got) {
+                const uint8_t *slice =
+                    ring + size_t(b) * g.region + size_t(kWarps) * g.gu_warp + size_t(warp) * g.dn_warp;
+                float xs[4][2];
+#pragma unroll
+                for (int bq = 0; bq < 4; ++bq) {
+                    xs[bq][0] = bq < nbh && 2 * tl < T ? s.hsb[bq][2 * tl] : 0.f;
+                    xs[bq][1] = bq < nbh && 2 * tl + 1 < T ? s.hsb[bq][2 * tl + 1] : 0.f;
+                }
+                for (int j = 0; j < g.NDRW; ++j) {
+                    const uint8_t *cb = slice + size_t(j) * (g.dn_c + g.dn_s);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    if constexpr (FMT == 2) {
+                        uint32_t B[2][8];
+#pragma unroll
+                        for (int bq = 0; bq < 2; ++bq)
+#pragma unroll
+                            for (int rho = 0; rho < 8; ++rho) B[bq][rho] = bfh[(bq * 8 + rho) * 32 + lane];
+                        const uint4 c = *reinterpret_cast<const uint4 *>(cb + lane * 16);
+                        const uint4 sv = *reinterpret_cast<const uint4 *>(cb + g.dn_c + gl * 16);
+                        const float xs2[2][2] = {{xs[0][0], xs[0][1]}, {xs[1][0], xs[1][1]}};
+                        pair_compute_q2(c, sv, B, xs2, acc);
+                    } else {
+                        uint32_t B[4][8];
+#pragma unroll
+                        for (int bq = 0; bq < 4; ++bq)
+#pragma unroll
+                            for (int rho = 0; rho < 8; ++rho) B[bq][rho] = bfh[(bq * 8 + rho) * 32 + lane];
+                        QuadRegs<FMT> q;
+                        quad_smem<FMT>(cb, cb + g.dn_c, 0, lane, q);
+                        quad_compute<FMT>(q, B, xs, acc);
+                    }
+                    const int rl = (warp * g.NDRW + j) * 16 + gl;  // row inside this CTA's DR rows
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int n = 2 * tl + (r & 1);
+                        if (n < NT) yst[n * g.DR + rl + ((r & 2) ? 8 : 0)] = acc[r];
+                    }
+                }
+            }
+            if (!got && ok && lane == 0) flag(p.status, MOE_DEV_TIMEOUT);
+            ok = ok && __all_sync(0xffffffffu, got);
+            __syncwarp();
+            if (ok) issue_upto(nmine, i + 1, i + 1);
+            ok = __syncthreads_and(ok) != 0;
+            if (i == 0) TRACE(8);
+            // ---- gate-weighted vector atomics into y
+            if (ok) {
+                const int nv = T * (g.DR / 4);
+                for (int e = tid; e < nv; e += kThreads) {
+                    const int n = e / (g.DR / 4), r4 = e % (g.DR / 4);
+                    const float gw = s.gsel[n];
+                    if (gw != 0.f) {
+                        const float4 v = *reinterpret_cast<const float4 *>(yst + n * g.DR + 4 * r4);
+                        red_add4(lp.y + size_t(n) * d + int(rank) * g.DR + 4 * r4, gw * v.x, gw * v.y, gw * v.z,
+                                 gw * v.w);
+                    }
+                }
+            }
+            __syncthreads();  // staging, h and fragments reused by the next task
+            if (i == 0) TRACE(9);
+        }
+        seq += nmine;
+        // copies issued for tasks that never ran (error paths) land before their buffers are reused
+        if (gu_next > nmine || dn_next > nmine) {
+            for (int i = nmine; i < max(gu_next, dn_next); ++i) {
+                const int b = (seq0 + i) % g.nbuf;
+                const uint32_t ph = uint32_t((seq0 + i) / g.nbuf) & 1u;
+                if (i < gu_next) bar_wait(&s.gu_bar[b][warp], ph);
+                if (i < dn_next) bar_wait(&s.dn_bar[b][warp], ph);
+            }
+            seq = seq0 + max(gu_next, dn_next);
+        }
+        if (ok && cta == G - 1) publish(p, s, l, T, k, E);
+        // ------------------------------------------------ grid barrier: the layer is complete
+        // (the next layer starts only once every contribution to this one is in y)
+        if (l + 1 < p.L) {
+            __syncthreads();
+            if (tid == 0) {
+                __threadfence();
+                atomicAdd(p.ctr, 1u);
+            }
+            bar_target += unsigned(G);
+            if (tid == 0) s.ok = wait_geq(p.ctr, bar_target, p.status);
+            __syncthreads();
+            ok = ok && s.ok;
+        }
+        TRACE(10);
     }
 
-finish:
-    if (tid == 0)  // copies still in flight (error paths only) land before the CTA leaves
-        for (int u = ring_used; u < ring_issued; ++u)
-            if (!ring_wait(&s.full[u % p.nslots], uint32_t(u / p.nslots) & 1u)) break;
     if (too_big) flag(p.status, MOE_DEV_NONFINITE);
-    __syncthreads();
-    TRACE(4);
+    // no CTA leaves while a peer may still read its shared memory
+    cluster_sync();
     if (tid == 0) {
         __threadfence();
         s.last = atomicAdd(p.ctr + 1, 1u) == unsigned(G - 1);
     }
     __syncthreads();
-    if (s.last) {  // every CTA is done with the counters: reset them for the next launch
-        for (int i = tid; i <= kMaxPairs; i += kThreads) p.done[i] = 0u;
-        if (tid == 0) p.ctr[0] = 0u;
+    if (s.last && tid == 0) {  // every CTA is done with the counters: reset them for the next launch
+        p.ctr[0] = 0u;
         __threadfence();
-        __syncthreads();
-        if (tid == 0) {
-            p.ctr[1] = 0u;
-            __threadfence();
-        }
+        p.ctr[1] = 0u;
+        __threadfence();
     }
 }
 
-struct LaunchCache {
-    int grid[8][64] = {};
-    int avail[8][64] = {};  // dynamic shared memory a CTA can have
-    bool ready[8][64] = {};
+
+// ---------------------------------------------------------------- host side
+size_t ws_align(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Launch geometry and shared-memory layout for (fmt, T, d, f) with `avail`
+// bytes of dynamic shared memory per CTA and G CTAs; false if it does not fit.
+bool plan(int fmt, int T, int d, int f, int E, int G, size_t avail, Geo &g) {
+    g.C = d % 1024 == 0 ? 4 : (d % 512 == 0 ? 2 : 1);
+    g.HB = fmt == 2 ? 128 : 256;
+    if (f % g.HB) return false;
+    g.NHB = f / g.HB;
+    g.KR = d / g.C;
+    g.NQR = g.KR / 256;
+    g.DR = d / g.C;
+    g.NDRW = g.DR / 128;
+    g.GUW = g.HB / 128;
+    if (g.NQR < 1 || g.NDRW < 1) return false;
+    g.gu_c = uint32_t(g.NQR) * (fmt == 2 ? 1024u : 1536u);
+    g.gu_s = uint32_t(g.NQR) * (fmt == 2 ? 256u : 128u);
+    g.dn_c = fmt == 2 ? 512u : 1536u;
+    g.dn_s = 128u;
+    g.gu_warp = uint32_t(g.GUW) * 2u * (g.gu_c + g.gu_s);
+    g.dn_warp = uint32_t(g.NDRW) * (g.dn_c + g.dn_s);
+    g.region = uint32_t(kWarps) * (g.gu_warp + g.dn_warp);
+    const int NTp = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8;
+    g.part_bytes = uint32_t((std::max<size_t>(size_t(g.HB) * 64, size_t(NTp) * g.DR * 4) + 127) & ~size_t(127));
+    size_t off = 0;
+    g.off_bfx = uint32_t(off);
+    off += size_t(g.NQR) * 4096;
+    g.off_part = uint32_t(off);
+    off += 2 * size_t(g.part_bytes);
+    g.off_h = uint32_t(off);
+    off += size_t(g.HB) * 8 * 4;
+    g.off_bfh = uint32_t(off);
+    off += size_t(g.HB / 64) * 1024;
+    off = (off + 127) & ~size_t(127);
+    g.off_ring = uint32_t(off);
+    if (avail < off + g.region) return false;
+    g.nbuf = int(std::min<size_t>(kMaxBuf, (avail - off) / g.region));
+    const int rows = (E + G - 1) / G;
+    const size_t router = size_t(rows) * d * 4 + size_t(T) * d * 2;  // router rows + x, staged in the ring
+    size_t ring = size_t(g.nbuf) * g.region;
+    if (ring < router) {
+        if (off + router > avail) return false;
+        ring = router;
+    }
+    g.total = uint32_t(off + ring);
+    return true;
+}
+
+struct LaunchInfo {
+    bool ready = false;
+    int sms = 0;
+    size_t avail = 0;   // dynamic shared memory a CTA can have
+    int grid[5] = {};   // CTAs per launch for cluster size C (index C), 0 = not known yet
+    bool coop = true;   // cooperative launches of clusters accepted
 };
 std::mutex g_mu;
-LaunchCache g_cache;
+LaunchInfo g_info[8][64];
 
 template <int FMT, int NT>
 moe_status launch(DecodeParams p, cudaStream_t stream) {
@@ -1106,42 +1115,73 @@ moe_status launch(DecodeParams p, cudaStream_t stream) {
         return MOE_ERR_CUDA;
     }
     constexpr int ci = (FMT - 2) * 4 + (NT == 1 ? 0 : NT == 2 ? 1 : NT == 4 ? 2 : 3);
-    int grid, avail;
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        if (!g_cache.ready[ci][dev]) {
-            int sms = 0, per = 0, optin = 0;
-            cudaFuncAttributes fa;
-            if (cudaFuncGetAttributes(&fa, decode_layer_kernel<FMT, NT>) != cudaSuccess ||
-                cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-                cudaGetLastError();
-                return MOE_ERR_CUDA;
-            }
-            const int av = optin - int(fa.sharedSizeBytes);
-            if (av <= 0 ||
-                cudaFuncSetAttribute(decode_layer_kernel<FMT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, av) !=
-                    cudaSuccess ||
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, decode_layer_kernel<FMT, NT>, kThreads, av) !=
-                    cudaSuccess ||
-                per < 1) {
-                cudaGetLastError();
-                return MOE_ERR_CUDA;
-            }
-            g_cache.grid[ci][dev] = sms * std::min(per, kCtasPerSm);
-            g_cache.avail[ci][dev] = av;
-            g_cache.ready[ci][dev] = true;
+    auto kern = decode_layer_kernel<FMT, NT>;
+    const int C = p.d % 1024 == 0 ? 4 : (p.d % 512 == 0 ? 2 : 1);
+    std::lock_guard<std::mutex> lock(g_mu);
+    LaunchInfo &li = g_info[ci][dev];
+    if (!li.ready) {
+        int optin = 0, sms = 0;
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
         }
-        grid = g_cache.grid[ci][dev];
-        avail = g_cache.avail[ci][dev];
+        const int av = optin - int(fa.sharedSizeBytes);
+        if (av <= 0 || cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, av) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        li.sms = sms;
+        li.avail = size_t(av);
+        li.ready = true;
     }
-    const size_t base = ring_off(p.T, p.d, p.f);
-    if (size_t(avail) < base + 2 * size_t(p.rslot)) return MOE_ERR_UNSUPPORTED;
-    p.nslots = int(std::min<size_t>(kMaxSlots, (size_t(avail) - base) / p.rslot));
-    const size_t smem = base + size_t(p.nslots) * p.rslot;
-    void *args[] = {&p};
-    if (cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(decode_layer_kernel<FMT, NT>), dim3(grid),
-                                    dim3(kThreads), args, smem, stream) != cudaSuccess) {
+    if (li.grid[C] == 0) {  // co-resident clusters of C CTAs with the largest shared-memory use
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = unsigned(C);
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(unsigned(C * (li.sms / C)));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = li.avail;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int ncl = 0;
+        if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess || ncl < 1) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        li.grid[C] = std::min(ncl * C, C * (li.sms / C));
+    }
+    const int G = li.grid[C];
+    if (!plan(FMT, p.T, p.d, p.f, p.E, G, li.avail, p.g)) return MOE_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = unsigned(C);
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeCooperative;
+    at[1].val.cooperative = 1;
+    cfg.gridDim = dim3(unsigned(G));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = p.g.total;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = li.coop ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess && li.coop) {
+        // cooperative launches of clusters refused: the grid is sized to the co-resident
+        // clusters and every grid-wide wait is bounded, so a plain cluster launch is used
+        cudaGetLastError();
+        li.coop = false;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, p);
+    }
+    if (e != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
@@ -1156,7 +1196,52 @@ moe_status launch_fmt(const DecodeParams &p, cudaStream_t stream) {
     return launch<FMT, 8>(p, stream);
 }
 
-size_t ws_align(size_t x) { return (x + 255) & ~size_t(255); }
+// Host-side checks and parameters shared by the one-layer and the stacked call.
+moe_status setup(DecodeParams &p, const moe_qpool *W, int L, const int32_t *slot_of, const uint16_t *x,
+                 const float *Wr, int T, int d, int f, int E, int k, int32_t miss_cap, moe_miss *miss, float *y,
+                 void *ws, size_t ws_bytes) {
+    if (!W || T < 0 || E <= 0 || k <= 0 || miss_cap < 0 || L < 1) return MOE_ERR_INVALID_ARG;
+    if (W->fmt != 2 && W->fmt != 3) return MOE_ERR_INVALID_ARG;
+    if (W->d != d || W->f != f) return MOE_ERR_INVALID_ARG;
+    if (!dims_ok(d, f) || d > kMaxDimDec || f > kMaxFDec || T > kMaxTokDec || E > kMaxEDec || k > kMaxK || k > E)
+        return MOE_ERR_UNSUPPORTED;
+    if (int64_t(L) * E * d >= (int64_t(1) << 40)) return MOE_ERR_OVERFLOW;
+    if (T == 0) return MOE_OK;
+    if (!slot_of || !x || !Wr || !y) return MOE_ERR_INVALID_ARG;
+    if (miss_cap > 0 && !miss) return MOE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(Wr) % 16 ||
+        reinterpret_cast<uintptr_t>(y) % 16)
+        return MOE_ERR_INVALID_ARG;
+    const ExpertGeom eg = expert_geom(W->fmt, d, f);
+    if (!W->base || W->num_slots <= 0 || W->slot_bytes < int64_t(eg.bytes) || W->slot_bytes % 256 ||
+        reinterpret_cast<uintptr_t>(W->base) % 256)
+        return MOE_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < moe_layer_decode_workspace_bytes(T, k, f, E)) return MOE_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) % 256) return MOE_ERR_INVALID_ARG;
+    p = DecodeParams{};
+    p.pool = static_cast<const uint8_t *>(W->base);
+    p.slot_bytes = W->slot_bytes;
+    p.num_slots = W->num_slots;
+    p.L = L;
+    p.slot_of = slot_of;
+    p.x = x;
+    p.Wr = Wr;
+    p.T = T;
+    p.d = d;
+    p.f = f;
+    p.E = E;
+    p.k = k;
+    p.miss = miss;
+    p.miss_cap = miss_cap;
+    p.y = y;
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    p.ctr = reinterpret_cast<unsigned *>(w);
+    p.logits = reinterpret_cast<float *>(w + 256);
+    p.gate = eg.m[0];
+    p.up = eg.m[1];
+    p.down = eg.m[2];
+    return MOE_OK;
+}
 
 }  // namespace
 }  // namespace moe
@@ -1165,9 +1250,11 @@ using namespace moe;
 
 MOE_API size_t moe_layer_decode_workspace_bytes(int T, int k, int f, int E) {
     if (T <= 0 || k <= 0 || f <= 0 || E <= 0) return 0;
-    const size_t rows = size_t(T) * k + T;
-    return ws_align(2 * sizeof(unsigned)) + ws_align((kMaxPairs + 1) * sizeof(unsigned)) +
-           ws_align(size_t(T) * E * sizeof(float)) + ws_align(rows * f * sizeof(float));
+    return 256 + ws_align(2 * size_t(T) * E * sizeof(float));
+}
+
+MOE_API size_t moe_stack_decode_workspace_bytes(int T, int k, int f, int E) {
+    return moe_layer_decode_workspace_bytes(T, k, f, E);
 }
 
 MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t shared_slot, int32_t layer,
@@ -1177,35 +1264,18 @@ MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, 
                                     int32_t *active, int32_t *slot_of_pair, moe_miss *miss, int32_t *miss_count,
                                     int32_t miss_cap, float *y, void *ws, size_t ws_bytes, int32_t *dev_status,
                                     moe_stream_t stream) {
-    if (!W || T < 0 || E <= 0 || k <= 0 || miss_cap < 0) return MOE_ERR_INVALID_ARG;
-    if (W->fmt != 2 && W->fmt != 3) return MOE_ERR_INVALID_ARG;
-    if (W->d != d || W->f != f) return MOE_ERR_INVALID_ARG;
-    if (!dims_ok(d, f) || d > kMaxDimDec || f > kMaxFDec || T > kMaxTokDec || E > kMaxEDec || k > kMaxK || k > E)
-        return MOE_ERR_UNSUPPORTED;
-    if (T == 0) return MOE_OK;
-    if (!slot_of || !x || !Wr || !y) return MOE_ERR_INVALID_ARG;
-    if (miss_cap > 0 && !miss) return MOE_ERR_INVALID_ARG;
-    const ExpertGeom eg = expert_geom(W->fmt, d, f);
-    if (!W->base || W->num_slots <= 0 || W->slot_bytes < int64_t(eg.bytes) || W->slot_bytes % 256 ||
-        reinterpret_cast<uintptr_t>(W->base) % 256 || shared_slot < 0 || shared_slot >= W->num_slots)
-        return MOE_ERR_INVALID_ARG;
-    if (!ws || ws_bytes < moe_layer_decode_workspace_bytes(T, k, f, E)) return MOE_ERR_WORKSPACE;
-    if (reinterpret_cast<uintptr_t>(ws) % 256) return MOE_ERR_INVALID_ARG;
     DecodeParams p;
-    p.pool = static_cast<const uint8_t *>(W->base);
-    p.slot_bytes = W->slot_bytes;
-    p.num_slots = W->num_slots;
-    p.slot_of = slot_of;
-    p.shared_slot = shared_slot;
-    p.layer = layer;
-    p.x = x;
-    p.Wr = Wr;
+    const moe_status st = setup(p, W, 1, slot_of, x, Wr, T, d, f, E, k, miss_cap, miss, y, ws, ws_bytes);
+    if (st != MOE_OK || T == 0) return st;
+    if (shared_slot < 0 || shared_slot >= W->num_slots) return MOE_ERR_INVALID_ARG;
+    p.shared_slot = nullptr;
+    p.shared_slot0 = shared_slot;
+    p.layer0 = layer;
     p.bias = bias;
-    p.T = T;
-    p.d = d;
-    p.f = f;
-    p.E = E;
-    p.k = k;
+    if (logits) {
+        p.logits = logits;
+        p.logits_out = true;
+    }
     p.topk_idx = topk_idx;
     p.topk_w = topk_w;
     p.counts = counts;
@@ -1215,43 +1285,29 @@ MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, 
     p.inv = inv;
     p.active = active;
     p.slot_of_pair = slot_of_pair;
-    p.miss = miss;
     p.miss_count = miss_count;
-    p.miss_cap = miss_cap;
-    p.y = y;
     p.status = dev_status;
-    unsigned char *w = static_cast<unsigned char *>(ws);
-    p.ctr = reinterpret_cast<unsigned *>(w);
-    w += ws_align(2 * sizeof(unsigned));
-    p.done = reinterpret_cast<unsigned *>(w);
-    w += ws_align((kMaxPairs + 1) * sizeof(unsigned));
-    float *lg = reinterpret_cast<float *>(w);
-    w += ws_align(size_t(T) * E * sizeof(float));
-    p.logits = logits ? logits : lg;
-    p.h = reinterpret_cast<float *>(w);
-    p.gate = eg.m[0];
-    p.up = eg.m[1];
-    p.down = eg.m[2];
-    // bytes of one row group's codes and scales (contiguous in the record), and
-    // the ring slot: a gate/up task (both matrices) or a down task (8 row groups)
-    const int fmt = W->fmt;
-    auto cbytes = [&](const MatGeom &m) {
-        return uint32_t(fmt == 2 ? q2_chunk_off(m, 1, 0, 0) - q2_chunk_off(m, 0, 0, 0)
-                                 : q3_word_off(m, 1, 0, 0, 0) - q3_word_off(m, 0, 0, 0, 0));
-    };
-    auto sbytes = [&](const MatGeom &m) { return uint32_t(scale_off(m, fmt, 1, 0, 0) - scale_off(m, fmt, 0, 0, 0)); };
-    p.gu_cb = cbytes(p.gate);
-    p.gu_sb = sbytes(p.gate);
-    p.dn_cb = cbytes(p.down);
-    p.dn_sb = sbytes(p.down);
-    if ((p.gu_cb | p.gu_sb | p.dn_cb | p.dn_sb) % 16 ||
-        (p.gate.codes_off | p.gate.scales_off | p.up.codes_off | p.up.scales_off | p.down.codes_off |
-         p.down.scales_off) % 16 ||
-        cbytes(p.up) != p.gu_cb || sbytes(p.up) != p.gu_sb)
-        return MOE_ERR_UNSUPPORTED;
-    p.rslot = (std::max(2u * (p.gu_cb + p.gu_sb), 8u * (p.dn_cb + p.dn_sb)) + 127u) & ~127u;
-    p.nslots = 0;
-    return fmt == 2 ? launch_fmt<2>(p, as_cuda(stream)) : launch_fmt<3>(p, as_cuda(stream));
+    return W->fmt == 2 ? launch_fmt<2>(p, as_cuda(stream)) : launch_fmt<3>(p, as_cuda(stream));
+}
+
+MOE_API moe_status moe_stack_decode(const moe_qpool *W, int L, const int32_t *slot_of, const int32_t *shared_slot,
+                                    int32_t layer0, const uint16_t *x, const float *Wr, const float *bias, int T,
+                                    int d, int f, int E, int k, int32_t *topk_idx, float *topk_w,
+                                    int32_t *slot_of_pair, moe_miss *miss, int32_t *miss_count, int32_t miss_cap,
+                                    float *y, void *ws, size_t ws_bytes, int32_t *dev_status, moe_stream_t stream) {
+    DecodeParams p;
+    const moe_status st = setup(p, W, L, slot_of, x, Wr, T, d, f, E, k, miss_cap, miss, y, ws, ws_bytes);
+    if (st != MOE_OK || T == 0) return st;
+    if (!shared_slot) return MOE_ERR_INVALID_ARG;
+    p.shared_slot = shared_slot;
+    p.layer0 = layer0;
+    p.bias = bias;
+    p.topk_idx = topk_idx;
+    p.topk_w = topk_w;
+    p.slot_of_pair = slot_of_pair;
+    p.miss_count = miss_count;
+    p.status = dev_status;
+    return W->fmt == 2 ? launch_fmt<2>(p, as_cuda(stream)) : launch_fmt<3>(p, as_cuda(stream));
 }
 
 MOE_API moe_status moe_debug_wait_probe(const uint32_t *counter, uint32_t target, uint64_t *elapsed_ns,

@@ -79,6 +79,18 @@ class Buffers:
     sh_active: torch.Tensor
 
 
+@dataclass
+class StackBuffers:
+    T: int
+    idx: torch.Tensor        # [L][T*k]
+    w: torch.Tensor          # [L][T*k]
+    sop: torch.Tensor        # [L][T*k]
+    miss: torch.Tensor       # [L][T*k] miss records (20 bytes each)
+    miss_count: torch.Tensor  # [L]
+    y: torch.Tensor          # [L][T][d]
+    status: torch.Tensor
+
+
 class MoEStack:
     def __init__(self, wl: Workload, device="cuda", seed: int | None = None, layers: int | None = None,
                  alpha: float = ZIPF_ALPHA):
@@ -93,6 +105,14 @@ class MoEStack:
         self.num_slots = self.L * self.R + self.L
         self.pool = torch.empty(self.num_slots * self.slot_bytes, dtype=torch.uint8, device=self.device)
         self.qpool = native.qpool(self.pool, self.slot_bytes, self.num_slots, wl.fmt, wl.d, wl.f)
+        # per-layer router weights, biases and slot tables live in [L][...] device
+        # tensors (the stacked call reads them with a layer stride); the lists
+        # hold per-layer views
+        self.Wr_all = torch.empty((self.L, wl.E, wl.d), dtype=torch.float32, device=self.device)
+        self.bias_all = torch.empty((self.L, wl.E), dtype=torch.float32, device=self.device) if wl.zipf else None
+        self.slot_of_all = torch.empty((self.L, wl.E), dtype=torch.int32, device=self.device)
+        self.shared_slot_all = torch.arange(self.L * self.R, self.L * self.R + self.L, dtype=torch.int32,
+                                            device=self.device)
         self.Wr, self.bias, self.rank, self.slot_of_host, self.slot_of, self.shared_slot = [], [], [], [], [], []
         for l in range(self.L):
             Wr = synth.gen_router(self.seed, l, wl.E, wl.d)
@@ -102,13 +122,16 @@ class MoEStack:
                 slot = np.arange(wl.E, dtype=np.int32) + l * self.R
             else:
                 slot = synth.slot_table_by_rank(rank, self.R, l * self.R)
-            self.Wr.append(_t(Wr, self.device))
-            self.bias.append(_t(bias, self.device))
+            self.Wr_all[l].copy_(torch.from_numpy(Wr))
+            self.Wr.append(self.Wr_all[l])
+            if bias is not None:
+                self.bias_all[l].copy_(torch.from_numpy(bias))
+            self.bias.append(None if bias is None else self.bias_all[l])
             self.rank.append(rank)
             self.slot_of_host.append(slot)
-            self.slot_of.append(_t(slot, self.device))
-            sh = self.L * self.R + l
-            self.shared_slot.append(torch.tensor([sh], dtype=torch.int32, device=self.device))
+            self.slot_of_all[l].copy_(torch.from_numpy(slot))
+            self.slot_of.append(self.slot_of_all[l])
+            self.shared_slot.append(self.shared_slot_all[l:l + 1])
         # every resident expert and each layer's shared expert: generated on host
         # threads, packed on the current stream in order, one wait at the end
         jobs = [(l, e, int(self.slot_of_host[l][e])) for l in range(self.L) for e in range(wl.E)
@@ -240,6 +263,42 @@ class MoEStack:
                             miss_cap=b.idx.numel() if o else 0, y=b.y, ws=ws, ws_bytes=ws.numel(),
                             dev_status=b.status, stream=stream)
         return b
+
+    def stack_buffers(self, T: int) -> "StackBuffers":
+        """Outputs of moe_stack_decode for T tokens through all L layers (kept per T)."""
+        key = ("stack", T)
+        if key not in self._ws:
+            wl, dev, L = self.wl, self.device, self.L
+            n = max(T * wl.k, 1)
+            i32 = dict(dtype=torch.int32, device=dev)
+            self._ws[key] = StackBuffers(
+                T=T, idx=torch.empty(L, n, **i32), w=torch.empty(L, n, dtype=torch.float32, device=dev),
+                sop=torch.empty(L, n, **i32), miss=torch.empty(L, n * native.MISS_BYTES, dtype=torch.uint8, device=dev),
+                miss_count=torch.zeros(L, **i32), y=torch.empty(L, max(T, 1), wl.d, dtype=torch.float32, device=dev),
+                status=torch.zeros(1, **i32))
+        return self._ws[key]
+
+    def forward_stack(self, x: torch.Tensor, b: "StackBuffers | None" = None, stream=None) -> "StackBuffers":
+        """Enqueue all L layers as one moe_stack_decode launch; x is [L][T][d]
+        (bf16 bits), layer l's input in x[l]. T <= 8."""
+        wl = self.wl
+        T = x.shape[1]
+        b = b or self.stack_buffers(T)
+        ws = self.decode_workspace(T)
+        n = max(T * wl.k, 1)
+        native.stack_decode(self.qpool, self.L, self.slot_of_all, self.shared_slot_all, 0, x, self.Wr_all,
+                            self.bias_all, T, wl.d, wl.f, wl.E, wl.k, topk_idx=b.idx, topk_w=b.w, slot_of_pair=b.sop,
+                            miss=b.miss, miss_count=b.miss_count, miss_cap=n, y=b.y, ws=ws, ws_bytes=ws.numel(),
+                            dev_status=b.status, stream=stream)
+        return b
+
+    def stack_misses(self, b: "StackBuffers", layer: int) -> list:
+        """Miss records of one layer of the last forward_stack (host copy; synchronises)."""
+        n = min(int(b.miss_count[layer].item()), b.idx.shape[1])
+        raw = b.miss[layer, : n * native.MISS_BYTES].cpu().numpy().tobytes()
+        rec = np.frombuffer(raw, dtype=np.dtype([("layer", "<i4"), ("expert", "<i4"), ("token", "<i4"),
+                                                 ("j", "<i4"), ("gate", "<f4")]))
+        return [(int(r["layer"]), int(r["expert"]), int(r["token"]), int(r["j"]), float(r["gate"])) for r in rec]
 
     def misses(self, b: Buffers) -> list:
         """Miss records of the last forward (host copy; synchronises)."""

@@ -69,6 +69,9 @@ SIGNATURES = {
     "moe_layer_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "moe_layer_decode": (_I, [C.POINTER(QPool), _P, _I32, _I32, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                               _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _SZ, _P, _P]),
+    "moe_stack_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "moe_stack_decode": (_I, [C.POINTER(QPool), _I, _P, _P, _I32, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P,
+                              _P, _I32, _P, _P, _SZ, _P, _P]),
     "moe_complete_misses_host": (_I, [_I, _I, _I, _P, _I, _P, _I32, _I32, _P, _I, _P, _I]),
     "moe_debug_wait_probe": (_I, [_P, C.c_uint32, _P, _P, _P]),
     "moe_cache_policy_bytes": (_SZ, [_I, _I]),
@@ -209,6 +212,16 @@ def layer_decode(pool: QPool, slot_of, shared_slot: int, layer: int, x, Wr, bias
           lib.moe_layer_decode(C.byref(pool), ptr(slot_of), shared_slot, layer, ptr(x), ptr(Wr), ptr(bias), T, d, f,
                                E, k, ptr(logits), ptr(topk_idx), ptr(topk_w), ptr(counts), ptr(offsets),
                                ptr(sorted_tok), ptr(sorted_j), ptr(inv), ptr(active), ptr(slot_of_pair), ptr(miss),
+                               ptr(miss_count), miss_cap, ptr(y), ptr(ws), ws_bytes, ptr(dev_status),
+                               stream_handle(stream)))
+
+
+def stack_decode(pool: QPool, L: int, slot_of, shared_slot, layer0: int, x, Wr, bias, T, d, f, E, k, topk_idx=None,
+                 topk_w=None, slot_of_pair=None, miss=None, miss_count=None, miss_cap=0, y=None, ws=None,
+                 ws_bytes=0, dev_status=None, stream=None) -> None:
+    check("moe_stack_decode",
+          lib.moe_stack_decode(C.byref(pool), L, ptr(slot_of), ptr(shared_slot), layer0, ptr(x), ptr(Wr), ptr(bias),
+                               T, d, f, E, k, ptr(topk_idx), ptr(topk_w), ptr(slot_of_pair), ptr(miss),
                                ptr(miss_count), miss_cap, ptr(y), ptr(ws), ws_bytes, ptr(dev_status),
                                stream_handle(stream)))
 

@@ -321,29 +321,37 @@ int32_t moe_cache_policy_plan(void *state, int32_t *slot_of, moe_swap *swaps, in
 moe_status moe_debug_wait_probe(const uint32_t *counter, uint32_t target, uint64_t *elapsed_ns,
                                 int32_t *dev_status, moe_stream_t stream);
 
-/* Workspace bytes moe_layer_decode needs for (T, k, f, E). */
+/* Workspace bytes moe_layer_decode and moe_stack_decode need for (T, k, f, E):
+ * two grid counters and two fp32 [T][E] logit buffers. */
 size_t moe_layer_decode_workspace_bytes(int T, int k, int f, int E);
+size_t moe_stack_decode_workspace_bytes(int T, int k, int f, int E);
 
 /*
  * The whole layer for a few tokens (decode, or an MTP verify batch of one token
  * plus drafts -- [SAITO] "命中率七成，代价是答案会变" verifies three drafts at once) in
- * one cooperative launch: router + top-k gates, permutation, cache lookup,
- * routed experts, shared expert and gate-weighted combine, as defined by
- * moe_route, moe_permute, moe_cache_lookup, moe_expert_ffn_q2/q3 and
- * moe_combine. Routing, permutation, slots and misses are identical to those
- * calls; y agrees with them up to the order of its fp32 additions (the experts'
- * contributions are added with atomics).
+ * one cooperative launch of thread-block clusters: router + top-k gates,
+ * permutation, cache lookup, routed experts, shared expert and gate-weighted
+ * combine, as defined by moe_route, moe_permute, moe_cache_lookup,
+ * moe_expert_ffn_q2/q3 and moe_combine. Routing, permutation, slots and misses
+ * are identical to those calls; y agrees with them up to the order of its fp32
+ * additions (each expert's hidden activations are formed from C partial sums
+ * over slices of d added in a fixed order, and the experts' contributions are
+ * added into y with atomics).
  *   W, slot_of   pool and this layer's expert -> slot table (W->fmt 2 or 3)
  *   shared_slot  pool slot of the layer's shared expert
  *   layer        copied into miss records
- *   x, Wr, bias  as moe_route; T <= 8, E <= 512, d <= 2048, f <= 1024
+ *   x, Wr, bias  as moe_route; T <= 8, E <= 512, d <= 2048, f <= 4096;
+ *                x, Wr and y 16-byte aligned
  *   logits .. miss_count  outputs of the step-by-step calls, each may be NULL
  *   y            fp32 [T][d] (output, overwritten)
  *   ws           moe_layer_decode_workspace_bytes() bytes, 256-byte aligned,
  *                zero-filled before first use; each launch leaves its counters
  *                zeroed again (zero it again after a MOE_DEV_TIMEOUT)
- * The launch uses every SM (cooperative); two launches on different streams
- * must not share a workspace.
+ * The launch uses every SM (one CTA per SM, clusters of 4 CTAs when d is a
+ * multiple of 1024, of 2 when a multiple of 512, else of 1); two launches on
+ * different streams must not share a workspace, and launches that would run
+ * at the same time as other work on the GPU wait for SMs (the grid must be
+ * co-resident; a grid-wide wait that gives up sets MOE_DEV_TIMEOUT).
  */
 moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t shared_slot, int32_t layer,
                             const uint16_t *x, const float *Wr, const float *bias, int T, int d, int f, int E, int k,
@@ -351,6 +359,31 @@ moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t 
                             int32_t *sorted_tok, int32_t *sorted_j, int32_t *inv, int32_t *active,
                             int32_t *slot_of_pair, moe_miss *miss, int32_t *miss_count, int32_t miss_cap, float *y,
                             void *ws, size_t ws_bytes, int32_t *dev_status, moe_stream_t stream);
+
+/*
+ * L layers of moe_layer_decode in one launch, in order: layer l + 1 starts
+ * once every contribution to layer l's y is in place (a grid barrier), so its
+ * input could have been derived from layer l's output; while layer l's experts
+ * stream, every CTA asks the L2 for its slice of layer l + 1's router rows and
+ * shared expert (weights that do not depend on routing). The ([SAITO]
+ * "1250 亿参数，每个词只用得上 2%") model has 48 such layers.
+ *   W            one pool holding every layer's resident experts
+ *   slot_of      int32 [L][E]: each layer's expert -> slot table (-1 = miss)
+ *   shared_slot  int32 [L] (device): each layer's shared-expert slot
+ *   layer0       layer id of the first layer (miss records carry layer0 + l)
+ *   x            bf16 [L][T][d]: each layer's input
+ *   Wr, bias     fp32 [L][E][d], [L][E] (bias may be NULL)
+ *   topk_idx, topk_w, slot_of_pair  [L][T*k] outputs as moe_layer_decode (may be NULL)
+ *   miss         moe_miss [L][miss_cap], miss_count int32 [L] (may be NULL)
+ *   y            fp32 [L][T][d] (output)
+ *   ws           moe_stack_decode_workspace_bytes() bytes, as moe_layer_decode
+ * Shapes and limits as moe_layer_decode.
+ */
+moe_status moe_stack_decode(const moe_qpool *W, int L, const int32_t *slot_of, const int32_t *shared_slot,
+                            int32_t layer0, const uint16_t *x, const float *Wr, const float *bias, int T, int d, int f,
+                            int E, int k, int32_t *topk_idx, float *topk_w, int32_t *slot_of_pair, moe_miss *miss,
+                            int32_t *miss_count, int32_t miss_cap, float *y, void *ws, size_t ws_bytes,
+                            int32_t *dev_status, moe_stream_t stream);
 
 /*
  * moe_expert_ffn_q2 without a caller-supplied workspace. The pages have no

@@ -79,14 +79,24 @@ def test_host_validation_rejects_before_launch():
     assert L.moe_expert_ffn_q2(C.byref(pool), *small) == 3
     pool.slot_bytes = 1000
     assert L.moe_expert_ffn_q2(C.byref(pool), *args) == 1
-    # one-launch decode layer: f above the 1024 it stages, T above 8
-    wide = native.QPool(dummy * 256, 1 << 22, 10, 2, 2048, 2048)
-    dec = [dummy, 0, 0, dummy, dummy, None, 1, 2048, 2048, 512, 10] + [None] * 12 + [0, dummy, dummy, 1 << 24,
-                                                                                   None, None]
+    # one-launch decode layer: d above the 2048 it stages, T above 8
+    wide = native.QPool(dummy * 256, 1 << 23, 10, 2, 4096, 768)
+    dec = [dummy, 0, 0, dummy, dummy, None, 1, 4096, 768, 512, 10] + [None] * 12 + [0, dummy, dummy, 1 << 24,
+                                                                                  None, None]
     assert L.moe_layer_decode(C.byref(wide), *dec) == 2
     dec9 = list(dec)
-    dec9[6], dec9[8] = 9, 768
+    dec9[6], dec9[7], dec9[8] = 9, 2048, 768
     assert L.moe_layer_decode(C.byref(pool), *dec9) == 2
+    # stacked layers: no shared-slot table, zero layers, misaligned x
+    st = [C.byref(pool), 4, dummy, None, 0, dummy, dummy, None, 1, 2048, 768, 512, 10, None, None, None, None, None, 0,
+          dummy, dummy, 1 << 24, None, None]
+    assert L.moe_stack_decode(*st) == 1
+    st0 = list(st)
+    st0[1] = 0
+    assert L.moe_stack_decode(*st0) == 1
+    st3 = list(st)
+    st3[3], st3[5] = dummy, dummy + 2
+    assert L.moe_stack_decode(*st3) == 1
     # wait probe: null pointers
     assert L.moe_debug_wait_probe(None, 1, dummy, dummy, None) == 1
     assert L.moe_debug_wait_probe(dummy, 1, None, dummy, None) == 1

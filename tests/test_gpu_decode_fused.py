@@ -141,6 +141,37 @@ def test_fused_with_misses():
         stack.slot_of[0].copy_(saved)
 
 
+def test_stacked_layers_one_launch():
+    """moe_stack_decode over 6 layers of the 48-layer workload (25% resident):
+    every layer's routing, slots and misses bit-exact and y within 2e-3 of the
+    oracle, and equal to the one-layer call on the same layer."""
+    wl = configs.STACK48
+    L = 6
+    stack = MoEStack(wl, layers=L)
+    xs = np.stack([synth.gen_x(0, l, 2, wl.d, stream=900) for l in range(L)])
+    x = torch.from_numpy(xs.view(np.int16)).cuda()
+    b = stack.stack_buffers(2)
+    b.status.zero_()
+    b.y.fill_(float("nan"))
+    stack.forward_stack(x, b)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    ws = stack.decode_workspace(2)
+    assert int(ws[:8].view(torch.int32).abs().sum().item()) == 0
+    n = 2 * wl.k
+    for l in range(L):
+        ref = oracle_layer(stack, l, xs[l])
+        np.testing.assert_array_equal(b.idx[l, :n].cpu().numpy().reshape(2, wl.k), ref["idx"])
+        np.testing.assert_allclose(b.w[l, :n].cpu().numpy().reshape(2, wl.k), ref["gate"], rtol=1e-5, atol=1e-7)
+        np.testing.assert_array_equal(b.sop[l, :n].cpu().numpy(), ref["slot_of_pair"])
+        assert [m[:4] for m in stack.stack_misses(b, l)] == [m[:4] for m in ref["misses"]]
+        assert int(b.miss_count[l].item()) == ref["miss_count"]
+        err = rel_err(b.y[l, :2].cpu().numpy().astype(np.float64), ref["y_partial"])
+        assert err <= OUT_TOL, (l, err)
+        one = _fused(stack, l, xs[l])
+        assert rel_err(b.y[l, :2].cpu().numpy(), one.y[:2].cpu().numpy()) < 1e-5
+
+
 def test_fused_rejects_unsupported(tiny):
     wl = configs.TINY
     x = torch.zeros(9, wl.d, dtype=torch.int16, device="cuda")
