@@ -23,16 +23,17 @@
 //          the routing tables and the task list itself;
 //  tasks   a task is (expert, block of HB hidden rows): HB = 128 for Q2 (one
 //          block pair of the down matrix) and 256 for Q3 (one block quad).
-//          The C CTAs of a cluster split a task: CTA r computes the gate/up
-//          partial sums of the HB rows over its d/C slice of K, the partials
-//          are exchanged through distributed shared memory (one cluster
-//          barrier), every CTA forms h = silu(a) * u for the HB rows, and CTA
-//          r computes down rows [r d/C, (r+1) d/C) over the HB columns and
-//          adds gate * y_e into y with vector atomics. No task waits for
-//          another cluster. The weights of a task stream into per-warp slices
-//          of a shared-memory ring with bulk copies (each warp copies and
-//          waits for its own rows), the next task's copies issued as soon as
-//          a warp's slice is free.
+//          The C CTAs of a cluster split a task: CTA r computes gate/up over
+//          all of d for hidden rows [r HB/C, (r+1) HB/C) of the block, forms
+//          h = silu(a) * u for them and pushes its h rows into every peer's
+//          shared memory (st.async, completion counted in bytes on the peer's
+//          mbarrier: no cluster barrier); then CTA r computes down rows
+//          [r d/C, (r+1) d/C) over the block's HB columns and adds gate * y_e
+//          into y with vector atomics. No task waits for another cluster. The
+//          weights of a task stream into per-warp slices of a shared-memory
+//          ring with bulk copies (each warp copies and waits for its own
+//          bytes), the next task's copies issued as soon as a warp's slice is
+//          free.
 //
 // Every wait on another CTA or on a copy is bounded (MOE_DEV_TIMEOUT after
 // 100 ms); the last CTA to leave resets the grid counters, so the workspace
@@ -80,21 +81,23 @@ constexpr int kMaxBuf = 2;                             // task buffers in the we
 
 // Geometry of one launch (host-computed; see plan()).
 struct Geo {
-    int C;        // CTAs per cluster: K of gate/up and the rows of down are split C ways
+    int C;        // CTAs per cluster (hidden rows of gate/up and output rows of down split C ways)
     int HB;       // hidden rows per task (128 Q2, 256 Q3)
     int NHB;      // tasks per expert, f / HB
-    int KR;       // gate/up K columns per CTA, d / C
-    int NQR;      // 256-column quads per CTA, KR / 256
+    int GR;       // gate/up row groups (16 rows) per CTA and task, HB / C / 16
+    int RPW;      // gate/up row groups per warp (GR > 8: 2)
+    int WPR;      // warps per gate/up row group (GR < 8: 8 / GR, each a share of the K quads)
+    int NQ;       // 256-column quads of d
+    int QPW;      // quads per warp, NQ / WPR
     int DR;       // down rows per CTA, d / C
     int NDRW;     // down row groups per warp, DR / 16 / 8
-    int GUW;      // gate/up row groups per warp, HB / 16 / 8
-    uint32_t gu_c, gu_s;  // codes / scales bytes of one gate/up row group (one matrix) over KR
+    uint32_t gu_c, gu_s;  // codes / scales bytes of one gate/up row group (one matrix) over a warp's quads
     uint32_t dn_c, dn_s;  // codes / scales bytes of one down row group over the task's HB columns
     uint32_t gu_warp, dn_warp, region;  // per-warp slices and one task buffer (8 warps)
     int nbuf;             // task buffers in the ring
-    uint32_t part_bytes;  // one partial-sum buffer (also the down-result staging)
+    uint32_t red_bytes;   // per-warp gate/up results, later the down-result staging
     // dynamic shared memory offsets
-    uint32_t off_bfx, off_part, off_h, off_bfh, off_ring, total;
+    uint32_t off_bfx, off_red, off_h, off_bfh, off_ring, total;
 };
 
 struct DecodeParams {
@@ -132,6 +135,9 @@ struct Smem {
     float w[kMaxTokDec][kMaxK];
     uint64_t wl[kWarps][kMaxK];             // per-warp top-k lists (keys)
     uint64_t sel[kMaxTokDec][kMaxK];        // merged top-k per token, best first
+    float ex_r[kMaxTokDec][kMaxK];          // exp(logit - max) of the selected, by ascending id
+    float inv_z[kMaxTokDec];
+    float rbias[8];                         // bias of this CTA's router rows
     int pair_e[kMaxPairs];                  // expert of sorted pair s
     int s_tok[kMaxPairs], s_j[kMaxPairs];   // sorted pairs
     int inv[kMaxPairs];
@@ -144,6 +150,7 @@ struct Smem {
     uint64_t rt_bar;                        // router rows landed
     uint64_t gu_bar[kMaxBuf][kWarps];       // per-warp gate/up slice landed
     uint64_t dn_bar[kMaxBuf][kWarps];       // per-warp down slice landed
+    uint64_t xbar[2];                       // peers' h rows landed (by task parity)
     int nact, nres, nmiss, ntask;
     int ok, last;
 };
@@ -251,6 +258,12 @@ __device__ __forceinline__ int ld_peer_int(uint32_t a) {
     asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
     return v;
 }
+// 16 bytes into a peer CTA's shared memory, counted on the peer's mbarrier.
+__device__ __forceinline__ void st_async4(uint32_t raddr, float4 v, uint32_t rbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1,%2,%3,%4}, [%5];" ::"r"(raddr),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(rbar)
+                 : "memory");
+}
 __device__ __forceinline__ void red_add4(float *p, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
@@ -288,8 +301,8 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 
 // One router row (fixed fp32 order, see moe.h) for NT tokens from shared memory.
 template <int NT>
-__device__ void router_row(const float *wrow, const uint16_t *sx, int T, int d, int lane, const float *bias, int e,
-                           float *logits, int E, int32_t *status) {
+__device__ void router_row(const float *wrow, const uint16_t *sx, int T, int d, int lane, bool has_bias, float b,
+                           int e, float *logits, int E, int32_t *status) {
     float acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.f;
@@ -313,9 +326,8 @@ __device__ void router_row(const float *wrow, const uint16_t *sx, int T, int d, 
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) acc[t] = __fadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], o));
     if (lane == 0) {
-        const float b = bias ? bias[e] : 0.f;
         for (int t = 0; t < T; ++t) {
-            const float v = bias ? __fadd_rn(acc[t], b) : acc[t];
+            const float v = has_bias ? __fadd_rn(acc[t], b) : acc[t];
             if (!isfinite(v)) flag(status, MOE_DEV_NONFINITE);
             __stcg(logits + size_t(t) * E + e, v);
         }
@@ -404,28 +416,34 @@ __device__ __forceinline__ int task_slot(const DecodeParams &p, const Smem &s, c
     return s.act_slot[a];
 }
 
+// Gate/up row group (task-local, 0 .. GR-1) and first quad of warp `warp`'s
+// ri-th share of the task.
+__device__ __forceinline__ int gu_rgl(const Geo &g, int warp, int ri) { return g.WPR > 1 ? warp / g.WPR : warp + 8 * ri; }
+__device__ __forceinline__ int gu_q0(const Geo &g, int warp) { return g.QPW * (warp % g.WPR); }
+
 // Lanes of one warp issue the bulk copies of the warp's gate/up slice of task
-// (slot, hb) into buffer b (lane 0 sets the expected bytes first).
+// (slot, hb) into buffer b (lane 0 sets the expected bytes first): for each of
+// its RPW row groups, gate and up, the codes and scales of its QPW quads.
 template <int FMT>
 __device__ __forceinline__ void issue_gu(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int warp, int lane,
                                          unsigned rank, int slot, int hb) {
     const Geo &g = p.g;
     uint8_t *dst = ring + size_t(b) * g.region + size_t(warp) * g.gu_warp;
     const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
-    const int kq0 = int(rank) * g.NQR;  // first quad of this CTA's K slice
+    const int q0 = gu_q0(g, warp);
     if (lane == 0) bar_expect(&s.gu_bar[b][warp], g.gu_warp);
     __syncwarp();
-    // copy c: row group gi = c / 4, matrix (c / 2) % 2, codes (c even) or scales
-    if (lane < 4 * g.GUW) {
-        const int gi = lane >> 2, mi = (lane >> 1) & 1, sc = lane & 1;
+    // copy c: share ri = c / 4, matrix (c / 2) % 2, codes (c even) or scales
+    if (lane < 4 * g.RPW) {
+        const int ri = lane >> 2, mi = (lane >> 1) & 1, sc = lane & 1;
         const MatGeom &m = mi ? p.up : p.gate;
-        const int rg = hb * (g.HB / 16) + warp + 8 * gi;
-        uint8_t *d0 = dst + size_t(gi * 2 + mi) * (g.gu_c + g.gu_s) + (sc ? g.gu_c : 0);
+        const int rg = hb * (g.HB / 16) + int(rank) * g.GR + gu_rgl(g, warp, ri);
+        uint8_t *d0 = dst + size_t(ri * 2 + mi) * (g.gu_c + g.gu_s) + (sc ? g.gu_c : 0);
         uint64_t off;
         if (sc)
-            off = scale_off(m, FMT, rg, 2 * kq0, 0);
+            off = scale_off(m, FMT, rg, 2 * q0, 0);
         else
-            off = FMT == 2 ? q2_chunk_off(m, rg, 2 * kq0, 0) : q3_word_off(m, rg, kq0, 0, 0);
+            off = FMT == 2 ? q2_chunk_off(m, rg, 2 * q0, 0) : q3_word_off(m, rg, q0, 0, 0);
         bulk_copy(d0, rec + off, sc ? g.gu_s : g.gu_c, &s.gu_bar[b][warp]);
     }
 }
@@ -440,8 +458,8 @@ __device__ __forceinline__ void issue_dn(const DecodeParams &p, Smem &s, uint8_t
     const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
     if (lane == 0) bar_expect(&s.dn_bar[b][warp], g.dn_warp);
     __syncwarp();
-    if (lane < 2 * g.NDRW) {
-        const int j = lane >> 1, sc = lane & 1;
+    for (int c = lane; c < 2 * g.NDRW; c += 32) {
+        const int j = c >> 1, sc = c & 1;
         const int rg = int(rank) * (g.DR / 16) + warp * g.NDRW + j;
         uint8_t *d0 = dst + size_t(j) * (g.dn_c + g.dn_s) + (sc ? g.dn_c : 0);
         uint64_t off;
@@ -505,44 +523,49 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
     }
     if (WPT > 1) {
         __syncthreads();
-        if (tt < T && lane < k) {
+        if (tt < T && lane < k) {  // rank = entries of all the token's lists above mine (independent loads)
             const uint64_t me = s.wl[warp][lane];
-            int rank = lane;
+            int rank = 0;
+#pragma unroll
             for (int o = 0; o < WPT; ++o) {
-                if (o == sub) continue;
                 const uint64_t *ol = s.wl[tt * WPT + o];
-                int lo = 0, hi = k;  // entries of list o above me (lists are descending)
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (ol[mid] > me) lo = mid + 1; else hi = mid;
-                }
-                rank += lo;
+                for (int q = 0; q < k; ++q) rank += ol[q] > me;
             }
             if (rank < k) s.sel[tt][rank] = me;
         }
     }
     __syncthreads();
-    if (warp < T) {  // one warp per token: softmax, ascending id order (as moe_route)
-        const uint64_t mine = lane < k ? s.sel[warp][lane] : 0ull;
+    // softmax over the selected logits in ascending-id order (the arithmetic of
+    // moe_route: z summed from 0 in that order, gate = ex * (1 / z))
+    const bool selt = warp < T && lane < k;
+    int my_id = 0, rank = 0;
+    float ex = 0.f;
+    if (selt) {
+        const uint64_t mine = s.sel[warp][lane];
         const uint32_t key = uint32_t(mine >> 32);
         // a round that found only NaN left takes expert 0 with logit -inf, as moe_route does
-        const int my_id = key ? int(~uint32_t(mine)) : 0;
+        my_id = key ? int(~uint32_t(mine)) : 0;
         const float my_v = key ? key_value(key) : -INFINITY;
-        const bool sel = lane < k;
-        int rank = 0;
-        for (int q = 0; q < k; ++q) rank += __shfl_sync(0xffffffffu, my_id, q) < my_id;
-        const float mx = __shfl_sync(0xffffffffu, my_v, 0);
-        const float ex = sel ? expf(my_v - mx) : 0.f;
+        const uint64_t top = s.sel[warp][0];
+        const float mx = uint32_t(top >> 32) ? key_value(uint32_t(top >> 32)) : -INFINITY;
+        for (int q = 0; q < k; ++q) {
+            const uint64_t o = s.sel[warp][q];
+            const int oid = uint32_t(o >> 32) ? int(~uint32_t(o)) : 0;
+            rank += oid < my_id;
+        }
+        ex = expf(my_v - mx);
+        s.ex_r[warp][rank] = ex;
+    }
+    __syncthreads();
+    if (warp < T && lane == 0) {
         float z = 0.0f;
-        for (int a = 0; a < k; ++a) {
-            const unsigned who = __ballot_sync(0xffffffffu, sel && rank == a);
-            z += __shfl_sync(0xffffffffu, ex, __ffs(who) - 1);
-        }
-        const float inv = 1.0f / z;
-        if (sel) {
-            s.idx[warp][rank] = my_id;
-            s.w[warp][rank] = ex * inv;
-        }
+        for (int a = 0; a < k; ++a) z += s.ex_r[warp][a];
+        s.inv_z[warp] = 1.0f / z;
+    }
+    __syncthreads();
+    if (selt) {
+        s.idx[warp][rank] = my_id;
+        s.w[warp][rank] = ex * s.inv_z[warp];
     }
     __syncthreads();
 }
@@ -552,6 +575,40 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
 __device__ void routing_tables(const DecodeParams &p, Smem &s, int T, int k) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int npairs = T * k;
+    if (T == 1) {  // one token: its k experts (ascending id) are the active experts, one pair each
+        if (warp == 0) {
+            const bool in = lane < k;
+            int sl = -1;
+            if (in) {
+                const int e = s.idx[0][lane];
+                s.pair_e[lane] = e;
+                s.s_tok[lane] = 0;
+                s.s_j[lane] = lane;
+                s.inv[lane] = lane;
+                sl = (e >= 0 && e < p.E) ? s.slot[e] : -1;
+                const bool bad = sl < -1 || sl >= p.num_slots;
+                if (bad && blockIdx.x == 0) flag(p.status, MOE_DEV_BAD_SLOT);
+                if (bad) sl = -1;
+                s.act_e[lane] = e;
+                s.act_beg[lane] = lane;
+                s.act_cnt[lane] = 1;
+                s.act_slot[lane] = sl;
+            }
+            const unsigned rm = __ballot_sync(0xffffffffu, in && sl >= 0);
+            const unsigned mm = __ballot_sync(0xffffffffu, in && sl < 0);
+            const unsigned lt = (1u << lane) - 1u;
+            if (in) s.act_mbase[lane] = __popc(mm & lt);
+            if (in && sl >= 0) s.res[__popc(rm & lt)] = lane;
+            if (lane == 0) {
+                s.nact = k;
+                s.nres = __popc(rm);
+                s.nmiss = __popc(mm);
+                s.ntask = (__popc(rm) + 1) * p.g.NHB;
+            }
+        }
+        __syncthreads();
+        return;
+    }
     if (tid < npairs) {  // stable sort of the pairs by (expert, pair index)
         const int pp = tid;
         const int e = s.idx[pp / k][pp % k];
@@ -683,16 +740,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
     const unsigned rank = cluster_rank(), cid = cluster_id(), ncl = cluster_count();
     const int T = p.T, k = p.k, E = p.E, d = p.d;
     const int gl = lane >> 2, tl = lane & 3;  // MMA fragment coordinates of this lane
-    uint4 *bfx = reinterpret_cast<uint4 *>(dyn + g.off_bfx);  // x B fragments [NQR][8][32]
-    float *part = reinterpret_cast<float *>(dyn + g.off_part);  // [2][HB/16][32][8] partials
-    float *hs = reinterpret_cast<float *>(dyn + g.off_h);       // [HB][8] h of the task
+    uint4 *bfx = reinterpret_cast<uint4 *>(dyn + g.off_bfx);  // x B fragments [NQ][8][NT*4] (lanes g < NT)
+    float *red = reinterpret_cast<float *>(dyn + g.off_red);  // [8 warps][RPW][32][8] gate/up results; down staging
+    float *hs_all = reinterpret_cast<float *>(dyn + g.off_h);  // [2][HB][NT] h of the task (by task parity)
     uint32_t *bfh = reinterpret_cast<uint32_t *>(dyn + g.off_bfh);  // [HB/64][8][32] h B fragments
     uint8_t *ring = dyn + g.off_ring;
-    const int part_floats = int(g.part_bytes / 4);
     bool too_big = false, ok = true;
     unsigned bar_target = 0;  // grid barrier arrivals this CTA has waited for
-    // per-warp ring bookkeeping (identical in every lane of a warp)
-    int seq = 0;  // tasks of this CTA started so far, over all layers (buffer = seq % nbuf)
+    int seq = 0;  // tasks of this CTA started so far, over all layers (buffer = seq % nbuf, h parity = seq % 2)
 
     if (tid == 0) {
         bar_init(&s.rt_bar, 1);
@@ -701,14 +756,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                 bar_init(&s.gu_bar[b][w], 1);
                 bar_init(&s.dn_bar[b][w], 1);
             }
+        bar_init(&s.xbar[0], 1);
+        bar_init(&s.xbar[1], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    __syncthreads();
+    // every CTA of the cluster has initialised its barriers before a peer sends to them
+    cluster_sync();
 
     // rows of the router this CTA computes (contiguous, about E/G)
     const int rb = int(int64_t(E) * cta / G), re = int(int64_t(E) * (cta + 1) / G);
     const int nrows = re - rb;
 
+#ifdef MOE_DECODE_TRACE
+    if (tid == 0)  // points this launch does not reach stay empty
+        for (int i = 1; i < 32; ++i) moe_decode_trace[blockIdx.x * 32 + i] = 0ull;
+#endif
     for (int l = 0; l < p.L; ++l) {
         const LayerPtrs lp = layer_ptrs(p, l);
         TRACE(0);
@@ -720,6 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
             bulk_copy(rrows, lp.Wr + size_t(rb) * d, uint32_t(nrows) * uint32_t(d) * 4u, &s.rt_bar);
         }
         {
+            if (tid < nrows && tid < 8) s.rbias[tid] = lp.bias ? __ldg(lp.bias + rb + tid) : 0.f;
             const uint4 *src = reinterpret_cast<const uint4 *>(lp.x);
             uint4 *dst = reinterpret_cast<uint4 *>(sx);
             for (int i = tid; i < T * d / 8; i += kThreads) dst[i] = __ldg(src + i);
@@ -728,26 +791,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
             for (int i = cta * kThreads + tid; i < T * d; i += G * kThreads) lp.y[i] = 0.f;
         }
         __syncthreads();
-        // block sums of x over this CTA's K slice, and its B fragments (all 8 token columns)
-        const int k0 = int(rank) * g.KR;
-        for (int job = warp; job < (g.KR / 64) * T; job += kWarps) {
+        TRACE(12);
+        // block sums of x and its B fragments (token columns < NT; the rest are zero)
+        for (int job = warp; job < (d / 64) * T; job += kWarps) {
             const int bb = job / T, n = job % T;
-            const uint32_t u = *reinterpret_cast<const uint32_t *>(sx + size_t(n) * d + k0 + 64 * bb + 2 * lane);
+            const uint32_t u = *reinterpret_cast<const uint32_t *>(sx + size_t(n) * d + 64 * bb + 2 * lane);
             float v = bf16_lo(u) + bf16_hi(u);
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
             if (lane == 0) s.xs[bb][n] = v;
         }
-        for (int e = tid; e < g.NQR * 256; e += kThreads) {
-            const int qi = e >> 8, ln = (e >> 3) & 31, r4 = e & 7;
+        for (int e = tid; e < g.NQ * 8 * NT * 4; e += kThreads) {
+            const int qi = e / (8 * NT * 4), r4 = (e / (NT * 4)) % 8, ln = e % (NT * 4);
             const int gg = ln >> 2, tt = ln & 3, bq = r4 >> 1;
-            const uint16_t *src = gg < T ? sx + size_t(gg) * d + k0 + 256 * qi + 64 * bq : nullptr;
+            const uint16_t *src = sx + size_t(gg) * d + 256 * qi + 64 * bq;
             uint32_t v[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int rho = (r4 & 1) * 4 + j;
                 float lo = 0.f, hi = 0.f;
-                if (src) {
+                if (gg < T) {
                     const uint32_t u = *reinterpret_cast<const uint32_t *>(src + slot_k(rho, tt, 0));
                     lo = bf16_lo(u);
                     hi = bf16_hi(u);
@@ -755,16 +818,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                 const float sc = __int_as_float((127 - slot_exp<FMT>(bq, rho)) << 23);  // 2^-exp
                 v[j] = pack_half2(lo * sc, hi * sc);
             }
-            bfx[(qi * 8 + r4) * 32 + ln] = make_uint4(v[0], v[1], v[2], v[3]);
+            bfx[e] = make_uint4(v[0], v[1], v[2], v[3]);
         }
         if (nrows > 0) {
             const bool got = bar_wait(&s.rt_bar, uint32_t(l & 1));
             if (!got && tid == 0) flag(p.status, MOE_DEV_TIMEOUT);
             ok = ok && got;
-            if (got && warp < nrows)
-                router_row<NT>(rrows + size_t(warp) * d, sx, T, d, lane, lp.bias, rb + warp, lp.logits, E, p.status);
-            for (int r = warp + kWarps; got && r < nrows; r += kWarps)
-                router_row<NT>(rrows + size_t(r) * d, sx, T, d, lane, lp.bias, rb + r, lp.logits, E, p.status);
+            TRACE(13);
+            for (int r = warp; got && r < nrows; r += kWarps)
+                router_row<NT>(rrows + size_t(r) * d, sx, T, d, lane, lp.bias != nullptr,
+                               r < 8 ? s.rbias[r] : (lp.bias ? __ldg(lp.bias + rb + r) : 0.f), rb + r, lp.logits, E,
+                               p.status);
         }
         ok = __syncthreads_and(ok) != 0;  // logits written; router rows and x consumed (the ring is free)
         if (tid == 0) {
@@ -815,41 +879,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
             routing_tables(p, s, T, k);
         }
         TRACE(4);
-        // every CTA of the cluster runs the same number of tasks (and cluster barriers):
-        // if any of them failed to route, none of them runs a task
-        if (tid == 0) s.last = ok ? s.ntask : -1;
-        cluster_sync();
-        int ntask = s.last;
-        for (int r = 0; r < g.C; ++r)
-            if (unsigned(r) != rank) ntask = min(ntask, ld_peer_int(peer_addr(&s.last, unsigned(r))));
-        cluster_sync();  // the peers' flags are read before anyone changes them
-        if (ntask < 0) {
-            ntask = 0;
-            ok = false;
-        }
+        // every CTA of a cluster derives the same task list from the same routing;
+        // a CTA that could not route runs none (its peers' waits for it give up)
+        const int ntask = ok ? s.ntask : 0;
         const int nmine = ntask > int(cid) ? (ntask - int(cid) + int(ncl) - 1) / int(ncl) : 0;
         if (ok) issue_upto(nmine, 0, 0);
+        TRACE(11);
         // ------------------------------------------------ tasks
+        const int hrows = g.GR * 16;  // hidden rows this CTA computes per task
         for (int i = 0; i < nmine; ++i) {
             const int b = (seq0 + i) % g.nbuf;
             const uint32_t ph = uint32_t((seq0 + i) / g.nbuf) & 1u;
+            const int xb = (seq0 + i) & 1;
+            const uint32_t xph = uint32_t((seq0 + i) >> 1) & 1u;
+            float *hs = hs_all + size_t(xb) * g.HB * NT;
             int hb, a;
             task_slot(p, s, lp, int(cid) + i * int(ncl), hb, a);
-            float *mypart = part + size_t(i & 1) * part_floats;
-            // gate/up partial sums of this warp's row groups over this CTA's K slice
+            // the peers' h rows of this task land on xbar[xb]
+            if (tid == 0) bar_expect(&s.xbar[xb], uint32_t(g.C - 1) * uint32_t(hrows * NT * 4));
+            // gate/up of this warp's row groups over its quads
             bool got = ok && bar_wait(&s.gu_bar[b][warp], ph);
             if (i == 0) TRACE(5);
             if (got) {
                 const uint8_t *slice = ring + size_t(b) * g.region + size_t(warp) * g.gu_warp;
-                for (int gi = 0; gi < g.GUW; ++gi) {
+                const int q0 = gu_q0(g, warp);
+                for (int ri = 0; ri < g.RPW; ++ri) {
                     float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
-                    const uint8_t *gc = slice + size_t(gi * 2) * (g.gu_c + g.gu_s);
+                    const uint8_t *gc = slice + size_t(ri * 2) * (g.gu_c + g.gu_s);
                     const uint8_t *uc = gc + (g.gu_c + g.gu_s);
-                    for (int qi = 0; qi < g.NQR; ++qi) {
+                    for (int qi = 0; qi < g.QPW; ++qi) {
                         uint32_t B[4][8];
+                        const uint4 *bq4 = bfx + size_t((q0 + qi) * 8) * (NT * 4) + lane;
 #pragma unroll
                         for (int r4 = 0; r4 < 8; ++r4) {
-                            const uint4 v = bfx[(qi * 8 + r4) * 32 + lane];
+                            const uint4 v = gl < NT ? bq4[r4 * (NT * 4)] : make_uint4(0u, 0u, 0u, 0u);
                             B[r4 >> 1][(r4 & 1) * 4 + 0] = v.x;
                             B[r4 >> 1][(r4 & 1) * 4 + 1] = v.y;
                             B[r4 >> 1][(r4 & 1) * 4 + 2] = v.z;
@@ -858,8 +921,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                         float xs[4][2];
 #pragma unroll
                         for (int bq = 0; bq < 4; ++bq) {
-                            xs[bq][0] = 2 * tl < T ? s.xs[4 * qi + bq][2 * tl] : 0.f;
-                            xs[bq][1] = 2 * tl + 1 < T ? s.xs[4 * qi + bq][2 * tl + 1] : 0.f;
+                            xs[bq][0] = 2 * tl < T ? s.xs[4 * (q0 + qi) + bq][2 * tl] : 0.f;
+                            xs[bq][1] = 2 * tl + 1 < T ? s.xs[4 * (q0 + qi) + bq][2 * tl + 1] : 0.f;
                         }
                         QuadRegs<FMT> qg, qu;
                         quad_smem<FMT>(gc, gc + g.gu_c, qi, lane, qg);
@@ -867,7 +930,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                         quad_compute<FMT>(qg, B, xs, ag);
                         quad_compute<FMT>(qu, B, xs, au);
                     }
-                    float4 *dst = reinterpret_cast<float4 *>(mypart + (size_t(warp + 8 * gi) * 32 + lane) * 8);
+                    float4 *dst = reinterpret_cast<float4 *>(red + (size_t(warp * g.RPW + ri) * 32 + lane) * 8);
                     dst[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
                     dst[1] = make_float4(au[0], au[1], au[2], au[3]);
                 }
@@ -877,33 +940,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
             __syncwarp();
             // this warp's gate/up slice of buffer b is free: copy ahead
             if (ok) issue_upto(nmine, i + 1, i);
-            if (i == 0) TRACE(6);
-            // ---- exchange the partials inside the cluster
-            cluster_sync();
-            if (i == 0) TRACE(7);
             ok = __syncthreads_and(ok) != 0;
-            // h = silu(a) * u for the HB rows x T tokens, partials summed in rank order
-            for (int e = tid; e < g.HB * NT; e += kThreads) {
-                const int row = e / NT, tok = e % NT;
-                const int lrg = row >> 4, rr = row & 15;
+            if (i == 0) TRACE(6);
+            // h = silu(a) * u of this CTA's hidden rows (the WPR warps of a row group
+            // summed in warp order), written to its rows of hs
+            for (int e = tid; e < hrows * NT; e += kThreads) {
+                const int r = e / NT, tok = e % NT;
+                const int rgl = r >> 4, rr = r & 15;
                 const int ln = 4 * (rr & 7) + (tok >> 1), ix = 2 * (rr >> 3) + (tok & 1);
-                const float *src = mypart + (size_t(lrg) * 32 + ln) * 8 + ix;
                 float A = 0.f, U = 0.f;
-                for (int r = 0; r < g.C; ++r) {
-                    float av, uv;
-                    if (unsigned(r) == rank) {
-                        av = src[0];
-                        uv = src[4];
-                    } else {
-                        av = ld_peer(peer_addr(src, unsigned(r)));
-                        uv = ld_peer(peer_addr(src + 4, unsigned(r)));
-                    }
-                    A = r == 0 ? av : A + av;
-                    U = r == 0 ? uv : U + uv;
+                for (int j = 0; j < g.WPR; ++j) {
+                    const int w = g.WPR > 1 ? rgl * g.WPR + j : (rgl & 7);
+                    const int ri = g.WPR > 1 ? 0 : (rgl >> 3);
+                    const float *src = red + (size_t(w * g.RPW + ri) * 32 + ln) * 8 + ix;
+                    A = j == 0 ? src[0] : A + src[0];
+                    U = j == 0 ? src[4] : U + src[4];
                 }
                 const float h = (ok && tok < T) ? A / (1.0f + expf(-A)) * U : 0.f;
                 too_big |= !(fabsf(h) <= 65504.f);
-                hs[row * 8 + tok] = h;
+                hs[(int(rank) * hrows + r) * NT + tok] = h;
             }
             if (tid < NT) {  // gate of each token for this task
                 float gw = 0.f;
@@ -920,26 +975,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                 s.gsel[tid] = gw;
             }
             __syncthreads();
-            // B fragments of h for the task's HB down columns (8 token columns) and block sums
+            // push this CTA's h rows into every peer (16 bytes per store)
+            {
+                const int nv = hrows * NT / 4;
+                const float4 *mine = reinterpret_cast<const float4 *>(hs + int(rank) * hrows * NT);
+                for (int e = tid; e < nv * (g.C - 1); e += kThreads) {
+                    const unsigned peer = (rank + 1 + unsigned(e / nv)) % unsigned(g.C);
+                    const int v = e % nv;
+                    st_async4(peer_addr(mine + v, peer), mine[v], peer_addr(&s.xbar[xb], peer));
+                }
+            }
+            // the peers' h rows
+            got = ok && bar_wait(&s.xbar[xb], xph);
+            if (!got && ok && tid == 0) flag(p.status, MOE_DEV_TIMEOUT);
+            ok = __syncthreads_and(got) != 0;
+            if (i == 0) TRACE(7);
+            // B fragments of h for the task's HB down columns (token columns < NT) and block sums
             const int nbh = g.HB / 64;
             for (int e = tid; e < nbh * 8 * 32; e += kThreads) {
                 const int bq = e >> 8, rho = (e >> 5) & 7, ln = e & 31;
                 const int gg = ln >> 2, tt = ln & 3;
                 const int kk = 64 * bq + slot_k(rho, tt, 0);
-                const float lo = gg < NT ? hs[kk * 8 + gg] : 0.f, hi = gg < NT ? hs[(kk + 1) * 8 + gg] : 0.f;
+                const float lo = gg < NT ? hs[kk * NT + gg] : 0.f, hi = gg < NT ? hs[(kk + 1) * NT + gg] : 0.f;
                 const float sc = __int_as_float((127 - slot_exp<FMT>(bq, rho)) << 23);
                 bfh[e] = pack_half2(lo * sc, hi * sc);
             }
             for (int job = warp; job < nbh * NT; job += kWarps) {
                 const int bq = job / NT, n = job % NT;
-                float v = hs[(64 * bq + lane) * 8 + n] + hs[(64 * bq + 32 + lane) * 8 + n];
+                float v = hs[(64 * bq + lane) * NT + n] + hs[(64 * bq + 32 + lane) * NT + n];
 #pragma unroll
                 for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
                 if (lane == 0) s.hsb[bq][n] = v;
             }
             __syncthreads();
-            // ---- down rows of this CTA over the task's columns
-            float *yst = part + size_t((i + 1) & 1) * part_floats;  // staging [NT][DR] in the other partial buffer
+            // ---- down rows of this CTA over the task's columns (results staged in red)
+            float *yst = red;
             got = ok && bar_wait(&s.dn_bar[b][warp], ph);
             if (got) {
                 const uint8_t *slice =
@@ -1032,8 +1102,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
     }
 
     if (too_big) flag(p.status, MOE_DEV_NONFINITE);
-    // no CTA leaves while a peer may still read its shared memory
-    cluster_sync();
+    // no CTA leaves while a peer may still send into its shared memory
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\nbarrier.cluster.wait.aligned;" ::: "memory");
     if (tid == 0) {
         __threadfence();
         s.last = atomicAdd(p.ctr + 1, 1u) == unsigned(G - 1);
@@ -1047,39 +1117,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
     }
 }
 
-
 // ---------------------------------------------------------------- host side
 size_t ws_align(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Launch geometry and shared-memory layout for (fmt, T, d, f) with `avail`
-// bytes of dynamic shared memory per CTA and G CTAs; false if it does not fit.
-bool plan(int fmt, int T, int d, int f, int E, int G, size_t avail, Geo &g) {
-    g.C = d % 1024 == 0 ? 4 : (d % 512 == 0 ? 2 : 1);
+// Cluster size for a format and hidden size: the hidden rows of a task (HB)
+// and the down rows are split C ways. Q2 uses pairs of SMs (a task's weights
+// on one CTA would be ~240 KB); Q3 (HB = 256) uses four.
+int cluster_size(int fmt, int d, int cmax) {
+    int c = fmt == 2 ? 2 : 4;
+    c = std::min(c, cmax);
+    while (c > 1 && d % (256 * c) != 0) c >>= 1;
+    return c;
+}
+// (the launcher takes a larger cluster when a task of this one does not fit, e.g. Q3 with 8 tokens)
+
+// Launch geometry and shared-memory layout for (fmt, T, d, f) with cluster size
+// C, `avail` bytes of dynamic shared memory per CTA and G CTAs; false if it
+// does not fit.
+bool plan(int fmt, int T, int d, int f, int E, int G, int C, size_t avail, Geo &g) {
+    g.C = C;
     g.HB = fmt == 2 ? 128 : 256;
-    if (f % g.HB) return false;
+    if (f % g.HB || d % 256 || g.HB % (16 * C)) return false;
     g.NHB = f / g.HB;
-    g.KR = d / g.C;
-    g.NQR = g.KR / 256;
-    g.DR = d / g.C;
+    g.GR = g.HB / C / 16;
+    if (g.GR > 16) return false;
+    g.RPW = g.GR > 8 ? g.GR / 8 : 1;
+    g.WPR = g.GR < 8 ? 8 / g.GR : 1;
+    g.NQ = d / 256;
+    if (g.NQ % g.WPR) return false;
+    g.QPW = g.NQ / g.WPR;
+    g.DR = d / C;
+    if (g.DR % 128) return false;
     g.NDRW = g.DR / 128;
-    g.GUW = g.HB / 128;
-    if (g.NQR < 1 || g.NDRW < 1) return false;
-    g.gu_c = uint32_t(g.NQR) * (fmt == 2 ? 1024u : 1536u);
-    g.gu_s = uint32_t(g.NQR) * (fmt == 2 ? 256u : 128u);
+    g.gu_c = uint32_t(g.QPW) * (fmt == 2 ? 1024u : 1536u);
+    g.gu_s = uint32_t(g.QPW) * (fmt == 2 ? 256u : 128u);
     g.dn_c = fmt == 2 ? 512u : 1536u;
     g.dn_s = 128u;
-    g.gu_warp = uint32_t(g.GUW) * 2u * (g.gu_c + g.gu_s);
+    g.gu_warp = uint32_t(g.RPW) * 2u * (g.gu_c + g.gu_s);
     g.dn_warp = uint32_t(g.NDRW) * (g.dn_c + g.dn_s);
     g.region = uint32_t(kWarps) * (g.gu_warp + g.dn_warp);
     const int NTp = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8;
-    g.part_bytes = uint32_t((std::max<size_t>(size_t(g.HB) * 64, size_t(NTp) * g.DR * 4) + 127) & ~size_t(127));
+    g.red_bytes = uint32_t((std::max<size_t>(size_t(kWarps) * g.RPW * 32 * 8 * 4, size_t(NTp) * g.DR * 4) + 127) &
+                           ~size_t(127));
     size_t off = 0;
     g.off_bfx = uint32_t(off);
-    off += size_t(g.NQR) * 4096;
-    g.off_part = uint32_t(off);
-    off += 2 * size_t(g.part_bytes);
+    off += size_t(g.NQ) * 8 * NTp * 4 * 16;
+    g.off_red = uint32_t(off);
+    off += g.red_bytes;
     g.off_h = uint32_t(off);
-    off += size_t(g.HB) * 8 * 4;
+    off += 2 * size_t(g.HB) * NTp * 4;
     g.off_bfh = uint32_t(off);
     off += size_t(g.HB / 64) * 1024;
     off = (off + 127) & ~size_t(127);
@@ -1101,7 +1187,7 @@ struct LaunchInfo {
     bool ready = false;
     int sms = 0;
     size_t avail = 0;   // dynamic shared memory a CTA can have
-    int grid[5] = {};   // CTAs per launch for cluster size C (index C), 0 = not known yet
+    int grid[9] = {};   // CTAs per launch for cluster size C (index C), 0 = not known yet
     bool coop = true;   // cooperative launches of clusters accepted
 };
 std::mutex g_mu;
@@ -1116,7 +1202,6 @@ moe_status launch(DecodeParams p, cudaStream_t stream) {
     }
     constexpr int ci = (FMT - 2) * 4 + (NT == 1 ? 0 : NT == 2 ? 1 : NT == 4 ? 2 : 3);
     auto kern = decode_layer_kernel<FMT, NT>;
-    const int C = p.d % 1024 == 0 ? 4 : (p.d % 512 == 0 ? 2 : 1);
     std::lock_guard<std::mutex> lock(g_mu);
     LaunchInfo &li = g_info[ci][dev];
     if (!li.ready) {
@@ -1137,27 +1222,32 @@ moe_status launch(DecodeParams p, cudaStream_t stream) {
         li.avail = size_t(av);
         li.ready = true;
     }
-    if (li.grid[C] == 0) {  // co-resident clusters of C CTAs with the largest shared-memory use
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute at[1];
-        at[0].id = cudaLaunchAttributeClusterDimension;
-        at[0].val.clusterDim.x = unsigned(C);
-        at[0].val.clusterDim.y = 1;
-        at[0].val.clusterDim.z = 1;
-        cfg.gridDim = dim3(unsigned(C * (li.sms / C)));
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = li.avail;
-        cfg.attrs = at;
-        cfg.numAttrs = 1;
-        int ncl = 0;
-        if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess || ncl < 1) {
-            cudaGetLastError();
-            return MOE_ERR_CUDA;
+    // the format's cluster size, doubled (up to 8) while a task does not fit in shared memory
+    int C = cluster_size(FMT, p.d, 8), G = 0;
+    for (;; C *= 2) {
+        if (C > 8 || p.d % (256 * C) != 0) return MOE_ERR_UNSUPPORTED;
+        if (li.grid[C] == 0) {  // co-resident clusters of C CTAs with the largest shared-memory use
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = unsigned(C);
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(unsigned(C * (li.sms / C)));
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = li.avail;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            int ncl = 0;
+            if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess || ncl < 1) {
+                cudaGetLastError();
+                return MOE_ERR_CUDA;
+            }
+            li.grid[C] = std::min(ncl * C, C * (li.sms / C));
         }
-        li.grid[C] = std::min(ncl * C, C * (li.sms / C));
+        G = li.grid[C];
+        if (plan(FMT, p.T, p.d, p.f, p.E, G, C, li.avail, p.g)) break;
     }
-    const int G = li.grid[C];
-    if (!plan(FMT, p.T, p.d, p.f, p.E, G, li.avail, p.g)) return MOE_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;

@@ -20,13 +20,10 @@ import torch
 from . import configs, native, synth
 from .layer import MoEStack, x_tensor
 
-POINTS = {8: "x staged", 10: "router rows (warp 0)", 1: "phase A done", 2: "all logits counted",
-          11: "top-k loads", 12: "top-k candidates", 13: "top-k selected", 6: "top-k + gates",
-          5: "routing tables", 3: "ring copies issued", 9: "C task 1 computed (warp 0)",
-          16: "C task 1 bytes landed", 17: "C task 1 partials synced", 14: "C task 1 done",
-          15: "C task 2 computed (warp 0)", 7: "phase C done", 18: "D unit 1 bytes landed",
-          19: "D unit 1 expert ready", 20: "D unit 1 h staged", 21: "D unit 1 computed (warp 0)",
-          22: "D unit 1 done", 4: "kernel end"}
+POINTS = {12: "x staged", 13: "router rows landed", 1: "logits written", 2: "grid barrier passed",
+          3: "top-k + gates", 4: "routing tables", 11: "cluster task count", 5: "task 1 gate/up landed (warp 0)",
+          6: "task 1 gate/up computed (warp 0)", 7: "task 1 partials exchanged", 8: "task 1 down computed",
+          9: "task 1 atomics done", 10: "layer end"}
 
 
 def main() -> None:
@@ -50,13 +47,20 @@ def main() -> None:
     flush = torch.empty(512 << 18, dtype=torch.float32, device="cuda")
     buf = np.zeros(4096 * 32, np.uint64)
     acc = {k: [] for k in POINTS}
+    starts = []
     skip = 10
+    ev = []
     for it in range(args.launches + skip):
         x = x_tensor(synth.gen_x(wl.seed, 0, wl.T, wl.d, stream=0 if args.warm else it))
         if not args.warm:
             flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
         stack.forward_fused(0, x, b)
+        e1.record()
         torch.cuda.synchronize()
+        if it >= skip:
+            ev.append(e0.elapsed_time(e1) * 1e3)
         tl.moe_decode_trace_read(buf.ctypes.data)
         if it < skip:
             continue
@@ -64,16 +68,19 @@ def main() -> None:
         G = int((tr[:, 0] > 0).sum())
         ns = tr[:G, :].astype(np.int64)
         rel = np.where(ns > 0, (ns - ns[:, 0].min()) / 1000.0, np.nan)
+        starts.append(float((ns[:, 0].max() - ns[:, 0].min()) / 1000.0))
         for k in POINTS:
             if np.isfinite(rel[:, k]).any():
                 acc[k].append((np.nanmedian(rel[:, k]), np.nanmax(rel[:, k])))
     print(f"{wl.name}: {G} CTAs, {'warm' if args.warm else 'L2 evicted before each launch'}, "
           f"status {int(b.status.item())}")
-    print(f"{'point':24s} {'median CTA':>11s} {'slowest CTA':>12s}  (us since first CTA start)")
+    print(f"launch time between CUDA events: median {np.median(ev):.2f} us; CTA start spread median "
+          f"{np.median(starts):.2f} us")
+    print(f"{'point':34s} {'median CTA':>11s} {'slowest CTA':>12s}  (us since first CTA start)")
     for k, nm in POINTS.items():
         if acc[k]:
             a = np.array(acc[k])
-            print(f"{nm:24s} {np.median(a[:, 0]):11.2f} {np.median(a[:, 1]):12.2f}")
+            print(f"{nm:34s} {np.median(a[:, 0]):11.2f} {np.median(a[:, 1]):12.2f}")
 
 
 if __name__ == "__main__":
