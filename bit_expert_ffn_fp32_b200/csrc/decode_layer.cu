@@ -38,6 +38,9 @@
 // Every wait on another CTA or on a copy is bounded (MOE_DEV_TIMEOUT after
 // 100 ms); the last CTA to leave resets the grid counters, so the workspace
 // stays zeroed between launches.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <math.h>
 #include <mutex>
@@ -91,9 +94,10 @@ struct Geo {
     int QPW;      // quads per warp, NQ / WPR
     int DR;       // down rows per CTA, d / C
     int NDRW;     // down row groups per warp, DR / 16 / 8
-    uint32_t gu_c, gu_s;  // codes / scales bytes of one gate/up row group (one matrix) over a warp's quads
+    uint32_t gu_c, gu_s;  // codes / scales bytes of one gate/up row group (one matrix, all of d)
     uint32_t dn_c, dn_s;  // codes / scales bytes of one down row group over the task's HB columns
-    uint32_t gu_warp, dn_warp, region;  // per-warp slices and one task buffer (8 warps)
+    uint32_t gu_rg;       // one row group's gate/up bytes in a task buffer (gate codes, scales, up codes, scales)
+    uint32_t gu_bytes, dn_bytes, region;  // a task buffer: GR gate/up row groups, then the down slice
     int nbuf;             // task buffers in the ring
     uint32_t red_bytes;   // per-warp gate/up results, later the down-result staging
     // dynamic shared memory offsets
@@ -127,6 +131,9 @@ struct DecodeParams {
     unsigned *ctr;               // [0] barrier arrivals, [1] CTAs finished
     MatGeom gate, up, down;
     Geo g;
+    // the down matrix of every pool slot as [slot][row group][chunk][bytes], one
+    // chunk = the codes (or scales) of one block pair (Q2) or block quad (Q3)
+    CUtensorMap dn_codes, dn_scales;
 };
 
 struct Smem {
@@ -148,8 +155,10 @@ struct Smem {
     float hsb[4][kMaxTokDec];               // block sums of the task's h columns
     float gsel[kMaxTokDec];                 // gate of each token for the current task (0 = not routed)
     uint64_t rt_bar;                        // router rows landed
-    uint64_t gu_bar[kMaxBuf][kWarps];       // per-warp gate/up slice landed
-    uint64_t dn_bar[kMaxBuf][kWarps];       // per-warp down slice landed
+    uint64_t gu_bar[kMaxBuf][16];           // per gate/up row group of a task buffer: its bytes landed
+    uint64_t dn_bar[kMaxBuf];               // the down slice of a task buffer landed
+    uint64_t cand[kMaxTokDec][64];          // top-k candidates above the threshold
+    int ncand[kMaxTokDec];
     uint64_t xbar[2];                       // peers' h rows landed (by task parity)
     int nact, nres, nmiss, ntask;
     int ok, last;
@@ -165,6 +174,12 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Grid barrier arrival: this CTA's writes (ordered before it by a CTA barrier)
+// are visible before the count is.
+__device__ __forceinline__ void arrive_release(unsigned *ctr) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
@@ -421,72 +436,91 @@ __device__ __forceinline__ int task_slot(const DecodeParams &p, const Smem &s, c
 __device__ __forceinline__ int gu_rgl(const Geo &g, int warp, int ri) { return g.WPR > 1 ? warp / g.WPR : warp + 8 * ri; }
 __device__ __forceinline__ int gu_q0(const Geo &g, int warp) { return g.QPW * (warp % g.WPR); }
 
-// Lanes of one warp issue the bulk copies of the warp's gate/up slice of task
-// (slot, hb) into buffer b (lane 0 sets the expected bytes first): for each of
-// its RPW row groups, gate and up, the codes and scales of its QPW quads.
-template <int FMT>
-__device__ __forceinline__ void issue_gu(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int warp, int lane,
-                                         unsigned rank, int slot, int hb) {
-    const Geo &g = p.g;
-    uint8_t *dst = ring + size_t(b) * g.region + size_t(warp) * g.gu_warp;
-    const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
-    const int q0 = gu_q0(g, warp);
-    if (lane == 0) bar_expect(&s.gu_bar[b][warp], g.gu_warp);
-    __syncwarp();
-    // copy c: share ri = c / 4, matrix (c / 2) % 2, codes (c even) or scales
-    if (lane < 4 * g.RPW) {
-        const int ri = lane >> 2, mi = (lane >> 1) & 1, sc = lane & 1;
-        const MatGeom &m = mi ? p.up : p.gate;
-        const int rg = hb * (g.HB / 16) + int(rank) * g.GR + gu_rgl(g, warp, ri);
-        uint8_t *d0 = dst + size_t(ri * 2 + mi) * (g.gu_c + g.gu_s) + (sc ? g.gu_c : 0);
-        uint64_t off;
-        if (sc)
-            off = scale_off(m, FMT, rg, 2 * q0, 0);
-        else
-            off = FMT == 2 ? q2_chunk_off(m, rg, 2 * q0, 0) : q3_word_off(m, rg, q0, 0, 0);
-        bulk_copy(d0, rec + off, sc ? g.gu_s : g.gu_c, &s.gu_bar[b][warp]);
-    }
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];" ::"r"(saddr(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(saddr(bar))
+        : "memory");
 }
 
-// The warp's down slice: row groups rank*DR/16 + warp*NDRW + j, the task's HB
-// columns (block pair hb for Q2, block quad hb for Q3).
+// Copies of task (slot, hb) into buffer b, issued by threads 0 .. 4*GR of the
+// CTA: for each of its GR gate/up row groups, the gate and up codes and scales
+// over all of d (4 bulk copies, completing on that row group's barrier).
 template <int FMT>
-__device__ __forceinline__ void issue_dn(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int warp, int lane,
+__device__ __forceinline__ void issue_gu(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int tid,
                                          unsigned rank, int slot, int hb) {
     const Geo &g = p.g;
-    uint8_t *dst = ring + size_t(b) * g.region + size_t(kWarps) * g.gu_warp + size_t(warp) * g.dn_warp;
+    if (tid >= 4 * g.GR) return;
+    const int rgl = tid >> 2, mi = (tid >> 1) & 1, sc = tid & 1;
     const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
-    if (lane == 0) bar_expect(&s.dn_bar[b][warp], g.dn_warp);
-    __syncwarp();
-    for (int c = lane; c < 2 * g.NDRW; c += 32) {
-        const int j = c >> 1, sc = c & 1;
-        const int rg = int(rank) * (g.DR / 16) + warp * g.NDRW + j;
-        uint8_t *d0 = dst + size_t(j) * (g.dn_c + g.dn_s) + (sc ? g.dn_c : 0);
-        uint64_t off;
-        if (sc)
-            off = scale_off(p.down, FMT, rg, FMT == 2 ? hb : 2 * hb, 0);
-        else
-            off = FMT == 2 ? q2_chunk_off(p.down, rg, hb, 0) : q3_word_off(p.down, rg, hb, 0, 0);
-        bulk_copy(d0, rec + off, sc ? g.dn_s : g.dn_c, &s.dn_bar[b][warp]);
+    const MatGeom &m = mi ? p.up : p.gate;
+    const int rg = hb * (g.HB / 16) + int(rank) * g.GR + rgl;
+    uint8_t *dst = ring + size_t(b) * g.region + size_t(rgl) * g.gu_rg + size_t(mi) * (g.gu_c + g.gu_s) +
+                   (sc ? g.gu_c : 0);
+    if ((tid & 3) == 0) bar_expect(&s.gu_bar[b][rgl], g.gu_rg);
+    const uint64_t off = sc ? scale_off(m, FMT, rg, 0, 0) : (FMT == 2 ? q2_chunk_off(m, rg, 0, 0) : q3_word_off(m, rg, 0, 0, 0));
+    bulk_copy(dst, rec + off, sc ? g.gu_s : g.gu_c, &s.gu_bar[b][rgl]);
+}
+
+// The down slice of task (slot, hb) into buffer b, by thread 0: this CTA's DR
+// rows over the task's HB columns (block pair hb for Q2, block quad hb for
+// Q3), codes then scales, as two tensor copies.
+__device__ __forceinline__ void issue_dn(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int tid,
+                                         unsigned rank, int slot, int hb) {
+    const Geo &g = p.g;
+    if (tid != 0) return;
+    uint8_t *dst = ring + size_t(b) * g.region + g.gu_bytes;
+    const int ndr = g.DR / 16;
+    bar_expect(&s.dn_bar[b], g.dn_bytes);
+    tma_load_4d(dst, &p.dn_codes, 0, hb, int(rank) * ndr, slot, &s.dn_bar[b]);
+    tma_load_4d(dst + size_t(ndr) * g.dn_c, &p.dn_scales, 0, hb, int(rank) * ndr, slot, &s.dn_bar[b]);
+}
+
+// k largest of a warp's M keys per lane (64-bit: logit key << 32 | ~id),
+// descending, by k rounds of a warp-wide maximum; lane r < k receives the r-th.
+template <int M>
+__device__ __forceinline__ uint64_t warp_topk(uint64_t (&c)[M], int k, int lane) {
+    uint64_t mine = 0ull;
+    for (int r = 0; r < k; ++r) {
+        uint64_t mx = 0ull;
+#pragma unroll
+        for (int m = 0; m < M; ++m) mx = c[m] > mx ? c[m] : mx;
+        const uint32_t hk = __reduce_max_sync(0xffffffffu, uint32_t(mx >> 32));
+        const uint32_t lk = __reduce_max_sync(0xffffffffu, uint32_t(mx >> 32) == hk ? uint32_t(mx) : 0u);
+        const uint64_t win = (uint64_t(hk) << 32) | lk;
+        if (lane == r) mine = win;
+        if (mx == win && win != 0ull) {
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+                if (c[m] == win) c[m] = 0ull;
+        }
     }
+    return mine;
 }
 
 // Top-k of every token from the logits in global memory (written by all CTAs
-// of this launch): WPT = 8 / NT warps per token each find the k best of their
-// share of the experts by k rounds of a warp-wide maximum of 64-bit keys
-// (logit key << 32 | ~id: larger logit first, then lower id); the WPT sorted
-// lists are merged by counting, for every entry, the entries of the other
-// lists above it. Then softmax over the selected logits and ascending-id order
-// (the arithmetic of moe_route).
+// of this launch). A candidate is the 64-bit key (logit key << 32 | ~id), so
+// the top k are the k largest keys (larger logit first, then lower id).
+// WPT = 8 / NT warps share a token's experts. With WPT > 1 each warp finds the
+// R-th largest of its keys (R = ceil(k / WPT) rounds of a warp-wide maximum);
+// the smallest of those, L, has at least R * WPT >= k keys at or above it, so
+// the top k are the k largest of the keys >= L (usually a few dozen), ranked
+// by counting. If more than 64 keys reach L (near-equal logits) every warp
+// finds its exact top k by rounds and the lists are merged by counting. With
+// WPT = 1 the warp's k rounds give the answer. Then softmax over the selected
+// logits in ascending-id order (the arithmetic of moe_route).
 template <int NT>
 __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, int T, int E, int k) {
     constexpr int WPT = kWarps / NT;       // warps per token
     constexpr int M = kMaxEDec / 32 / WPT;  // keys per lane
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tt = warp / WPT, sub = warp % WPT;
+    uint64_t c[M], orig[WPT > 1 ? M : 1];
+    if (tid < kMaxTokDec) s.ncand[tid] = 0;
     if (tt < T) {
         const float *row = logits + size_t(tt) * E;
-        uint64_t c[M];
         bool nan = false;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
@@ -498,40 +532,67 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
             } else {
                 c[m] = 0ull;
             }
+            if constexpr (WPT > 1) orig[m] = c[m];
         }
         if (__any_sync(0xffffffffu, nan) && lane == 0 && blockIdx.x == 0) flag(p.status, MOE_DEV_NONFINITE);
-        uint64_t mine = 0ull;
-        for (int r = 0; r < k; ++r) {
-            uint64_t mx = 0ull;
-#pragma unroll
-            for (int m = 0; m < M; ++m) mx = c[m] > mx ? c[m] : mx;
-            const uint32_t hk = __reduce_max_sync(0xffffffffu, uint32_t(mx >> 32));
-            const uint32_t lk = __reduce_max_sync(0xffffffffu, uint32_t(mx >> 32) == hk ? uint32_t(mx) : 0u);
-            const uint64_t win = (uint64_t(hk) << 32) | lk;
-            if (lane == r) mine = win;
-            if (mx == win && win != 0ull) {
-#pragma unroll
-                for (int m = 0; m < M; ++m)
-                    if (c[m] == win) c[m] = 0ull;
-            }
-        }
-        if (WPT == 1) {
+        if constexpr (WPT == 1) {
+            const uint64_t mine = warp_topk<M>(c, k, lane);
             if (lane < k) s.sel[tt][lane] = mine;
-        } else if (lane < k) {
-            s.wl[warp][lane] = mine;
+        } else {
+            const int R = (k + WPT - 1) / WPT;
+            const uint64_t mine = warp_topk<M>(c, R, lane);
+            if (lane == R - 1) s.wl[warp][0] = mine;  // this warp's R-th largest
         }
     }
-    if (WPT > 1) {
+    if constexpr (WPT > 1) {
         __syncthreads();
-        if (tt < T && lane < k) {  // rank = entries of all the token's lists above mine (independent loads)
-            const uint64_t me = s.wl[warp][lane];
-            int rank = 0;
+        if (tt < T) {  // gather the keys >= L
+            uint64_t L = ~0ull;
 #pragma unroll
             for (int o = 0; o < WPT; ++o) {
-                const uint64_t *ol = s.wl[tt * WPT + o];
-                for (int q = 0; q < k; ++q) rank += ol[q] > me;
+                const uint64_t v = s.wl[tt * WPT + o][0];
+                L = v < L ? v : L;
             }
-            if (rank < k) s.sel[tt][rank] = me;
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                const bool in = orig[m] != 0ull && orig[m] >= L;
+                const unsigned bal = __ballot_sync(0xffffffffu, in);
+                int base = 0;
+                if (lane == 0 && bal) base = atomicAdd(&s.ncand[tt], __popc(bal));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                const int pos = base + __popc(bal & ((1u << lane) - 1u));
+                if (in && pos < 64) s.cand[tt][pos] = orig[m];
+            }
+        }
+        __syncthreads();
+        const bool many = tt < T && s.ncand[tt] > 64;
+        if (tt < T && !many) {  // rank the candidates: keys above mine
+            const int n = s.ncand[tt];
+            for (int i = sub * 32 + lane; i < n; i += WPT * 32) {
+                const uint64_t me = s.cand[tt][i];
+                int rank = 0;
+#pragma unroll 16
+                for (int q = 0; q < 64; ++q) rank += (q < n && s.cand[tt][q] > me);
+                if (rank < k) s.sel[tt][rank] = me;
+            }
+        }
+        if (__syncthreads_or(many)) {  // near-equal logits: exact lists per warp, merged by counting
+            if (many) {
+#pragma unroll
+                for (int m = 0; m < M; ++m) c[m] = orig[m];
+                const uint64_t mine = warp_topk<M>(c, k, lane);
+                if (lane < k) s.wl[warp][lane] = mine;
+            }
+            __syncthreads();
+            if (many && lane < k) {
+                const uint64_t me = s.wl[warp][lane];
+                int rank = 0;
+#pragma unroll
+                for (int o = 0; o < WPT; ++o)
+#pragma unroll 16
+                    for (int q = 0; q < kMaxK; ++q) rank += (q < k && s.wl[tt * WPT + o][q] > me);
+                if (rank < k) s.sel[tt][rank] = me;
+            }
         }
     }
     __syncthreads();
@@ -548,10 +609,13 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
         const float my_v = key ? key_value(key) : -INFINITY;
         const uint64_t top = s.sel[warp][0];
         const float mx = uint32_t(top >> 32) ? key_value(uint32_t(top >> 32)) : -INFINITY;
-        for (int q = 0; q < k; ++q) {
-            const uint64_t o = s.sel[warp][q];
-            const int oid = uint32_t(o >> 32) ? int(~uint32_t(o)) : 0;
-            rank += oid < my_id;
+#pragma unroll 16
+        for (int q = 0; q < kMaxK; ++q) {
+            if (q < k) {
+                const uint64_t o = s.sel[warp][q];
+                const int oid = uint32_t(o >> 32) ? int(~uint32_t(o)) : 0;
+                rank += oid < my_id;
+            }
         }
         ex = expf(my_v - mx);
         s.ex_r[warp][rank] = ex;
@@ -731,7 +795,7 @@ __device__ void publish(const DecodeParams &p, Smem &s, int l, int T, int k, int
 }
 
 template <int FMT, int NT>
-__global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_constant__ DecodeParams p) {
     extern __shared__ __align__(128) unsigned char dyn[];
     __shared__ Smem s;
     const Geo &g = p.g;
@@ -751,11 +815,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
 
     if (tid == 0) {
         bar_init(&s.rt_bar, 1);
-        for (int b = 0; b < kMaxBuf; ++b)
-            for (int w = 0; w < kWarps; ++w) {
-                bar_init(&s.gu_bar[b][w], 1);
-                bar_init(&s.dn_bar[b][w], 1);
-            }
+        for (int b = 0; b < kMaxBuf; ++b) {
+            for (int r = 0; r < 16; ++r) bar_init(&s.gu_bar[b][r], 1);
+            bar_init(&s.dn_bar[b], 1);
+        }
         bar_init(&s.xbar[0], 1);
         bar_init(&s.xbar[1], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -831,10 +894,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                                p.status);
         }
         ok = __syncthreads_and(ok) != 0;  // logits written; router rows and x consumed (the ring is free)
-        if (tid == 0) {
-            __threadfence();
-            atomicAdd(p.ctr, 1u);
-        }
+        if (tid == 0) arrive_release(p.ctr);
         bar_target += unsigned(G);
         TRACE(1);
         // this cluster's tasks known before routing: the shared expert's blocks
@@ -842,18 +902,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
         int known = 0;  // tasks of this cluster whose index is known (its list: cid, cid + ncl, ...)
         while (int(cid) + known * int(ncl) < nsh) ++known;
         const int seq0 = seq;  // this layer's first task of this CTA
-        int gu_next = 0, dn_next = 0;  // next task (layer-local) whose slices this warp copies
+        int gu_next = 0, dn_next = 0;  // next task (layer-local) whose copies are issued (CTA-uniform)
+        // called by every thread at the same points, after a CTA barrier that
+        // frees the buffers being refilled
         auto issue_upto = [&](int n_known, int gu_done, int dn_done) {
             while (gu_next < n_known && gu_next < gu_done + g.nbuf) {
                 int hb, a;
                 const int slot = task_slot(p, s, lp, int(cid) + gu_next * int(ncl), hb, a);
-                issue_gu<FMT>(p, s, ring, (seq0 + gu_next) % g.nbuf, warp, lane, rank, slot, hb);
+                issue_gu<FMT>(p, s, ring, (seq0 + gu_next) % g.nbuf, tid, rank, slot, hb);
                 ++gu_next;
             }
             while (dn_next < n_known && dn_next < dn_done + g.nbuf) {
                 int hb, a;
                 const int slot = task_slot(p, s, lp, int(cid) + dn_next * int(ncl), hb, a);
-                issue_dn<FMT>(p, s, ring, (seq0 + dn_next) % g.nbuf, warp, lane, rank, slot, hb);
+                issue_dn(p, s, ring, (seq0 + dn_next) % g.nbuf, tid, rank, slot, hb);
                 ++dn_next;
             }
         };
@@ -898,14 +960,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
             // the peers' h rows of this task land on xbar[xb]
             if (tid == 0) bar_expect(&s.xbar[xb], uint32_t(g.C - 1) * uint32_t(hrows * NT * 4));
             // gate/up of this warp's row groups over its quads
-            bool got = ok && bar_wait(&s.gu_bar[b][warp], ph);
-            if (i == 0) TRACE(5);
-            if (got) {
-                const uint8_t *slice = ring + size_t(b) * g.region + size_t(warp) * g.gu_warp;
-                const int q0 = gu_q0(g, warp);
-                for (int ri = 0; ri < g.RPW; ++ri) {
+            bool got = ok;
+            const int q0 = gu_q0(g, warp);
+            for (int ri = 0; ri < g.RPW && got; ++ri) {
+                const int rgl = gu_rgl(g, warp, ri);
+                got = bar_wait(&s.gu_bar[b][rgl], ph);
+                if (i == 0 && ri == 0) TRACE(5);
+                if (got) {
                     float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
-                    const uint8_t *gc = slice + size_t(ri * 2) * (g.gu_c + g.gu_s);
+                    const uint8_t *gc = ring + size_t(b) * g.region + size_t(rgl) * g.gu_rg;
                     const uint8_t *uc = gc + (g.gu_c + g.gu_s);
                     for (int qi = 0; qi < g.QPW; ++qi) {
                         uint32_t B[4][8];
@@ -925,8 +988,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                             xs[bq][1] = 2 * tl + 1 < T ? s.xs[4 * (q0 + qi) + bq][2 * tl + 1] : 0.f;
                         }
                         QuadRegs<FMT> qg, qu;
-                        quad_smem<FMT>(gc, gc + g.gu_c, qi, lane, qg);
-                        quad_smem<FMT>(uc, uc + g.gu_c, qi, lane, qu);
+                        quad_smem<FMT>(gc, gc + g.gu_c, q0 + qi, lane, qg);
+                        quad_smem<FMT>(uc, uc + g.gu_c, q0 + qi, lane, qu);
                         quad_compute<FMT>(qg, B, xs, ag);
                         quad_compute<FMT>(qu, B, xs, au);
                     }
@@ -936,11 +999,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                 }
             }
             if (!got && ok && lane == 0) flag(p.status, MOE_DEV_TIMEOUT);
-            ok = ok && __all_sync(0xffffffffu, got);
-            __syncwarp();
-            // this warp's gate/up slice of buffer b is free: copy ahead
+            ok = __syncthreads_and(ok && got) != 0;
+            // the gate/up part of buffer b is free: copy ahead
             if (ok) issue_upto(nmine, i + 1, i);
-            ok = __syncthreads_and(ok) != 0;
             if (i == 0) TRACE(6);
             // h = silu(a) * u of this CTA's hidden rows (the WPR warps of a row group
             // summed in warp order), written to its rows of hs
@@ -1010,10 +1071,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
             __syncthreads();
             // ---- down rows of this CTA over the task's columns (results staged in red)
             float *yst = red;
-            got = ok && bar_wait(&s.dn_bar[b][warp], ph);
+            got = ok && bar_wait(&s.dn_bar[b], ph);
             if (got) {
-                const uint8_t *slice =
-                    ring + size_t(b) * g.region + size_t(kWarps) * g.gu_warp + size_t(warp) * g.dn_warp;
+                const uint8_t *dcodes = ring + size_t(b) * g.region + g.gu_bytes;
+                const uint8_t *dscales = dcodes + size_t(g.DR / 16) * g.dn_c;
                 float xs[4][2];
 #pragma unroll
                 for (int bq = 0; bq < 4; ++bq) {
@@ -1021,7 +1082,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                     xs[bq][1] = bq < nbh && 2 * tl + 1 < T ? s.hsb[bq][2 * tl + 1] : 0.f;
                 }
                 for (int j = 0; j < g.NDRW; ++j) {
-                    const uint8_t *cb = slice + size_t(j) * (g.dn_c + g.dn_s);
+                    const uint8_t *cb = dcodes + size_t(warp * g.NDRW + j) * g.dn_c;
+                    const uint8_t *sb = dscales + size_t(warp * g.NDRW + j) * g.dn_s;
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
                     if constexpr (FMT == 2) {
                         uint32_t B[2][8];
@@ -1030,7 +1092,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
 #pragma unroll
                             for (int rho = 0; rho < 8; ++rho) B[bq][rho] = bfh[(bq * 8 + rho) * 32 + lane];
                         const uint4 c = *reinterpret_cast<const uint4 *>(cb + lane * 16);
-                        const uint4 sv = *reinterpret_cast<const uint4 *>(cb + g.dn_c + gl * 16);
+                        const uint4 sv = *reinterpret_cast<const uint4 *>(sb + gl * 16);
                         const float xs2[2][2] = {{xs[0][0], xs[0][1]}, {xs[1][0], xs[1][1]}};
                         pair_compute_q2(c, sv, B, xs2, acc);
                     } else {
@@ -1040,7 +1102,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
 #pragma unroll
                             for (int rho = 0; rho < 8; ++rho) B[bq][rho] = bfh[(bq * 8 + rho) * 32 + lane];
                         QuadRegs<FMT> q;
-                        quad_smem<FMT>(cb, cb + g.dn_c, 0, lane, q);
+                        quad_smem<FMT>(cb, sb, 0, lane, q);
                         quad_compute<FMT>(q, B, xs, acc);
                     }
                     const int rl = (warp * g.NDRW + j) * 16 + gl;  // row inside this CTA's DR rows
@@ -1052,10 +1114,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
                 }
             }
             if (!got && ok && lane == 0) flag(p.status, MOE_DEV_TIMEOUT);
-            ok = ok && __all_sync(0xffffffffu, got);
-            __syncwarp();
-            if (ok) issue_upto(nmine, i + 1, i + 1);
-            ok = __syncthreads_and(ok) != 0;
+            ok = __syncthreads_and(ok && got) != 0;
+            if (ok) issue_upto(nmine, i + 1, i + 1);  // the down part of buffer b is free
             if (i == 0) TRACE(8);
             // ---- gate-weighted vector atomics into y
             if (ok) {
@@ -1076,12 +1136,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
         seq += nmine;
         // copies issued for tasks that never ran (error paths) land before their buffers are reused
         if (gu_next > nmine || dn_next > nmine) {
-            for (int i = nmine; i < max(gu_next, dn_next); ++i) {
-                const int b = (seq0 + i) % g.nbuf;
-                const uint32_t ph = uint32_t((seq0 + i) / g.nbuf) & 1u;
-                if (i < gu_next) bar_wait(&s.gu_bar[b][warp], ph);
-                if (i < dn_next) bar_wait(&s.dn_bar[b][warp], ph);
-            }
+            if (tid == 0)
+                for (int i = nmine; i < max(gu_next, dn_next); ++i) {
+                    const int b = (seq0 + i) % g.nbuf;
+                    const uint32_t ph = uint32_t((seq0 + i) / g.nbuf) & 1u;
+                    for (int r = 0; i < gu_next && r < g.GR; ++r) bar_wait(&s.gu_bar[b][r], ph);
+                    if (i < dn_next) bar_wait(&s.dn_bar[b], ph);
+                }
+            __syncthreads();
             seq = seq0 + max(gu_next, dn_next);
         }
         if (ok && cta == G - 1) publish(p, s, l, T, k, E);
@@ -1089,10 +1151,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(DecodeParams 
         // (the next layer starts only once every contribution to this one is in y)
         if (l + 1 < p.L) {
             __syncthreads();
-            if (tid == 0) {
-                __threadfence();
-                atomicAdd(p.ctr, 1u);
-            }
+            if (tid == 0) arrive_release(p.ctr);
             bar_target += unsigned(G);
             if (tid == 0) s.ok = wait_geq(p.ctr, bar_target, p.status);
             __syncthreads();
@@ -1149,13 +1208,15 @@ bool plan(int fmt, int T, int d, int f, int E, int G, int C, size_t avail, Geo &
     g.DR = d / C;
     if (g.DR % 128) return false;
     g.NDRW = g.DR / 128;
-    g.gu_c = uint32_t(g.QPW) * (fmt == 2 ? 1024u : 1536u);
-    g.gu_s = uint32_t(g.QPW) * (fmt == 2 ? 256u : 128u);
+    g.gu_c = uint32_t(g.NQ) * (fmt == 2 ? 1024u : 1536u);
+    g.gu_s = uint32_t(g.NQ) * (fmt == 2 ? 256u : 128u);
     g.dn_c = fmt == 2 ? 512u : 1536u;
     g.dn_s = 128u;
-    g.gu_warp = uint32_t(g.RPW) * 2u * (g.gu_c + g.gu_s);
-    g.dn_warp = uint32_t(g.NDRW) * (g.dn_c + g.dn_s);
-    g.region = uint32_t(kWarps) * (g.gu_warp + g.dn_warp);
+    g.gu_rg = 2u * (g.gu_c + g.gu_s);
+    g.gu_bytes = uint32_t(g.GR) * g.gu_rg;
+    g.dn_bytes = uint32_t(g.DR / 16) * (g.dn_c + g.dn_s);
+    if (g.gu_bytes % 128) return false;
+    g.region = g.gu_bytes + g.dn_bytes;
     const int NTp = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8;
     g.red_bytes = uint32_t((std::max<size_t>(size_t(kWarps) * g.RPW * 32 * 8 * 4, size_t(NTp) * g.DR * 4) + 127) &
                            ~size_t(127));
@@ -1181,6 +1242,36 @@ bool plan(int fmt, int T, int d, int f, int E, int G, int C, size_t avail, Geo &
     }
     g.total = uint32_t(off + ring);
     return true;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// The down matrix of every slot of the pool as a 4D uint64 tensor [slot][row
+// group][chunk][elements] for its codes and for its scales; a chunk is the
+// codes (scales) of one row group over one block pair (Q2) or quad (Q3), and
+// a box is one chunk of nrg consecutive row groups.
+bool dn_maps(DecodeParams &p, int fmt, int d, int f, int nrg) {
+    const MatGeom &m = p.down;
+    const uint64_t nchunk = fmt == 2 ? uint64_t(m.NB / 2) : uint64_t(m.NB / 4);
+    const uint64_t cb = fmt == 2 ? 512 : 1536;          // code bytes of a chunk
+    const uint64_t sb = 128;                           // scale bytes of a chunk
+    const uint64_t srow = fmt == 2 ? uint64_t(m.NB / 2) * 128 : uint64_t(m.NB / 2) * 64;  // scale bytes per row group
+    const cuuint64_t cd[4] = {cb / 8, nchunk, cuuint64_t(d / 16), cuuint64_t(p.num_slots)};
+    const cuuint64_t cs[3] = {cb, nchunk * cb, cuuint64_t(p.slot_bytes)};
+    const cuuint32_t cbox[4] = {cuuint32_t(cb / 8), 1, cuuint32_t(nrg), 1};
+    const cuuint64_t sd[4] = {sb / 8, nchunk, cuuint64_t(d / 16), cuuint64_t(p.num_slots)};
+    const cuuint64_t ss[3] = {sb, srow, cuuint64_t(p.slot_bytes)};
+    const cuuint32_t sbox[4] = {cuuint32_t(sb / 8), 1, cuuint32_t(nrg), 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    (void)f;
+    auto enc = [&](CUtensorMap *map, const uint8_t *base, const cuuint64_t *dims, const cuuint64_t *strides,
+                   const cuuint32_t *box) {
+        return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 4, const_cast<uint8_t *>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    return enc(&p.dn_codes, p.pool + m.codes_off, cd, cs, cbox) &&
+           enc(&p.dn_scales, p.pool + m.scales_off, sd, ss, sbox);
 }
 
 struct LaunchInfo {
@@ -1248,6 +1339,18 @@ moe_status launch(DecodeParams p, cudaStream_t stream) {
         G = li.grid[C];
         if (plan(FMT, p.T, p.d, p.f, p.E, G, C, li.avail, p.g)) break;
     }
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (!dn_maps(p, FMT, p.d, p.f, p.g.DR / 16)) return MOE_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;

@@ -182,6 +182,21 @@ def test_fused_rejects_unsupported(tiny):
     assert ei.value.code == 2
 
 
+@pytest.mark.parametrize("T", [1, 2, 4])
+def test_fused_all_logits_equal(decode, T):
+    """x = 0 and no bias: all 512 logits tie, so far more than 64 keys reach the
+    selection threshold and the exact per-warp path runs; the experts must be
+    0..k-1 (ties go to the lower id) with equal gates."""
+    wl = configs.DECODE
+    saved = decode.bias[0].clone()
+    try:
+        decode.bias[0].zero_()
+        b, ref = _check(decode, 0, np.zeros((T, wl.d), np.uint16))
+        np.testing.assert_array_equal(ref["idx"], np.tile(np.arange(wl.k), (T, 1)))
+    finally:
+        decode.bias[0].copy_(saved)
+
+
 def test_fused_many_candidates_fallback(decode):
     """Experts in 10 of the 32 lanes (id % 32 < 10) all outrank the rest, so more
     than 64 candidates clear the k-th lane maximum and the round-based path runs."""
