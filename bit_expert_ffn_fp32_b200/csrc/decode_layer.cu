@@ -349,24 +349,95 @@ __device__ void router_row(const float *wrow, const uint16_t *sx, int T, int d, 
     }
 }
 
-// Q2 down tile of one block pair (16 rows x 128 columns): c = the lane's 16
-// code bytes, s = its 16 scale bytes (see layout.h), B / xs for the pair's two
-// blocks.
-__device__ __forceinline__ void pair_compute_q2(uint4 c, uint4 s, const uint32_t (&B)[2][8], const float (&xs)[2][2],
-                                                float (&acc)[4]) {
-    const uint32_t wg[2] = {c.x, c.z}, wg8[2] = {c.y, c.w};
-    const uint32_t sc[2] = {s.x, s.z}, mn[2] = {s.y, s.w};
+// One 64-weight block of a 16-row tile against B (4 MMAs over k 0..63): the
+// four MMAs start from zero accumulators and their results are summed
+// afterwards, so they are independent (no chain through the accumulator).
+template <int FMT>
+__device__ __forceinline__ void block_mma(const QuadRegs<FMT> &q, int bq, const uint32_t (&Bb)[8], float (&c)[4]) {
+    float p[4][4];
 #pragma unroll
-    for (int bq = 0; bq < 2; ++bq) {
-        float cc[4];
-        mma16816_zc(cc, q2_reg(wg[bq], 0), q2_reg(wg8[bq], 0), q2_reg(wg[bq], 1), q2_reg(wg8[bq], 1), B[bq][0],
-                    B[bq][1]);
-#pragma unroll
-        for (int i = 1; i < 4; ++i)
-            mma16816(cc, q2_reg(wg[bq], 2 * i), q2_reg(wg8[bq], 2 * i), q2_reg(wg[bq], 2 * i + 1),
-                     q2_reg(wg8[bq], 2 * i + 1), B[bq][2 * i], B[bq][2 * i + 1]);
-        block_epilogue<2>(cc, sc[bq], mn[bq], xs[bq][0], xs[bq][1], acc);
+    for (int i = 0; i < 4; ++i) {
+        uint32_t a0, a1, a2, a3;
+        if constexpr (FMT == 2) {
+            const uint32_t wg = bq == 0 ? q.c0.x : bq == 1 ? q.c0.z : bq == 2 ? q.c1.x : q.c1.z;
+            const uint32_t wg8 = bq == 0 ? q.c0.y : bq == 1 ? q.c0.w : bq == 2 ? q.c1.y : q.c1.w;
+            a0 = q2_reg(wg, 2 * i);
+            a1 = q2_reg(wg8, 2 * i);
+            a2 = q2_reg(wg, 2 * i + 1);
+            a3 = q2_reg(wg8, 2 * i + 1);
+        } else {
+            const int u0 = 8 * bq + 2 * i, u1 = u0 + 1;
+            a0 = q3_reg(q.W, u0, 0);
+            a1 = q3_reg(q.W, u0, 1);
+            a2 = q3_reg(q.W, u1, 0);
+            a3 = q3_reg(q.W, u1, 1);
+        }
+        mma16816_zc(p[i], a0, a1, a2, a3, Bb[2 * i], Bb[2 * i + 1]);
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) c[j] = (p[0][j] + p[1][j]) + (p[2][j] + p[3][j]);
+}
+
+template <int FMT>
+__device__ __forceinline__ uint32_t block_scale(const QuadRegs<FMT> &q, int bq) {
+    if constexpr (FMT == 2) return bq == 0 ? q.s0.x : bq == 1 ? q.s0.z : bq == 2 ? q.s1.x : q.s1.z;
+    else return bq == 0 ? q.s0.x : bq == 1 ? q.s0.y : bq == 2 ? q.s1.x : q.s1.y;
+}
+template <int FMT>
+__device__ __forceinline__ uint32_t block_min(const QuadRegs<FMT> &q, int bq) {
+    if constexpr (FMT == 2) return bq == 0 ? q.s0.y : bq == 1 ? q.s0.w : bq == 2 ? q.s1.y : q.s1.w;
+    else return 0u;
+}
+
+// Gate and up tiles of one 16-row x 256-column quad against the same B,
+// block by block with the two matrices interleaved (8 independent MMAs per block).
+template <int FMT>
+__device__ __forceinline__ void quad_pair_compute(const QuadRegs<FMT> &qg, const QuadRegs<FMT> &qu,
+                                                  const uint32_t (&B)[4][8], const float (&xs)[4][2],
+                                                  float (&ag)[4], float (&au)[4]) {
+#pragma unroll
+    for (int bq = 0; bq < 4; ++bq) {
+        float cg[4], cu[4];
+        block_mma<FMT>(qg, bq, B[bq], cg);
+        block_mma<FMT>(qu, bq, B[bq], cu);
+        block_epilogue<FMT>(cg, block_scale<FMT>(qg, bq), block_min<FMT>(qg, bq), xs[bq][0], xs[bq][1], ag);
+        block_epilogue<FMT>(cu, block_scale<FMT>(qu, bq), block_min<FMT>(qu, bq), xs[bq][0], xs[bq][1], au);
+    }
+}
+
+// One quad (4 blocks) of one matrix.
+template <int FMT>
+__device__ __forceinline__ void quad_compute_ilp(const QuadRegs<FMT> &q, const uint32_t (&B)[4][8],
+                                                 const float (&xs)[4][2], float (&acc)[4]) {
+    float c[4][4];
+#pragma unroll
+    for (int bq = 0; bq < 4; ++bq) block_mma<FMT>(q, bq, B[bq], c[bq]);
+#pragma unroll
+    for (int bq = 0; bq < 4; ++bq)
+        block_epilogue<FMT>(c[bq], block_scale<FMT>(q, bq), block_min<FMT>(q, bq), xs[bq][0], xs[bq][1], acc);
+}
+
+// Q2 down tiles of one block pair (16 rows x 128 columns) for two row groups:
+// c = a lane's 16 code bytes, s = its 16 scale bytes (see layout.h), B / xs of
+// the pair's two blocks; 16 independent MMAs.
+__device__ __forceinline__ void pair2_compute_q2(uint4 c0, uint4 s0, uint4 c1, uint4 s1, const uint32_t (&B)[2][8],
+                                                 const float (&xs)[2][2], float (&acc0)[4], float (&acc1)[4]) {
+    QuadRegs<2> q0, q1;  // blocks 0, 1 of each pair in the first half of a quad's registers
+    q0.c0 = c0;
+    q0.s0 = s0;
+    q1.c0 = c1;
+    q1.s0 = s1;
+    q0.c1 = q1.c1 = make_uint4(0u, 0u, 0u, 0u);
+    q0.s1 = q1.s1 = make_uint4(0u, 0u, 0u, 0u);
+    float r[4][4];
+    block_mma<2>(q0, 0, B[0], r[0]);
+    block_mma<2>(q0, 1, B[1], r[1]);
+    block_mma<2>(q1, 0, B[0], r[2]);
+    block_mma<2>(q1, 1, B[1], r[3]);
+    block_epilogue<2>(r[0], s0.x, s0.y, xs[0][0], xs[0][1], acc0);
+    block_epilogue<2>(r[1], s0.z, s0.w, xs[1][0], xs[1][1], acc0);
+    block_epilogue<2>(r[2], s1.x, s1.y, xs[0][0], xs[0][1], acc1);
+    block_epilogue<2>(r[3], s1.z, s1.w, xs[1][0], xs[1][1], acc1);
 }
 
 // Packed codes and scales of one 16-row x 256-column tile from shared memory:
@@ -445,21 +516,23 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// Copies of task (slot, hb) into buffer b, issued by threads 0 .. 4*GR of the
-// CTA: for each of its GR gate/up row groups, the gate and up codes and scales
-// over all of d (4 bulk copies, completing on that row group's barrier).
+// Copies of task (slot, hb) into buffer b: for each of its GR gate/up row
+// groups, the gate and up codes and scales over all of d (4 bulk copies,
+// completing on that row group's barrier). Copy c is issued by lane c / 8 of
+// warp c % 8, so the copies of a task leave from all warps at once.
 template <int FMT>
 __device__ __forceinline__ void issue_gu(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int tid,
                                          unsigned rank, int slot, int hb) {
     const Geo &g = p.g;
-    if (tid >= 4 * g.GR) return;
-    const int rgl = tid >> 2, mi = (tid >> 1) & 1, sc = tid & 1;
+    const int c = (tid & 31) * kWarps + (tid >> 5);
+    if (c >= 4 * g.GR) return;
+    const int rgl = c >> 2, mi = (c >> 1) & 1, sc = c & 1;
     const uint8_t *rec = p.pool + int64_t(slot) * p.slot_bytes;
     const MatGeom &m = mi ? p.up : p.gate;
     const int rg = hb * (g.HB / 16) + int(rank) * g.GR + rgl;
     uint8_t *dst = ring + size_t(b) * g.region + size_t(rgl) * g.gu_rg + size_t(mi) * (g.gu_c + g.gu_s) +
                    (sc ? g.gu_c : 0);
-    if ((tid & 3) == 0) bar_expect(&s.gu_bar[b][rgl], g.gu_rg);
+    if ((c & 3) == 0) bar_expect(&s.gu_bar[b][rgl], g.gu_rg);
     const uint64_t off = sc ? scale_off(m, FMT, rg, 0, 0) : (FMT == 2 ? q2_chunk_off(m, rg, 0, 0) : q3_word_off(m, rg, 0, 0, 0));
     bulk_copy(dst, rec + off, sc ? g.gu_s : g.gu_c, &s.gu_bar[b][rgl]);
 }
@@ -519,6 +592,8 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
     const int tt = warp / WPT, sub = warp % WPT;
     uint64_t c[M], orig[WPT > 1 ? M : 1];
     if (tid < kMaxTokDec) s.ncand[tid] = 0;
+    const int l = 0;  // (trace points are recorded for the first layer)
+    (void)l;
     if (tt < T) {
         const float *row = logits + size_t(tt) * E;
         bool nan = false;
@@ -535,6 +610,7 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
             if constexpr (WPT > 1) orig[m] = c[m];
         }
         if (__any_sync(0xffffffffu, nan) && lane == 0 && blockIdx.x == 0) flag(p.status, MOE_DEV_NONFINITE);
+        TRACE(14);
         if constexpr (WPT == 1) {
             const uint64_t mine = warp_topk<M>(c, k, lane);
             if (lane < k) s.sel[tt][lane] = mine;
@@ -546,6 +622,7 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
     }
     if constexpr (WPT > 1) {
         __syncthreads();
+        TRACE(15);
         if (tt < T) {  // gather the keys >= L
             uint64_t L = ~0ull;
 #pragma unroll
@@ -565,6 +642,7 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
             }
         }
         __syncthreads();
+        TRACE(16);
         const bool many = tt < T && s.ncand[tt] > 64;
         if (tt < T && !many) {  // rank the candidates: keys above mine
             const int n = s.ncand[tt];
@@ -596,6 +674,7 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
         }
     }
     __syncthreads();
+    TRACE(17);
     // softmax over the selected logits in ascending-id order (the arithmetic of
     // moe_route: z summed from 0 in that order, gate = ex * (1 / z))
     const bool selt = warp < T && lane < k;
@@ -831,8 +910,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
     const int nrows = re - rb;
 
 #ifdef MOE_DECODE_TRACE
-    if (tid == 0)  // points this launch does not reach stay empty
+    if (tid == 0) {  // points this launch does not reach stay empty; 30/31: SM cycles at start / end
         for (int i = 1; i < 32; ++i) moe_decode_trace[blockIdx.x * 32 + i] = 0ull;
+        moe_decode_trace[blockIdx.x * 32 + 30] = clock64();
+    }
 #endif
     for (int l = 0; l < p.L; ++l) {
         const LayerPtrs lp = layer_ptrs(p, l);
@@ -990,8 +1071,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
                         QuadRegs<FMT> qg, qu;
                         quad_smem<FMT>(gc, gc + g.gu_c, q0 + qi, lane, qg);
                         quad_smem<FMT>(uc, uc + g.gu_c, q0 + qi, lane, qu);
-                        quad_compute<FMT>(qg, B, xs, ag);
-                        quad_compute<FMT>(qu, B, xs, au);
+                        quad_pair_compute<FMT>(qg, qu, B, xs, ag, au);
                     }
                     float4 *dst = reinterpret_cast<float4 *>(red + (size_t(warp * g.RPW + ri) * 32 + lane) * 8);
                     dst[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
@@ -1081,35 +1161,47 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
                     xs[bq][0] = bq < nbh && 2 * tl < T ? s.hsb[bq][2 * tl] : 0.f;
                     xs[bq][1] = bq < nbh && 2 * tl + 1 < T ? s.hsb[bq][2 * tl + 1] : 0.f;
                 }
-                for (int j = 0; j < g.NDRW; ++j) {
-                    const uint8_t *cb = dcodes + size_t(warp * g.NDRW + j) * g.dn_c;
-                    const uint8_t *sb = dscales + size_t(warp * g.NDRW + j) * g.dn_s;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    if constexpr (FMT == 2) {
-                        uint32_t B[2][8];
-#pragma unroll
-                        for (int bq = 0; bq < 2; ++bq)
-#pragma unroll
-                            for (int rho = 0; rho < 8; ++rho) B[bq][rho] = bfh[(bq * 8 + rho) * 32 + lane];
-                        const uint4 c = *reinterpret_cast<const uint4 *>(cb + lane * 16);
-                        const uint4 sv = *reinterpret_cast<const uint4 *>(sb + gl * 16);
-                        const float xs2[2][2] = {{xs[0][0], xs[0][1]}, {xs[1][0], xs[1][1]}};
-                        pair_compute_q2(c, sv, B, xs2, acc);
-                    } else {
-                        uint32_t B[4][8];
-#pragma unroll
-                        for (int bq = 0; bq < 4; ++bq)
-#pragma unroll
-                            for (int rho = 0; rho < 8; ++rho) B[bq][rho] = bfh[(bq * 8 + rho) * 32 + lane];
-                        QuadRegs<FMT> q;
-                        quad_smem<FMT>(cb, sb, 0, lane, q);
-                        quad_compute<FMT>(q, B, xs, acc);
-                    }
+                auto stage = [&](int j, const float (&acc)[4]) {
                     const int rl = (warp * g.NDRW + j) * 16 + gl;  // row inside this CTA's DR rows
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
                         const int n = 2 * tl + (r & 1);
                         if (n < NT) yst[n * g.DR + rl + ((r & 2) ? 8 : 0)] = acc[r];
+                    }
+                };
+                if constexpr (FMT == 2) {
+                    uint32_t B[2][8];
+#pragma unroll
+                    for (int bq = 0; bq < 2; ++bq)
+#pragma unroll
+                        for (int rho = 0; rho < 8; ++rho) B[bq][rho] = bfh[(bq * 8 + rho) * 32 + lane];
+                    const float xs2[2][2] = {{xs[0][0], xs[0][1]}, {xs[1][0], xs[1][1]}};
+                    for (int j = 0; j < g.NDRW; j += 2) {  // NDRW is even (DR is a multiple of 256)
+                        const int r0 = warp * g.NDRW + j;
+                        const uint4 c0 = *reinterpret_cast<const uint4 *>(dcodes + size_t(r0) * g.dn_c + lane * 16);
+                        const uint4 c1 =
+                            *reinterpret_cast<const uint4 *>(dcodes + size_t(r0 + 1) * g.dn_c + lane * 16);
+                        const uint4 s0 = *reinterpret_cast<const uint4 *>(dscales + size_t(r0) * g.dn_s + gl * 16);
+                        const uint4 s1 =
+                            *reinterpret_cast<const uint4 *>(dscales + size_t(r0 + 1) * g.dn_s + gl * 16);
+                        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+                        pair2_compute_q2(c0, s0, c1, s1, B, xs2, acc0, acc1);
+                        stage(j, acc0);
+                        stage(j + 1, acc1);
+                    }
+                } else {
+                    uint32_t B[4][8];
+#pragma unroll
+                    for (int bq = 0; bq < 4; ++bq)
+#pragma unroll
+                        for (int rho = 0; rho < 8; ++rho) B[bq][rho] = bfh[(bq * 8 + rho) * 32 + lane];
+                    for (int j = 0; j < g.NDRW; ++j) {
+                        const int r0 = warp * g.NDRW + j;
+                        QuadRegs<FMT> q;
+                        quad_smem<FMT>(dcodes + size_t(r0) * g.dn_c, dscales + size_t(r0) * g.dn_s, 0, lane, q);
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                        quad_compute_ilp<FMT>(q, B, xs, acc);
+                        stage(j, acc);
                     }
                 }
             }
@@ -1161,6 +1253,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
     }
 
     if (too_big) flag(p.status, MOE_DEV_NONFINITE);
+#ifdef MOE_DECODE_TRACE
+    if (tid == 0) {
+        unsigned long long t_;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));
+        moe_decode_trace[blockIdx.x * 32 + 29] = t_;
+        moe_decode_trace[blockIdx.x * 32 + 31] = clock64();
+    }
+#endif
     // no CTA leaves while a peer may still send into its shared memory
     asm volatile("barrier.cluster.arrive.relaxed.aligned;\nbarrier.cluster.wait.aligned;" ::: "memory");
     if (tid == 0) {

@@ -3,10 +3,14 @@
     python -m bit_expert_ffn_fp32_b200.build --trace
     python -m bit_expert_ffn_fp32_b200.trace_decode [WORKLOAD] [--launches N] [--warm]
 
-Loads libmoe_trace.so (the library built with -DMOE_DECODE_TRACE), runs the
-layer N times on fresh tokens with the L2 evicted before each launch (unless
---warm), and prints, for each phase boundary, the median over launches of the
-median and the slowest CTA, in microseconds since the first CTA started.
+Loads libmoe_trace.so (the library built with -DMOE_DECODE_TRACE) and runs
+the layer as the benchmark does: bursts of back-to-back steps on fresh tokens
+(resident in HBM), each step after a 512 MiB write and a 256 MiB read of other
+buffers (unless --warm), CUDA events around every launch. The trace of the last
+launch of each burst is read; the report gives, for each phase boundary, the
+median over bursts of the median and the slowest CTA (microseconds since the
+first CTA started), the launch time between events and the SM clock the kernel
+ran at (cycles over nanoseconds between kernel start and end).
 """
 from __future__ import annotations
 
@@ -21,7 +25,8 @@ from . import configs, native, synth
 from .layer import MoEStack, x_tensor
 
 POINTS = {12: "x staged", 13: "router rows landed", 1: "logits written", 2: "grid barrier passed",
-          3: "top-k + gates", 4: "routing tables", 11: "cluster task count", 5: "task 1 gate/up landed (warp 0)",
+          14: "top-k: logits loaded", 15: "top-k: threshold rounds", 16: "top-k: candidates gathered",
+          17: "top-k: ranked", 3: "top-k + gates", 4: "routing tables", 11: "cluster task count", 5: "task 1 gate/up landed (warp 0)",
           6: "task 1 gate/up computed (warp 0)", 7: "task 1 partials exchanged", 8: "task 1 down computed",
           9: "task 1 atomics done", 10: "layer end"}
 
@@ -44,29 +49,37 @@ def main() -> None:
     wl = configs.WORKLOADS[args.workload]
     stack = MoEStack(wl)
     b = stack.buffers(wl.T)
-    flush = torch.empty(512 << 18, dtype=torch.float32, device="cuda")
+    wbuf = torch.empty(512 << 18, dtype=torch.float32, device="cuda")
+    rbuf = torch.ones(256 << 18, dtype=torch.float32, device="cuda")
+    out = torch.empty((), dtype=torch.float32, device="cuda")
+    xs = [x_tensor(synth.gen_x(wl.seed, 0, wl.T, wl.d, stream=s), "cuda") for s in range(16)]
     buf = np.zeros(4096 * 32, np.uint64)
     acc = {k: [] for k in POINTS}
-    starts = []
-    skip = 10
-    ev = []
-    for it in range(args.launches + skip):
-        x = x_tensor(synth.gen_x(wl.seed, 0, wl.T, wl.d, stream=0 if args.warm else it))
-        if not args.warm:
-            flush.fill_(1.0)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        stack.forward_fused(0, x, b)
-        e1.record()
+    starts, ev, mhz = [], [], []
+    burst = 6
+    for it in range(args.launches + 3):
+        evs = []
+        for j in range(burst):
+            if not args.warm:
+                wbuf.fill_(float(j))
+                torch.sum(rbuf, 0, out=out)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            stack.forward_fused(0, xs[0 if args.warm else (it * burst + j) % len(xs)], b)
+            e1.record()
+            evs.append((e0, e1))
         torch.cuda.synchronize()
-        if it >= skip:
-            ev.append(e0.elapsed_time(e1) * 1e3)
-        tl.moe_decode_trace_read(buf.ctypes.data)
-        if it < skip:
+        if it < 3:
             continue
+        ev.extend(a.elapsed_time(c) * 1e3 for a, c in evs[1:])
+        tl.moe_decode_trace_read(buf.ctypes.data)
         tr = buf.reshape(4096, 32)
         G = int((tr[:, 0] > 0).sum())
         ns = tr[:G, :].astype(np.int64)
+        cyc = (ns[:, 31] - ns[:, 30]).astype(np.float64)
+        dur = (ns[:, 29] - ns[:, 0]).astype(np.float64)
+        mhz.append(float(np.median(cyc / dur * 1e3)))
+        ns = ns[:, :29]
         rel = np.where(ns > 0, (ns - ns[:, 0].min()) / 1000.0, np.nan)
         starts.append(float((ns[:, 0].max() - ns[:, 0].min()) / 1000.0))
         for k in POINTS:
@@ -75,7 +88,7 @@ def main() -> None:
     print(f"{wl.name}: {G} CTAs, {'warm' if args.warm else 'L2 evicted before each launch'}, "
           f"status {int(b.status.item())}")
     print(f"launch time between CUDA events: median {np.median(ev):.2f} us; CTA start spread median "
-          f"{np.median(starts):.2f} us")
+          f"{np.median(starts):.2f} us; SM clock during the kernel: median {np.median(mhz):.0f} MHz")
     print(f"{'point':34s} {'median CTA':>11s} {'slowest CTA':>12s}  (us since first CTA start)")
     for k, nm in POINTS.items():
         if acc[k]:
