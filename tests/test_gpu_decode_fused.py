@@ -136,7 +136,9 @@ def test_fused_with_misses():
         assert int(b.miss_count.item()) == 2 * wl.k
         stack.forward(0, x_tensor(x_bits), b)
         torch.cuda.synchronize()
-        assert rel_err(y_sh.cpu().numpy(), b.y_sh[:2].cpu().numpy()) < 1e-6
+        # the same fp32 sums in another association (the fused kernel adds each block's
+        # four MMA partials after the fact; the step-by-step kernels chain them)
+        assert rel_err(y_sh.cpu().numpy(), b.y_sh[:2].cpu().numpy()) < 1e-5
     finally:
         stack.slot_of[0].copy_(saved)
 
