@@ -62,9 +62,21 @@ __device__ unsigned long long moe_decode_trace[4096 * 32];
             moe_decode_trace[blockIdx.x * 32 + (i)] = t_;                                             \
         }                                                                                             \
     } while (0)
+// the same, recorded by lane 0 of the calling warp
+#define TRACEW(i)                                                                                     \
+    do {                                                                                              \
+        if ((threadIdx.x & 31) == 0 && l == 0) {                                                      \
+            unsigned long long t_;                                                                    \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                    \
+            moe_decode_trace[blockIdx.x * 32 + (i)] = t_;                                             \
+        }                                                                                             \
+    } while (0)
 #else
 #define TRACE(i) \
     do {         \
+    } while (0)
+#define TRACEW(i) \
+    do {          \
     } while (0)
 #endif
 
@@ -1046,7 +1058,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
             for (int ri = 0; ri < g.RPW && got; ++ri) {
                 const int rgl = gu_rgl(g, warp, ri);
                 got = bar_wait(&s.gu_bar[b][rgl], ph);
-                if (i == 0 && ri == 0) TRACE(5);
+                if (i == 0 && ri == 0) TRACEW(18 + warp);
                 if (got) {
                     float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
                     const uint8_t *gc = ring + size_t(b) * g.region + size_t(rgl) * g.gu_rg;
@@ -1078,6 +1090,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
                     dst[1] = make_float4(au[0], au[1], au[2], au[3]);
                 }
             }
+            if (i == 0 && warp == 0) TRACEW(26);
             if (!got && ok && lane == 0) flag(p.status, MOE_DEV_TIMEOUT);
             ok = __syncthreads_and(ok && got) != 0;
             // the gate/up part of buffer b is free: copy ahead
@@ -1152,6 +1165,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
             // ---- down rows of this CTA over the task's columns (results staged in red)
             float *yst = red;
             got = ok && bar_wait(&s.dn_bar[b], ph);
+            if (i == 0 && warp == 0) TRACEW(27);
             if (got) {
                 const uint8_t *dcodes = ring + size_t(b) * g.region + g.gu_bytes;
                 const uint8_t *dscales = dcodes + size_t(g.DR / 16) * g.dn_c;
@@ -1205,6 +1219,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
                     }
                 }
             }
+            if (i == 0 && warp == 0) TRACEW(28);
             if (!got && ok && lane == 0) flag(p.status, MOE_DEV_TIMEOUT);
             ok = __syncthreads_and(ok && got) != 0;
             if (ok) issue_upto(nmine, i + 1, i + 1);  // the down part of buffer b is free

@@ -26,8 +26,11 @@ from .layer import MoEStack, x_tensor
 
 POINTS = {12: "x staged", 13: "router rows landed", 1: "logits written", 2: "grid barrier passed",
           14: "top-k: logits loaded", 15: "top-k: threshold rounds", 16: "top-k: candidates gathered",
-          17: "top-k: ranked", 3: "top-k + gates", 4: "routing tables", 11: "cluster task count", 5: "task 1 gate/up landed (warp 0)",
-          6: "task 1 gate/up computed (warp 0)", 7: "task 1 partials exchanged", 8: "task 1 down computed",
+          17: "top-k: ranked", 3: "top-k + gates", 4: "routing tables", 11: "copies of the first tasks issued",
+          **{18 + w: f"task 1 row group landed (warp {w})" for w in range(8)},
+          26: "task 1 gate/up computed (warp 0 alone)", 6: "task 1 gate/up computed (all warps)",
+          7: "task 1 h exchanged", 27: "task 1 down slice landed (warp 0)",
+          28: "task 1 down computed (warp 0 alone)", 8: "task 1 down computed (all warps)",
           9: "task 1 atomics done", 10: "layer end"}
 
 
