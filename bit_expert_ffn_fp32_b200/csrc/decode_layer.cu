@@ -50,13 +50,13 @@
 #include "mma_q.cuh"
 
 // Optional phase timestamps (build with -DMOE_DECODE_TRACE): thread 0 of every
-// CTA records %globaltimer at each phase boundary of the first layer into
-// moe_decode_trace.
+// CTA records %globaltimer at each phase boundary of layer L / 2 (the only
+// layer of a one-layer call) into moe_decode_trace.
 #ifdef MOE_DECODE_TRACE
 __device__ unsigned long long moe_decode_trace[4096 * 32];
 #define TRACE(i)                                                                                      \
     do {                                                                                              \
-        if (threadIdx.x == 0 && l == 0) {                                                             \
+        if (threadIdx.x == 0 && l == p.L / 2) {                                                       \
             unsigned long long t_;                                                                    \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                    \
             moe_decode_trace[blockIdx.x * 32 + (i)] = t_;                                             \
@@ -65,7 +65,7 @@ __device__ unsigned long long moe_decode_trace[4096 * 32];
 // the same, recorded by lane 0 of the calling warp
 #define TRACEW(i)                                                                                     \
     do {                                                                                              \
-        if ((threadIdx.x & 31) == 0 && l == 0) {                                                      \
+        if ((threadIdx.x & 31) == 0 && l == p.L / 2) {                                                \
             unsigned long long t_;                                                                    \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                    \
             moe_decode_trace[blockIdx.x * 32 + (i)] = t_;                                             \
@@ -604,7 +604,7 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
     const int tt = warp / WPT, sub = warp % WPT;
     uint64_t c[M], orig[WPT > 1 ? M : 1];
     if (tid < kMaxTokDec) s.ncand[tid] = 0;
-    const int l = 0;  // (trace points are recorded for the first layer)
+    const int l = p.L / 2;  // (trace points of the traced layer only; the caller passes that layer's logits)
     (void)l;
     if (tt < T) {
         const float *row = logits + size_t(tt) * E;

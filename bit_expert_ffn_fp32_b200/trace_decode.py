@@ -4,7 +4,8 @@
     python -m bit_expert_ffn_fp32_b200.trace_decode [WORKLOAD] [--launches N] [--warm]
 
 Loads libmoe_trace.so (the library built with -DMOE_DECODE_TRACE) and runs
-the layer as the benchmark does: bursts of back-to-back steps on fresh tokens
+the layer (or, for a stacked workload, all layers in one launch, tracing
+layer L/2) as the benchmark does: bursts of back-to-back steps on fresh tokens
 (resident in HBM), each step after a 512 MiB write and a 256 MiB read of other
 buffers (unless --warm), CUDA events around every launch. The trace of the last
 launch of each burst is read; the report gives, for each phase boundary, the
@@ -56,6 +57,9 @@ def main() -> None:
     rbuf = torch.ones(256 << 18, dtype=torch.float32, device="cuda")
     out = torch.empty((), dtype=torch.float32, device="cuda")
     xs = [x_tensor(synth.gen_x(wl.seed, 0, wl.T, wl.d, stream=s), "cuda") for s in range(16)]
+    sb = stack.stack_buffers(wl.T) if stack.L > 1 else None
+    xst = [torch.stack([x_tensor(synth.gen_x(wl.seed, l, wl.T, wl.d, stream=s), "cuda") for l in range(stack.L)])
+           for s in range(4)] if stack.L > 1 else None
     buf = np.zeros(4096 * 32, np.uint64)
     acc = {k: [] for k in POINTS}
     starts, ev, mhz = [], [], []
@@ -68,7 +72,10 @@ def main() -> None:
                 torch.sum(rbuf, 0, out=out)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            stack.forward_fused(0, xs[0 if args.warm else (it * burst + j) % len(xs)], b)
+            if stack.L > 1:
+                stack.forward_stack(xst[0 if args.warm else (it * burst + j) % len(xst)], sb)
+            else:
+                stack.forward_fused(0, xs[0 if args.warm else (it * burst + j) % len(xs)], b)
             e1.record()
             evs.append((e0, e1))
         torch.cuda.synchronize()
@@ -88,8 +95,9 @@ def main() -> None:
         for k in POINTS:
             if np.isfinite(rel[:, k]).any():
                 acc[k].append((np.nanmedian(rel[:, k]), np.nanmax(rel[:, k])))
-    print(f"{wl.name}: {G} CTAs, {'warm' if args.warm else 'L2 evicted before each launch'}, "
-          f"status {int(b.status.item())}")
+    st = int((sb.status if sb is not None else b.status).item())
+    print(f"{wl.name}: {G} CTAs, {'warm' if args.warm else 'L2 evicted before each launch'}, status {st}"
+          + (f"; layer {stack.L // 2} of {stack.L} traced" if stack.L > 1 else ""))
     print(f"launch time between CUDA events: median {np.median(ev):.2f} us; CTA start spread median "
           f"{np.median(starts):.2f} us; SM clock during the kernel: median {np.median(mhz):.0f} MHz")
     print(f"{'point':34s} {'median CTA':>11s} {'slowest CTA':>12s}  (us since first CTA start)")
