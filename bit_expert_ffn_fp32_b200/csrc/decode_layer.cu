@@ -93,6 +93,10 @@ constexpr int kMaxFDec = 4096;
 constexpr unsigned long long kWaitNs = 100ull * 1000 * 1000;
 constexpr unsigned long long kWaitSteps = 1ull << 27;  // polls: >= 4 s of 32 ns sleeps
 constexpr int kMaxBuf = 2;                             // task buffers in the weight ring
+// Copies of the logits in the workspace: every CTA reads all logits right after
+// the grid barrier; CTA c reads copy c % kLogitCopies, so those reads spread
+// over more L2 lines than one copy (one copy would be read by every SM at once).
+constexpr int kLogitCopies = 8;
 
 // Geometry of one launch (host-computed; see plan()).
 struct Geo {
@@ -129,8 +133,8 @@ struct DecodeParams {
     const float *Wr;             // [L][E][d]
     const float *bias;           // [L][E] or NULL
     int T, d, f, E, k;
-    float *logits;               // [2][T][E] workspace, or [T][E] output for L == 1
-    bool logits_out;
+    float *logits;               // [2][kLogitCopies][T][E] workspace
+    float *logits_out;           // [T][E] output (L == 1) or NULL
     int32_t *topk_idx;           // [L][T*k] or NULL
     float *topk_w;
     int32_t *counts, *offsets, *sorted_tok, *sorted_j, *inv, *active;  // L == 1 only (else NULL)
@@ -329,7 +333,7 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 // One router row (fixed fp32 order, see moe.h) for NT tokens from shared memory.
 template <int NT>
 __device__ void router_row(const float *wrow, const uint16_t *sx, int T, int d, int lane, bool has_bias, float b,
-                           int e, float *logits, int E, int32_t *status) {
+                           int e, float *logits, float *logits_out, int E, int32_t *status) {
     float acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.f;
@@ -352,21 +356,21 @@ __device__ void router_row(const float *wrow, const uint16_t *sx, int T, int d, 
     for (int t = 0; t < NT; ++t)
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) acc[t] = __fadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], o));
-    if (lane == 0) {
+    if (lane < kLogitCopies) {  // lane c writes copy c
         for (int t = 0; t < T; ++t) {
             const float v = has_bias ? __fadd_rn(acc[t], b) : acc[t];
-            if (!isfinite(v)) flag(status, MOE_DEV_NONFINITE);
-            __stcg(logits + size_t(t) * E + e, v);
+            if (lane == 0 && !isfinite(v)) flag(status, MOE_DEV_NONFINITE);
+            __stcg(logits + (size_t(lane) * T + t) * E + e, v);
+            if (lane == 0 && logits_out) logits_out[size_t(t) * E + e] = v;
         }
     }
 }
 
-// One 64-weight block of a 16-row tile against B (4 MMAs over k 0..63): the
-// four MMAs start from zero accumulators and their results are summed
-// afterwards, so they are independent (no chain through the accumulator).
+// One 64-weight block of a 16-row tile against B (4 MMAs over k 0..63) as two
+// independent chains of two MMAs (k 0..31 and 32..63) summed at the end.
 template <int FMT>
 __device__ __forceinline__ void block_mma(const QuadRegs<FMT> &q, int bq, const uint32_t (&Bb)[8], float (&c)[4]) {
-    float p[4][4];
+    float p[2][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         uint32_t a0, a1, a2, a3;
@@ -384,10 +388,13 @@ __device__ __forceinline__ void block_mma(const QuadRegs<FMT> &q, int bq, const 
             a2 = q3_reg(q.W, u1, 0);
             a3 = q3_reg(q.W, u1, 1);
         }
-        mma16816_zc(p[i], a0, a1, a2, a3, Bb[2 * i], Bb[2 * i + 1]);
+        if (i < 2)
+            mma16816_zc(p[i], a0, a1, a2, a3, Bb[2 * i], Bb[2 * i + 1]);
+        else
+            mma16816(p[i - 2], a0, a1, a2, a3, Bb[2 * i], Bb[2 * i + 1]);
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) c[j] = (p[0][j] + p[1][j]) + (p[2][j] + p[3][j]);
+    for (int j = 0; j < 4; ++j) c[j] = p[0][j] + p[1][j];
 }
 
 template <int FMT>
@@ -482,7 +489,7 @@ struct LayerPtrs {
     const int32_t *slot_of;
     const uint16_t *x;
     const float *Wr, *bias;
-    float *y, *logits;
+    float *y, *logits;  // logits: this layer's copies in the workspace
     int shared_slot;
 };
 __device__ __forceinline__ LayerPtrs layer_ptrs(const DecodeParams &p, int l) {
@@ -492,7 +499,7 @@ __device__ __forceinline__ LayerPtrs layer_ptrs(const DecodeParams &p, int l) {
     q.Wr = p.Wr + size_t(l) * p.E * p.d;
     q.bias = p.bias ? p.bias + size_t(l) * p.E : nullptr;
     q.y = p.y + size_t(l) * p.T * p.d;
-    q.logits = p.logits + (p.logits_out ? 0 : size_t(l & 1) * p.T * p.E);
+    q.logits = p.logits + size_t(l & 1) * kLogitCopies * p.T * p.E;
     q.shared_slot = p.shared_slot ? __ldg(p.shared_slot + l) : p.shared_slot0;
     return q;
 }
@@ -764,18 +771,26 @@ __device__ void routing_tables(const DecodeParams &p, Smem &s, int T, int k) {
         __syncthreads();
         return;
     }
+    if (tid < npairs) s.pair_e[tid] = s.idx[tid / k][tid % k];  // flat ids (pair p = t*k + j)
+    __syncthreads();
+    int my_e = 0, my_rank = 0;
     if (tid < npairs) {  // stable sort of the pairs by (expert, pair index)
-        const int pp = tid;
-        const int e = s.idx[pp / k][pp % k];
-        int rank = 0;
-        for (int q = 0; q < npairs; ++q) {
-            const int eq = s.idx[q / k][q % k];
-            rank += (eq < e) || (eq == e && q < pp);
+        my_e = s.pair_e[tid];
+#pragma unroll 8
+        for (int q = 0; q < kMaxPairs; ++q) {
+            if (q < npairs) {
+                const int eq = s.pair_e[q];
+                my_rank += (eq < my_e) || (eq == my_e && q < tid);
+            }
         }
-        s.pair_e[rank] = e;
-        s.s_tok[rank] = pp / k;
-        s.s_j[rank] = pp % k;
-        s.inv[pp] = rank;
+    }
+    __syncthreads();
+    if (tid < npairs) {
+        const int t = tid / k;
+        s.pair_e[my_rank] = my_e;
+        s.s_tok[my_rank] = t;
+        s.s_j[my_rank] = tid - t * k;
+        s.inv[tid] = my_rank;
     }
     __syncthreads();
     const bool in = tid < npairs;
@@ -983,8 +998,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
             TRACE(13);
             for (int r = warp; got && r < nrows; r += kWarps)
                 router_row<NT>(rrows + size_t(r) * d, sx, T, d, lane, lp.bias != nullptr,
-                               r < 8 ? s.rbias[r] : (lp.bias ? __ldg(lp.bias + rb + r) : 0.f), rb + r, lp.logits, E,
-                               p.status);
+                               r < 8 ? s.rbias[r] : (lp.bias ? __ldg(lp.bias + rb + r) : 0.f), rb + r, lp.logits,
+                               p.logits_out, E, p.status);
         }
         ok = __syncthreads_and(ok) != 0;  // logits written; router rows and x consumed (the ring is free)
         if (tid == 0) arrive_release(p.ctr);
@@ -1022,6 +1037,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
             const uint64_t c1 = (eb * uint64_t(cta + 1) / uint64_t(G)) & ~uint64_t(15);
             if (c1 > c0) prefetch_l2(p.pool + int64_t(np.shared_slot) * p.slot_bytes + c0, uint32_t(c1 - c0));
             if (cta == 0) prefetch_l2(np.slot_of, uint32_t(E) * 4u);
+            if (cta == 1) prefetch_l2(np.x, uint32_t(T) * uint32_t(d) * 2u);
         }
         // ------------------------------------------------ grid barrier: all logits written
         if (tid == 0) s.ok = wait_geq(p.ctr, bar_target, p.status);
@@ -1029,7 +1045,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
         ok = ok && s.ok;
         TRACE(2);
         if (ok) {
-            topk_cta<NT>(p, s, lp.logits, T, E, k);
+            topk_cta<NT>(p, s, lp.logits + size_t(cta % kLogitCopies) * T * E, T, E, k);
             TRACE(3);
             routing_tables(p, s, T, k);
         }
@@ -1558,7 +1574,7 @@ using namespace moe;
 
 MOE_API size_t moe_layer_decode_workspace_bytes(int T, int k, int f, int E) {
     if (T <= 0 || k <= 0 || f <= 0 || E <= 0) return 0;
-    return 256 + ws_align(2 * size_t(T) * E * sizeof(float));
+    return 256 + ws_align(2 * size_t(kLogitCopies) * T * E * sizeof(float));
 }
 
 MOE_API size_t moe_stack_decode_workspace_bytes(int T, int k, int f, int E) {
@@ -1580,10 +1596,7 @@ MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, 
     p.shared_slot0 = shared_slot;
     p.layer0 = layer;
     p.bias = bias;
-    if (logits) {
-        p.logits = logits;
-        p.logits_out = true;
-    }
+    p.logits_out = logits;
     p.topk_idx = topk_idx;
     p.topk_w = topk_w;
     p.counts = counts;

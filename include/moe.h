@@ -322,7 +322,8 @@ moe_status moe_debug_wait_probe(const uint32_t *counter, uint32_t target, uint64
                                 int32_t *dev_status, moe_stream_t stream);
 
 /* Workspace bytes moe_layer_decode and moe_stack_decode need for (T, k, f, E):
- * two grid counters and two fp32 [T][E] logit buffers. */
+ * two grid counters and 2 x 8 fp32 [T][E] logit buffers (the logits are
+ * written in 8 copies, which the launch's CTAs read in turn). */
 size_t moe_layer_decode_workspace_bytes(int T, int k, int f, int E);
 size_t moe_stack_decode_workspace_bytes(int T, int k, int f, int E);
 
