@@ -279,16 +279,6 @@ __device__ __forceinline__ uint32_t peer_addr(const void *p, unsigned rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr(p)), "r"(rank));
     return r;
 }
-__device__ __forceinline__ float ld_peer(uint32_t a) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-    return v;
-}
-__device__ __forceinline__ int ld_peer_int(uint32_t a) {
-    int v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-    return v;
-}
 // 16 bytes into a peer CTA's shared memory, counted on the peer's mbarrier.
 __device__ __forceinline__ void st_async4(uint32_t raddr, float4 v, uint32_t rbar) {
     asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1,%2,%3,%4}, [%5];" ::"r"(raddr),
@@ -414,7 +404,7 @@ template <int FMT>
 __device__ __forceinline__ void quad_pair_compute(const QuadRegs<FMT> &qg, const QuadRegs<FMT> &qu,
                                                   const uint32_t (&B)[4][8], const float (&xs)[4][2],
                                                   float (&ag)[4], float (&au)[4]) {
-#pragma unroll
+#pragma unroll 2
     for (int bq = 0; bq < 4; ++bq) {
         float cg[4], cu[4];
         block_mma<FMT>(qg, bq, B[bq], cg);
@@ -540,8 +530,8 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
 // completing on that row group's barrier). Copy c is issued by lane c / 8 of
 // warp c % 8, so the copies of a task leave from all warps at once.
 template <int FMT>
-__device__ __forceinline__ void issue_gu(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int tid,
-                                         unsigned rank, int slot, int hb) {
+__device__ __noinline__ void issue_gu(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int tid, unsigned rank,
+                                      int slot, int hb) {
     const Geo &g = p.g;
     const int c = (tid & 31) * kWarps + (tid >> 5);
     if (c >= 4 * g.GR) return;
@@ -559,8 +549,8 @@ __device__ __forceinline__ void issue_gu(const DecodeParams &p, Smem &s, uint8_t
 // The down slice of task (slot, hb) into buffer b, by thread 0: this CTA's DR
 // rows over the task's HB columns (block pair hb for Q2, block quad hb for
 // Q3), codes then scales, as two tensor copies.
-__device__ __forceinline__ void issue_dn(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int tid,
-                                         unsigned rank, int slot, int hb) {
+__device__ __noinline__ void issue_dn(const DecodeParams &p, Smem &s, uint8_t *ring, int b, int tid, unsigned rank,
+                                      int slot, int hb) {
     const Geo &g = p.g;
     if (tid != 0) return;
     uint8_t *dst = ring + size_t(b) * g.region + g.gu_bytes;
@@ -592,6 +582,30 @@ __device__ __forceinline__ uint64_t warp_topk(uint64_t (&c)[M], int k, int lane)
     return mine;
 }
 
+// Near-equal logits (more than 64 keys reach the threshold): every warp finds
+// its exact top k by rounds and each token's lists are merged by counting.
+template <int NT, int M>
+__device__ __noinline__ void topk_exact(Smem &s, const uint64_t (&orig)[M], bool many, int k) {
+    constexpr int WPT = kWarps / NT;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int tt = warp / WPT;
+    if (many) {
+        uint64_t c[M];
+#pragma unroll
+        for (int m = 0; m < M; ++m) c[m] = orig[m];
+        const uint64_t mine = warp_topk<M>(c, k, lane);
+        if (lane < k) s.wl[warp][lane] = mine;
+    }
+    __syncthreads();
+    if (many && lane < k) {
+        const uint64_t me = s.wl[warp][lane];
+        int rank = 0;
+        for (int o = 0; o < WPT; ++o)
+            for (int q = 0; q < k; ++q) rank += s.wl[tt * WPT + o][q] > me;
+        if (rank < k) s.sel[tt][rank] = me;
+    }
+}
+
 // Top-k of every token from the logits in global memory (written by all CTAs
 // of this launch). A candidate is the 64-bit key (logit key << 32 | ~id), so
 // the top k are the k largest keys (larger logit first, then lower id).
@@ -604,7 +618,7 @@ __device__ __forceinline__ uint64_t warp_topk(uint64_t (&c)[M], int k, int lane)
 // WPT = 1 the warp's k rounds give the answer. Then softmax over the selected
 // logits in ascending-id order (the arithmetic of moe_route).
 template <int NT>
-__device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, int T, int E, int k) {
+__device__ __noinline__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, int T, int E, int k) {
     constexpr int WPT = kWarps / NT;       // warps per token
     constexpr int M = kMaxEDec / 32 / WPT;  // keys per lane
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -668,29 +682,12 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
             for (int i = sub * 32 + lane; i < n; i += WPT * 32) {
                 const uint64_t me = s.cand[tt][i];
                 int rank = 0;
-#pragma unroll 16
+#pragma unroll 4
                 for (int q = 0; q < 64; ++q) rank += (q < n && s.cand[tt][q] > me);
                 if (rank < k) s.sel[tt][rank] = me;
             }
         }
-        if (__syncthreads_or(many)) {  // near-equal logits: exact lists per warp, merged by counting
-            if (many) {
-#pragma unroll
-                for (int m = 0; m < M; ++m) c[m] = orig[m];
-                const uint64_t mine = warp_topk<M>(c, k, lane);
-                if (lane < k) s.wl[warp][lane] = mine;
-            }
-            __syncthreads();
-            if (many && lane < k) {
-                const uint64_t me = s.wl[warp][lane];
-                int rank = 0;
-#pragma unroll
-                for (int o = 0; o < WPT; ++o)
-#pragma unroll 16
-                    for (int q = 0; q < kMaxK; ++q) rank += (q < k && s.wl[tt * WPT + o][q] > me);
-                if (rank < k) s.sel[tt][rank] = me;
-            }
-        }
+        if (__syncthreads_or(many)) topk_exact<NT, M>(s, orig, many, k);
     }
     __syncthreads();
     TRACE(17);
@@ -707,7 +704,7 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
         const float my_v = key ? key_value(key) : -INFINITY;
         const uint64_t top = s.sel[warp][0];
         const float mx = uint32_t(top >> 32) ? key_value(uint32_t(top >> 32)) : -INFINITY;
-#pragma unroll 16
+#pragma unroll 4
         for (int q = 0; q < kMaxK; ++q) {
             if (q < k) {
                 const uint64_t o = s.sel[warp][q];
@@ -734,7 +731,7 @@ __device__ void topk_cta(const DecodeParams &p, Smem &s, const float *logits, in
 
 // Routing tables from s.idx: sorted pairs, active experts with their slots,
 // resident list, miss bases, and the task count. Whole CTA.
-__device__ void routing_tables(const DecodeParams &p, Smem &s, int T, int k) {
+__device__ __noinline__ void routing_tables(const DecodeParams &p, Smem &s, int T, int k) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int npairs = T * k;
     if (T == 1) {  // one token: its k experts (ascending id) are the active experts, one pair each
@@ -776,7 +773,7 @@ __device__ void routing_tables(const DecodeParams &p, Smem &s, int T, int k) {
     int my_e = 0, my_rank = 0;
     if (tid < npairs) {  // stable sort of the pairs by (expert, pair index)
         my_e = s.pair_e[tid];
-#pragma unroll 8
+#pragma unroll 4
         for (int q = 0; q < kMaxPairs; ++q) {
             if (q < npairs) {
                 const int eq = s.pair_e[q];
@@ -847,7 +844,7 @@ __device__ void routing_tables(const DecodeParams &p, Smem &s, int T, int k) {
 }
 
 // Routing, permutation, slots and misses of layer l to global memory (one CTA).
-__device__ void publish(const DecodeParams &p, Smem &s, int l, int T, int k, int E) {
+__device__ __noinline__ void publish(const DecodeParams &p, Smem &s, int l, int T, int k, int E) {
     const int tid = threadIdx.x;
     const int npairs = T * k;
     const size_t po = size_t(l) * npairs;
