@@ -248,34 +248,66 @@ def run_reference(args, wl, rank):
 
 
 # ------------------------------------------------------------------ host completion of misses
-MISS_DTYPE = [("layer", "<i4"), ("expert", "<i4"), ("token", "<i4"), ("j", "<i4"), ("gate", "<f4")]
+def _host_miss_leg(stack, wl, x_dev, x_host, reps=3):
+    """The stacked layers' misses completed on the host (moe_miss_engine, every
+    host thread) for one step's tokens: GPU alone, host alone after the GPU
+    (serial), and both overlapped -- the launch writes each layer's miss list
+    to mapped pinned memory as the layer ends and the engine starts on it while
+    the GPU runs the later layers. Host wall-clock times (the host is the one
+    waiting), median of `reps`; the missed experts are generated into host
+    storage first (not timed)."""
+    import torch
 
-
-def _time_host_misses(stack, wl, sb, x_step):
-    """moe_complete_misses_host over one step's miss lists (all layers), the
-    missed experts in canonical host storage (generated first, not timed), the
-    completion of every layer timed on the host clock with all threads."""
     from bit_expert_ffn_fp32_b200 import native
+    from bit_expert_ffn_fp32_b200.layer import MISS_DTYPE
 
     L, T = wl.layers, wl.T
-    work, n_rec, n_exp = [], 0, 0
-    for l in range(L):
-        recs = np.array(stack.stack_misses(sb, l), dtype=MISS_DTYPE)
-        if len(recs) == 0:
-            continue
-        y = np.ascontiguousarray(sb.y[l, :T].cpu().numpy())
-        canon = {e: stack.canonical_expert(l, e) for e in sorted(set(recs["expert"].tolist()))}
-        work.append((l, recs, y, canon, native.expert_table(wl.E, canon), np.ascontiguousarray(x_step[l])))
-        n_rec += len(recs)
-        n_exp += len(canon)
+    sb = stack.stack_buffers(T)
+    stack.forward_stack(x_dev, sb)
+    torch.cuda.synchronize()
+    missed = [sorted(set(m[1] for m in stack.stack_misses(sb, l))) for l in range(L)]
+    tabs = [native.expert_table(wl.E, {e: stack.canonical_expert(l, e) for e in missed[l]}) for l in range(L)]
+    hb = stack.stack_buffers(T, host_misses=True)
+    cap = hb.idx.shape[1]
+    cnt = hb.miss_count.view(np.int32)
+    miss_h = hb.miss.view(MISS_DTYPE, (L, cap))
+    xs = [np.ascontiguousarray(x_host[l]) for l in range(L)]
+    y_add = np.zeros((L, T, wl.d), np.float32)
     threads = len(os.sched_getaffinity(0))
-    t0 = time.perf_counter()
-    for l, recs, y, _canon, tab, xl in work:
-        native.complete_misses_host(wl.fmt, wl.d, wl.f, tab, wl.E, recs, len(recs), l, xl, T, y, 0)
-    dt = time.perf_counter() - t0
-    return {"ms_per_step": dt * 1e3, "misses_per_step": n_rec, "distinct_experts_per_step": n_exp,
-            "threads": threads, "call": "moe_complete_misses_host (host C++, fp32 lookup-table dot products), "
-            "one call per layer", "sample": "the misses of the last end-to-end step"}
+    eng = native.MissEngine(0)
+    gpu, host, both = [], [], []
+    try:
+        for _ in range(reps):
+            cnt[:] = -1
+            t0 = time.perf_counter()
+            stack.forward_stack(x_dev, hb)
+            torch.cuda.synchronize()
+            gpu.append(time.perf_counter() - t0)
+            y_add[:] = 0
+            t0 = time.perf_counter()
+            for l in range(L):
+                eng.submit(wl.fmt, wl.d, wl.f, tabs[l], wl.E, miss_h[l], cnt[l:l + 1], cap, l, xs[l], T, y_add[l])
+            eng.wait()
+            host.append(time.perf_counter() - t0)
+            cnt[:] = -1
+            y_add[:] = 0
+            t0 = time.perf_counter()
+            stack.forward_stack(x_dev, hb)
+            for l in range(L):
+                eng.submit(wl.fmt, wl.d, wl.f, tabs[l], wl.E, miss_h[l], cnt[l:l + 1], cap, l, xs[l], T, y_add[l])
+            eng.wait()
+            torch.cuda.synchronize()
+            both.append(time.perf_counter() - t0)
+    finally:
+        eng.close()
+    n_rec = int(sum(int(c) for c in cnt))
+    g, h, o = (1e3 * float(np.median(v)) for v in (gpu, host, both))
+    return {"gpu_ms": g, "host_ms": h, "serial_ms": g + h, "overlapped_ms": o,
+            "tokens_per_s_overlapped": T / (o / 1e3), "misses_per_step": n_rec,
+            "distinct_experts_per_step": int(sum(len(m) for m in missed)), "threads": threads,
+            "call": "moe_stack_decode writing miss lists to mapped host memory + moe_miss_engine (host C++ workers, "
+                    "fp32 dot products on the canonical codes)",
+            "timing": f"host wall clock, median of {reps}; serial = GPU alone + host alone"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -490,7 +522,8 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
         "clocks": clocks, "gpu_launches": launches_per_step * steps, "dev_status": status,
     }
     if stacked and not args.no_host_misses and rank == 0:
-        line["host_miss_completion"] = _time_host_misses(stack, wl, sb, xs_host[(steps - 1) % n_x])
+        i_last = (warmup + steps - 1) % n_x
+        line["host_miss_completion"] = _host_miss_leg(stack, wl, xs(warmup + steps - 1), xs_host[i_last])
     return line
 
 

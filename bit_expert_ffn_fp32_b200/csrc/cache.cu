@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(kThreads)
     cache_lookup_kernel(const int32_t *slot_of, int num_slots, int layer, const int32_t *topk_idx,
                         const float *topk_w, const int32_t *offsets, const int32_t *sorted_tok,
                         const int32_t *sorted_j, int T, int k, int E, int32_t *slot_of_pair, moe_miss *miss,
-                        int32_t *miss_count, int miss_cap, int32_t *status) {
+                        int32_t *miss_count, int miss_cap, int32_t *expert_counts, int32_t *status) {
     __shared__ int s_mbase[kMaxE];
     __shared__ int s_warp[32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(kThreads)
             slot_of_pair[p] = -1;
             continue;
         }
+        if (expert_counts) atomicAdd(expert_counts + e, 1);
         const int sl = slot_of[e];
         const bool resident = sl >= 0 && sl < num_slots;
         slot_of_pair[p] = resident ? sl : -1;
@@ -109,8 +110,8 @@ using namespace moe;
 MOE_API moe_status moe_cache_lookup(const int32_t *slot_of, int32_t num_slots, int32_t layer, const int32_t *topk_idx,
                                     const float *topk_w, const int32_t *offsets, const int32_t *sorted_tok,
                                     const int32_t *sorted_j, int T, int k, int E, int32_t *slot_of_pair,
-                                    moe_miss *miss, int32_t *miss_count, int32_t miss_cap, int32_t *dev_status,
-                                    moe_stream_t stream) {
+                                    moe_miss *miss, int32_t *miss_count, int32_t miss_cap, int32_t *expert_counts,
+                                    int32_t *dev_status, moe_stream_t stream) {
     if (T < 0 || k <= 0 || E <= 0 || num_slots < 0 || miss_cap < 0) return MOE_ERR_INVALID_ARG;
     if (E > kMaxE || k > kMaxK) return MOE_ERR_UNSUPPORTED;
     if (int64_t(T) * k >= (int64_t(1) << 31)) return MOE_ERR_OVERFLOW;
@@ -120,6 +121,6 @@ MOE_API moe_status moe_cache_lookup(const int32_t *slot_of, int32_t num_slots, i
     const int grid = int(std::min<int64_t>((int64_t(T) * k + kThreads - 1) / kThreads, 148));
     cache_lookup_kernel<<<std::max(grid, 1), kThreads, 0, as_cuda(stream)>>>(slot_of, num_slots, layer, topk_idx, topk_w, offsets,
                                                              sorted_tok, sorted_j, T, k, E, slot_of_pair, miss,
-                                                             miss_count, miss_cap, dev_status);
+                                                             miss_count, miss_cap, expert_counts, dev_status);
     return launch_status();
 }

@@ -88,6 +88,23 @@ MOE_API moe_status moe_cache_policy_observe(void *state, int layer, const int32_
     return MOE_OK;
 }
 
+MOE_API moe_status moe_cache_policy_observe_counts(void *state, const int32_t *counts_host, int tokens) {
+    if (!state || header(state)->magic != kPolicyMagic) return MOE_ERR_INVALID_ARG;
+    PolicyHeader *h = header(state);
+    const int64_t LE = int64_t(h->L) * h->E;
+    if (tokens < 0 || !counts_host) return MOE_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < LE; ++i)
+        if (counts_host[i] < 0) return MOE_ERR_INVALID_ARG;
+    uint32_t *c = counts(state);
+    h->clock += tokens;  // the token clock first, as for one call per layer of a token step
+    while (h->clock >= h->epoch) {
+        h->clock -= h->epoch;
+        for (int64_t i = 0; i < LE; ++i) c[i] >>= 1;
+    }
+    for (int64_t i = 0; i < LE; ++i) c[i] = uint32_t(std::min<uint64_t>(uint64_t(c[i]) + uint32_t(counts_host[i]), 0xffffffffull));
+    return MOE_OK;
+}
+
 MOE_API int32_t moe_cache_policy_plan(void *state, int32_t *slot_of, moe_swap *swaps, int32_t max_swaps) {
     if (!state || header(state)->magic != kPolicyMagic || !slot_of || max_swaps < 0 || (max_swaps > 0 && !swaps))
         return -int32_t(MOE_ERR_INVALID_ARG);

@@ -142,6 +142,7 @@ struct DecodeParams {
     moe_miss *miss;              // [L][miss_cap] or NULL
     int32_t *miss_count;         // [L] or NULL
     int miss_cap;
+    int32_t *expert_counts;      // [L][E] routed pairs per expert, added to (or NULL)
     float *y;                    // [L][T][d]
     int32_t *status;
     unsigned *ctr;               // [0] barrier arrivals, [1] CTAs finished
@@ -871,6 +872,8 @@ __device__ __noinline__ void publish(const DecodeParams &p, Smem &s, int l, int 
         for (int a = tid; a < s.nact; a += kThreads) p.active[1 + a] = s.act_e[a];
         if (tid == 0) p.active[0] = s.nact;
     }
+    if (p.expert_counts)
+        for (int i = tid; i < npairs; i += kThreads) atomicAdd(p.expert_counts + size_t(l) * E + s.idx[i / k][i % k], 1);
     moe_miss *miss = p.miss ? p.miss + size_t(l) * p.miss_cap : nullptr;
     for (int sp = tid; sp < npairs; sp += kThreads) {
         int a = 0;
@@ -891,8 +894,12 @@ __device__ __noinline__ void publish(const DecodeParams &p, Smem &s, int l, int 
             }
         }
     }
+    // the count last, after every record is visible system-wide: a host reader of
+    // mapped memory that sees the count sees the records
+    __syncthreads();
     if (tid == 0) {
-        if (p.miss_count) p.miss_count[l] = s.nmiss;
+        __threadfence_system();
+        if (p.miss_count) *reinterpret_cast<volatile int32_t *>(p.miss_count + l) = s.nmiss;
         if (s.nmiss > p.miss_cap && p.miss) flag(p.status, MOE_DEV_MISS_OVERFLOW);
     }
 }
@@ -1583,8 +1590,8 @@ MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, 
                                     int k, float *logits, int32_t *topk_idx, float *topk_w, int32_t *counts,
                                     int32_t *offsets, int32_t *sorted_tok, int32_t *sorted_j, int32_t *inv,
                                     int32_t *active, int32_t *slot_of_pair, moe_miss *miss, int32_t *miss_count,
-                                    int32_t miss_cap, float *y, void *ws, size_t ws_bytes, int32_t *dev_status,
-                                    moe_stream_t stream) {
+                                    int32_t miss_cap, int32_t *expert_counts, float *y, void *ws, size_t ws_bytes,
+                                    int32_t *dev_status, moe_stream_t stream) {
     DecodeParams p;
     const moe_status st = setup(p, W, 1, slot_of, x, Wr, T, d, f, E, k, miss_cap, miss, y, ws, ws_bytes);
     if (st != MOE_OK || T == 0) return st;
@@ -1604,6 +1611,7 @@ MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, 
     p.active = active;
     p.slot_of_pair = slot_of_pair;
     p.miss_count = miss_count;
+    p.expert_counts = expert_counts;
     p.status = dev_status;
     return W->fmt == 2 ? launch_fmt<2>(p, as_cuda(stream)) : launch_fmt<3>(p, as_cuda(stream));
 }
@@ -1612,7 +1620,8 @@ MOE_API moe_status moe_stack_decode(const moe_qpool *W, int L, const int32_t *sl
                                     int32_t layer0, const uint16_t *x, const float *Wr, const float *bias, int T,
                                     int d, int f, int E, int k, int32_t *topk_idx, float *topk_w,
                                     int32_t *slot_of_pair, moe_miss *miss, int32_t *miss_count, int32_t miss_cap,
-                                    float *y, void *ws, size_t ws_bytes, int32_t *dev_status, moe_stream_t stream) {
+                                    int32_t *expert_counts, float *y, void *ws, size_t ws_bytes,
+                                    int32_t *dev_status, moe_stream_t stream) {
     DecodeParams p;
     const moe_status st = setup(p, W, L, slot_of, x, Wr, T, d, f, E, k, miss_cap, miss, y, ws, ws_bytes);
     if (st != MOE_OK || T == 0) return st;
@@ -1624,6 +1633,7 @@ MOE_API moe_status moe_stack_decode(const moe_qpool *W, int L, const int32_t *sl
     p.topk_w = topk_w;
     p.slot_of_pair = slot_of_pair;
     p.miss_count = miss_count;
+    p.expert_counts = expert_counts;
     p.status = dev_status;
     return W->fmt == 2 ? launch_fmt<2>(p, as_cuda(stream)) : launch_fmt<3>(p, as_cuda(stream));
 }

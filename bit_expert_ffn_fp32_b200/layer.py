@@ -79,6 +79,43 @@ class Buffers:
     sh_active: torch.Tensor
 
 
+MISS_DTYPE = np.dtype([("layer", "<i4"), ("expert", "<i4"), ("token", "<i4"), ("j", "<i4"), ("gate", "<f4")])
+
+
+class MappedHostBuffer:
+    """Pinned host memory mapped into the device address space: kernels write it
+    through `data_ptr()` (a device address), the host reads `host` (a numpy
+    view of the same bytes)."""
+
+    def __init__(self, nbytes: int):
+        from cuda.bindings import runtime as rt
+
+        self._rt = rt
+        err, hp = rt.cudaHostAlloc(max(int(nbytes), 16), rt.cudaHostAllocMapped | rt.cudaHostAllocPortable)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaHostAlloc failed: {err}")
+        err, dp = rt.cudaHostGetDevicePointer(hp, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            rt.cudaFreeHost(hp)
+            raise RuntimeError(f"cudaHostGetDevicePointer failed: {err}")
+        self._hp, self._dp, self.nbytes = int(hp), int(dp), int(nbytes)
+        import ctypes as _C
+        self.host = np.ctypeslib.as_array((_C.c_uint8 * self.nbytes).from_address(self._hp))
+
+    def data_ptr(self) -> int:
+        return self._dp
+
+    def view(self, dtype, shape=None) -> np.ndarray:
+        v = self.host.view(dtype)
+        return v if shape is None else v.reshape(shape)
+
+    def __del__(self):
+        try:
+            self._rt.cudaFreeHost(self._hp)
+        except Exception:
+            pass
+
+
 @dataclass
 class StackBuffers:
     T: int
@@ -145,6 +182,10 @@ class MoEStack:
                                   self.device, sync=False)
         torch.cuda.current_stream().synchronize()
         self._bufs: dict[int, Buffers] = {}
+        # routed pairs per (layer, expert), added to by every forward (device
+        # counters the cache policy reads in bulk); zero it to start a window
+        self.count_experts = True
+        self.expert_counts = torch.zeros((self.L, wl.E), dtype=torch.int32, device=self.device)
         self._ws: dict = {}
 
     # expert e == E is the layer's shared expert
@@ -168,6 +209,60 @@ class MoEStack:
             self._pack(l_in, e_in, slot)
         for l in changed:
             self.slot_of[l].copy_(torch.from_numpy(np.ascontiguousarray(self.slot_of_host[l], dtype=np.int32)))
+
+    def _set_rows(self, layers) -> None:
+        for l in sorted(layers):
+            self.slot_of[l].copy_(torch.from_numpy(np.ascontiguousarray(self.slot_of_host[l], dtype=np.int32)),
+                                  non_blocking=True)
+
+    def prepare_swaps(self, swaps) -> list:
+        """Pack every admitted expert of a plan into a pinned host record (host
+        work, no GPU): [(slot, layer_in, expert_in, layer_out, expert_out, record)]."""
+        out = []
+        for slot, l_in, e_in, l_out, e_out in swaps:
+            if not 0 <= slot < self.L * self.R:
+                raise ValueError("slot %d outside the routed slots" % slot)
+            ex = self.canonical_expert(l_in, e_in)
+            rec = torch.empty(self.slot_bytes, dtype=torch.uint8).pin_memory()
+            mats = [native.qmatrix(ex[m]["codes"], ex[m]["scale"], ex[m]["min"], ex[m]["hi"]) for m in
+                    ("gate", "up", "down")]
+            native.pack_expert_host(self.wl.fmt, self.wl.d, self.wl.f, *mats, rec.data_ptr())
+            out.append((slot, l_in, e_in, l_out, e_out, rec))
+        return out
+
+    def begin_swaps(self, prepared: list, side_stream) -> dict:
+        """Start a plan without stopping the layers: on the current stream the
+        outgoing experts leave the slot tables (later layers count them as
+        misses); once every layer queued before that point is done, the side
+        stream copies the new records into their slots while the current stream
+        goes on. commit_swaps() then makes the incoming experts resident."""
+        main = torch.cuda.current_stream()
+        changed = set()
+        for slot, l_in, e_in, l_out, e_out, _ in prepared:
+            if l_out >= 0:
+                self.slot_of_host[l_out][e_out] = -1
+                changed.add(l_out)
+        self._set_rows(changed)
+        unmapped = torch.cuda.Event()
+        unmapped.record(main)
+        side_stream.wait_event(unmapped)
+        with torch.cuda.stream(side_stream):
+            for slot, _, _, _, _, rec in prepared:
+                dst = self.pool[slot * self.slot_bytes: slot * self.slot_bytes + rec.numel()]
+                dst.copy_(rec, non_blocking=True)
+        copied = torch.cuda.Event()
+        copied.record(side_stream)
+        return {"prepared": prepared, "copied": copied}
+
+    def commit_swaps(self, handle: dict) -> None:
+        """The current stream waits for the record copies, then the incoming
+        experts take their slots in the slot tables."""
+        torch.cuda.current_stream().wait_event(handle["copied"])
+        changed = set()
+        for slot, l_in, e_in, _, _, _ in handle["prepared"]:
+            self.slot_of_host[l_in][e_in] = slot
+            changed.add(l_in)
+        self._set_rows(changed)
 
     def _pack(self, layer: int, e: int, slot: int) -> None:
         upload_expert(self.canonical_expert(layer, e), self.wl.fmt, self.wl.d, self.wl.f,
@@ -221,7 +316,8 @@ class MoEStack:
         native.permute(b.idx, T, k, E, b.counts, b.offsets, b.sorted_tok, b.sorted_j, b.inv, b.active, b.perm_ws,
                        0 if b.perm_ws is None else b.perm_ws.numel(), b.status, stream)
         native.cache_lookup(self.slot_of[layer], self.num_slots, layer, b.idx, b.w, b.offsets, b.sorted_tok,
-                            b.sorted_j, T, k, E, b.sop, b.miss, b.miss_count, b.idx.numel(), b.status, stream)
+                            b.sorted_j, T, k, E, b.sop, b.miss, b.miss_count, b.idx.numel(), b.status, stream,
+                            expert_counts=self.expert_counts[layer] if self.count_experts else None)
         if combine == "atomic":
             native.expert_ffn(self.qpool, self.shared_slot[layer], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
                               b.sh_sorted_j, b.sh_active, None, b.y, b.h_sh, b.h_sh.numel(), b.status, stream)
@@ -261,21 +357,31 @@ class MoEStack:
                             active=b.active if o else None, slot_of_pair=b.sop if o else None,
                             miss=b.miss if o else None, miss_count=b.miss_count if o else None,
                             miss_cap=b.idx.numel() if o else 0, y=b.y, ws=ws, ws_bytes=ws.numel(),
-                            dev_status=b.status, stream=stream)
+                            dev_status=b.status, stream=stream,
+                            expert_counts=self.expert_counts[layer] if self.count_experts else None)
         return b
 
-    def stack_buffers(self, T: int) -> "StackBuffers":
-        """Outputs of moe_stack_decode for T tokens through all L layers (kept per T)."""
-        key = ("stack", T)
+    def stack_buffers(self, T: int, host_misses: bool = False) -> "StackBuffers":
+        """Outputs of moe_stack_decode for T tokens through all L layers (kept per
+        T). With host_misses the miss records and counts live in mapped pinned
+        host memory (the kernel writes them there layer by layer; see
+        MissEngine), else on the device."""
+        key = ("stack", T, host_misses)
         if key not in self._ws:
             wl, dev, L = self.wl, self.device, self.L
             n = max(T * wl.k, 1)
             i32 = dict(dtype=torch.int32, device=dev)
+            if host_misses:
+                miss = MappedHostBuffer(L * n * native.MISS_BYTES)
+                count = MappedHostBuffer(L * 4)
+                count.view(np.int32)[:] = -1
+            else:
+                miss = torch.empty(L, n * native.MISS_BYTES, dtype=torch.uint8, device=dev)
+                count = torch.zeros(L, **i32)
             self._ws[key] = StackBuffers(
                 T=T, idx=torch.empty(L, n, **i32), w=torch.empty(L, n, dtype=torch.float32, device=dev),
-                sop=torch.empty(L, n, **i32), miss=torch.empty(L, n * native.MISS_BYTES, dtype=torch.uint8, device=dev),
-                miss_count=torch.zeros(L, **i32), y=torch.empty(L, max(T, 1), wl.d, dtype=torch.float32, device=dev),
-                status=torch.zeros(1, **i32))
+                sop=torch.empty(L, n, **i32), miss=miss, miss_count=count,
+                y=torch.empty(L, max(T, 1), wl.d, dtype=torch.float32, device=dev), status=torch.zeros(1, **i32))
         return self._ws[key]
 
     def forward_stack(self, x: torch.Tensor, b: "StackBuffers | None" = None, stream=None) -> "StackBuffers":
@@ -289,15 +395,21 @@ class MoEStack:
         native.stack_decode(self.qpool, self.L, self.slot_of_all, self.shared_slot_all, 0, x, self.Wr_all,
                             self.bias_all, T, wl.d, wl.f, wl.E, wl.k, topk_idx=b.idx, topk_w=b.w, slot_of_pair=b.sop,
                             miss=b.miss, miss_count=b.miss_count, miss_cap=n, y=b.y, ws=ws, ws_bytes=ws.numel(),
-                            dev_status=b.status, stream=stream)
+                            dev_status=b.status, stream=stream,
+                            expert_counts=self.expert_counts if self.count_experts else None)
         return b
 
     def stack_misses(self, b: "StackBuffers", layer: int) -> list:
         """Miss records of one layer of the last forward_stack (host copy; synchronises)."""
-        n = min(int(b.miss_count[layer].item()), b.idx.shape[1])
-        raw = b.miss[layer, : n * native.MISS_BYTES].cpu().numpy().tobytes()
-        rec = np.frombuffer(raw, dtype=np.dtype([("layer", "<i4"), ("expert", "<i4"), ("token", "<i4"),
-                                                 ("j", "<i4"), ("gate", "<f4")]))
+        cap = b.idx.shape[1]
+        if isinstance(b.miss, MappedHostBuffer):
+            torch.cuda.synchronize()
+            n = min(int(b.miss_count.view(np.int32)[layer]), cap)
+            rec = b.miss.view(MISS_DTYPE, (self.L, cap))[layer, :n].copy()
+        else:
+            n = min(int(b.miss_count[layer].item()), cap)
+            raw = b.miss[layer, : n * native.MISS_BYTES].cpu().numpy().tobytes()
+            rec = np.frombuffer(raw, dtype=MISS_DTYPE)
         return [(int(r["layer"]), int(r["expert"]), int(r["token"]), int(r["j"]), float(r["gate"])) for r in rec]
 
     def misses(self, b: Buffers) -> list:

@@ -57,7 +57,7 @@ SIGNATURES = {
     "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_permute_workspace_bytes": (_SZ, [_I, _I, _I]),
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
-    "moe_cache_lookup": (_I, [_P, _I32, _I32, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I32, _P, _P]),
+    "moe_cache_lookup": (_I, [_P, _I32, _I32, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I32, _P, _P, _P]),
     "moe_expert_ffn_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "moe_expert_ffn_q2": (_I, [C.POINTER(QPool), _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P,
                                _P]),
@@ -68,15 +68,20 @@ SIGNATURES = {
     "moe_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "moe_layer_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "moe_layer_decode": (_I, [C.POINTER(QPool), _P, _I32, _I32, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
-                              _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _SZ, _P, _P]),
+                              _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _SZ, _P, _P]),
     "moe_stack_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "moe_stack_decode": (_I, [C.POINTER(QPool), _I, _P, _P, _I32, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P,
-                              _P, _I32, _P, _P, _SZ, _P, _P]),
+                              _P, _I32, _P, _P, _P, _SZ, _P, _P]),
     "moe_complete_misses_host": (_I, [_I, _I, _I, _P, _I, _P, _I32, _I32, _P, _I, _P, _I]),
     "moe_debug_wait_probe": (_I, [_P, C.c_uint32, _P, _P, _P]),
+    "moe_miss_engine_create": (_I, [_I, C.POINTER(_P)]),
+    "moe_miss_engine_submit": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _I32, _I32, _P, _I, _P]),
+    "moe_miss_engine_wait": (_I, [_P]),
+    "moe_miss_engine_destroy": (None, [_P]),
     "moe_cache_policy_bytes": (_SZ, [_I, _I]),
     "moe_cache_policy_init": (_I, [_P, _SZ, _I, _I, _I, _I, _I]),
     "moe_cache_policy_observe": (_I, [_P, _I, _P, _I, _I]),
+    "moe_cache_policy_observe_counts": (_I, [_P, _P, _I]),
     "moe_cache_policy_plan": (_I32, [_P, _P, _P, _I32]),
 }
 
@@ -166,11 +171,11 @@ def permute(topk_idx, T, k, E, counts, offsets, sorted_tok, sorted_j, inv, activ
 
 
 def cache_lookup(slot_of, num_slots, layer, topk_idx, topk_w, offsets, sorted_tok, sorted_j, T, k, E,
-                 slot_of_pair, miss, miss_count, miss_cap, dev_status=None, stream=None) -> None:
+                 slot_of_pair, miss, miss_count, miss_cap, dev_status=None, stream=None, expert_counts=None) -> None:
     check("moe_cache_lookup", lib.moe_cache_lookup(ptr(slot_of), num_slots, layer, ptr(topk_idx), ptr(topk_w),
                                                    ptr(offsets), ptr(sorted_tok), ptr(sorted_j), T, k, E,
                                                    ptr(slot_of_pair), ptr(miss), ptr(miss_count), miss_cap,
-                                                   ptr(dev_status), stream_handle(stream)))
+                                                   ptr(expert_counts), ptr(dev_status), stream_handle(stream)))
 
 
 def expert_ffn_workspace_bytes(T, k, d, f) -> int:
@@ -207,23 +212,23 @@ def layer_decode_workspace_bytes(T, k, f, E) -> int:
 def layer_decode(pool: QPool, slot_of, shared_slot: int, layer: int, x, Wr, bias, T, d, f, E, k, logits=None,
                  topk_idx=None, topk_w=None, counts=None, offsets=None, sorted_tok=None, sorted_j=None, inv=None,
                  active=None, slot_of_pair=None, miss=None, miss_count=None, miss_cap=0, y=None, ws=None,
-                 ws_bytes=0, dev_status=None, stream=None) -> None:
+                 ws_bytes=0, dev_status=None, stream=None, expert_counts=None) -> None:
     check("moe_layer_decode",
           lib.moe_layer_decode(C.byref(pool), ptr(slot_of), shared_slot, layer, ptr(x), ptr(Wr), ptr(bias), T, d, f,
                                E, k, ptr(logits), ptr(topk_idx), ptr(topk_w), ptr(counts), ptr(offsets),
                                ptr(sorted_tok), ptr(sorted_j), ptr(inv), ptr(active), ptr(slot_of_pair), ptr(miss),
-                               ptr(miss_count), miss_cap, ptr(y), ptr(ws), ws_bytes, ptr(dev_status),
-                               stream_handle(stream)))
+                               ptr(miss_count), miss_cap, ptr(expert_counts), ptr(y), ptr(ws), ws_bytes,
+                               ptr(dev_status), stream_handle(stream)))
 
 
 def stack_decode(pool: QPool, L: int, slot_of, shared_slot, layer0: int, x, Wr, bias, T, d, f, E, k, topk_idx=None,
                  topk_w=None, slot_of_pair=None, miss=None, miss_count=None, miss_cap=0, y=None, ws=None,
-                 ws_bytes=0, dev_status=None, stream=None) -> None:
+                 ws_bytes=0, dev_status=None, stream=None, expert_counts=None) -> None:
     check("moe_stack_decode",
           lib.moe_stack_decode(C.byref(pool), L, ptr(slot_of), ptr(shared_slot), layer0, ptr(x), ptr(Wr), ptr(bias),
                                T, d, f, E, k, ptr(topk_idx), ptr(topk_w), ptr(slot_of_pair), ptr(miss),
-                               ptr(miss_count), miss_cap, ptr(y), ptr(ws), ws_bytes, ptr(dev_status),
-                               stream_handle(stream)))
+                               ptr(miss_count), miss_cap, ptr(expert_counts), ptr(y), ptr(ws), ws_bytes,
+                               ptr(dev_status), stream_handle(stream)))
 
 
 def expert_table(E: int, experts: dict) -> C.Array:
@@ -247,6 +252,44 @@ def complete_misses_host(fmt: int, d: int, f: int, experts: C.Array, E: int, mis
                                        nthreads))
 
 
+class MissEngine:
+    """moe_miss_engine: host worker threads completing miss lists as they are
+    published (see include/moe.h). Submitted arrays must stay alive until
+    wait() returns; the engine keeps references to them until then."""
+
+    def __init__(self, nthreads: int = 0):
+        h = _P()
+        check("moe_miss_engine_create", lib.moe_miss_engine_create(nthreads, C.byref(h)))
+        self.h = h
+        self._keep = []
+
+    def submit(self, fmt: int, d: int, f: int, experts: C.Array, E: int, miss, count, miss_cap: int, layer: int, x,
+               T: int, y) -> None:
+        """miss: host records (e.g. a pinned tensor the GPU writes), count: host
+        int32 whose value becomes >= 0 when the records are complete."""
+        self._keep.append((experts, miss, count, x, y))
+        check("moe_miss_engine_submit",
+              lib.moe_miss_engine_submit(self.h, fmt, d, f, C.cast(experts, _P), E, ptr(miss), ptr(count), miss_cap,
+                                         layer, ptr(x), T, ptr(y)))
+
+    def wait(self) -> None:
+        code = lib.moe_miss_engine_wait(self.h)
+        self._keep.clear()
+        check("moe_miss_engine_wait", code)
+
+    def close(self) -> None:
+        if self.h:
+            lib.moe_miss_engine_destroy(self.h)
+            self.h = None
+            self._keep.clear()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 class CachePolicy:
     """Host expert-cache policy (moe_cache_policy_*): counts of routed pairs,
     halved every `epoch` tokens, and slot plans against an [L][E] slot table."""
@@ -268,6 +311,14 @@ class CachePolicy:
         T, k = idx.shape
         check("moe_cache_policy_observe", lib.moe_cache_policy_observe(self.state.ctypes.data, layer, idx.ctypes.data,
                                                                        T, k))
+
+    def observe_counts(self, counts, tokens: int) -> None:
+        """A window of `tokens` token steps from per-expert counts (int32 [L][E])."""
+        import numpy as np
+
+        c = np.ascontiguousarray(counts, dtype=np.int32)
+        check("moe_cache_policy_observe_counts",
+              lib.moe_cache_policy_observe_counts(self.state.ctypes.data, c.ctypes.data, tokens))
 
     def plan(self, slot_of, max_swaps: int) -> list:
         """Update slot_of (int32 [L][E] numpy, in place); the changes as tuples

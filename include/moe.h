@@ -195,11 +195,16 @@ moe_status moe_permute(const int32_t *topk_idx, int T, int k, int E, int32_t *co
  *                resident, ordered by (expert, token); entries past miss_cap are
  *                dropped and set MOE_DEV_MISS_OVERFLOW
  *   miss_count   int32 [1] (output): the true number of misses
+ *   expert_counts int32 [E] or NULL: every routed pair (hit or miss) adds 1
+ *                to its expert's entry (atomically; the caller zeroes it when
+ *                a counting window starts) -- the use counts the cache policy
+ *                reads in bulk (moe_cache_policy_observe_counts)
  */
 moe_status moe_cache_lookup(const int32_t *slot_of, int32_t num_slots, int32_t layer, const int32_t *topk_idx,
                             const float *topk_w, const int32_t *offsets, const int32_t *sorted_tok,
                             const int32_t *sorted_j, int T, int k, int E, int32_t *slot_of_pair, moe_miss *miss,
-                            int32_t *miss_count, int32_t miss_cap, int32_t *dev_status, moe_stream_t stream);
+                            int32_t *miss_count, int32_t miss_cap, int32_t *expert_counts, int32_t *dev_status,
+                            moe_stream_t stream);
 
 /* Workspace bytes moe_expert_ffn_q2/q3 need for (T, k, d, f). With T*k < 512
  * only the weight-streaming path can run and the workspace is h as fp32,
@@ -250,8 +255,9 @@ moe_status moe_expert_ffn_q3(const moe_qpool *W, const int32_t *slot_of, const u
  * with the experts kept in system RAM. For every record i of miss[0..n):
  *   y[miss[i].token] += miss[i].gate * down(silu(gate_proj x) * up_proj x),
  * x = x[miss[i].token], in fp32 from the expert's canonical storage (w = s*q+m
- * or s*(q-4) applied per 64-block to the block's code-weighted sum). Results
- * are added in record order, so y does not depend on nthreads.
+ * or s*(q-4) applied per 64-block to the block's code-weighted sum, that sum
+ * formed from 16 per-byte-position partial sums added in a fixed order).
+ * Results are added in record order, so y does not depend on nthreads.
  *   fmt, d, f  format and shapes (as for the pool)
  *   experts    moe_qmatrix [E][3] (host): gate [f][d], up [f][d], down [d][f]
  *              of every expert of this layer in canonical host storage; only
@@ -271,6 +277,36 @@ moe_status moe_expert_ffn_q3(const moe_qpool *W, const int32_t *slot_of, const u
  */
 moe_status moe_complete_misses_host(int fmt, int d, int f, const moe_qmatrix *experts, int E, const moe_miss *miss,
                                     int32_t n, int32_t layer, const uint16_t *x, int T, float *y, int nthreads);
+
+/*
+ * Miss engine: a pool of host worker threads that completes miss lists as the
+ * GPU publishes them, so that the host works on one layer's misses while the
+ * GPU runs the next layers ([SAITO] "命中率七成，代价是答案会变": the CPU computes
+ * the experts that are not in GPU memory during the same round as the GPU).
+ *   create   nthreads workers (0 = the machine's hardware threads);
+ *            MOE_ERR_HOST if threads or memory cannot be had
+ *   submit   queue one layer: the arguments of moe_complete_misses_host, with
+ *            the record count read from *count (host memory) once it is >= 0
+ *            (at most miss_cap records are used). A miss list and count that
+ *            moe_layer_decode / moe_stack_decode write to mapped pinned host
+ *            memory are published in that order (the count last, after a
+ *            system-wide fence): set *count to -1 before the launch and submit
+ *            at once. All pointers must stay valid until wait returns. A count
+ *            still negative after 10 s fails the job with MOE_ERR_HOST.
+ *            Jobs run in any order and concurrently; each job adds its records
+ *            into its y in record order (y independent of the thread count).
+ *   wait     block until every submitted job has finished; returns the first
+ *            error among them (MOE_OK if none) and forgets them
+ *   destroy  wait, then stop the workers
+ * One thread at a time may call submit/wait on an engine.
+ */
+typedef struct moe_miss_engine moe_miss_engine;
+moe_status moe_miss_engine_create(int nthreads, moe_miss_engine **engine);
+moe_status moe_miss_engine_submit(moe_miss_engine *engine, int fmt, int d, int f, const moe_qmatrix *experts, int E,
+                                  const moe_miss *miss, const int32_t *count, int32_t miss_cap, int32_t layer,
+                                  const uint16_t *x, int T, float *y);
+moe_status moe_miss_engine_wait(moe_miss_engine *engine);
+void moe_miss_engine_destroy(moe_miss_engine *engine);
 
 /*
  * Expert-cache policy ([SAITO] "命中率七成，代价是答案会变": the free GPU room is
@@ -303,6 +339,14 @@ moe_status moe_cache_policy_init(void *state, size_t bytes, int L, int E, int S,
 
 /* Count one layer call's routing: topk_idx int32 [T][k] (host). */
 moe_status moe_cache_policy_observe(void *state, int layer, const int32_t *topk_idx, int T, int k);
+
+/* Count a window of `tokens` token steps at once from per-expert counts
+ * (host int32 [L][E], e.g. a copy of the device counters that
+ * moe_cache_lookup / moe_layer_decode / moe_stack_decode add to): the token
+ * clock advances by `tokens` first (halving all counts once per full epoch),
+ * then every count is added. For a window of one token step through all
+ * layers this equals moe_cache_policy_observe on each layer in order. */
+moe_status moe_cache_policy_observe_counts(void *state, const int32_t *counts_host, int tokens);
 
 /* Plan slot changes; returns the number written to swaps (<= max_swaps), or
  * -(moe_status) on an invalid state or slot table (slot_of then unchanged). */
@@ -344,6 +388,8 @@ size_t moe_stack_decode_workspace_bytes(int T, int k, int f, int E);
  *   x, Wr, bias  as moe_route; T <= 8, E <= 512, d <= 2048, f <= 4096;
  *                x, Wr and y 16-byte aligned
  *   logits .. miss_count  outputs of the step-by-step calls, each may be NULL
+ *   expert_counts int32 [E] or NULL: routed pairs added per expert, as for
+ *                moe_cache_lookup
  *   y            fp32 [T][d] (output, overwritten)
  *   ws           moe_layer_decode_workspace_bytes() bytes, 256-byte aligned,
  *                zero-filled before first use; each launch leaves its counters
@@ -358,8 +404,9 @@ moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t 
                             const uint16_t *x, const float *Wr, const float *bias, int T, int d, int f, int E, int k,
                             float *logits, int32_t *topk_idx, float *topk_w, int32_t *counts, int32_t *offsets,
                             int32_t *sorted_tok, int32_t *sorted_j, int32_t *inv, int32_t *active,
-                            int32_t *slot_of_pair, moe_miss *miss, int32_t *miss_count, int32_t miss_cap, float *y,
-                            void *ws, size_t ws_bytes, int32_t *dev_status, moe_stream_t stream);
+                            int32_t *slot_of_pair, moe_miss *miss, int32_t *miss_count, int32_t miss_cap,
+                            int32_t *expert_counts, float *y, void *ws, size_t ws_bytes, int32_t *dev_status,
+                            moe_stream_t stream);
 
 /*
  * L layers of moe_layer_decode in one launch, in order: layer l + 1 starts
@@ -375,7 +422,11 @@ moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t 
  *   x            bf16 [L][T][d]: each layer's input
  *   Wr, bias     fp32 [L][E][d], [L][E] (bias may be NULL)
  *   topk_idx, topk_w, slot_of_pair  [L][T*k] outputs as moe_layer_decode (may be NULL)
- *   miss         moe_miss [L][miss_cap], miss_count int32 [L] (may be NULL)
+ *   miss         moe_miss [L][miss_cap], miss_count int32 [L] (may be NULL);
+ *                layer l's records and then its count are written as the
+ *                layer ends (the count after a system-wide fence), so they may
+ *                live in mapped pinned host memory read while the launch runs
+ *   expert_counts int32 [L][E] or NULL: routed pairs added per (layer, expert)
  *   y            fp32 [L][T][d] (output)
  *   ws           moe_stack_decode_workspace_bytes() bytes, as moe_layer_decode
  * Shapes and limits as moe_layer_decode.
@@ -383,8 +434,8 @@ moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t 
 moe_status moe_stack_decode(const moe_qpool *W, int L, const int32_t *slot_of, const int32_t *shared_slot,
                             int32_t layer0, const uint16_t *x, const float *Wr, const float *bias, int T, int d, int f,
                             int E, int k, int32_t *topk_idx, float *topk_w, int32_t *slot_of_pair, moe_miss *miss,
-                            int32_t *miss_count, int32_t miss_cap, float *y, void *ws, size_t ws_bytes,
-                            int32_t *dev_status, moe_stream_t stream);
+                            int32_t *miss_count, int32_t miss_cap, int32_t *expert_counts, float *y, void *ws,
+                            size_t ws_bytes, int32_t *dev_status, moe_stream_t stream);
 
 /*
  * moe_expert_ffn_q2 without a caller-supplied workspace. The pages have no

@@ -10,6 +10,8 @@ reading used here (written out in plain Python loops, integers only):
   observe(layer, rows): on layer 0 the token clock advances by len(rows); for
       every full `epoch` of tokens every count is halved (floor). Then every
       expert id in rows adds 1 to count[layer][id].
+  observe_counts(counts, tokens): the clock advances by `tokens` (halving as
+      above), then counts[layer][expert] is added to every count.
   plan(slot_of, max_swaps): free slots (ascending) go to the non-resident
       (layer, expert) with count > 0 in order (count desc, layer*E+expert asc);
       then the next candidate in that order replaces the next resident in order
@@ -36,6 +38,21 @@ class PolicyOracle:
         for row in rows:
             for e in row:
                 self.count[layer][int(e)] += 1
+
+    def observe_counts(self, counts, tokens: int) -> None:
+        """A window of `tokens` token steps given as counts[layer][expert]: the
+        token clock advances (halving once per full epoch) before the counts are
+        added -- for one token step through every layer this is observe() on
+        each layer in order."""
+        self.clock += tokens
+        while self.clock >= self.epoch:
+            self.clock -= self.epoch
+            for l in range(self.L):
+                for e in range(self.E):
+                    self.count[l][e] //= 2
+        for l in range(self.L):
+            for e in range(self.E):
+                self.count[l][e] += int(counts[l][e])
 
     def plan(self, slot_of, max_swaps: int) -> list:
         """slot_of: list of L lists of E ints (-1 = not resident), changed in place."""

@@ -67,7 +67,7 @@ def test_host_validation_rejects_before_launch():
     assert L.moe_permute(dummy, 8, 10, 5000, dummy, dummy, dummy, dummy, dummy, dummy, None, 0, None, None) == 2
     # cache lookup: null offsets
     assert L.moe_cache_lookup(dummy, 10, 0, dummy, dummy, None, dummy, dummy, 1, 10, 512, dummy, dummy, dummy, 10,
-                              None, None) == 1
+                              None, None, None) == 1
     # ffn: format mismatch, bad dims, small workspace
     pool = native.QPool(dummy * 256, 1474560, 10, 3, 2048, 768)
     args = [dummy, dummy, 1, 2048, 768, 512, 10, dummy, dummy, dummy, dummy, None, dummy, dummy, 1 << 20, None, None]
@@ -81,7 +81,7 @@ def test_host_validation_rejects_before_launch():
     assert L.moe_expert_ffn_q2(C.byref(pool), *args) == 1
     # one-launch decode layer: d above the 2048 it stages, T above 8
     wide = native.QPool(dummy * 256, 1 << 23, 10, 2, 4096, 768)
-    dec = [dummy, 0, 0, dummy, dummy, None, 1, 4096, 768, 512, 10] + [None] * 12 + [0, dummy, dummy, 1 << 24,
+    dec = [dummy, 0, 0, dummy, dummy, None, 1, 4096, 768, 512, 10] + [None] * 12 + [0, None, dummy, dummy, 1 << 24,
                                                                                   None, None]
     assert L.moe_layer_decode(C.byref(wide), *dec) == 2
     dec9 = list(dec)
@@ -89,7 +89,7 @@ def test_host_validation_rejects_before_launch():
     assert L.moe_layer_decode(C.byref(pool), *dec9) == 2
     # stacked layers: no shared-slot table, zero layers, misaligned x
     st = [C.byref(pool), 4, dummy, None, 0, dummy, dummy, None, 1, 2048, 768, 512, 10, None, None, None, None, None, 0,
-          dummy, dummy, 1 << 24, None, None]
+          None, dummy, dummy, 1 << 24, None, None]
     assert L.moe_stack_decode(*st) == 1
     st0 = list(st)
     st0[1] = 0

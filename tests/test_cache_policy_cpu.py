@@ -142,3 +142,43 @@ def test_cache_sim_tool_small():
     r = cache_sim.simulate(L=2, E=16, S=8, k=2, tokens=60, s=1.1, drift_every=20, drift_swaps=3, epoch=16,
                            margin=0, plan_every=4, max_swaps=4, warm=10)
     assert 0.0 <= r["fixed_hit_rate"] <= 1.0 and 0.0 < r["online_hit_rate"] <= 1.0 and r["swaps"] > 0
+
+
+def test_bulk_counts_match_oracle_and_per_layer_observation():
+    """moe_cache_policy_observe_counts against the oracle on windows of several
+    token steps; and for windows of one token step it equals observing each
+    layer's routing in order (both libraries' plans compared with the oracle)."""
+    L, E, S, k = 3, 24, 16, 3
+    trace = synth.gen_routing_trace(12, L, E, k, 120, drift_every=30, drift_swaps=5)
+    # windows of 1..7 token steps, counts summed per (layer, expert)
+    bulk = native.CachePolicy(L, E, S, epoch=9, margin=1)
+    orc = PolicyOracle(L, E, S, epoch=9, margin=1)
+    slot_b = np.full((L, E), -1, np.int32)
+    slot_o = [[-1] * E for _ in range(L)]
+    rng = np.random.default_rng(3)
+    t = 0
+    while t < trace.shape[0]:
+        w = int(rng.integers(1, 8))
+        win = trace[t:t + w]
+        counts = np.zeros((L, E), np.int32)
+        for l in range(L):
+            np.add.at(counts[l], win[:, l].ravel(), 1)
+        bulk.observe_counts(counts, win.shape[0])
+        orc.observe_counts(counts.tolist(), win.shape[0])
+        assert bulk.plan(slot_b, 3) == orc.plan(slot_o, 3)
+        np.testing.assert_array_equal(slot_b, np.array(slot_o, np.int32))
+        t += w
+    # one token step per window == per-layer observe
+    per = native.CachePolicy(L, E, S, epoch=5, margin=0)
+    one = native.CachePolicy(L, E, S, epoch=5, margin=0)
+    s1 = np.full((L, E), -1, np.int32)
+    s2 = np.full((L, E), -1, np.int32)
+    for t in range(40):
+        counts = np.zeros((L, E), np.int32)
+        for l in range(L):
+            per.observe(l, trace[t, l][None, :])
+            np.add.at(counts[l], trace[t, l], 1)
+        one.observe_counts(counts, 1)
+        if t % 4 == 3:
+            assert per.plan(s1, 5) == one.plan(s2, 5)
+            np.testing.assert_array_equal(s1, s2)

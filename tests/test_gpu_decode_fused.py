@@ -174,6 +174,52 @@ def test_stacked_layers_one_launch():
         assert rel_err(b.y[l, :2].cpu().numpy(), one.y[:2].cpu().numpy()) < 1e-5
 
 
+def test_stacked_layers_host_misses_overlapped():
+    """The stacked launch writes each layer's miss list into mapped pinned host
+    memory (count last); the miss engine, given the layers before the launch
+    has finished, completes them on host threads while the GPU runs. GPU y plus
+    the engine's sums must equal the oracle's full layer output (misses
+    included) within 2e-3, and the published lists the oracle's."""
+    from bit_expert_ffn_fp32_b200.layer import MISS_DTYPE
+
+    wl = configs.STACK48
+    L, T = 6, 1
+    stack = MoEStack(wl, layers=L)
+    xs = np.stack([synth.gen_x(0, l, T, wl.d, stream=901) for l in range(L)])
+    x = torch.from_numpy(xs.view(np.int16)).cuda()
+    b0 = stack.stack_buffers(T)        # a first pass tells which experts miss
+    stack.forward_stack(x, b0)
+    torch.cuda.synchronize()
+    missed = [sorted(set(m[1] for m in stack.stack_misses(b0, l))) for l in range(L)]
+    assert sum(len(m) for m in missed) > 0
+    canon = [{e: stack.canonical_expert(l, e) for e in missed[l]} for l in range(L)]
+    tabs = [native.expert_table(wl.E, c) for c in canon]
+    b = stack.stack_buffers(T, host_misses=True)
+    cap = b.idx.shape[1]
+    cnt = b.miss_count.view(np.int32)
+    miss_h = b.miss.view(MISS_DTYPE, (L, cap))
+    y_add = np.zeros((L, T, wl.d), np.float32)
+    eng = native.MissEngine(0)
+    try:
+        cnt[:] = -1
+        b.status.zero_()
+        stack.forward_stack(x, b)
+        for l in range(L):
+            eng.submit(wl.fmt, wl.d, wl.f, tabs[l], wl.E, miss_h[l], cnt[l:l + 1], cap, l,
+                       np.ascontiguousarray(xs[l]), T, y_add[l])
+        eng.wait()
+    finally:
+        eng.close()
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    y_full = b.y[:, :T].cpu().numpy().astype(np.float64) + y_add
+    for l in range(L):
+        ref = oracle_layer(stack, l, xs[l])
+        assert [tuple(r)[:4] for r in miss_h[l, : int(cnt[l])]] == [m[:4] for m in ref["misses"]]
+        err = rel_err(y_full[l], ref["y_full"])
+        assert err <= OUT_TOL, (l, err)
+
+
 def test_fused_rejects_unsupported(tiny):
     wl = configs.TINY
     x = torch.zeros(9, wl.d, dtype=torch.int16, device="cuda")

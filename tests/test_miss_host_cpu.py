@@ -118,3 +118,74 @@ def test_complete_misses_rejects_bad_records_before_writing():
     assert np.all(y == 1.0)
     assert call(np.zeros(0, MISS_DT)) == 0
     assert np.all(y == 1.0)
+
+
+# ---------------------------------------------------------------- miss engine
+def test_miss_engine_matches_blocking_call_as_counts_are_published():
+    """Layers submitted before their records exist: each count starts at -1 and
+    another thread fills the records and then the count (as the GPU does
+    through mapped memory), layer by layer. The engine's y equals the blocking
+    moe_complete_misses_host result bit for bit."""
+    import threading
+    import time
+
+    d, f, E, T, L = 512, 256, 8, 4, 5
+    fmt = 2
+    canons = [_experts(fmt, d, f, range(E), seed=20 + l, layer=l) for l in range(L)]
+    tabs = [native.expert_table(E, c) for c in canons]
+    xs = [synth.gen_x(4, l, T, d, stream=2) for l in range(L)]
+    rng = np.random.default_rng(8)
+    recs = []
+    for l in range(L):
+        n = int(rng.integers(1, 7))
+        recs.append(np.array([(l, int(rng.integers(0, E)), int(rng.integers(0, T)), j, float(rng.random()))
+                              for j in range(n)], MISS_DT))
+    cap = 8
+    miss_bufs = [np.zeros(cap, MISS_DT) for _ in range(L)]
+    counts = np.full(L, -1, np.int32)
+    ys = [np.zeros((T, d), np.float32) for _ in range(L)]
+    eng = native.MissEngine(3)
+    try:
+        for l in range(L):
+            eng.submit(fmt, d, f, tabs[l], E, miss_bufs[l], counts[l:l + 1], cap, l, xs[l], T, ys[l])
+
+        def publish():
+            for l in range(L):
+                time.sleep(0.02)
+                miss_bufs[l][: len(recs[l])] = recs[l]
+                counts[l] = len(recs[l])
+
+        th = threading.Thread(target=publish)
+        th.start()
+        eng.wait()
+        th.join()
+    finally:
+        eng.close()
+    for l in range(L):
+        ref = np.zeros((T, d), np.float32)
+        native.complete_misses_host(fmt, d, f, tabs[l], E, recs[l], len(recs[l]), l, xs[l], T, ref, 2)
+        np.testing.assert_array_equal(ys[l], ref)
+
+
+def test_miss_engine_reports_bad_records_and_keeps_y():
+    d, f, E, T = 512, 256, 3, 2
+    canon = _experts(2, d, f, [0, 1])
+    tab = native.expert_table(E, canon)
+    x = synth.gen_x(1, 0, T, d)
+    y = np.ones((T, d), np.float32)
+    recs = np.array([(0, 1, 1, 0, 0.5), (0, 2, 0, 0, 0.5)], MISS_DT)   # expert 2 not given
+    count = np.array([2], np.int32)
+    eng = native.MissEngine(2)
+    try:
+        eng.submit(2, d, f, tab, E, recs, count, 2, 0, x, T, y)
+        with pytest.raises(native.MoeError) as ei:
+            eng.wait()
+        assert ei.value.code == 1
+        assert np.all(y == 1.0)
+        # the engine stays usable
+        good = np.array([(0, 1, 1, 0, 0.5)], MISS_DT)
+        eng.submit(2, d, f, tab, E, good, np.array([1], np.int32), 1, 0, x, T, y)
+        eng.wait()
+        assert not np.all(y == 1.0)
+    finally:
+        eng.close()
