@@ -147,7 +147,7 @@ def ffn(W, x):
     return [sum(W["down"][r][c] * h[c] for c in range(f)) for r in range(d)]
 
 
-def layer(x_bits, Wr, bias, experts, shared, k, fmt, slot_of=None):
+def layer(x_bits, Wr, bias, experts, shared, k, fmt, slot_of=None, fmt_of=None):
     T, d = len(x_bits), len(x_bits[0])
     E = len(Wr)
     logits = [[router_logit(x_bits[t], Wr[e], None if bias is None else bias[e]) for e in range(E)]
@@ -167,7 +167,8 @@ def layer(x_bits, Wr, bias, experts, shared, k, fmt, slot_of=None):
         for j in range(k):
             e = idx[t][j]
             if e not in Wd:
-                Wd[e] = {m: dequant(experts[e][m], fmt) for m in ("gate", "up", "down")}
+                fe = fmt if fmt_of is None else fmt_of[e]
+                Wd[e] = {m: dequant(experts[e][m], fe) for m in ("gate", "up", "down")}
             ye = ffn(Wd[e], xf[t])
             full = [a + gate[t][j] * b for a, b in zip(full, ye)]
             if slot_of[e] >= 0:

@@ -205,11 +205,15 @@ def expert_hidden(W: dict, x_row: np.ndarray) -> np.ndarray:
 
 
 def layer(x: np.ndarray, Wr: np.ndarray, bias, get_expert, shared: dict, k: int, fmt: int,
-          slot_of: np.ndarray | None = None, layer_id: int = 0, tokens=None, miss_cap=None) -> dict:
+          slot_of: np.ndarray | None = None, layer_id: int = 0, tokens=None, miss_cap=None,
+          fmt_of=None) -> dict:
     """One MoE FFN layer.
 
     get_expert(e) returns expert e in canonical storage; shared is the shared
     expert. slot_of (int32 [E], -1 = not resident) defaults to all resident.
+    fmt is the storage format of every expert, unless fmt_of (int [E]) gives
+    each routed expert its own (a pool holding both tiers: each expert is
+    dequantised by its own format's rule, the shared expert by fmt).
     tokens restricts the FFN work to those token indices (routing, permutation
     and lookup always cover all T tokens); y_partial / y_full rows of other
     tokens are NaN.
@@ -236,7 +240,7 @@ def layer(x: np.ndarray, Wr: np.ndarray, bias, get_expert, shared: dict, k: int,
         for j in range(k):
             need.setdefault(int(idx[t, j]), []).append(t)
     for e in sorted(need):
-        W = dequant_expert(get_expert(e), fmt)
+        W = dequant_expert(get_expert(e), fmt if fmt_of is None else int(fmt_of[e]))
         ts = sorted(set(need[e]))
         rows = expert_ffn(W, xf[ts])
         for i, t in enumerate(ts):

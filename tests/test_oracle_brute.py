@@ -54,6 +54,32 @@ def test_layer_vs_brute(orc, brute, fmt, seed, bias, ties):
     np.testing.assert_allclose(o["y_full"], np.array(br["y_full"]), rtol=1e-10, atol=1e-12)
 
 
+def test_mixed_format_layer_vs_brute(orc, brute):
+    """A pool holding both tiers: each routed expert dequantised by its own
+    format (Q3 for the odd ids, Q2 for the rest, shared Q2), the oracle against
+    the brute force; and the routed part differs from the all-Q2 layer exactly
+    where a Q3 expert was routed."""
+    k, E, d, f, seed = 3, 8, 128, 64, 5
+    x, Wr, b, _, shared = _tiny(2, seed)
+    fmt_of = [3 if e % 2 else 2 for e in range(E)]
+    experts = {e: synth.gen_expert(seed, 0, e, fmt_of[e], d, f) for e in range(E)}
+    slot_of = np.array([0, 1, 2, -1, 3, 4, -1, 5], np.int32)
+    o = orc.layer(x, Wr, b, experts.__getitem__, shared, k, 2, slot_of=slot_of, fmt_of=np.array(fmt_of))
+    lst = lambda m: {kk: (None if v is None else v.tolist()) for kk, v in m.items()}
+    br = brute.layer(x.tolist(), Wr.tolist(), b.tolist(),
+                     {e: {m: lst(experts[e][m]) for m in experts[e]} for e in experts},
+                     {m: lst(shared[m]) for m in shared}, k, 2, slot_of=slot_of.tolist(), fmt_of=fmt_of)
+    np.testing.assert_array_equal(o["idx"], np.array(br["idx"]))
+    np.testing.assert_allclose(o["y_partial"], np.array(br["y_partial"]), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(o["y_full"], np.array(br["y_full"]), rtol=1e-10, atol=1e-12)
+    assert any(fmt_of[int(e)] == 3 for e in o["idx"].ravel())
+    q2 = {e: synth.gen_expert(seed, 0, e, 2, d, f) for e in range(E)}
+    o2 = orc.layer(x, Wr, b, q2.__getitem__, shared, k, 2, slot_of=slot_of)
+    for t in range(x.shape[0]):
+        same = all(fmt_of[int(e)] == 2 for e in o["idx"][t])
+        assert np.array_equal(o["y_full"][t], o2["y_full"][t]) == same
+
+
 def test_round_f32_matches_numpy(brute):
     from fractions import Fraction
     rng = np.random.default_rng(0)
