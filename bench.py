@@ -42,7 +42,11 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s (decode T=1/4, 8K prefill); % of HBM / tensor roofline"
 HEADLINE = "decode_T1_d2048_E512_k10_f768_q2"
 NESTED = ("prefill_T8192_d2048_E512_k10_f768_q2", "verify_T4_d2048_E512_k10_f768_q3",
-          "stack48_T1_d2048_E512_k10_f768_q2_res25")
+          "stack48_T1_d2048_E512_k10_f768_q2_res25",
+          # beyond the metric's own workloads: a 32K prompt in 8192-token chunks,
+          # the 3-bit tier at prefill size and a pool holding both tiers
+          "prefill_chunks4_T32768_d2048_E512_k10_f768_q2", "prefill_T8192_d2048_E512_k10_f768_q3",
+          "prefill_T8192_d2048_E512_k10_f768_mixed_q3top128")
 FLUSH_WRITE_BYTES = 512 << 20
 FLUSH_READ_BYTES = 256 << 20
 
@@ -148,9 +152,11 @@ def _oracle_worker_init(wl_name):
     from bit_expert_ffn_fp32_b200.configs import WORKLOADS, ZIPF_ALPHA
 
     wl = WORKLOADS[wl_name]
+    rank = synth.gen_rank_perm(wl.seed, 0, wl.E)
     _ORC_CTX.update(
         orc=orc, wl=wl, Wr=synth.gen_router(wl.seed, 0, wl.E, wl.d),
-        bias=synth.zipf_bias(synth.gen_rank_perm(wl.seed, 0, wl.E), ZIPF_ALPHA) if wl.zipf else None,
+        bias=synth.zipf_bias(rank, ZIPF_ALPHA) if wl.zipf else None,
+        fmt_of=np.array([wl.expert_fmt(int(r)) for r in rank]),
         shared=synth.gen_expert(wl.seed, 0, wl.E, wl.fmt, wl.d, wl.f), synth=synth)
 
 
@@ -159,9 +165,9 @@ def _oracle_one_token(stream_id):
     c = _ORC_CTX
     wl, synth = c["wl"], c["synth"]
     x = synth.gen_x(wl.seed, 0, 1, wl.d, stream=stream_id)
-    get = lambda e: synth.gen_expert(wl.seed, 0, e, wl.fmt, wl.d, wl.f)  # noqa: E731
+    get = lambda e: synth.gen_expert(wl.seed, 0, e, int(c["fmt_of"][e]), wl.d, wl.f)  # noqa: E731
     t0 = time.perf_counter()
-    c["orc"].layer(x, c["Wr"], c["bias"], get, c["shared"], wl.k, wl.fmt)
+    c["orc"].layer(x, c["Wr"], c["bias"], get, c["shared"], wl.k, wl.fmt, fmt_of=c["fmt_of"])
     return time.perf_counter() - t0
 
 
@@ -334,8 +340,6 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
     from bit_expert_ffn_fp32_b200.layer import x_tensor
 
     L, T = wl.layers, wl.T
-    bufs = [stack.buffers(T)]
-    b = bufs[0]
     stream = torch.cuda.current_stream()
     steps, warmup = args.steps, args.warmup
     n_steps = warmup + steps
@@ -347,43 +351,35 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
     xs_dev = torch.stack([torch.stack([x_tensor(xl, dev) for xl in x]) for x in xs_host])
     xs = lambda i: xs_dev[i % n_x]  # noqa: E731
 
-    fused = T <= 8
+    fused = T <= 8 and not stack.mixed
     stacked = fused and L > 1  # all layers in one moe_stack_decode launch
     sb = stack.stack_buffers(T) if stacked else None
-    k, E, d, f = wl.k, wl.E, wl.d, wl.f
+    C = wl.chunk if wl.chunk and not fused else T   # tokens per forward() (a prompt's chunks)
+    chunks = [(c0, min(C, T - c0)) for c0 in range(0, T, C)]
+    y_long = torch.empty((T, wl.d), dtype=torch.float32, device=dev) if len(chunks) > 1 else None
+    b = stack.buffers(T) if y_long is None else None
 
     def layer_step(xset, evs=None):
+        """One step; evs: one event pair per chunk, recorded around the expert
+        calls (or the whole launch on the one-launch paths). Returns y."""
         if fused:
             if evs:
-                evs[0].record(stream)
+                evs[0][0].record(stream)
             if stacked:
                 stack.forward_stack(xset, sb)
             else:
                 stack.forward_fused(0, xset[0], b)
             if evs:
-                evs[1].record(stream)
-            return
-        x = xset[0]
-        native.route(x, stack.Wr[0], stack.bias[0], T, d, E, k, b.logits, b.idx, b.w, b.status)
-        native.permute(b.idx, T, k, E, b.counts, b.offsets, b.sorted_tok, b.sorted_j, b.inv, b.active, b.perm_ws,
-                       0 if b.perm_ws is None else b.perm_ws.numel(), b.status)
-        native.cache_lookup(stack.slot_of[0], stack.num_slots, 0, b.idx, b.w, b.offsets, b.sorted_tok,
-                            b.sorted_j, T, k, E, b.sop, b.miss, b.miss_count, b.idx.numel(), b.status)
-        if evs:
-            evs[0].record(stream)
-        native.expert_ffn(stack.qpool, stack.slot_of[0], x, T, d, f, E, k, b.offsets, b.sorted_tok, b.sorted_j,
-                          b.active, None, b.y_perm, b.h_ws, b.h_ws.numel(), b.status)
-        native.expert_ffn(stack.qpool, stack.shared_slot[0], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
-                          b.sh_sorted_j, b.sh_active, None, b.y_sh, b.h_sh, b.h_sh.numel(), b.status)
-        if evs:
-            evs[1].record(stream)
-        native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y)
+                evs[0][1].record(stream)
+            return sb.y if stacked else b.y
+        if y_long is not None:
+            return stack.forward_chunked(0, xset[0], C, y=y_long, ffn_events=evs)
+        stack.forward(0, xset[0], b, ffn_events=evs[0] if evs else None)
+        return b.y
 
-    tc_path = T * wl.k >= 512 and wl.fmt == 2
-    ffn_launches = 3 if tc_path else 2  # (+ the fp16 gather on the tensor-core path)
-    perm_launches = 1 if native.permute_workspace_bytes(T, wl.k, wl.E) == 0 else 3
-    launches_per_step = 1 if fused else 2 + perm_launches + 1 + 2 * ffn_launches + 1
-    statuses = [sb.status] if stacked else [bl.status for bl in bufs]
+    tc_path = not fused and C * wl.k >= 512
+    launches_per_step = 1 if fused else sum(stack.launches(n) for _, n in chunks)
+    statuses = [sb.status] if stacked else [stack.buffers(n).status for n in sorted({n for _, n in chunks})]
 
     for st in statuses:
         st.zero_()
@@ -413,38 +409,52 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
     if fused:
         kern_ms = step_ms
     else:
-        kev = [(mk(), mk()) for _ in range(steps)]
+        kev = [[(mk(), mk()) for _ in chunks] for _ in range(steps)]
         for i in range(steps):
             evict(i)
             layer_step(xs(warmup + i), kev[i])
         torch.cuda.synchronize()
-        kern_ms = [kev[i][0].elapsed_time(kev[i][1]) for i in range(steps)]
+        kern_ms = [sum(a.elapsed_time(c) for a, c in kev[i]) for i in range(steps)]
     status = 0
     for st in statuses:
         status |= int(st.item())
 
-    # distinct resident experts, resident pairs and misses of each step's routing,
-    # summed over the layers (not timed)
-    n_act, n_pairs, n_miss = [], [], []
+    # distinct resident experts (and their packed bytes), resident pairs and
+    # misses of each step's routing, summed over the layers and the chunks (not timed)
+    ebytes = [np.array([native.expert_bytes(stack.expert_fmt(l, e), wl.d, wl.f) for e in range(wl.E)])
+              for l in range(L)]
+    n_act, n_bytes, n_pairs, n_miss = [], [], [], []
     for i in range(min(steps, (64 if T <= 64 else 4) if L == 1 else 4)):
-        layer_step(xs(warmup + i))
-        a_sum = p_sum = m_sum = 0
+        a_sum = p_sum = m_sum = by_sum = 0
         if stacked:
+            layer_step(xs(warmup + i))
             idx_h = sb.idx[:, : T * wl.k].cpu().numpy()
             sop_h = sb.sop[:, : T * wl.k].cpu().numpy()
             mc_h = sb.miss_count.cpu().numpy()
             for l in range(L):
                 ids = np.unique(idx_h[l])
-                a_sum += int((stack.slot_of_host[l][ids] >= 0).sum())
+                ids = ids[stack.slot_of_host[l][ids] >= 0]
+                a_sum += len(ids)
+                by_sum += int(ebytes[l][ids].sum())
                 p_sum += int((sop_h[l] >= 0).sum())
                 m_sum += int(mc_h[l])
-        for l, bl in enumerate(bufs if not stacked else []):
-            na = int(bl.active[0].item())
-            ids = bl.active[1:1 + na].cpu().numpy()
-            a_sum += int((stack.slot_of_host[l][ids] >= 0).sum())
-            p_sum += int((bl.sop[: T * wl.k] >= 0).sum().item())
-            m_sum += int(bl.miss_count.item())
+        else:
+            x0 = xs(warmup + i)[0]
+            for c0, n in chunks:
+                bl = stack.buffers(n)
+                if fused:
+                    stack.forward_fused(0, x0, bl)
+                else:
+                    stack.forward(0, x0[c0:c0 + n], bl)
+                na = int(bl.active[0].item())
+                ids = bl.active[1:1 + na].cpu().numpy()
+                ids = ids[stack.slot_of_host[0][ids] >= 0]
+                a_sum += len(ids)
+                by_sum += int(ebytes[0][ids].sum())
+                p_sum += int((bl.sop[: n * wl.k] >= 0).sum().item())
+                m_sum += int(bl.miss_count.item())
         n_act.append(a_sum)
+        n_bytes.append(by_sum)
         n_pairs.append(p_sum)
         n_miss.append(m_sum)
     mean_act = float(np.mean(n_act))
@@ -464,11 +474,11 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
         evict(i)
         e2e_ev[i][0].record(stream)
         x_dev.copy_(x_pin[i % n_x], non_blocking=True)
-        layer_step(x_dev)
+        y_out = layer_step(x_dev)
         if stacked:
-            y_pin[i % n_y].copy_(sb.y[:, :T], non_blocking=True)
-        for l in range(L if not stacked else 0):
-            y_pin[i % n_y, l].copy_(bufs[l].y[:T], non_blocking=True)
+            y_pin[i % n_y].copy_(y_out[:, :T], non_blocking=True)
+        else:
+            y_pin[i % n_y, 0].copy_(y_out[:T], non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -477,14 +487,17 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
 
     hbm_peak, tc_peak, peak_kind = _measured_peaks()
     eb = native.expert_bytes(wl.fmt, wl.d, wl.f)
-    ffn_bytes = (mean_act + L) * eb                # routed resident experts + the shared experts, read once
+    # routed resident experts (each in its own format) + the shared experts, read once
+    ffn_bytes = float(np.mean(n_bytes)) + L * eb
     layer_bytes = L * wl.E * wl.d * 4 + ffn_bytes  # + the fp32 router weights (all L layers of a step)
     kern_avg_s = kern_total / steps / 1e3
     ffn_flops = 2.0 * 3 * wl.d * wl.f * (res_pairs_mean + T)   # routed resident pairs + shared, per step
     traffic = _profiled_traffic(wl.name)
+    fmt_names = "/".join("q%d" % fm for fm in stack.fmts)
     if tc_path and not fused:
         roof = {"bound": "tensor",
-                "kernel": "moe_expert_ffn_q2 tcgen05 grouped GEMMs (gate/up + down, routed + shared)",
+                "kernel": "moe_expert_ffn_%s tcgen05 grouped GEMMs (gate/up + down, routed + shared%s)"
+                          % (fmt_names, ", every chunk" if len(chunks) > 1 else ""),
                 "achieved": ffn_flops / kern_avg_s / 1e12, "peak": tc_peak, "peak_kind": peak_kind + " bf16 burst",
                 "unit": "TFLOP/s", "frac": ffn_flops / kern_avg_s / 1e12 / tc_peak, "traffic": traffic,
                 "traffic_scope": "the expert FFN launches of one step (fp16 gathers, gate/up, down; routed + shared)",
@@ -494,7 +507,7 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
         roof = {"bound": "hbm",
                 "kernel": ("decode_layer_kernel (moe_stack_decode: %d layers in one launch)" % L if stacked else
                            "decode_layer_kernel (moe_layer_decode: whole layer, one launch)") if fused else
-                          "moe_expert_ffn_q%d (gate/up + down, routed + shared)" % wl.fmt,
+                          "moe_expert_ffn_%s (gate/up + down, routed + shared)" % fmt_names,
                 "achieved": kb / kern_avg_s / 1e9, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                 "frac": kb / kern_avg_s / 1e9 / hbm_peak, "traffic": traffic,
                 "traffic_scope": "DRAM bytes per step (all launches of the step)",
@@ -505,12 +518,16 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
         "step_ms_quantiles": {"median": float(np.median(step_ms)), "p90": float(np.percentile(step_ms, 90)),
                               "min": float(np.min(step_ms)), "max": float(np.max(step_ms)),
                               "note": "this rank's per-step CUDA-event times"},
-        "dtype": ("f16 (dequantised q2) x f16 -> f32" if tc_path and not fused
-                  else "q2xf16->f32" if wl.fmt == 2 else "q3xf16->f32"),
+        "dtype": ("f16 (dequantised %s) x f16 -> f32" % fmt_names if tc_path and not fused
+                  else "%sxf16->f32" % fmt_names),
         "config": {"workload": wl.name, "tokens_per_step": T,
                    "l2": "512 MiB write + 256 MiB read of other buffers between steps (flushed, clean)",
                    "path": ("moe_stack_decode (all layers, one launch)" if stacked else
-                            "moe_layer_decode (one launch)") if fused else "step-by-step calls, y_perm + moe_combine",
+                            "moe_layer_decode (one launch)") if fused else
+                           ("step-by-step calls, y_perm + moe_combine"
+                            + (", %d chunks of <= %d tokens back to back" % (len(chunks), C) if len(chunks) > 1
+                               else "")
+                            + (", one expert call per format (mixed pool)" if stack.mixed else "")),
                    "parallelism": f"replicas x{world}", "layers_per_step": L,
                    "step_algorithmic_bytes": layer_bytes,
                    "step_GBps": layer_bytes / (total_ms / steps / 1e3) / 1e9,
@@ -544,7 +561,7 @@ def run_ours(args, names, rank, world, local_rank):
         for name in names:
             wl = WORKLOADS[name]
             # workloads that differ only in T share one pool of experts
-            key = (wl.d, wl.E, wl.f, wl.fmt, wl.layers, wl.resident, wl.seed, wl.zipf)
+            key = (wl.d, wl.E, wl.f, wl.fmt, wl.layers, wl.resident, wl.seed, wl.zipf, wl.q3_top)
             if key not in stacks:
                 stacks.clear()
                 torch.cuda.empty_cache()

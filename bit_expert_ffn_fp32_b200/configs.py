@@ -34,10 +34,16 @@ class Workload:
     zipf: bool = True
     resident: int = -1   # resident experts per layer (-1 = all)
     seed: int = 0
+    q3_top: int = 0      # mixed pool: the q3_top most popular experts of a layer are stored Q3, the rest fmt
+    chunk: int = 0       # prefill chunk loop: T tokens processed in chunks of this many (0 = one call)
 
     @property
     def resident_count(self) -> int:
         return self.E if self.resident < 0 else self.resident
+
+    def expert_fmt(self, rank: int) -> int:
+        """Storage format of an expert of popularity rank `rank` (1 = most popular)."""
+        return 3 if self.q3_top > 0 and rank <= self.q3_top else self.fmt
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -53,6 +59,15 @@ WORKLOADS = {
     "prefill_T8192_d2048_E512_k10_f768_q2": Workload("prefill_T8192_d2048_E512_k10_f768_q2", 8192, 2048, 512, 10, 768, 2),
     "stack48_T1_d2048_E512_k10_f768_q2_res25": Workload(
         "stack48_T1_d2048_E512_k10_f768_q2_res25", 1, 2048, 512, 10, 768, 2, layers=48, resident=128),
+    # a 32K-token prompt through one layer in four 8192-token chunks
+    "prefill_chunks4_T32768_d2048_E512_k10_f768_q2": Workload(
+        "prefill_chunks4_T32768_d2048_E512_k10_f768_q2", 32768, 2048, 512, 10, 768, 2, chunk=8192),
+    # the 3-bit tier at prefill size
+    "prefill_T8192_d2048_E512_k10_f768_q3": Workload("prefill_T8192_d2048_E512_k10_f768_q3", 8192, 2048, 512, 10,
+                                                      768, 3),
+    # a pool with both tiers: the 128 most popular experts of the layer in Q3, the rest in Q2
+    "prefill_T8192_d2048_E512_k10_f768_mixed_q3top128": Workload(
+        "prefill_T8192_d2048_E512_k10_f768_mixed_q3top128", 8192, 2048, 512, 10, 768, 2, q3_top=128),
 }
 
 TINY = WORKLOADS["tiny_T16_d512_E64_k4_f256_q2"]

@@ -37,8 +37,9 @@ inline bool dims_ok(int d, int f) {
     return d > 0 && f > 0 && d % 256 == 0 && f % 256 == 0 && d <= kMaxDim && f <= kMaxDim;
 }
 
-// Prefill path (ffn_tc05.cu): grouped tcgen05 GEMMs for Q2 experts. Used by
-// moe_expert_ffn_q2 when T*k >= kTcMinPairs; the caller has validated arguments.
+// Prefill path (ffn_tc05.cu): grouped tcgen05 GEMMs for Q2 or Q3 experts. Used
+// by moe_expert_ffn_q2/q3 when T*k >= kTcMinPairs; the caller has validated
+// arguments.
 constexpr int kTcMinPairs = 512;
 constexpr int kTcMaxE = 1024;
 // Byte offset of the permuted fp16 activations (fp16 [T*k][d]) inside the
@@ -46,8 +47,9 @@ constexpr int kTcMaxE = 1024;
 inline size_t tc05_xperm_offset(int T, int k, int f) {
     return (size_t(T) * size_t(k) * size_t(f) * 2 + 255) & ~size_t(255);
 }
-moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f, int E, int k,
-                       const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j, const int32_t *active,
-                       const float *topk_w, float *out, void *ws, int32_t *dev_status, cudaStream_t stream);
+moe_status tc05_ffn(int fmt, const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f, int E,
+                    int k, const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j,
+                    const int32_t *active, const float *topk_w, float *out, void *ws, int32_t *dev_status,
+                    cudaStream_t stream);
 
 }  // namespace moe

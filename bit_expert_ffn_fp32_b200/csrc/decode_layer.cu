@@ -143,6 +143,7 @@ struct DecodeParams {
     int32_t *miss_count;         // [L] or NULL
     int miss_cap;
     int32_t *expert_counts;      // [L][E] routed pairs per expert, added to (or NULL)
+    int miss_host;               // miss records / counts in mapped host memory: publish with a system fence
     float *y;                    // [L][T][d]
     int32_t *status;
     unsigned *ctr;               // [0] barrier arrivals, [1] CTAs finished
@@ -405,7 +406,7 @@ template <int FMT>
 __device__ __forceinline__ void quad_pair_compute(const QuadRegs<FMT> &qg, const QuadRegs<FMT> &qu,
                                                   const uint32_t (&B)[4][8], const float (&xs)[4][2],
                                                   float (&ag)[4], float (&au)[4]) {
-#pragma unroll 2
+#pragma unroll
     for (int bq = 0; bq < 4; ++bq) {
         float cg[4], cu[4];
         block_mma<FMT>(qg, bq, B[bq], cg);
@@ -895,10 +896,11 @@ __device__ __noinline__ void publish(const DecodeParams &p, Smem &s, int l, int 
         }
     }
     // the count last, after every record is visible system-wide: a host reader of
-    // mapped memory that sees the count sees the records
+    // mapped memory that sees the count sees the records (device readers run
+    // after the kernel and need no fence)
     __syncthreads();
     if (tid == 0) {
-        __threadfence_system();
+        if (p.miss_host) __threadfence_system();
         if (p.miss_count) *reinterpret_cast<volatile int32_t *>(p.miss_count + l) = s.nmiss;
         if (s.nmiss > p.miss_cap && p.miss) flag(p.status, MOE_DEV_MISS_OVERFLOW);
     }
@@ -1585,6 +1587,17 @@ MOE_API size_t moe_stack_decode_workspace_bytes(int T, int k, int f, int E) {
     return moe_layer_decode_workspace_bytes(T, k, f, E);
 }
 
+// True for pinned host memory (mapped into the device's address space).
+static bool in_host_memory(const void *ptr) {
+    if (!ptr) return false;
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeHost;
+}
+
 MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, int32_t shared_slot, int32_t layer,
                                     const uint16_t *x, const float *Wr, const float *bias, int T, int d, int f, int E,
                                     int k, float *logits, int32_t *topk_idx, float *topk_w, int32_t *counts,
@@ -1612,6 +1625,7 @@ MOE_API moe_status moe_layer_decode(const moe_qpool *W, const int32_t *slot_of, 
     p.slot_of_pair = slot_of_pair;
     p.miss_count = miss_count;
     p.expert_counts = expert_counts;
+    p.miss_host = in_host_memory(miss) || in_host_memory(miss_count);
     p.status = dev_status;
     return W->fmt == 2 ? launch_fmt<2>(p, as_cuda(stream)) : launch_fmt<3>(p, as_cuda(stream));
 }
@@ -1634,6 +1648,7 @@ MOE_API moe_status moe_stack_decode(const moe_qpool *W, int L, const int32_t *sl
     p.slot_of_pair = slot_of_pair;
     p.miss_count = miss_count;
     p.expert_counts = expert_counts;
+    p.miss_host = in_host_memory(miss) || in_host_memory(miss_count);
     p.status = dev_status;
     return W->fmt == 2 ? launch_fmt<2>(p, as_cuda(stream)) : launch_fmt<3>(p, as_cuda(stream));
 }

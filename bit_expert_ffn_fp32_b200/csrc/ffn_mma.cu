@@ -230,9 +230,9 @@ moe_status ffn_launch(const moe_qpool *W, const int32_t *slot_of, const uint16_t
     p.up = eg.m[1];
     p.down = eg.m[2];
     cudaStream_t s = as_cuda(stream);
-    if (FMT == 2 && int64_t(T) * k >= kTcMinPairs && E <= kTcMaxE)  // many tokens per expert: tensor-core GEMMs
-        return tc05_ffn_q2(W, slot_of, x, T, d, f, E, k, offsets, sorted_tok, sorted_j, active, topk_w, out, ws,
-                           dev_status, s);
+    if (int64_t(T) * k >= kTcMinPairs && E <= kTcMaxE)  // many tokens per expert: tensor-core GEMMs
+        return tc05_ffn(FMT, W, slot_of, x, T, d, f, E, k, offsets, sorted_tok, sorted_j, active, topk_w, out, ws,
+                        dev_status, s);
     const int na_max = int(std::min<int64_t>(E, int64_t(T) * k));
     gateup_kernel<FMT><<<dim3(f / 16, na_max), 256, 0, s>>>(p);
     down_kernel<FMT><<<dim3(d / 64, na_max), 128, 0, s>>>(p);

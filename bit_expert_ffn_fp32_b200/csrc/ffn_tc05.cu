@@ -8,11 +8,11 @@
 //
 // One persistent CTA per SM walks the (expert, M-tile, N-tile) list; warps are
 // specialised:
-//   producers (8 warps)  dequantise each K stage's packed Q2 codes (staged in
+//   producers (8 warps)  dequantise each K stage's packed codes (staged in
 //                        shared memory by the TMA thread) into the fp16 A tile
-//                        in 128-byte-swizzled shared memory (w = s*q + m, one
-//                        fp16 rounding); the B rows (fp16 activation rows in
-//                        sorted order, or hidden rows) come straight from TMA;
+//                        in tensor memory (Q2 w = s*q + m, Q3 w = s*(q-4), one
+//                        fp16 rounding each); the B rows (fp16 activation rows
+//                        in sorted order, or hidden rows) come straight from TMA;
 //   MMA (1 thread)       issues tcgen05.mma per 16-wide K step into a TMEM
 //                        accumulator;
 //   TMA (2 threads)      issue the tensor-memory-accelerator loads of the
@@ -31,6 +31,7 @@
 
 #include "common.cuh"
 #include "layout.h"
+#include "mma_q.cuh"
 #include "tc05.cuh"
 
 namespace moe {
@@ -263,44 +264,70 @@ __device__ __forceinline__ void dequant_half_q2(const HalfQ2 &c, uint32_t (&v)[1
     }
 }
 
+// Dequantise block BQ of a Q3 lane chunk (the 12 words of a block quad; s01 =
+// {s(g), s(g+8)} of the block) into fp16 pairs in the same register order as
+// dequant_half_q2: w = s*(q-4), q-4 exact in fp16 (1024-offset trick), one
+// rounding in the product.
+template <int BQ>
+__device__ __forceinline__ void dequant_block_q3(const uint32_t (&W)[12], uint32_t s01, uint32_t (&v)[16]) {
+    const __half2 k1028 = __half2half2(__ushort_as_half(0x6404));
+    const __half2 s2x = *reinterpret_cast<const __half2 *>(&s01);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const __half2 s2 = r ? __high2half2(s2x) : __low2half2(s2x);
+#pragma unroll
+        for (int rho = 0; rho < 8; ++rho) {
+            const int u = 8 * BQ + rho;
+            const uint32_t qbits = (q3_reg(W, u, r) >> q3_exp(u)) | 0x64006400u;
+            const __half2 q = __hsub2(*reinterpret_cast<const __half2 *>(&qbits), k1028);
+            const __half2 wv = __hmul2(s2, q);
+            v[2 * rho + r] = *reinterpret_cast<const uint32_t *>(&wv);
+        }
+    }
+}
+
+// Block bq (run time) of the quad; every register index stays a compile-time constant.
+__device__ __forceinline__ void dequant_q3(const uint32_t (&W)[12], const uint32_t (&s)[4], int bq,
+                                           uint32_t (&v)[16]) {
+    switch (bq) {
+        case 0: dequant_block_q3<0>(W, s[0], v); break;
+        case 1: dequant_block_q3<1>(W, s[1], v); break;
+        case 2: dequant_block_q3<2>(W, s[2], v); break;
+        default: dequant_block_q3<3>(W, s[3], v); break;
+    }
+}
+
 __device__ __forceinline__ void set_abort(TcSmem &s, int32_t *status) {
     if (atomicExch(&s.abort, 1) == 0) flag(status, MOE_DEV_TIMEOUT);
 }
 
-// Ask the L2 for tile tau's packed weight rows (codes and scales, one
-// contiguous range per matrix and region) and its B rows (K fp16 each).
-template <int NMAT>
-__device__ __forceinline__ void prefetch_tile(const TcParams &p, const TcSmem &s, int tau, int MT, int TN, int K,
-                                              const __half *bsrc) {
-    const TileInfo t = tile_info(p, s, tau, MT, TN);
-    const uint8_t *rec = p.pool + int64_t(t.slot) * p.slot_bytes;
-    const MatGeom *mats[2] = {NMAT == 2 ? &p.gate : &p.down, &p.up};
-#pragma unroll
-    for (int i = 0; i < NMAT; ++i) {
-        tc::prefetch_l2(rec + q2_chunk_off(*mats[i], 8 * t.mi, 0, 0), uint32_t(8 * (K / 128) * 512));
-        tc::prefetch_l2(rec + scale_off(*mats[i], 2, 8 * t.mi, 0, 0), uint32_t(8 * (K / 128) * 128));
-    }
-    tc::prefetch_l2(bsrc + int64_t(t.beg) * K, uint32_t(t.rows) * uint32_t(K) * 2u);
-}
+// Packed bytes of one code unit of a 128-row tile, per matrix: a block pair
+// (two K stages) for Q2, 8 row groups x 32 lanes x 16 B of codes, then 8 row
+// groups x 8 x 16 B of scales; a block quad (four K stages) for Q3, 8 row
+// groups x 3 x 32 lanes x 16 B of codes, then 8 row groups x 2 x 8 x 8 B of
+// scales.
+template <int FMT>
+struct RawUnit {
+    static constexpr int kStages = FMT == 2 ? 2 : 4;
+    static constexpr int kCodes = FMT == 2 ? 8 * 512 : 8 * 1536;
+    static constexpr int kMat = kCodes + 8 * 128;
+};
 
-// Packed bytes of one block pair (two K stages) of a 128-row tile, per matrix:
-// 8 row groups x 32 lanes x 16 B of codes, then 8 row groups x 8 x 16 B of scales.
-constexpr int kRawCodes = 8 * 512;
-constexpr int kRawPairMat = kRawCodes + 8 * 128;
-
-// Shared-memory rings of a kernel: SB B stages (256 rows x 64 fp16) and SRP
-// slots of packed A bytes (one block pair each). The dequantised A stages live
+// Shared-memory rings of a kernel: SB B stages (192 rows x 64 fp16) and SRP
+// slots of packed A bytes (one code unit each). The dequantised A stages live
 // in tensor memory.
-template <int NMAT, int SB, int SRP>
+template <int FMT, int NMAT, int SB, int SRP>
 struct Rings {
-    static constexpr int kRaw = NMAT * kRawPairMat;
+    static constexpr int kRaw = NMAT * RawUnit<FMT>::kMat;
     static constexpr int kBytes = SB * kSubB + SRP * kRaw;
     __device__ static unsigned char *b(unsigned char *dyn, int it) { return dyn + (it % SB) * kSubB; }
     __device__ static unsigned char *raw(unsigned char *dyn, int pp) { return dyn + SB * kSubB + (pp % SRP) * kRaw; }
 };
 
-// Tensor maps of the packed weights, per matrix: codes as uint32 [slot][row
-// group][pair * 128 words], scales as [slot][row group][pair * 32 words].
+// Tensor maps of the packed weights, per matrix. Q2: codes as uint32 [slot][row
+// group][pair * 128 words], scales as [slot][row group][pair * 32 words]. Q3:
+// codes as uint32 [slot][row group][quad * 3 sub-chunks][128 words], scales as
+// [slot][row group][quad * 32 words].
 struct RawMaps {
     CUtensorMap code[2], scale[2];
 };
@@ -313,16 +340,17 @@ struct StageCursor {
 // TMA threads (lane 0 of warps 17 and 18), each walking this CTA's stages in
 // order and blocking only on the slot it refills next:
 //   A codes  (warp 17) one load of codes and one of scales per matrix and
-//            block pair (two stages) into slot pp % SRP once every producer
-//            is done with it (emptyR); complete on fullR;
+//            code unit (two stages Q2, four Q3) into slot pp % SRP once every
+//            producer is done with it (emptyR); complete on fullR;
 //   B rows   (warp 18) TMA loads of the tile's rows, 64 per box, into B slot
 //            it % SB once the MMA has released it (emptyB); complete on
 //            fullB. On entering a tile it asks the L2 for the next tile.
-template <int NMAT, int SA, int SB, int SRP>
+template <int FMT, int NMAT, int SA, int SB, int SRP>
 __device__ __forceinline__ void issue_codes(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int TN,
                                             int KS, const RawMaps &rm) {
-    using R = Rings<NMAT, SB, SRP>;
-    const int PS = KS / 2;
+    using R = Rings<FMT, NMAT, SB, SRP>;
+    using U = RawUnit<FMT>;
+    const int PS = KS / U::kStages;
     const int mine = blockIdx.x < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
     const int npairs = mine * PS;
     TcClock ck;
@@ -347,11 +375,14 @@ __device__ __forceinline__ void issue_codes(const TcParams &p, TcSmem &s, unsign
         const long long t1 = ck.now();
         unsigned char *raw = R::raw(dyn, pr);
         uint64_t *bar = &s.fullR[pr % SRP];
-        tc::mbar_arrive_expect_tx(bar, uint32_t(NMAT * kRawPairMat));
+        tc::mbar_arrive_expect_tx(bar, uint32_t(NMAT * U::kMat));
 #pragma unroll
         for (int i = 0; i < NMAT; ++i) {
-            tc::tma_load_3d(raw + i * kRawPairMat, &rm.code[i], 128 * pk, 8 * t.mi, t.slot, bar);
-            tc::tma_load_3d(raw + i * kRawPairMat + kRawCodes, &rm.scale[i], 32 * pk, 8 * t.mi, t.slot, bar);
+            if (FMT == 2)
+                tc::tma_load_3d(raw + i * U::kMat, &rm.code[i], 128 * pk, 8 * t.mi, t.slot, bar);
+            else
+                tc::tma_load_4d(raw + i * U::kMat, &rm.code[i], 0, 3 * pk, 8 * t.mi, t.slot, bar);
+            tc::tma_load_3d(raw + i * U::kMat + U::kCodes, &rm.scale[i], 32 * pk, 8 * t.mi, t.slot, bar);
         }
         ck.add(3, t1);
         ck.count(6);
@@ -365,10 +396,10 @@ __device__ __forceinline__ void issue_codes(const TcParams &p, TcSmem &s, unsign
     ck.store(NMAT == 2 ? 0 : 1, 3, true);
 }
 
-template <int NMAT, int SA, int SB, int SRP>
+template <int FMT, int NMAT, int SA, int SB, int SRP>
 __device__ __forceinline__ void issue_rows(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int MT, int TN,
                                            int KS, const void *tmap_b, const __half *bsrc) {
-    using R = Rings<NMAT, SB, SRP>;
+    using R = Rings<FMT, NMAT, SB, SRP>;
     const int mine = blockIdx.x < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
     const int nstages = mine * KS;
     tc::prefetch_tensormap(tmap_b);
@@ -398,16 +429,19 @@ __device__ __forceinline__ void issue_rows(const TcParams &p, TcSmem &s, unsigne
 
 // Producer warps (0-7): warp w owns row group rgl = 2(w%4) + w/4 of the
 // 128-row tile (its tensor-memory lane quadrant is w%4). For each stage, once
-// the block pair's packed bytes have landed (fullR), each thread loads its lane
-// chunk (rows g, g+8 of the row group; k-slots of t), releases the code slot
-// after the pair's second block (emptyR) and dequantises into registers; once
+// the code unit's packed bytes have landed (fullR), each thread loads its lane
+// chunk (rows g, g+8 of the row group; k-slots of t) -- Q2 one block's 8 B of
+// codes and scales per stage, releasing the slot (emptyR) after the pair's
+// second block; Q3 the quad's 48 B of codes and 16 B of scales at its first
+// block, releasing the slot at once -- and dequantises into registers; once
 // the MMA has released the A stage (emptyA) it stores the chunk to the stage's
 // TMEM columns (lane g / g+8, column 4*rho + t = k/2) and arrives on fullA. a_col0: TMEM column of A
 // stage 0, matrix 0; stages are 32*NMAT columns apart.
-template <int NMAT, int SA, int SB, int SRP>
+template <int FMT, int NMAT, int SA, int SB, int SRP>
 __device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned char *dyn, int total, int KS,
                                         uint32_t tmem, int a_col0) {
-    using R = Rings<NMAT, SB, SRP>;
+    using R = Rings<FMT, NMAT, SB, SRP>;
+    using U = RawUnit<FMT>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rgl = 2 * (warp & 3) + (warp >> 2);
     const uint32_t ta = tmem + (uint32_t(16 * rgl) << 16) + uint32_t(a_col0);
@@ -416,9 +450,10 @@ __device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned c
     TcClock ck;
     ck.start();
     bool ok = true;
+    uint32_t w3[NMAT][12], s3[NMAT][4];  // Q3: the quad's lane chunk, kept for its four stages
 #pragma unroll 1
     for (int it = 0; it < nstages; ++it) {
-        const int pp = it >> 1, bb = it & 1;
+        const int pp = it / U::kStages, bb = it % U::kStages;
         long long t0 = ck.now();
         if (bb == 0 && !tc::mbar_wait(&s.fullR[pp % SRP], (pp / SRP) & 1, kTcWaitNs)) {
             ok = false;
@@ -427,18 +462,46 @@ __device__ __forceinline__ void produce(const TcParams &p, TcSmem &s, unsigned c
         ck.add(1, t0);
         t0 = ck.now();
         const unsigned char *raw = R::raw(dyn, pp);
-        HalfQ2 c[NMAT];  // both matrices' bytes first, then both dequantised together
-#pragma unroll
-        for (int i = 0; i < NMAT; ++i) {
-            c[i].cw = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + rgl * 512 + lane * 16 + 8 * bb);
-            c[i].sc = *reinterpret_cast<const uint2 *>(raw + i * kRawPairMat + kRawCodes + rgl * 128 +
-                                                       (lane >> 2) * 16 + 8 * bb);
-        }
-        if (bb) tc::mbar_arrive(&s.emptyR[pp % SRP]);  // both blocks of the pair are in registers
-        // dequantise into registers while the MMA may still be reading this A stage
         uint32_t v[NMAT][16];
+        if (FMT == 2) {
+            HalfQ2 c[NMAT];  // both matrices' bytes first, then both dequantised together
 #pragma unroll
-        for (int i = 0; i < NMAT; ++i) dequant_half_q2(c[i], v[i]);
+            for (int i = 0; i < NMAT; ++i) {
+                c[i].cw = *reinterpret_cast<const uint2 *>(raw + i * U::kMat + rgl * 512 + lane * 16 + 8 * bb);
+                c[i].sc = *reinterpret_cast<const uint2 *>(raw + i * U::kMat + U::kCodes + rgl * 128 +
+                                                           (lane >> 2) * 16 + 8 * bb);
+            }
+            if (bb) tc::mbar_arrive(&s.emptyR[pp % SRP]);  // both blocks of the pair are in registers
+            // dequantise into registers while the MMA may still be reading this A stage
+#pragma unroll
+            for (int i = 0; i < NMAT; ++i) dequant_half_q2(c[i], v[i]);
+        } else {
+            if (bb == 0) {
+#pragma unroll
+                for (int i = 0; i < NMAT; ++i) {
+                    const unsigned char *cb = raw + i * U::kMat + rgl * 1536 + lane * 16;
+#pragma unroll
+                    for (int sub = 0; sub < 3; ++sub) {
+                        const uint4 q = *reinterpret_cast<const uint4 *>(cb + sub * 512);
+                        w3[i][4 * sub + 0] = q.x;
+                        w3[i][4 * sub + 1] = q.y;
+                        w3[i][4 * sub + 2] = q.z;
+                        w3[i][4 * sub + 3] = q.w;
+                    }
+                    // scale entries of the quad's two pairs: {s(g), s(g+8)} per block
+                    const unsigned char *sb = raw + i * U::kMat + U::kCodes + rgl * 128 + (lane >> 2) * 8;
+                    const uint2 a = *reinterpret_cast<const uint2 *>(sb);
+                    const uint2 b = *reinterpret_cast<const uint2 *>(sb + 64);
+                    s3[i][0] = a.x;
+                    s3[i][1] = a.y;
+                    s3[i][2] = b.x;
+                    s3[i][3] = b.y;
+                }
+                tc::mbar_arrive(&s.emptyR[pp % SRP]);  // the whole quad is in registers
+            }
+#pragma unroll
+            for (int i = 0; i < NMAT; ++i) dequant_q3(w3[i], s3[i], bb, v[i]);
+        }
         ck.add(4, t0);
         t0 = ck.now();
         if (!tc::mbar_wait(&s.emptyA[it % SA], ((it / SA) & 1) ^ 1, kTcWaitNs)) {
@@ -510,25 +573,33 @@ __device__ __forceinline__ void mma_release_stage(TcSmem &s, int it) {
 }
 
 // -------------------------------------------------------------------- gate/up
-// Shared memory: 5 B stages (up to 192 tokens, 24 KB each), 4 packed-code
-// slots (one block pair, 10 KB each), 1 KB of h staging per epilogue warp.
-// TMEM: D_gate columns 0..191, D_up 192..383 (one accumulator pair), A stages
-// at 384 and 448 (gate 32 columns, then up 32 columns).
-constexpr int kGuSA = 2, kGuSB = 5, kGuSR = 4;
+// Shared memory: 5 B stages (up to 192 tokens, 24 KB each), packed-code slots
+// (Q2: 4 of one block pair, 10 KB each; Q3: 2 of one block quad, 26 KB each),
+// 1 KB of h staging per epilogue warp. TMEM: D_gate columns 0..191, D_up
+// 192..383 (one accumulator pair), A stages at 384 and 448 (gate 32 columns,
+// then up 32 columns).
+constexpr int kGuSA = 2, kGuSB = 5;
+template <int FMT>
+struct GuSR {
+    static constexpr int v = FMT == 2 ? 4 : 2;
+};
 constexpr int kHStage = 1024;  // per epilogue warp: 16 tokens x 32 rows of h (fp16)
 constexpr int kGuColU = kTileGu, kGuColA = 2 * kTileGu;
-using GuRings = Rings<2, kGuSB, kGuSR>;
+template <int FMT>
+using GuRings = Rings<FMT, 2, kGuSB, GuSR<FMT>::v>;
 
+template <int FMT>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_gateup_q2_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmap_b,
-                        const __grid_constant__ RawMaps rm) {
+    tc_gateup_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmap_b,
+                     const __grid_constant__ RawMaps rm) {
+    constexpr int kGuSR = GuSR<FMT>::v;
     extern __shared__ __align__(1024) unsigned char dyn_raw[];
     unsigned char *dyn =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
     __shared__ TcSmem s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int MT = p.f / 128, KS = p.d / 64, TN = kTileGu;
-    unsigned char *hstage = dyn + GuRings::kBytes;  // epilogue staging of h
+    unsigned char *hstage = dyn + GuRings<FMT>::kBytes;  // epilogue staging of h
     if (tid == 0) init_barriers<kGuSA, kGuSB, kGuSR>(s, 1);
     if (warp == kMmaWarp) tc::tmem_alloc(&s.tmem_base, 512);
     const int total = build_schedule(p, s, MT, TN, reinterpret_cast<int *>(dyn));
@@ -538,7 +609,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tmem = s.tmem_base;
 
     if (warp < kProdWarps) {  // --------------------------------------- producers
-        produce<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, KS, tmem, kGuColA);
+        produce<FMT, 2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, KS, tmem, kGuColA);
     } else if (warp < kMmaWarp) {  // ---------------------------------- epilogue
         const int q = warp & 3, half = (warp - kEpiWarp0) >> 2;  // TMEM lane quadrant, column half
         int tcount = 0;
@@ -589,9 +660,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (too_big) flag(p.status, MOE_DEV_NONFINITE);
         ck.store(0, 1, warp == kEpiWarp0 && lane == 0);
     } else if (warp == kTmaWarp) {  // -------------------------------------- TMA
-        if (lane == 0) issue_codes<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, TN, KS, rm);
+        if (lane == 0) issue_codes<FMT, 2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, TN, KS, rm);
     } else if (warp == kTmaBWarp) {
-        if (lane == 0) issue_rows<2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, TN, KS, &tmap_b, p.xperm);
+        if (lane == 0) issue_rows<FMT, 2, kGuSA, kGuSB, kGuSR>(p, s, dyn, total, MT, TN, KS, &tmap_b, p.xperm);
     } else if (lane == 0) {  // --------------------------------------------- MMA
         int it = 0, tcount = 0;
         bool ok = true;
@@ -615,7 +686,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
                 const uint32_t a = tmem + uint32_t(kGuColA + (it % kGuSA) * 64);  // gate, then up at +32
-                const uint32_t b = tc::smem_u32(GuRings::b(dyn, it));
+                const uint32_t b = tc::smem_u32(GuRings<FMT>::b(dyn, it));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t bd = tc::desc_sw128(b + 32 * kk);
@@ -639,17 +710,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ----------------------------------------------------------------------- down
-// Shared memory: 7 B stages (up to 192 hidden rows, 24 KB each), 4
-// packed-code slots (one block pair, 5 KB each). TMEM: two 192-column
-// accumulators at 0 and 192 (the epilogue of one tile overlaps the MMAs of the
-// next), A stages at 384 and 416.
-constexpr int kDnSA = 2, kDnSB = 7, kDnSR = 4;
+// Shared memory: 7 B stages (up to 192 hidden rows, 24 KB each), packed-code
+// slots (Q2: 4 of one block pair, 5 KB each; Q3: 2 of one block quad, 13 KB
+// each). TMEM: two 192-column accumulators at 0 and 192 (the epilogue of one
+// tile overlaps the MMAs of the next), A stages at 384 and 416.
+constexpr int kDnSA = 2, kDnSB = 7;
+template <int FMT>
+struct DnSR {
+    static constexpr int v = FMT == 2 ? 4 : 2;
+};
 constexpr int kDnColA = 2 * kTileDn;
-using DnRings = Rings<1, kDnSB, kDnSR>;
+template <int FMT>
+using DnRings = Rings<FMT, 1, kDnSB, DnSR<FMT>::v>;
 
+template <int FMT>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_down_q2_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmap_b,
-                      const __grid_constant__ RawMaps rm) {
+    tc_down_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmap_b,
+                   const __grid_constant__ RawMaps rm) {
+    constexpr int kDnSR = DnSR<FMT>::v;
     extern __shared__ __align__(1024) unsigned char dyn_raw[];
     unsigned char *dyn =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
@@ -665,7 +743,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tmem = s.tmem_base;
 
     if (warp < kProdWarps) {  // --------------------------------------- producers
-        produce<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, KS, tmem, kDnColA);
+        produce<FMT, 1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, KS, tmem, kDnColA);
     } else if (warp < kMmaWarp) {  // ---------------------------------- epilogue
         const int q = warp & 3, half = (warp - kEpiWarp0) >> 2;
         int tcount = 0;
@@ -706,9 +784,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         ck.store(1, 1, warp == kEpiWarp0 && lane == 0);
     } else if (warp == kTmaWarp) {  // -------------------------------------- TMA
-        if (lane == 0) issue_codes<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, TN, KS, rm);
+        if (lane == 0) issue_codes<FMT, 1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, TN, KS, rm);
     } else if (warp == kTmaBWarp) {
-        if (lane == 0) issue_rows<1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, TN, KS, &tmap_b, p.h);
+        if (lane == 0) issue_rows<FMT, 1, kDnSA, kDnSB, kDnSR>(p, s, dyn, total, MT, TN, KS, &tmap_b, p.h);
     } else if (lane == 0) {  // --------------------------------------------- MMA
         int it = 0, tcount = 0;
         bool ok = true;
@@ -734,7 +812,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
                 const uint32_t a = tmem + uint32_t(kDnColA + (it % kDnSA) * 32);
-                const uint32_t bb = tc::smem_u32(DnRings::b(dyn, it));
+                const uint32_t bb = tc::smem_u32(DnRings<FMT>::b(dyn, it));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_f16_ta(dd, a + 8 * kk, tc::desc_sw128(bb + 32 * kk), idesc, (ks | kk) ? 1u : 0u);
@@ -812,32 +890,62 @@ bool raw_map(CUtensorMap *map, const uint8_t *pool, int64_t slot_bytes, int num_
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Q3 codes as a 4D uint32 view [slots][row groups][quads * 3 sub-chunks][128
+// words], read in boxes of one quad's 3 sub-chunks x 8 row groups (12 KB).
+bool q3_code_map(CUtensorMap *map, const uint8_t *pool, int64_t slot_bytes, int num_slots, const MatGeom &m) {
+    const cuuint64_t dims[4] = {128, cuuint64_t(m.NB / 4) * 3, cuuint64_t(m.NG), cuuint64_t(num_slots)};
+    const cuuint64_t strides[3] = {512, cuuint64_t(m.NB / 4) * 1536, cuuint64_t(slot_bytes)};
+    const cuuint32_t box[4] = {128, 3, 8, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<uint8_t *>(pool + m.codes_off), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT>
 bool raw_maps(RawMaps *rm, const TcParams &p, const MatGeom *const *mats, int nmat) {
     for (int i = 0; i < nmat; ++i) {
         const MatGeom &m = *mats[i];
-        if (!raw_map(&rm->code[i], p.pool, p.slot_bytes, p.num_slots, m.codes_off, int64_t(m.NB / 2) * 128, m.NG,
-                     128) ||
-            !raw_map(&rm->scale[i], p.pool, p.slot_bytes, p.num_slots, m.scales_off, int64_t(m.NB / 2) * 32, m.NG,
-                     32))
+        const bool codes = FMT == 2 ? raw_map(&rm->code[i], p.pool, p.slot_bytes, p.num_slots, m.codes_off,
+                                              int64_t(m.NB / 2) * 128, m.NG, 128)
+                                    : q3_code_map(&rm->code[i], p.pool, p.slot_bytes, p.num_slots, m);
+        // scales: 32 words per code unit (Q2 one pair of 16 B entries, Q3 two pairs of 8 B entries)
+        if (!codes || !raw_map(&rm->scale[i], p.pool, p.slot_bytes, p.num_slots, m.scales_off,
+                               int64_t(m.NB / 2) * (FMT == 2 ? 32 : 16), m.NG, 32))
             return false;
     }
     return true;
 }
 
-constexpr size_t kGuSmem = size_t(GuRings::kBytes) + size_t(kEpiWarps) * kHStage + 1024;
-constexpr size_t kDnSmem = size_t(DnRings::kBytes) + 1024;
-static_assert(kDnSB <= kMaxSB && kGuSB <= kMaxSB && kDnSR <= kMaxSRP && kGuSR <= kMaxSRP,
+template <int FMT>
+constexpr size_t gu_smem() { return size_t(GuRings<FMT>::kBytes) + size_t(kEpiWarps) * kHStage + 1024; }
+template <int FMT>
+constexpr size_t dn_smem() { return size_t(DnRings<FMT>::kBytes) + 1024; }
+static_assert(kDnSB <= kMaxSB && kGuSB <= kMaxSB && DnSR<2>::v <= kMaxSRP && GuSR<2>::v <= kMaxSRP &&
+                  DnSR<3>::v <= kMaxSRP && GuSR<3>::v <= kMaxSRP,
               "ring larger than its barrier array");
-static_assert(size_t(kKeys + 2 * kMaxActive) * 4 <= size_t(GuRings::kBytes) &&
-                  size_t(kKeys + 2 * kMaxActive) * 4 <= size_t(DnRings::kBytes),
+static_assert(size_t(kKeys + 2 * kMaxActive) * 4 <= size_t(GuRings<2>::kBytes) &&
+                  size_t(kKeys + 2 * kMaxActive) * 4 <= size_t(DnRings<2>::kBytes) &&
+                  size_t(kKeys + 2 * kMaxActive) * 4 <= size_t(GuRings<3>::kBytes) &&
+                  size_t(kKeys + 2 * kMaxActive) * 4 <= size_t(DnRings<3>::kBytes),
               "schedule scratch does not fit the stage memory");
+static_assert(gu_smem<2>() + sizeof(TcSmem) <= 232448 && dn_smem<2>() + sizeof(TcSmem) <= 232448 &&
+                  gu_smem<3>() + sizeof(TcSmem) <= 232448 && dn_smem<3>() + sizeof(TcSmem) <= 232448,
+              "shared memory above the 227 KB a CTA may use");
 
-}  // namespace
+template <int FMT>
+bool set_smem_attrs() {
+    return cudaFuncSetAttribute(tc_gateup_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(gu_smem<FMT>())) == cudaSuccess &&
+           cudaFuncSetAttribute(tc_down_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(dn_smem<FMT>())) == cudaSuccess;
+}
 
-// Launch the two grouped GEMMs (Q2); h is fp16 [T*k][f] inside the caller's workspace.
-moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f, int E, int k,
-                       const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j, const int32_t *active,
-                       const float *topk_w, float *out, void *ws, int32_t *dev_status, cudaStream_t stream) {
+template <int FMT>
+moe_status tc05_ffn_fmt(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f, int E,
+                        int k, const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j,
+                        const int32_t *active, const float *topk_w, float *out, void *ws, int32_t *dev_status,
+                        cudaStream_t stream) {
     if (reinterpret_cast<uintptr_t>(ws) % 256 || reinterpret_cast<uintptr_t>(x) % 16) return MOE_ERR_INVALID_ARG;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
@@ -847,10 +955,7 @@ moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_
     {
         std::lock_guard<std::mutex> lock(g_tc_mu);
         if (!g_tc_ready[dev]) {
-            if (cudaFuncSetAttribute(tc_gateup_q2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGuSmem)) !=
-                    cudaSuccess ||
-                cudaFuncSetAttribute(tc_down_q2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kDnSmem)) !=
-                    cudaSuccess ||
+            if (!set_smem_attrs<2>() || !set_smem_attrs<3>() ||
                 cudaDeviceGetAttribute(&g_tc_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
                 cudaGetLastError();
                 return MOE_ERR_CUDA;
@@ -869,7 +974,7 @@ moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_
             g_tc_ready[dev] = true;
         }
     }
-    const ExpertGeom eg = expert_geom(2, d, f);
+    const ExpertGeom eg = expert_geom(FMT, d, f);
     TcParams p;
     p.pool = static_cast<const uint8_t *>(W->base);
     p.slot_bytes = W->slot_bytes;
@@ -899,12 +1004,25 @@ moe_status tc05_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_
     CUtensorMap map_x, map_h;  // B operands: activation rows (gate/up), hidden rows (down)
     RawMaps rm_gu, rm_dn;
     const MatGeom *gu[2] = {&p.gate, &p.up}, *dn[1] = {&p.down};
-    if (!f16_map(&map_x, p.xperm, d, pairs, 64) || !f16_map(&map_h, p.h, f, pairs, 64) || !raw_maps(&rm_gu, p, gu, 2) ||
-        !raw_maps(&rm_dn, p, dn, 1))
+    if (!f16_map(&map_x, p.xperm, d, pairs, 64) || !f16_map(&map_h, p.h, f, pairs, 64) ||
+        !raw_maps<FMT>(&rm_gu, p, gu, 2) || !raw_maps<FMT>(&rm_dn, p, dn, 1))
         return MOE_ERR_CUDA;
-    tc_gateup_q2_kernel<<<grid, kTcThreads, kGuSmem, stream>>>(p, map_x, rm_gu);
-    tc_down_q2_kernel<<<grid, kTcThreads, kDnSmem, stream>>>(p, map_h, rm_dn);
+    tc_gateup_kernel<FMT><<<grid, kTcThreads, gu_smem<FMT>(), stream>>>(p, map_x, rm_gu);
+    tc_down_kernel<FMT><<<grid, kTcThreads, dn_smem<FMT>(), stream>>>(p, map_h, rm_dn);
     return launch_status();
+}
+
+}  // namespace
+
+// Launch the two grouped GEMMs; h is fp16 [T*k][f] inside the caller's workspace.
+moe_status tc05_ffn(int fmt, const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f, int E,
+                    int k, const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j,
+                    const int32_t *active, const float *topk_w, float *out, void *ws, int32_t *dev_status,
+                    cudaStream_t stream) {
+    return fmt == 2 ? tc05_ffn_fmt<2>(W, slot_of, x, T, d, f, E, k, offsets, sorted_tok, sorted_j, active, topk_w, out,
+                                      ws, dev_status, stream)
+                    : tc05_ffn_fmt<3>(W, slot_of, x, T, d, f, E, k, offsets, sorted_tok, sorted_j, active, topk_w, out,
+                                      ws, dev_status, stream);
 }
 
 }  // namespace moe

@@ -10,9 +10,17 @@ layer). ``forward`` enqueues the layer's steps on the current stream:
 
 Inputs are the seeded synthetic tensors of ``synth``; weights are generated on
 the host and packed on the device by ``moe_pack_expert``.
+
+A workload with ``q3_top > 0`` holds a mixed pool: per layer the ``q3_top``
+most popular experts are stored Q3 and the rest (and the shared expert) in the
+workload's format. Every slot is sized for the larger record; two pool
+descriptions (one per format) share the base, and per-format slot tables keep
+each ``moe_expert_ffn_q2/q3`` call to its own experts (the other format's
+experts read as -1 there, so their rows are left to the other call).
 """
 from __future__ import annotations
 
+import dataclasses
 import os
 from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
@@ -136,12 +144,16 @@ class MoEStack:
         self.seed = wl.seed if seed is None else seed
         self.L = wl.layers if layers is None else layers
         self.R = wl.resident_count
-        self.slot_bytes = native.expert_bytes(wl.fmt, wl.d, wl.f)
+        self.mixed = wl.q3_top > 0 and wl.fmt != 3
+        self.fmts = (wl.fmt, 3) if self.mixed else (wl.fmt,)
+        self.slot_bytes = max(native.expert_bytes(fm, wl.d, wl.f) for fm in self.fmts)
         if self.slot_bytes == 0:
             raise ValueError("unsupported shape")
         self.num_slots = self.L * self.R + self.L
         self.pool = torch.empty(self.num_slots * self.slot_bytes, dtype=torch.uint8, device=self.device)
-        self.qpool = native.qpool(self.pool, self.slot_bytes, self.num_slots, wl.fmt, wl.d, wl.f)
+        self.qpools = {fm: native.qpool(self.pool, self.slot_bytes, self.num_slots, fm, wl.d, wl.f)
+                       for fm in self.fmts}
+        self.qpool = self.qpools[wl.fmt]
         # per-layer router weights, biases and slot tables live in [L][...] device
         # tensors (the stacked call reads them with a layer stride); the lists
         # hold per-layer views
@@ -151,9 +163,15 @@ class MoEStack:
         self.shared_slot_all = torch.arange(self.L * self.R, self.L * self.R + self.L, dtype=torch.int32,
                                             device=self.device)
         self.Wr, self.bias, self.rank, self.slot_of_host, self.slot_of, self.shared_slot = [], [], [], [], [], []
+        # storage format of every routed expert, per layer (host); per-format
+        # device slot tables [L][E] for the two calls of a mixed pool
+        self.fmt_of_host = []
+        self.slot_of_fmt_all = {fm: torch.empty((self.L, wl.E), dtype=torch.int32, device=self.device)
+                                for fm in self.fmts} if self.mixed else {}
         for l in range(self.L):
             Wr = synth.gen_router(self.seed, l, wl.E, wl.d)
             rank = synth.gen_rank_perm(self.seed, l, wl.E)
+            self.fmt_of_host.append(np.array([wl.expert_fmt(int(r)) for r in rank], np.int32))
             bias = synth.zipf_bias(rank, alpha) if wl.zipf else None
             if self.R >= wl.E:
                 slot = np.arange(wl.E, dtype=np.int32) + l * self.R
@@ -169,6 +187,7 @@ class MoEStack:
             self.slot_of_all[l].copy_(torch.from_numpy(slot))
             self.slot_of.append(self.slot_of_all[l])
             self.shared_slot.append(self.shared_slot_all[l:l + 1])
+            self._copy_fmt_rows(l, non_blocking=False)
         # every resident expert and each layer's shared expert: generated on host
         # threads, packed on the current stream in order, one wait at the end
         jobs = [(l, e, int(self.slot_of_host[l][e])) for l in range(self.L) for e in range(wl.E)
@@ -178,8 +197,8 @@ class MoEStack:
             for c0 in range(0, len(jobs), 64):  # at most 64 generated experts held at once
                 chunk = jobs[c0:c0 + 64]
                 for (l, e, slot), canon in zip(chunk, ex.map(lambda j: self.canonical_expert(j[0], j[1]), chunk)):
-                    upload_expert(canon, wl.fmt, wl.d, wl.f, self.pool.data_ptr() + slot * self.slot_bytes,
-                                  self.device, sync=False)
+                    upload_expert(canon, self.expert_fmt(l, e), wl.d, wl.f,
+                                  self.pool.data_ptr() + slot * self.slot_bytes, self.device, sync=False)
         torch.cuda.current_stream().synchronize()
         self._bufs: dict[int, Buffers] = {}
         # routed pairs per (layer, expert), added to by every forward (device
@@ -189,8 +208,17 @@ class MoEStack:
         self._ws: dict = {}
 
     # expert e == E is the layer's shared expert
+    def expert_fmt(self, layer: int, e: int) -> int:
+        return self.wl.fmt if e >= self.wl.E else int(self.fmt_of_host[layer][e])
+
     def canonical_expert(self, layer: int, e: int) -> dict:
-        return synth.gen_expert(self.seed, layer, e, self.wl.fmt, self.wl.d, self.wl.f)
+        return synth.gen_expert(self.seed, layer, e, self.expert_fmt(layer, e), self.wl.d, self.wl.f)
+
+    def _copy_fmt_rows(self, l: int, non_blocking: bool = True) -> None:
+        """Per-format device slot tables of layer l from the host tables."""
+        for fm, tab in self.slot_of_fmt_all.items():
+            row = np.where(self.fmt_of_host[l] == fm, self.slot_of_host[l], -1).astype(np.int32)
+            tab[l].copy_(torch.from_numpy(row), non_blocking=non_blocking)
 
     def apply_swaps(self, swaps) -> None:
         """Carry out a cache-policy plan: every (slot, layer_in, expert_in,
@@ -209,11 +237,13 @@ class MoEStack:
             self._pack(l_in, e_in, slot)
         for l in changed:
             self.slot_of[l].copy_(torch.from_numpy(np.ascontiguousarray(self.slot_of_host[l], dtype=np.int32)))
+            self._copy_fmt_rows(l, non_blocking=False)
 
     def _set_rows(self, layers) -> None:
         for l in sorted(layers):
             self.slot_of[l].copy_(torch.from_numpy(np.ascontiguousarray(self.slot_of_host[l], dtype=np.int32)),
                                   non_blocking=True)
+            self._copy_fmt_rows(l)
 
     def prepare_swaps(self, swaps) -> list:
         """Pack every admitted expert of a plan into a pinned host record (host
@@ -226,7 +256,7 @@ class MoEStack:
             rec = torch.empty(self.slot_bytes, dtype=torch.uint8).pin_memory()
             mats = [native.qmatrix(ex[m]["codes"], ex[m]["scale"], ex[m]["min"], ex[m]["hi"]) for m in
                     ("gate", "up", "down")]
-            native.pack_expert_host(self.wl.fmt, self.wl.d, self.wl.f, *mats, rec.data_ptr())
+            native.pack_expert_host(self.expert_fmt(l_in, e_in), self.wl.d, self.wl.f, *mats, rec.data_ptr())
             out.append((slot, l_in, e_in, l_out, e_out, rec))
         return out
 
@@ -265,7 +295,7 @@ class MoEStack:
         self._set_rows(changed)
 
     def _pack(self, layer: int, e: int, slot: int) -> None:
-        upload_expert(self.canonical_expert(layer, e), self.wl.fmt, self.wl.d, self.wl.f,
+        upload_expert(self.canonical_expert(layer, e), self.expert_fmt(layer, e), self.wl.d, self.wl.f,
                       self.pool.data_ptr() + slot * self.slot_bytes, self.device)
 
     def buffers(self, T: int, fresh: bool = False) -> Buffers:
@@ -301,13 +331,15 @@ class MoEStack:
         return b
 
     def forward(self, layer: int, x: torch.Tensor, b: Buffers | None = None, stream=None,
-                combine: str = "kernel") -> Buffers:
+                combine: str = "kernel", ffn_events=None) -> Buffers:
         """Enqueue one layer on x (bf16 bits as int16/uint16-sized tensor [T][d]).
 
         combine="kernel": routed experts write y_e rows (y_perm), the shared
         expert y_sh, and moe_combine forms y. combine="atomic": the shared
         expert writes y directly and the routed call adds gate * y_e into it
-        (moe_expert_ffn with topk_w), with no y_perm and no combine pass."""
+        (moe_expert_ffn with topk_w), with no y_perm and no combine pass.
+        ffn_events: a pair of CUDA events recorded around the expert calls
+        (routed and shared), on the stream the layer runs on."""
         wl = self.wl
         T = x.shape[0]
         b = b or self.buffers(T)
@@ -318,18 +350,54 @@ class MoEStack:
         native.cache_lookup(self.slot_of[layer], self.num_slots, layer, b.idx, b.w, b.offsets, b.sorted_tok,
                             b.sorted_j, T, k, E, b.sop, b.miss, b.miss_count, b.idx.numel(), b.status, stream,
                             expert_counts=self.expert_counts[layer] if self.count_experts else None)
+        routed = [(self.qpools[fm], self.slot_of_fmt_all[fm][layer]) for fm in self.fmts] if self.mixed \
+            else [(self.qpool, self.slot_of[layer])]
+        st = torch.cuda.current_stream() if stream is None else stream
+        if ffn_events:
+            ffn_events[0].record(st)
         if combine == "atomic":
             native.expert_ffn(self.qpool, self.shared_slot[layer], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
                               b.sh_sorted_j, b.sh_active, None, b.y, b.h_sh, b.h_sh.numel(), b.status, stream)
-            native.expert_ffn(self.qpool, self.slot_of[layer], x, T, d, f, E, k, b.offsets, b.sorted_tok,
-                              b.sorted_j, b.active, b.w, b.y, b.h_ws, b.h_ws.numel(), b.status, stream)
+            for pool, table in routed:
+                native.expert_ffn(pool, table, x, T, d, f, E, k, b.offsets, b.sorted_tok, b.sorted_j, b.active, b.w,
+                                  b.y, b.h_ws, b.h_ws.numel(), b.status, stream)
+            if ffn_events:
+                ffn_events[1].record(st)
             return b
-        native.expert_ffn(self.qpool, self.slot_of[layer], x, T, d, f, E, k, b.offsets, b.sorted_tok, b.sorted_j,
-                          b.active, None, b.y_perm, b.h_ws, b.h_ws.numel(), b.status, stream)
+        for pool, table in routed:
+            native.expert_ffn(pool, table, x, T, d, f, E, k, b.offsets, b.sorted_tok, b.sorted_j, b.active, None,
+                              b.y_perm, b.h_ws, b.h_ws.numel(), b.status, stream)
         native.expert_ffn(self.qpool, self.shared_slot[layer], x, T, d, f, 1, 1, b.sh_offsets, b.sh_sorted_tok,
                           b.sh_sorted_j, b.sh_active, None, b.y_sh, b.h_sh, b.h_sh.numel(), b.status, stream)
+        if ffn_events:
+            ffn_events[1].record(st)
         native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y, stream)
         return b
+
+    def launches(self, T: int, combine: str = "kernel") -> int:
+        """Kernel launches forward() makes for T tokens (route 2, permute 1 or
+        3, lookup 1, each expert call 2, or 3 on the tensor-core path, combine 1)."""
+        wl = self.wl
+        ffn = lambda n, fm: 3 if n >= 512 and fm == 2 else 2  # noqa: E731
+        perm = 1 if native.permute_workspace_bytes(T, wl.k, wl.E) == 0 else 3
+        routed = sum(ffn(T * wl.k, fm) for fm in self.fmts)
+        return 2 + perm + 1 + routed + ffn(T, wl.fmt) + (1 if combine == "kernel" else 0)
+
+    def forward_chunked(self, layer: int, x: torch.Tensor, chunk: int = 8192, y: torch.Tensor | None = None,
+                        stream=None, combine: str = "kernel", ffn_events=None) -> torch.Tensor:
+        """A long prompt through one layer in chunks of at most `chunk` tokens,
+        back to back on one stream (each chunk is one forward(); the last may
+        be shorter). Returns y fp32 [T][d] (``y`` if given). ffn_events: one
+        pair of events per chunk (see forward)."""
+        T = x.shape[0]
+        y = torch.empty((T, self.wl.d), dtype=torch.float32, device=self.device) if y is None else y
+        for i, c0 in enumerate(range(0, T, chunk)):
+            n = min(chunk, T - c0)
+            # the chunk's buffers, with its output rows written in place in y
+            b = dataclasses.replace(self.buffers(n), y=y[c0:c0 + n])
+            self.forward(layer, x[c0:c0 + n], b, stream=stream, combine=combine,
+                         ffn_events=None if ffn_events is None else ffn_events[i])
+        return y
 
     def decode_workspace(self, T: int) -> torch.Tensor:
         """Zero-filled workspace of moe_layer_decode for T tokens (kept per T)."""
@@ -343,6 +411,8 @@ class MoEStack:
                       outputs: bool = True) -> Buffers:
         """Enqueue one layer as a single moe_layer_decode launch (T <= 8).
         outputs=False skips the routing/permutation side outputs (only y)."""
+        if self.mixed:
+            raise ValueError("the one-launch decode kernel reads a single-format pool; use forward()")
         wl = self.wl
         T = x.shape[0]
         b = b or self.buffers(T)
@@ -387,6 +457,8 @@ class MoEStack:
     def forward_stack(self, x: torch.Tensor, b: "StackBuffers | None" = None, stream=None) -> "StackBuffers":
         """Enqueue all L layers as one moe_stack_decode launch; x is [L][T][d]
         (bf16 bits), layer l's input in x[l]. T <= 8."""
+        if self.mixed:
+            raise ValueError("the stacked decode kernel reads a single-format pool; use forward()")
         wl = self.wl
         T = x.shape[1]
         b = b or self.stack_buffers(T)

@@ -232,12 +232,15 @@ size_t moe_expert_ffn_workspace_bytes(int T, int k, int d, int f);
  * 65504 sets MOE_DEV_NONFINITE.
  * Paths: with T*k < 512 a weight-streaming kernel reads each expert's packed
  * codes once per 8 tokens (mma.sync fragments built from the codes); with
- * T*k >= 512 and E <= 1024 (prefill) the Q2 call runs grouped GEMMs on the tcgen05 tensor
- * cores, dequantising each 128-row weight tile to fp16 in registers and storing
- * it to tensor memory (fp16 rounding of w = s*q + m, one fused multiply-add);
+ * T*k >= 512 and E <= 1024 (prefill) both calls run grouped GEMMs on the
+ * tcgen05 tensor cores, dequantising each 128-row weight tile to fp16 in
+ * registers and storing it to tensor memory (one fp16 rounding of
+ * w = s*q + m (Q2, one fused multiply-add) or w = s*(q-4) (Q3));
  * the workspace then holds h as fp16 [T*k][f]
  * followed by the activation rows in sorted pair order as fp16 [T*k][d]; ws
  * must then be 256-byte and x 16-byte aligned (else MOE_ERR_INVALID_ARG).
+ * A pool may hold records of both formats (slot_bytes >= the larger record):
+ * give each call a slot table in which the other format's experts are -1.
  */
 moe_status moe_expert_ffn_q2(const moe_qpool *W, const int32_t *slot_of, const uint16_t *x, int T, int d, int f,
                              int E, int k, const int32_t *offsets, const int32_t *sorted_tok, const int32_t *sorted_j,

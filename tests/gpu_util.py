@@ -30,7 +30,7 @@ def oracle_layer(stack: MoEStack, layer: int, x_bits: np.ndarray, tokens=None):
     assert np.array_equal(Wr, Wr_gen)
     return orc.layer(x_bits, Wr_gen, bias, lambda e: stack.canonical_expert(layer, e),
                      stack.canonical_expert(layer, wl.E), wl.k, wl.fmt, slot_of=stack.slot_of_host[layer],
-                     layer_id=layer, tokens=tokens)
+                     layer_id=layer, tokens=tokens, fmt_of=stack.fmt_of_host[layer] if stack.mixed else None)
 
 
 def rel_err(y: np.ndarray, ref: np.ndarray) -> float:
@@ -68,7 +68,26 @@ def oracle_pair_rows(stack: MoEStack, layer: int, x_bits: np.ndarray, perm: dict
         e = int(np.searchsorted(offs, s, side="right") - 1)
         by_e.setdefault(e, []).append(i)
     for e, rows in by_e.items():
-        W = orc.dequant_expert(stack.canonical_expert(layer, e), wl.fmt)
+        W = orc.dequant_expert(stack.canonical_expert(layer, e), stack.expert_fmt(layer, e))
         toks = [int(perm["sorted_tok"][positions[i]]) for i in rows]
         out[rows] = orc.expert_ffn(W, xf[toks])
     return out
+
+
+def full_check(stack, layer, x_bits, tokens=None, combine="kernel"):
+    """One forward() against the oracle: routing, permutation, slots and the
+    miss list bit for bit, y within OUT_TOL at `tokens` (default every token)."""
+    wl = stack.wl
+    T = x_bits.shape[0]
+    b = run_layer(stack, layer, x_bits, combine)
+    ref = oracle_layer(stack, layer, x_bits, tokens=tokens)
+    assert int(b.status.item()) == 0
+    check_routing(b, ref, T, wl.k, wl.E)
+    misses = stack.misses(b)
+    assert [m[:4] for m in misses] == [m[:4] for m in ref["misses"]]
+    assert int(b.miss_count.item()) == ref["miss_count"]
+    toks = ref["tokens"]
+    y = b.y[:T].cpu().numpy().astype(np.float64)
+    err = rel_err(y[toks], ref["y_partial"][toks])
+    assert err <= OUT_TOL, err
+    return b, ref, err

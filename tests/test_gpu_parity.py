@@ -10,26 +10,12 @@ import torch
 
 from bit_expert_ffn_fp32_b200 import configs, native, synth
 from bit_expert_ffn_fp32_b200.layer import MoEStack, x_tensor
-from gpu_util import OUT_TOL, check_routing, oracle_layer, oracle_pair_rows, rel_err, run_layer
+from gpu_util import OUT_TOL, check_routing, full_check, oracle_layer, oracle_pair_rows, rel_err, run_layer
 
 pytestmark = pytest.mark.gpu
 
 
-def _full_check(stack, layer, x_bits, tokens=None, combine="kernel"):
-    wl = stack.wl
-    T = x_bits.shape[0]
-    b = run_layer(stack, layer, x_bits, combine)
-    ref = oracle_layer(stack, layer, x_bits, tokens=tokens)
-    assert int(b.status.item()) == 0
-    check_routing(b, ref, T, wl.k, wl.E)
-    misses = stack.misses(b)
-    assert [m[:4] for m in misses] == [m[:4] for m in ref["misses"]]
-    assert int(b.miss_count.item()) == ref["miss_count"]
-    toks = ref["tokens"]
-    y = b.y[:T].cpu().numpy().astype(np.float64)
-    err = rel_err(y[toks], ref["y_partial"][toks])
-    assert err <= OUT_TOL, err
-    return b, ref, err
+_full_check = full_check
 
 
 @pytest.fixture(scope="module")
