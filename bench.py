@@ -60,7 +60,15 @@ def _env_int(name, default):
 # workload, from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum;
 # see profiles/), valid only while the sources it was captured on are unchanged
 # (sha256 of the listed csrc files, first 16 hex digits).
-PROFILED_TRAFFIC: dict[str, tuple[tuple[str, ...], str, float]] = {}
+_TC_FILES = ("ffn_tc05.cu", "ffn_mma.cu", "common.cuh", "tc05.cuh", "layout.h", "mma_q.cuh")
+_TC_DIGEST = "994a7bb37e842b2b"
+PROFILED_TRAFFIC: dict[str, tuple[tuple[str, ...], str, float]] = {
+    # the expert-FFN launches of one step (gathers, gate/up, down; routed + shared)
+    "prefill_T8192_d2048_E512_k10_f768_q2": (_TC_FILES, _TC_DIGEST, 2503245056.0),
+    "prefill_T8192_d2048_E512_k10_f768_q3": (_TC_FILES, _TC_DIGEST, 2738534144.0),
+    "prefill_T8192_d2048_E512_k10_f768_mixed_q3top128": (_TC_FILES, _TC_DIGEST, 2874947840.0),
+    "prefill_chunks4_T32768_d2048_E512_k10_f768_q2": (_TC_FILES, _TC_DIGEST, 10012321792.0),
+}
 
 
 def _source_digest(files) -> str:
@@ -511,6 +519,10 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
                 "achieved": kb / kern_avg_s / 1e9, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                 "frac": kb / kern_avg_s / 1e9 / hbm_peak, "traffic": traffic,
                 "traffic_scope": "DRAM bytes per step (all launches of the step)",
+                "traffic_note": None if traffic is not None else
+                ("no ncu capture: its kernel replay of the cooperative cluster launch failed to launch; "
+                 "the phase trace build times the kernel instead" if fused else
+                 "no ncu capture of these sources"),
                 "bytes_per_launch": kb, "avg_launch_us": kern_avg_s * 1e6}
     line = {
         "value": replicas.job_throughput(T * steps, world, total_ms), "unit": "tokens/s",
