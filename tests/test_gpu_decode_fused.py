@@ -245,9 +245,10 @@ def test_fused_all_logits_equal(decode, T):
         decode.bias[0].copy_(saved)
 
 
-def test_fused_many_candidates_fallback(decode):
+@pytest.mark.parametrize("T", [1, 2])
+def test_fused_many_candidates_fallback(decode, T):
     """Experts in 10 of the 32 lanes (id % 32 < 10) all outrank the rest, so more
-    than 64 candidates clear the k-th lane maximum and the round-based path runs."""
+    than 64 candidates clear the selection threshold and the round-based path runs."""
     wl = configs.DECODE
     saved = decode.bias[0].clone()
     try:
@@ -255,6 +256,6 @@ def test_fused_many_candidates_fallback(decode):
         boost[(torch.arange(wl.E, device=saved.device) % 32) < 10] = 100.0
         decode.bias[0].copy_(saved + boost)
         for s in range(2):
-            _check(decode, 0, synth.gen_x(0, 0, 2, wl.d, stream=600 + s))
+            _check(decode, 0, synth.gen_x(0, 0, T, wl.d, stream=600 + s))
     finally:
         decode.bias[0].copy_(saved)
