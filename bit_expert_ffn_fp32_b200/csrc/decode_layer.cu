@@ -685,7 +685,7 @@ __device__ __noinline__ void topk_cta(const DecodeParams &p, Smem &s, const floa
                 const uint64_t me = s.cand[tt][i];
                 int rank = 0;
 #pragma unroll 4
-                for (int q = 0; q < 64; ++q) rank += (q < n && s.cand[tt][q] > me);
+                for (int q = 0; q < n; ++q) rank += s.cand[tt][q] > me;
                 if (rank < k) s.sel[tt][rank] = me;
             }
         }
@@ -776,11 +776,9 @@ __device__ __noinline__ void routing_tables(const DecodeParams &p, Smem &s, int 
     if (tid < npairs) {  // stable sort of the pairs by (expert, pair index)
         my_e = s.pair_e[tid];
 #pragma unroll 4
-        for (int q = 0; q < kMaxPairs; ++q) {
-            if (q < npairs) {
-                const int eq = s.pair_e[q];
-                my_rank += (eq < my_e) || (eq == my_e && q < tid);
-            }
+        for (int q = 0; q < npairs; ++q) {
+            const int eq = s.pair_e[q];
+            my_rank += (eq < my_e) || (eq == my_e && q < tid);
         }
     }
     __syncthreads();
