@@ -481,12 +481,15 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
     for i in range(steps):
         evict(i)
         e2e_ev[i][0].record(stream)
-        x_dev.copy_(x_pin[i % n_x], non_blocking=True)
-        y_out = layer_step(x_dev)
-        if stacked:
-            y_pin[i % n_y].copy_(y_out[:, :T], non_blocking=True)
+        if y_long is not None:  # a chunked prompt: copies of chunks c+1 and c-1 overlap chunk c
+            stack.forward_chunked_host(0, x_pin[i % n_x][0], y_pin[i % n_y, 0], C)
         else:
-            y_pin[i % n_y, 0].copy_(y_out[:T], non_blocking=True)
+            x_dev.copy_(x_pin[i % n_x], non_blocking=True)
+            y_out = layer_step(x_dev)
+            if stacked:
+                y_pin[i % n_y].copy_(y_out[:, :T], non_blocking=True)
+            else:
+                y_pin[i % n_y, 0].copy_(y_out[:T], non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -547,7 +550,10 @@ def measure(wl, stack, args, rank, world, local_rank, dev, evict):
                    "misses_per_step": float(np.mean(n_miss))},
         "roofline": roof,
         "e2e": {"value": replicas.job_throughput(T * steps, world, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": L * T * wl.d * 2, "d2h_bytes_per_step": L * T * wl.d * 4},
+                "h2d_bytes_per_step": L * T * wl.d * 2, "d2h_bytes_per_step": L * T * wl.d * 4,
+                "path": ("MoEStack.forward_chunked_host: chunk copies in and out on two side streams, "
+                         "overlapped with the neighbouring chunks' layers" if y_long is not None else
+                         "pinned x copied in, the step, y copied out, on one stream")},
         "clocks": clocks, "gpu_launches": launches_per_step * steps, "dev_status": status,
     }
     if stacked and not args.no_host_misses and rank == 0:

@@ -374,6 +374,56 @@ class MoEStack:
         native.combine(b.y_perm, b.inv, b.w, b.sop, b.y_sh, T, k, d, b.y, stream)
         return b
 
+    def forward_chunked_host(self, layer: int, x_host: torch.Tensor, y_host: torch.Tensor, chunk: int = 8192,
+                             combine: str = "kernel") -> None:
+        """A long prompt from pinned host memory to pinned host memory in chunks
+        of at most `chunk` tokens, copies overlapped with the layer: chunk c+1
+        is copied in on one side stream and chunk c-1's y copied out on another
+        while chunk c runs on the current stream (two device buffers of each).
+        x_host: pinned int16 [T][d] (bf16 bits); y_host: pinned fp32 [T][d].
+        When the current stream reaches the end of what this enqueues, y_host
+        holds every chunk's output."""
+        wl, dev = self.wl, self.device
+        T = x_host.shape[0]
+        main = torch.cuda.current_stream()
+        key = ("chunk_io", chunk)
+        if key not in self._ws:
+            self._ws[key] = {
+                "h2d": torch.cuda.Stream(device=dev), "d2h": torch.cuda.Stream(device=dev),
+                "x": [torch.empty((chunk, wl.d), dtype=torch.int16, device=dev) for _ in range(2)],
+                "y": [torch.empty((chunk, wl.d), dtype=torch.float32, device=dev) for _ in range(2)],
+            }
+        io = self._ws[key]
+        h2d, d2h = io["h2d"], io["d2h"]
+        h2d.wait_stream(main)             # nothing is copied before the work queued so far
+        d2h.wait_stream(main)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [None, None]
+        ev_out = [None, None]
+        last = None
+        for c, c0 in enumerate(range(0, T, chunk)):
+            i, n = c % 2, min(chunk, T - c0)
+            with torch.cuda.stream(h2d):
+                if ev_done[i] is not None:
+                    h2d.wait_event(ev_done[i])       # the layer that read x buffer i is done
+                io["x"][i][:n].copy_(x_host[c0:c0 + n], non_blocking=True)
+                ev_in[i].record(h2d)
+            main.wait_event(ev_in[i])
+            if ev_out[i] is not None:
+                main.wait_event(ev_out[i])           # y buffer i has been copied out
+            b = dataclasses.replace(self.buffers(n), y=io["y"][i][:n])
+            self.forward(layer, io["x"][i][:n], b, combine=combine)
+            ev_done[i] = torch.cuda.Event()
+            ev_done[i].record(main)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(ev_done[i])
+                y_host[c0:c0 + n].copy_(io["y"][i][:n], non_blocking=True)
+                ev_out[i] = torch.cuda.Event()
+                ev_out[i].record(d2h)
+                last = ev_out[i]
+        if last is not None:
+            main.wait_event(last)
+
     def launches(self, T: int, combine: str = "kernel") -> int:
         """Kernel launches forward() makes for T tokens (route 2, permute 1 or
         3, lookup 1, each expert call 2, or 3 on the tensor-core path, combine 1)."""

@@ -152,6 +152,24 @@ def test_chunk_loop_ragged_prompt():
     assert err <= OUT_TOL, err
 
 
+def test_chunk_loop_from_host_overlapped():
+    """The pipelined host-to-host chunk loop (copies of the neighbouring chunks
+    on side streams) gives the device chunk loop's output bit for bit, ragged
+    last chunk included, and leaves nothing pending on the current stream's
+    reader."""
+    wl = CHUNKS
+    T = 2 * wl.chunk + 1000
+    stack = MoEStack(wl)
+    x = synth.gen_x(0, 0, T, wl.d, stream=34)
+    want = stack.forward_chunked(0, x_tensor(x), wl.chunk)
+    torch.cuda.synchronize()
+    x_host = torch.from_numpy(x.view(np.int16)).pin_memory()
+    y_host = torch.full((T, wl.d), float("nan"), dtype=torch.float32).pin_memory()
+    stack.forward_chunked_host(0, x_host, y_host, wl.chunk)
+    torch.cuda.current_stream().synchronize()
+    np.testing.assert_array_equal(y_host.numpy(), want.cpu().numpy())
+
+
 # ---------------------------------------------------------------- Q3 on the tensor-core path
 @pytest.fixture(scope="module")
 def tiny_q3():
