@@ -59,6 +59,9 @@ WORKLOADS = {
     "prefill_T8192_d2048_E512_k10_f768_q2": Workload("prefill_T8192_d2048_E512_k10_f768_q2", 8192, 2048, 512, 10, 768, 2),
     "stack48_T1_d2048_E512_k10_f768_q2_res25": Workload(
         "stack48_T1_d2048_E512_k10_f768_q2_res25", 1, 2048, 512, 10, 768, 2, layers=48, resident=128),
+    # the prefill layer with uniform routing (no popularity bias): ~160 tokens per expert
+    "prefill_T8192_d2048_E512_k10_f768_q2_uniform": Workload(
+        "prefill_T8192_d2048_E512_k10_f768_q2_uniform", 8192, 2048, 512, 10, 768, 2, zipf=False),
     # a 32K-token prompt through one layer in four 8192-token chunks
     "prefill_chunks4_T32768_d2048_E512_k10_f768_q2": Workload(
         "prefill_chunks4_T32768_d2048_E512_k10_f768_q2", 32768, 2048, 512, 10, 768, 2, chunk=8192),
