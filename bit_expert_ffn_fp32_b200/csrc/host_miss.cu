@@ -134,11 +134,16 @@ __attribute__((target_clones("avx512f", "avx2", "default"), noinline)) void moe_
             } else {
                 const uint8_t *hb = h + 8 * b;
                 const float *hbv = hi + size_t(b) * 64;
-                float hp[8];
-                for (int j = 0; j < 8; ++j) hp[j] = 0.f;
-                for (int i = 0; i < 8; ++i)
-                    for (int j = 0; j < 8; ++j) hp[j] += float((hb[j] >> i) & 1) * hbv[i * 8 + j];
-                const float hq = ((hp[0] + hp[1]) + (hp[2] + hp[3])) + ((hp[4] + hp[5]) + (hp[6] + hp[7]));
+                // 16 lanes: lane l takes bit 2ii + l/8 of byte l%8 (weight 8(l%8) + 2ii + l/8),
+                // whose permuted input sits at hbv[16 ii + l]
+                uint32_t hw[16];
+                for (int l = 0; l < 16; ++l) hw[l] = uint32_t(hb[l & 7]) >> (l >> 3);
+                float hp[16];
+                for (int l = 0; l < 16; ++l) hp[l] = 0.f;
+                for (int ii = 0; ii < 4; ++ii)
+                    for (int l = 0; l < 16; ++l) hp[l] += float((hw[l] >> (2 * ii)) & 1u) * hbv[16 * ii + l];
+                float hq = 0.f;
+                for (int l = 0; l < 16; l += 4) hq += (hp[l] + hp[l + 1]) + (hp[l + 2] + hp[l + 3]);
                 acc += s * ((q + 4.0f * hq) - 4.0f * bsum[b]);
             }
         }
