@@ -952,7 +952,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
         // ------------------------------------------------ router rows + activations
         float *rrows = reinterpret_cast<float *>(ring);  // router rows, then x, in the ring
         uint16_t *sx = reinterpret_cast<uint16_t *>(ring + size_t(nrows) * d * 4);
-        if (tid == 0 && nrows > 0) {
+        // layers after the first had their router rows and x staged at the end of
+        // the previous layer (while its grid barrier was pending)
+        if (l == 0 && tid == 0 && nrows > 0) {
             bar_expect(&s.rt_bar, uint32_t(nrows) * uint32_t(d) * 4u);
             bulk_copy(rrows, lp.Wr + size_t(rb) * d, uint32_t(nrows) * uint32_t(d) * 4u, &s.rt_bar);
         }
@@ -960,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
             if (tid < nrows && tid < 8) s.rbias[tid] = lp.bias ? __ldg(lp.bias + rb + tid) : 0.f;
             const uint4 *src = reinterpret_cast<const uint4 *>(lp.x);
             uint4 *dst = reinterpret_cast<uint4 *>(sx);
-            for (int i = tid; i < T * d / 8; i += kThreads) dst[i] = __ldg(src + i);
+            for (int i = tid; l == 0 && i < T * d / 8; i += kThreads) dst[i] = __ldg(src + i);
             for (int e = tid; e < E; e += kThreads) s.slot[e] = __ldg(lp.slot_of + e);
             // this CTA's slice of y starts at zero (before the grid barrier, so before any atomic)
             for (int i = cta * kThreads + tid; i < T * d; i += G * kThreads) lp.y[i] = 0.f;
@@ -1277,9 +1279,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
         // ------------------------------------------------ grid barrier: the layer is complete
         // (the next layer starts only once every contribution to this one is in y)
         if (l + 1 < p.L) {
-            __syncthreads();
+            __syncthreads();  // this layer's tasks are done with the ring
             if (tid == 0) arrive_release(p.ctr);
             bar_target += unsigned(G);
+            // the next layer's inputs (its own router rows and activations, which
+            // this layer does not produce) into the ring while the barrier is pending
+            const LayerPtrs np = layer_ptrs(p, l + 1);
+            if (tid == 0 && nrows > 0) {
+                bar_expect(&s.rt_bar, uint32_t(nrows) * uint32_t(d) * 4u);
+                bulk_copy(rrows, np.Wr + size_t(rb) * d, uint32_t(nrows) * uint32_t(d) * 4u, &s.rt_bar);
+            }
+            {
+                const uint4 *src = reinterpret_cast<const uint4 *>(np.x);
+                uint4 *dst = reinterpret_cast<uint4 *>(sx);
+                for (int i = tid; i < T * d / 8; i += kThreads) dst[i] = __ldg(src + i);
+            }
             if (tid == 0) s.ok = wait_geq(p.ctr, bar_target, p.status);
             __syncthreads();
             ok = ok && s.ok;
