@@ -13,7 +13,9 @@ Layer definition (per token t):
   4. the cache lookup: pairs whose expert has no HBM slot are misses;
   5. y_partial[t] = FFN_shared(x_t) + sum over resident selected experts of
      gate * FFN_e(x_t); y_full adds the missed experts too.
-FFN_e is the SwiGLU expert on dequantised fp64 weights.
+FFN_e is the SwiGLU expert on dequantised fp64 weights; every expert is
+dequantised by its own storage format (the layer's, or fmt_of[e] for a pool
+holding both tiers).
 """
 from __future__ import annotations
 
