@@ -42,6 +42,8 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s (decode T=1/4, 8K prefill); % of HBM / tensor roofline"
 HEADLINE = "decode_T1_d2048_E512_k10_f768_q2"
 NESTED = ("prefill_T8192_d2048_E512_k10_f768_q2", "verify_T4_d2048_E512_k10_f768_q3",
+          # wider MTP verify batches (1 token + 1 or 7 drafts) through the same layer
+          "verify_T2_d2048_E512_k10_f768_q3", "verify_T8_d2048_E512_k10_f768_q3",
           "stack48_T1_d2048_E512_k10_f768_q2_res25",
           # beyond the metric's own workloads: a 32K prompt in 8192-token chunks,
           # the 3-bit tier at prefill size and a pool holding both tiers
